@@ -1,0 +1,221 @@
+"""CPU oracle for the DSA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import this package.  The product path (``sparse_attention_long_04_b200``) never does, and
+this package never imports the product path: the two share no code.  Inputs come from the
+seeded generators in ``dsa_workloads``, which hold none of the method's arithmetic.
+
+Stages (the pages' order: "FP8 index -> top-k selection -> sparse core attention",
+"DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention (DSA)", pipeline
+summary):
+
+  indexer_rows      S[t,s] = s_k[s] sum_j w[t,j] s_q[t,j] ReLU(q[t,j].k[s]),  s <= pos(t)
+  topk_rows         k largest S per row, ties -> smaller index, all keys if fewer than k
+  sparse_mla_rows   MQA-mode attention over the selected latent rows, fp64, with LSE
+
+The C library ``dsa_oracle.c`` does the arithmetic (OpenMP over rows); this module only
+resolves which physical cache row holds logical key s of a sequence and moves bytes.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against things other
+than itself (the OCP FP8 spec values and torch's e4m3 cast, numpy matmul on the one-head
+special case, hand-worked fixtures in ``tests/golden/``, brute-force sorting, torch's fp64
+scaled-dot-product attention on the k >= context special case, and closed forms).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        L.dsa_oracle_e4m3_to_f64.restype = ctypes.c_double
+        L.dsa_oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.dsa_oracle_bf16_to_f64.restype = ctypes.c_double
+        L.dsa_oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.dsa_oracle_indexer_seq.restype = None
+        L.dsa_oracle_indexer_seq.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int64, f64p, ctypes.c_int]
+        L.dsa_oracle_topk.restype = None
+        L.dsa_oracle_topk.argtypes = [ctypes.c_int, ctypes.c_int, f64p, ctypes.c_int64,
+                                      ctypes.c_void_p, ctypes.c_void_p]
+        L.dsa_oracle_sparse_mla.restype = None
+        L.dsa_oracle_sparse_mla.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, f64p, f64p]
+        L.dsa_oracle_num_threads.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def num_threads() -> int:
+    return int(lib().dsa_oracle_num_threads())
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _np(t, dtype=None) -> np.ndarray:
+    """torch tensor / numpy array -> contiguous numpy (bf16 tensors as uint16 bit patterns)."""
+    if t is None:
+        return None
+    if hasattr(t, "detach"):
+        import torch
+        t = t.detach().cpu()
+        if t.dtype == torch.bfloat16:
+            t = t.view(torch.int16)
+            return np.ascontiguousarray(t.numpy().view(np.uint16))
+        if t.dtype == torch.float8_e4m3fn:
+            t = t.view(torch.uint8)
+        t = t.numpy()
+    a = np.ascontiguousarray(t)
+    return a.astype(dtype) if dtype is not None and a.dtype != dtype else a
+
+
+def e4m3_to_f64(byte: int) -> float:
+    return float(lib().dsa_oracle_e4m3_to_f64(int(byte)))
+
+
+def bf16_to_f64(bits: int) -> float:
+    return float(lib().dsa_oracle_bf16_to_f64(int(bits)))
+
+
+# ---- sequence geometry ------------------------------------------------------------------
+
+class Geometry:
+    """Where each query row and each logical key lives.
+
+    prefill: packed rows; row r of sequence b (cu[b] <= r < cu[b+1]) has position r - cu[b];
+             logical key s of sequence b is physical row cu[b] + s.
+    decode : row b is the new token of sequence b at position seq_lens[b] - 1; logical key s
+             is physical row block_table[b, s // bs] * bs + s % bs when a block table is
+             given, else b * max_seqlen + s.
+    """
+
+    def __init__(self, mode: str, seqlens: Sequence[int], block_table=None,
+                 max_seqlen: int = 0, block_size: int = 64):
+        self.mode = mode
+        self.seqlens = [int(x) for x in seqlens]
+        self.block_table = _np(block_table)
+        self.max_seqlen = int(max_seqlen) or max(self.seqlens)
+        self.block_size = block_size
+        self.cu = np.concatenate([[0], np.cumsum(self.seqlens)]).astype(np.int64)
+
+    @classmethod
+    def of(cls, wl) -> "Geometry":
+        return cls(wl.mode, wl.seqlens, wl.block_table, wl.max_seqlen)
+
+    def row_seq_pos(self, row: int):
+        if self.mode == "decode":
+            return row, self.seqlens[row] - 1
+        b = int(np.searchsorted(self.cu, row, side="right") - 1)
+        return b, int(row - self.cu[b])
+
+    def phys(self, b: int, s: np.ndarray) -> np.ndarray:
+        s = np.asarray(s, dtype=np.int64)
+        if self.mode == "prefill":
+            return self.cu[b] + s
+        if self.block_table is not None:
+            bs = self.block_size
+            return self.block_table[b, s // bs].astype(np.int64) * bs + s % bs
+        return b * self.max_seqlen + s
+
+
+# ---- stages --------------------------------------------------------------------------------
+
+def indexer_rows(wl, rows: Sequence[int], fp32: bool = False) -> Dict[int, np.ndarray]:
+    """Scores of each packed query row against keys 0..pos(row) of its sequence.
+    Returns {row: float64 array of length pos+1}."""
+    geo = Geometry.of(wl)
+    d = wl.dims
+    h_idx, d_idx = d["h_idx"], d["d_idx"]
+    q8 = _np(wl.q_idx, np.uint8)
+    qs = _np(wl.q_scale, np.float32)
+    w = _np(wl.w, np.float32)
+    k8 = _np(wl.k_idx, np.uint8)
+    ks = _np(wl.k_scale, np.float32)
+    by_seq: Dict[int, List[int]] = {}
+    for r in rows:
+        b, _ = geo.row_seq_pos(r)
+        by_seq.setdefault(b, []).append(int(r))
+    out: Dict[int, np.ndarray] = {}
+    for b, rs in by_seq.items():
+        pos = np.array([geo.row_seq_pos(r)[1] for r in rs], dtype=np.int32)
+        n_keys = int(pos.max()) + 1
+        phys = geo.phys(b, np.arange(n_keys))
+        kseq = np.ascontiguousarray(k8[phys])
+        kss = np.ascontiguousarray(ks[phys])
+        qq = np.ascontiguousarray(q8[rs])
+        qsc = np.ascontiguousarray(qs[rs])
+        ww = np.ascontiguousarray(w[rs])
+        res = np.full((len(rs), n_keys), np.nan, dtype=np.float64)
+        lib().dsa_oracle_indexer_seq(len(rs), h_idx, d_idx, _ptr(qq), _ptr(qsc), _ptr(ww),
+                                     _ptr(pos), n_keys, _ptr(kseq), _ptr(kss), n_keys,
+                                     _f64p(res), 1 if fp32 else 0)
+        for i, r in enumerate(rs):
+            out[r] = res[i, : pos[i] + 1].copy()
+    return out
+
+
+def topk_rows(scores: Sequence[np.ndarray], topk: int) -> np.ndarray:
+    """Selection per row under (score descending, index ascending); -1 padded.
+    Returns int32 [n_rows, topk] in selection order."""
+    n = len(scores)
+    ld = max(1, max((len(s) for s in scores), default=1))
+    mat = np.zeros((n, ld), dtype=np.float64)
+    nv = np.zeros(n, dtype=np.int32)
+    for i, s in enumerate(scores):
+        mat[i, : len(s)] = s
+        nv[i] = len(s)
+    idx = np.empty((n, topk), dtype=np.int32)
+    lib().dsa_oracle_topk(n, topk, _f64p(mat), ld, _ptr(nv), _ptr(idx))
+    return idx
+
+
+def sparse_mla_rows(wl, rows: Sequence[int], idx: np.ndarray):
+    """Attention of each packed query row over its selected logical keys ``idx`` (int32
+    [n_rows, k], -1 = unused).  Returns (O float64 [n, h, d_v], LSE float64 [n, h])."""
+    geo = Geometry.of(wl)
+    d = wl.dims
+    h, d_qk, d_v = d["h"], d["d_qk"], d["d_v"]
+    idx = np.asarray(idx)
+    k = idx.shape[1]
+    phys = np.full(idx.shape, -1, dtype=np.int64)
+    for i, r in enumerate(rows):
+        b, _ = geo.row_seq_pos(r)
+        sel = idx[i] >= 0
+        phys[i, sel] = geo.phys(b, idx[i, sel])
+    q = _np(wl.q)
+    qq = np.ascontiguousarray(q[list(rows)])
+    kv = _np(wl.kv)
+    out = np.empty((len(rows), h, d_v), dtype=np.float64)
+    lse = np.empty((len(rows), h), dtype=np.float64)
+    lib().dsa_oracle_sparse_mla(len(rows), h, d_qk, d_v, float(wl.softmax_scale), _ptr(qq),
+                                _ptr(kv), _ptr(phys), k, _f64p(out), _f64p(lse))
+    return out, lse
+
+
+def forward_rows(wl, rows: Sequence[int]):
+    """All three stages for the given rows: (scores dict, idx, O, LSE)."""
+    sc = indexer_rows(wl, rows)
+    idx = topk_rows([sc[r] for r in rows], wl.dims["topk"])
+    o, lse = sparse_mla_rows(wl, rows, idx)
+    return sc, idx, o, lse

@@ -1,0 +1,309 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+Runs without a GPU.  Sources of truth used here: the OCP FP8 E4M3 field definition and
+torch's float8_e4m3fn cast; numpy matmul (the one-head, unit-weight special case of the
+indexer); hand-worked fixtures under tests/golden/; brute-force sorting; torch's fp64
+scaled_dot_product_attention and logsumexp (the k >= context special case); closed forms.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import reference_np
+from dsa_workloads import make_prefill, make_decode, quantize_e4m3_rows
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- input decoding
+
+def test_e4m3_spec_values():
+    # OCP FP8 E4M3: max finite 448 (0x7E), min subnormal 2^-9 (0x01), min normal 2^-6 (0x08),
+    # 1.0 = 0x38, NaN = 0x7F / 0xFF, negative zero 0x80
+    assert oracle.e4m3_to_f64(0x7E) == 448.0
+    assert oracle.e4m3_to_f64(0xFE) == -448.0
+    assert oracle.e4m3_to_f64(0x01) == 2.0 ** -9
+    assert oracle.e4m3_to_f64(0x07) == 7 * 2.0 ** -9
+    assert oracle.e4m3_to_f64(0x08) == 2.0 ** -6
+    assert oracle.e4m3_to_f64(0x38) == 1.0
+    assert oracle.e4m3_to_f64(0x39) == 1.125
+    assert math.isnan(oracle.e4m3_to_f64(0x7F)) and math.isnan(oracle.e4m3_to_f64(0xFF))
+    assert math.copysign(1.0, oracle.e4m3_to_f64(0x80)) == -1.0
+
+
+def test_e4m3_all_codes_match_torch_cast():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle.e4m3_to_f64(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(mine))
+    assert np.array_equal(ref[~nan], mine[~nan])
+    tw = reference_np.e4m3_table()
+    assert np.array_equal(np.isnan(tw), nan) and np.array_equal(tw[~nan], ref[~nan])
+
+
+def test_bf16_decode_matches_torch():
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn(4096, generator=g) * 1e3).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    mine = np.array([oracle.bf16_to_f64(b) for b in bits[:512]])
+    assert np.array_equal(mine, x[:512].to(torch.float64).numpy())
+    assert np.array_equal(reference_np.bf16_to_f64(bits), x.to(torch.float64).numpy())
+
+
+# ---------------------------------------------------------------- indexer
+
+class _W:
+    """Minimal workload stand-in for the oracle's duck-typed inputs."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def _one_seq(q8, qs, w, k8, ks, h_idx, d_idx, d=None):
+    T = q8.shape[0]
+    return _W(mode="prefill", seqlens=[T], block_table=None, max_seqlen=T,
+              dims=dict(h_idx=h_idx, d_idx=d_idx, **(d or {})), q_idx=q8, q_scale=qs, w=w,
+              k_idx=k8, k_scale=ks)
+
+
+def test_indexer_hand_fixture():
+    g = _load("indexer_hand.json")
+    q8 = np.array([g["q_codes"]], dtype=np.uint8)              # one query row
+    k8 = np.array(g["k_codes"], dtype=np.uint8)
+    # the codes decode to the stated values (pins the fixture itself)
+    dec = torch.from_numpy(k8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(dec, np.array(g["k_values"], dtype=np.float64))
+    # query row sits at position pos = 2 of a 3-token sequence: pad with two dummy rows
+    q8 = np.concatenate([np.zeros((2, 2, 4), np.uint8), q8])
+    qs = np.array([[1, 1], [1, 1], g["q_scale"]], np.float32)
+    w = np.array([[0, 0], [0, 0], g["w"]], np.float32)
+    wl = _one_seq(q8, qs, w, k8, np.array(g["k_scale"], np.float32), 2, 4)
+    for fp32 in (False, True):
+        got = oracle.indexer_rows(wl, [2], fp32=fp32)[2]
+        assert np.array_equal(got, np.array(g["expected"]))
+    # causality: the row at position 1 sees keys 0..1 only
+    assert len(oracle.indexer_rows(wl, [1])[1]) == 2
+
+
+def test_indexer_one_head_is_relu_matmul():
+    rng = np.random.default_rng(0)
+    T, D = 37, 32
+    q = torch.from_numpy(rng.standard_normal((T, 1, D)) * 4).float()
+    k = torch.from_numpy(rng.standard_normal((T, D)) * 4).float()
+    q8 = q.to(torch.float8_e4m3fn)
+    k8 = k.to(torch.float8_e4m3fn)
+    ones_q = np.ones((T, 1), np.float32)
+    wl = _one_seq(q8.view(torch.uint8).numpy(), ones_q, ones_q, k8.view(torch.uint8).numpy(),
+                  np.ones(T, np.float32), 1, D)
+    ref = np.maximum(q8.double().numpy()[:, 0, :] @ k8.double().numpy().T, 0.0)  # numpy matmul
+    got = oracle.indexer_rows(wl, list(range(T)))
+    for t in range(T):
+        assert np.array_equal(got[t], ref[t, : t + 1])
+
+
+def test_indexer_scale_homogeneity_and_head_additivity():
+    rng = np.random.default_rng(1)
+    T, H, D = 20, 3, 32
+    q8 = rng.integers(0, 256, (T, H, D), dtype=np.uint8)
+    q8[(q8 & 0x7F) == 0x7F] = 0x38                   # no NaN codes
+    k8 = rng.integers(0, 256, (T, D), dtype=np.uint8)
+    k8[(k8 & 0x7F) == 0x7F] = 0x38
+    qs = rng.uniform(0.5, 2, (T, H)).astype(np.float32)
+    w = rng.uniform(0, 1, (T, H)).astype(np.float32)
+    ks = rng.uniform(0.5, 2, T).astype(np.float32)
+    base = oracle.indexer_rows(_one_seq(q8, qs, w, k8, ks, H, D), range(T))
+    scaled = oracle.indexer_rows(_one_seq(q8, qs * 2, w * 4, k8, ks * 0.5, H, D), range(T))
+    for t in range(T):
+        assert np.array_equal(scaled[t], base[t] * 4.0)       # powers of two: exact
+    # additivity over heads: S(all heads) = sum_j S(head j alone)
+    tot = np.zeros(T)
+    parts = [oracle.indexer_rows(_one_seq(np.ascontiguousarray(q8[:, j:j + 1]),
+                                          np.ascontiguousarray(qs[:, j:j + 1]),
+                                          np.ascontiguousarray(w[:, j:j + 1]), k8, ks, 1, D),
+                                 [T - 1])[T - 1] for j in range(H)]
+    np.testing.assert_allclose(base[T - 1], sum(parts), rtol=1e-12, atol=0)
+    # and each part really is one head: a head with weight 0 contributes nothing
+    w0 = w.copy()
+    w0[:, 1] = 0
+    no1 = oracle.indexer_rows(_one_seq(q8, qs, w0, k8, ks, H, D), [T - 1])[T - 1]
+    np.testing.assert_allclose(no1, parts[0] + parts[2], rtol=1e-12, atol=0)
+
+
+def test_indexer_fp32_path_close_to_fp64_and_numpy_twin():
+    wl = make_prefill(99, [300], dict(h_idx=4, d_idx=32, topk=64, h=4, d_qk=32, d_v=16),
+                      needles=8, device="cpu", seed=5)
+    rows = [0, 1, 127, 128, 299]
+    a = oracle.indexer_rows(wl, rows)
+    b = oracle.indexer_rows(wl, rows, fp32=True)
+    tw = reference_np.indexer(wl.q_idx.numpy(), wl.q_scale.numpy(), wl.w.numpy(),
+                              wl.k_idx.numpy(), wl.k_scale.numpy())
+    for r in rows:
+        np.testing.assert_allclose(b[r], a[r], rtol=1e-5, atol=1e-6 * a[r].max())
+        np.testing.assert_allclose(a[r], tw[r, : r + 1], rtol=1e-12, atol=1e-12)
+
+
+def test_paged_geometry_hand_and_equivalence():
+    geo = oracle.Geometry("decode", [100], block_table=np.array([[3, 1]]), max_seqlen=100)
+    assert geo.phys(0, np.array([5, 70])).tolist() == [3 * 64 + 5, 1 * 64 + 6]
+    dims = dict(h_idx=4, d_idx=32, topk=64, h=4, d_qk=32, d_v=16)
+    wp = make_decode(98, 3, [130, 64, 200], dims, boost=0.05, paged=True, device="cpu",
+                     seed=11, total_blocks=20)
+    # the same data laid out contiguously per sequence (gathered here with torch indexing)
+    bt = wp.block_table.long()
+    L = max(wp.seqlens)
+    idx = torch.stack([bt[b, torch.arange(L) // 64] * 64 + torch.arange(L) % 64
+                       for b in range(3)]).reshape(-1)
+    wc = _W(**{**wp.__dict__, "block_table": None, "k_idx": wp.k_idx[idx],
+               "k_scale": wp.k_scale[idx], "kv": wp.kv[idx]})
+    a = oracle.indexer_rows(wp, [0, 1, 2])
+    c = oracle.indexer_rows(wc, [0, 1, 2])
+    for r in range(3):
+        assert len(a[r]) == wp.seqlens[r]
+        assert np.array_equal(a[r], c[r])
+
+
+# ---------------------------------------------------------------- top-k
+
+def test_topk_hand_fixture():
+    for case in _load("topk_hand.json")["cases"]:
+        got = oracle.topk_rows([np.array(case["scores"], float)], case["k"])[0]
+        assert got.tolist() == case["expected"], case
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_brute_force(ties):
+    rng = np.random.default_rng(7 + ties)
+    rows = []
+    for n in [1, 5, 63, 64, 65, 500, 3000]:
+        s = rng.integers(0, 6, n).astype(float) if ties else rng.standard_normal(n)
+        rows.append(s)
+    k = 64
+    got = oracle.topk_rows(rows, k)
+    for s, g in zip(rows, got):
+        brute = sorted(range(len(s)), key=lambda i: (-s[i], i))[:k]
+        assert g.tolist() == brute + [-1] * (k - len(brute))
+        assert g.tolist() == reference_np.topk(s, k).tolist()
+
+
+def test_topk_permutation_invariance_tie_free():
+    rng = np.random.default_rng(8)
+    s = rng.standard_normal(5000)
+    assert len(np.unique(s)) == len(s)
+    perm = rng.permutation(len(s))
+    a = set(oracle.topk_rows([s], 100)[0].tolist())
+    b = oracle.topk_rows([s[perm]], 100)[0]
+    assert set(perm[b].tolist()) == a
+
+
+# ---------------------------------------------------------------- sparse attention
+
+def _tiny_attn_workload(L=40, h=4, d_qk=24, d_v=16, seed=2):
+    return make_prefill(97, [L], dict(h_idx=4, d_idx=32, topk=8, h=h, d_qk=d_qk, d_v=d_v),
+                        needles=0, device="cpu", seed=seed, softmax_scale=0.3)
+
+
+def test_attention_full_set_equals_torch_sdpa_causal_mqa():
+    wl = _tiny_attn_workload()
+    L, h, d_v = 40, 4, 16
+    rows = list(range(L))
+    idx = np.array([list(range(t + 1)) + [-1] * (L - t - 1) for t in rows], np.int32)
+    o, lse = oracle.sparse_mla_rows(wl, rows, idx)
+    q = wl.q.double().permute(1, 0, 2)                  # [h, L, d_qk]
+    kv = wl.kv.double()
+    k = kv.unsqueeze(0).expand(h, -1, -1)               # MQA: one KV row shared by all heads
+    v = kv[:, :d_v].unsqueeze(0).expand(h, -1, -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=0.3)
+    np.testing.assert_allclose(o, ref.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+    logits = torch.matmul(q, k.transpose(1, 2)) * 0.3
+    logits = logits.masked_fill(torch.triu(torch.ones(L, L, dtype=torch.bool), 1), -math.inf)
+    ref_lse = torch.logsumexp(logits, dim=-1).permute(1, 0).numpy()
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_k1_and_identical_rows_closed_forms():
+    wl = _tiny_attn_workload()
+    qd = wl.q.double().numpy()
+    kvd = wl.kv.double().numpy()
+    # k = 1: output is that row's value part, LSE is its scaled logit
+    o, lse = oracle.sparse_mla_rows(wl, [30], np.array([[17, -1, -1]], np.int32))
+    assert np.array_equal(o[0], np.broadcast_to(kvd[17, :16], (4, 16)))
+    np.testing.assert_allclose(lse[0], 0.3 * qd[30] @ kvd[17], rtol=1e-13)
+    # n identical rows: output that row, LSE = ln n + logit
+    o, lse = oracle.sparse_mla_rows(wl, [30], np.array([[9] * 5], np.int32))
+    np.testing.assert_allclose(o[0], np.broadcast_to(kvd[9, :16], (4, 16)), rtol=1e-14)
+    np.testing.assert_allclose(lse[0], math.log(5) + 0.3 * qd[30] @ kvd[9], rtol=1e-13)
+
+
+def test_attention_order_and_padding_invariance_and_numpy_twin():
+    wl = _tiny_attn_workload()
+    sel = np.array([[3, 11, 0, 25, 7, 30, -1, -1]], np.int32)
+    o1, l1 = oracle.sparse_mla_rows(wl, [30], sel)
+    o2, l2 = oracle.sparse_mla_rows(wl, [30], np.array([[-1, 30, 7, -1, 25, 0, 11, 3]],
+                                                       np.int32))
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13)
+    qb = wl.q.view(torch.int16).numpy().view(np.uint16)[30]
+    kvb = wl.kv.view(torch.int16).numpy().view(np.uint16)
+    o3, l3 = reference_np.sparse_attention(qb, kvb, sel[0], 0.3, 16)
+    np.testing.assert_allclose(o1[0], o3, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l1[0], l3, rtol=1e-12)
+
+
+def test_attention_dense_masked_softmax_equals_sparse():
+    """Dense attention with a top-k mask (numpy, all keys, -inf outside the set) equals the
+    sparse oracle over the set."""
+    wl = _tiny_attn_workload()
+    qd = wl.q.double().numpy()[33]
+    kvd = wl.kv.double().numpy()
+    sel = [2, 5, 8, 13, 21, 33]
+    logits = 0.3 * qd @ kvd[:34].T
+    mask = np.full(34, -np.inf)
+    mask[sel] = 0
+    z = logits + mask
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    ref = (p / p.sum(axis=1, keepdims=True)) @ kvd[:34, :16]
+    o, _ = oracle.sparse_mla_rows(wl, [33], np.array([sel], np.int32))
+    np.testing.assert_allclose(o[0], ref, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- whole pipeline
+
+def test_pipeline_rows_before_k_equal_dense_causal():
+    """Rows with fewer than k prior tokens keep all of them, so the sparse result is dense
+    causal MQA attention (torch fp64 SDPA)."""
+    dims = dict(h_idx=4, d_idx=32, topk=64, h=4, d_qk=32, d_v=16)
+    wl = make_prefill(96, [100], dims, needles=8, device="cpu", seed=4)
+    rows = [0, 1, 30, 63]
+    _, idx, o, lse = oracle.forward_rows(wl, rows)
+    for i, t in enumerate(rows):
+        assert sorted(idx[i][idx[i] >= 0].tolist()) == list(range(t + 1))
+    q = wl.q.double().permute(1, 0, 2)[:, :64]
+    kv = wl.kv.double()[:64]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, kv.unsqueeze(0).expand(4, -1, -1), kv[:, :16].unsqueeze(0).expand(4, -1, -1),
+        is_causal=True, scale=wl.softmax_scale).permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(o, ref[rows], rtol=1e-10, atol=1e-12)
+
+
+def test_workload_quantiser_roundtrip_bound():
+    """The generator's e4m3 bytes decode to within half an e4m3 ulp (2^-4 relative) of the
+    drawn values: the inputs the oracle and the kernels share are what they claim."""
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(64, 8, 32, generator=g)
+    q8, s = quantize_e4m3_rows(x, 2)
+    dec = q8.view(torch.float8_e4m3fn).double() * s.double()[:, None, None]
+    err = (dec - x.double()).abs()
+    amax = x.abs().amax(dim=(1, 2)).double()
+    assert bool((err <= torch.maximum(x.double().abs() * 2 ** -4,
+                                      (amax / 448 * 2 ** -9)[:, None, None] * 1.0001)).all())
