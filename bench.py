@@ -1,0 +1,441 @@
+"""Benchmark of the DSA hot path on B200: decode at 128k context (primary line) and varlen
+prefill up to 128k (secondary), plus the CPU oracle as the reported baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-prefill]
+
+One step = one pass of the whole path (indexer -> top-k -> sparse MLA-MQA) over one batch:
+  decode  : 64 sequences x 131072 context, 64-token pages, random block table (one new token
+            each); inputs (11 GB of caches) are far larger than L2, so no flush is needed
+  prefill : 8 packed causal sequences {4096 ... 131072}, T = 276480 rows
+With N > 1 (torchrun) every rank runs its own independent decode batch (weak scaling, no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DECODE_CFG, PREFILL_CFG = 3, 5
+METRIC = "DSA decode tokens/s and prefill tokens/s at 128k ctx; % of HBM/tensor roofline"
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            sel = str(device_index)
+        self.sel = sel
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ work model
+
+def decode_algorithmic_bytes(wl):
+    """Bytes the decode step must move at minimum: indexer keys + scales of every context token,
+    the selected latent rows, the per-token query inputs and the outputs."""
+    d = wl.dims
+    ctx = sum(wl.seqlens)
+    k_i = ctx * (d["d_idx"] + 4)
+    sel = sum(min(L, d["topk"]) for L in wl.seqlens) * d["d_qk"] * 2
+    q_in = wl.batch * (d["h"] * d["d_qk"] * 2 + d["h_idx"] * (d["d_idx"] + 8))
+    out = wl.batch * d["h"] * (d["d_v"] * 2 + 4)
+    return dict(indexer=k_i, total=k_i + sel + q_in + out)
+
+
+def prefill_flops(seqlens, d):
+    """Causal algorithmic FLOPs: indexer 2*H_I*D_I per (query, prior key) pair (fp8); attention
+    2*H*(D_qk + D_v) per (query, selected key) pair (bf16)."""
+    K = d["topk"]
+    pairs = sum(L * (L + 1) // 2 for L in seqlens)
+    sel = 0
+    for L in seqlens:
+        m = min(L, K)
+        sel += m * (m + 1) // 2 + (L - m) * K
+    return (2 * d["h_idx"] * d["d_idx"] * pairs, 2 * d["h"] * (d["d_qk"] + d["d_v"]) * sel)
+
+
+# ------------------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    import sparse_attention_long_04_b200 as dsa
+    from dsa_workloads import make_config, CONFIGS
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = read_peaks()
+    stream = torch.cuda.current_stream()
+    wl = make_config(DECODE_CFG, device=dev, seed=1000 + DECODE_CFG + 7919 * rank)
+    d = wl.dims
+    pb = dsa.problem_of(wl)
+    B = wl.batch
+    ld = (wl.max_seqlen + 3) // 4 * 4
+    scores = torch.empty(B, ld, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, d["topk"], dtype=torch.int32, device=dev)
+    out = torch.empty(B, d["h"], d["d_v"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, d["h"], dtype=torch.float32, device=dev)
+    mla_ws_bytes = dsa.dsa_sparse_mla_workspace_size(pb, B)
+    mla_ws = torch.empty(max(mla_ws_bytes, 16), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    launches_per_step = 3 + (1 if mla_ws_bytes > 0 else 0)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.check(dsa.dsa_indexer_scores(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx, wl.k_scale,
+                                         0, B, scores, ld, status, stream), "indexer")
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.check(dsa.dsa_topk(pb, scores, ld, 0, B, idx, status, stream), "topk")
+        if ev is not None:
+            ev[2].record(stream)
+        dsa.check(dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, idx, 0, B, out, lse, mla_ws,
+                                         mla_ws_bytes, status, stream), "sparse_mla")
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, raw = dsa.dsa_read_device_status(status, stream)
+    dsa.check(st, "device status after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.25)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    k_ms = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+            for e in evs]
+    per_kernel = [sum(x[j] for x in k_ms) / len(k_ms) for j in range(3)]
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    value = world * B / (ms_step / 1e3)
+
+    # ---- end to end through the public call, host buffers, copies inside the timed region
+    fwd = dsa.Forward(wl, keep_idx=False)
+    host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("q", "q_idx", "q_scale", "w",
+                                                              "seq_lens")}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4
+
+    def e2e_step():
+        for k, t in host_in.items():
+            getattr(wl, k).copy_(t, non_blocking=True)
+        dsa.check(fwd(stream), "dsa_forward")
+        host_out.copy_(fwd.out, non_blocking=True)
+        host_lse.copy_(fwd.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * B / (e2e_ms / args.steps / 1e3)
+    st, raw = dsa.dsa_read_device_status(status, stream)
+    dsa.check(st, "device status after timing")
+
+    work = decode_algorithmic_bytes(wl)
+    idx_gbs = work["indexer"] / (per_kernel[0] / 1e3) / 1e9
+    step_gbs = work["total"] / (ms_step / 1e3) / 1e9
+    traffic = load_traffic("indexer_decode")
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3+bf16",
+        "data": "synthetic",
+        "config": {"workload": CONFIGS[DECODE_CFG]["name"], "batch": B,
+                   "context": wl.max_seqlen, "page": 64, "topk": d["topk"],
+                   "indexer": f"{d['h_idx']}x{d['d_idx']} e4m3", "heads": d["h"],
+                   "latent": d["d_qk"], "d_v": d["d_v"],
+                   "l2": "inputs larger than L2 (11 GB of caches per step)",
+                   "parallelism": f"replicas{world}"},
+        "roofline": {"kernel": "dsa_indexer_kernel (decode)", "bound": "hbm",
+                     "achieved": round(idx_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": round(idx_gbs / peaks["hbm"], 4),
+                     "traffic": traffic, "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_launch": work["indexer"]},
+        "step_roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "unit": "GB/s",
+                          "frac": round(step_gbs / peaks["hbm"], 4),
+                          "algorithmic_bytes_per_step": work["total"]},
+        "kernel_ms": {"indexer": round(per_kernel[0], 4), "topk": round(per_kernel[1], 4),
+                      "sparse_mla": round(per_kernel[2], 4)},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "per step: new-token inputs (q, q_idx, q_scale, w, seq_lens) copied "
+                        "from pinned host memory, dsa_forward, out + lse copied back; the "
+                        "paged caches stay resident"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    del fwd
+    if not args.no_prefill:
+        del scores, idx, out, lse
+        line["prefill"] = run_prefill(args, dsa, dev, stream, peaks, rank, world)
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    return line
+
+
+def run_prefill(args, dsa, dev, stream, peaks, rank, world):
+    from dsa_workloads import make_config, CONFIGS
+    wl = make_config(PREFILL_CFG, device=dev, seed=1000 + PREFILL_CFG + 7919 * rank)
+    fwd = dsa.Forward(wl, keep_idx=False)
+    steps = max(1, min(args.steps, args.prefill_steps))
+    for _ in range(max(1, min(args.warmup, 3))):
+        dsa.check(fwd(stream), "prefill forward")
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        dsa.check(fwd(stream), "prefill forward")
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / steps
+    st, raw = dsa.dsa_read_device_status(fwd.status, stream)
+    dsa.check(st, "prefill device status")
+    f8, f16 = prefill_flops(wl.seqlens, wl.dims)
+    p8 = 2.0 * peaks["bf16_sustained"]
+    ideal_ms = (f8 / (p8 * 1e12) + f16 / (peaks["bf16_sustained"] * 1e12)) * 1e3
+    T = wl.total_rows
+    res = {"workload": CONFIGS[PREFILL_CFG]["name"], "value": round(world * T / (ms_step / 1e3), 1),
+           "unit": "tokens/s", "ms_per_step": round(ms_step, 3), "steps": steps,
+           "roofline": {"bound": "tensor", "frac": round(ideal_ms / ms_step, 4),
+                        "ideal_ms": round(ideal_ms, 3), "flops_fp8": f8, "flops_bf16": f16,
+                        "peak_bf16_tflops": peaks["bf16_sustained"],
+                        "peak_fp8_tflops": p8,
+                        "peak_note": "bf16 sustained measured; fp8 = 2x bf16 (nominal ratio)"}}
+    del fwd, wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def load_traffic(name):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        return json.load(f).get(name)
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(wl, n_rows):
+    """A decode workload holding only `n_rows` sequences of `wl`, laid out contiguously on the
+    host (a gather of the inputs; no arithmetic), for timing the oracle."""
+    from dsa_workloads import Workload
+    rows = list(range(n_rows))
+    L = wl.max_seqlen
+    bt = wl.block_table[:n_rows].long()
+    phys = (bt[:, torch.arange(L, device=bt.device) // 64] * 64 +
+            torch.arange(L, device=bt.device) % 64).reshape(-1)
+    return Workload(cfg_id=wl.cfg_id, name=wl.name, mode="decode", dims=wl.dims,
+                    softmax_scale=wl.softmax_scale, seqlens=wl.seqlens[:n_rows],
+                    q_idx=wl.q_idx[rows].cpu(), q_scale=wl.q_scale[rows].cpu(),
+                    w=wl.w[rows].cpu(), k_idx=wl.k_idx[phys].cpu(),
+                    k_scale=wl.k_scale[phys].cpu(), q=wl.q[rows].cpu(), kv=wl.kv[phys].cpu(),
+                    seq_lens=wl.seq_lens[:n_rows].cpu(), block_table=None, max_seqlen=L)
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    import oracle
+    threads = oracle.num_threads()
+    n = max(1, min(wl.batch, threads))
+    sub = oracle_sample(wl, n)
+    t0 = time.perf_counter()
+    oracle.forward_rows(sub, list(range(n)))
+    dt = time.perf_counter() - t0
+    if dt < budget_s / 3 and n < wl.batch:          # grow the sample toward the budget
+        n2 = min(wl.batch, max(n + 1, int(n * budget_s / 2 / max(dt, 1e-3))))
+        sub = oracle_sample(wl, n2)
+        t0 = time.perf_counter()
+        oracle.forward_rows(sub, list(range(n2)))
+        dt = time.perf_counter() - t0
+        n = n2
+    return {"value": round(n / dt, 4), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {wl.batch} decode rows of {wl.name} (full 131072-key indexer, "
+                      f"top-k, fp64 attention per row), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores, on the decode workload's metric."""
+    if rank != 0:
+        return None
+    from dsa_workloads import make_config, CONFIGS
+    import oracle
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    wl = make_config(DECODE_CFG, device=dev)
+    threads = oracle.num_threads()
+    n = max(1, min(wl.batch, threads))
+    sub = oracle_sample(wl, n)
+    for _ in range(args.warmup):
+        oracle.forward_rows(sub, [0])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward_rows(sub, list(range(n)))
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": CONFIGS[DECODE_CFG]["name"], "batch": wl.batch,
+                       "context": wl.max_seqlen, "parallelism": "replicas1"},
+            "cpu_baseline": {"value": round(value, 4), "kind": "oracle", "cores": threads,
+                             "sample": f"{n} decode rows per step of {wl.name}"},
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

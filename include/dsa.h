@@ -1,0 +1,184 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The path has three stages, in the order "FP8 index -> top-k selection -> sparse core
+ * attention" ("DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention
+ * (DSA)", pipeline summary):
+ *
+ *   dsa_indexer_scores  lightning indexer: for query row t and every prior key s <= pos(t)
+ *                       of its sequence,
+ *                         S[t,s] = k_scale[s] * sum_j w[t,j] * q_scale[t,j]
+ *                                    * ReLU( sum_i q_idx[t,j,i] * k_idx[s,i] )
+ *                       with e4m3 q_idx / k_idx and fp32 accumulation (the indexer "scores
+ *                       context tokens", same page, two-stage attention path; "Lightning
+ *                       Indexer computes lightweight index scores", maplevalley page,
+ *                       section 1; the weighted sum of ReLU(q.k) over indexer heads is the
+ *                       formula this library implements)
+ *   dsa_topk            per query row, the topk keys with the largest S; equal scores go to
+ *                       the smaller key index; rows with fewer than topk prior keys keep
+ *                       all of them (top-k=2048, same page, "Training signal"; "the Top-k
+ *                       selector keeps only k key-value pairs per query", maplevalley page,
+ *                       section 1)
+ *   dsa_sparse_mla_fwd  MLA in MQA mode over the selected latent rows: every selected
+ *                       576-d latent row is shared by all query heads (same page,
+ *                       "Instantiation"); logits sigma * q.kv, softmax, output = weighted
+ *                       sum of the first d_v latent dims, plus the natural-log LSE
+ *   dsa_forward         the three stages back to back, for prefill (packed varlen causal
+ *                       rows) and decode (one new token per sequence, paged or contiguous
+ *                       caches)
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and contiguous.
+ *     The library allocates nothing and keeps no state apart from a per-device attribute
+ *     cache.  dims / seqs structs are HOST pointers, read during the call only.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Argument errors are returned synchronously, before anything is launched.
+ *     A failed launch returns DSA_ERR_CUDA.
+ *   - `dev_status` is an optional caller-owned DEVICE int32.  Kernels OR in
+ *     DSA_DEVICE_TIMEOUT when a bounded wait gave up (the kernel then unwinds instead of
+ *     hanging) and DSA_DEVICE_BAD_INDEX when an index or block-table entry points outside
+ *     the caches (that entry is then skipped).  Clear it before the call; read it with
+ *     dsa_read_device_status.  NULL disables the reporting (the kernels still unwind).
+ *   - Alignment: every tensor pointer must be 16-byte aligned, ld_scores a multiple of 4;
+ *     otherwise DSA_ERR_MISALIGNED.
+ *   - Supported shapes: (h_idx, d_idx) in {(64,128), (4,32)}; (h, d_qk, d_v) in
+ *     {(128,576,512), (16,160,128)}; topk a multiple of 64 in [64, 2048]; block_size 64.
+ *     Decode needs (h_idx, d_idx) = (64,128).  Anything else: DSA_ERR_UNSUPPORTED_SHAPE.
+ *
+ * Geometry (dsa_seqs_t):
+ *   PREFILL: total_rows packed query rows; row r of sequence b (cu[b] <= r < cu[b+1]) has
+ *            position pos = r - cu[b] and sees keys 0..pos of its own sequence, which are
+ *            the same packed rows of k_idx / k_scale / kv (physical row cu[b] + s).
+ *   DECODE : one query row per sequence b (total_rows = batch) at position seq_lens[b]-1;
+ *            it sees keys 0..seq_lens[b]-1.  Logical key s of sequence b is physical row
+ *            block_table[b, s / block_size] * block_size + s % block_size, or, with
+ *            block_table == NULL, b * max_seqlen + s.
+ *   Key indices returned by dsa_topk and consumed by dsa_sparse_mla_fwd are LOGICAL
+ *   positions within the sequence.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+typedef struct CUstream_st* dsa_stream_t; /* cudaStream_t */
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, inconsistent geometry */
+  DSA_ERR_UNSUPPORTED_SHAPE = 2,   /* dims outside the supported set */
+  DSA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the *_workspace_size answer */
+  DSA_ERR_MISALIGNED = 4,          /* pointer not 16-byte aligned or ld not a multiple of 4 */
+  DSA_ERR_BAD_INDEX = 5,           /* device status: an index left the caches */
+  DSA_ERR_TIMEOUT = 6,             /* device status: a bounded wait gave up */
+  DSA_ERR_CUDA = 7                 /* a CUDA runtime call or launch failed */
+} dsa_status_t;
+
+/* Bits of the device status word. */
+#define DSA_DEVICE_TIMEOUT 1
+#define DSA_DEVICE_BAD_INDEX 2
+
+enum { DSA_PREFILL = 0, DSA_DECODE = 1 };
+
+typedef struct {
+  int32_t h_idx;        /* indexer heads */
+  int32_t d_idx;        /* indexer head dim (e4m3 bytes per key row) */
+  int32_t h;            /* query heads */
+  int32_t d_qk;         /* latent + RoPE dims of q and of a latent KV row */
+  int32_t d_v;          /* value dims = the first d_v dims of a latent KV row */
+  int32_t topk;         /* keys kept per query row */
+  int32_t block_size;   /* page size of the decode caches (64) */
+  float softmax_scale;  /* sigma in the logits sigma * q.kv */
+} dsa_dims_t;
+
+typedef struct {
+  int32_t mode;                  /* DSA_PREFILL or DSA_DECODE */
+  int32_t batch;                 /* sequences */
+  int32_t total_rows;            /* query rows: prefill cu_seqlens[batch]; decode batch */
+  int32_t max_seqlen;            /* longest sequence; decode without block table: row stride */
+  int64_t num_kv_rows;           /* physical rows of k_idx, k_scale and kv */
+  const int32_t* cu_seqlens;     /* PREFILL: device [batch+1], cu[0] = 0, non-decreasing */
+  const int32_t* cu_seqlens_host;/* PREFILL: host copy of cu_seqlens, used for planning */
+  const int32_t* seq_lens;       /* DECODE : device [batch], each in [1, max_seqlen] */
+  const int32_t* block_table;    /* DECODE : device [batch, max_blocks] or NULL */
+  int32_t max_blocks;            /* DECODE : columns of block_table */
+} dsa_seqs_t;
+
+/* Stage 1.  Scores of query rows [row_begin, row_begin + row_count) against their prior
+ * keys.  PREFILL rows may span several sequences.
+ *   q_idx   e4m3 [total_rows, h_idx, d_idx]      q_scale, w  fp32 [total_rows, h_idx]
+ *   k_idx   e4m3 [num_kv_rows, d_idx]            k_scale     fp32 [num_kv_rows]
+ *   scores  fp32 [row_count, ld_scores]: scores[(t - row_begin) * ld + s] for s <= pos(t);
+ *           entries past pos(t) are left untouched.  ld_scores >= max pos(t) + 1 over
+ *           the rows and a multiple of 4. */
+DSA_API dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                const uint8_t* q_idx, const float* q_scale, const float* w,
+                                const uint8_t* k_idx, const float* k_scale, int32_t row_begin,
+                                int32_t row_count, float* scores, int64_t ld_scores,
+                                int32_t* dev_status, dsa_stream_t stream);
+
+/* Stage 2.  Exact top-k of each row of `scores` (layout as written by dsa_indexer_scores)
+ * over keys 0..pos(t).  idx int32 [row_count, topk]: the selected LOGICAL key indices in
+ * increasing order, then -1 padding when pos(t) + 1 < topk.  The set is unique: larger
+ * score first, equal scores broken by the smaller index (-0 and +0 compare equal). */
+DSA_API dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
+                      int64_t ld_scores, int32_t row_begin, int32_t row_count, int32_t* idx,
+                      int32_t* dev_status, dsa_stream_t stream);
+
+/* Bytes of workspace dsa_sparse_mla_fwd needs for `row_count` rows (split-KV partials when
+ * few rows leave SMs idle).  0 is a valid answer. */
+DSA_API size_t dsa_sparse_mla_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                     int32_t row_count);
+
+/* Stage 3.  Sparse MLA-MQA forward for rows [row_begin, row_begin + row_count).
+ *   q    bf16 [total_rows, h, d_qk]   (indexed by absolute row)
+ *   kv   bf16 [num_kv_rows, d_qk]
+ *   idx  int32 [row_count, topk] logical key indices (-1 = unused), relative to row_begin
+ *   out  bf16 [total_rows, h, d_v] and lse fp32 [total_rows, h] (absolute rows); a row
+ *        with no valid index gets out = 0 and lse = -inf. */
+DSA_API dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                int32_t row_begin, int32_t row_count, uint16_t* out,
+                                float* lse, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, dsa_stream_t stream);
+
+/* Bytes of workspace dsa_forward needs (score slab for one row chunk, chunk indices when
+ * idx_out is NULL, split-KV partials).  Larger workspaces allow larger prefill chunks. */
+DSA_API size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs);
+
+/* The whole path for all seqs->total_rows query rows.  Inputs as for the three stages.
+ *   idx_out  optional int32 [total_rows, topk]: the selected indices (NULL = not kept)
+ *   out, lse as for dsa_sparse_mla_fwd. */
+DSA_API dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
+                         const float* q_scale, const float* w, const uint8_t* k_idx,
+                         const float* k_scale, const uint16_t* q, const uint16_t* kv,
+                         int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream);
+
+/* Synchronises `stream`, reads the device status word and maps it: 0 -> DSA_OK,
+ * DSA_DEVICE_TIMEOUT -> DSA_ERR_TIMEOUT, DSA_DEVICE_BAD_INDEX -> DSA_ERR_BAD_INDEX.
+ * *raw (optional, host) receives the word. */
+DSA_API dsa_status_t dsa_read_device_status(const int32_t* dev_status, dsa_stream_t stream,
+                                    int32_t* raw);
+
+DSA_API const char* dsa_status_string(dsa_status_t status);
+DSA_API int32_t dsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

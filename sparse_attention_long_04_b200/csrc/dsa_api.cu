@@ -1,0 +1,572 @@
+// C ABI of the DSA hot path (see include/dsa.h): argument checks, planning and launches.
+// Nothing here allocates device memory; the only state is a per-device attribute cache.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "dsa.h"
+#include "indexer.cuh"
+#include "sparse_mla.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using namespace dsa;
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kSlabBudget = size_t(96) << 20;   // prefill score slab per row chunk
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int max_smem = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_info[kMaxDevices];
+bool g_info_ok[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+dsa_status_t device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_info_ok[dev]) {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return DSA_ERR_CUDA;
+    g_info[dev] = d;
+    g_info_ok[dev] = true;
+  }
+  *out = g_info[dev];
+  return DSA_OK;
+}
+
+dsa_status_t encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return DSA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return DSA_OK;
+}
+
+// Per (kernel, device): the kernel's dynamic shared-memory limit has been raised.
+struct SmemRaised {
+  const void* fn;
+  uint64_t devices;
+};
+SmemRaised g_raised[32];
+int g_n_raised = 0;
+
+template <typename Kernel>
+dsa_status_t prepare_kernel(Kernel k, int smem_bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  const uint64_t bit = uint64_t(1) << dev;
+  const void* fn = reinterpret_cast<const void*>(k);
+  std::lock_guard<std::mutex> lk(g_mu);
+  int slot = -1;
+  for (int i = 0; i < g_n_raised; ++i)
+    if (g_raised[i].fn == fn) slot = i;
+  if (slot >= 0 && (g_raised[slot].devices & bit)) return DSA_OK;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (slot < 0) {
+    if (g_n_raised == 32) return DSA_OK;   // not cached: raised again next time
+    slot = g_n_raised++;
+    g_raised[slot] = SmemRaised{fn, 0};
+  }
+  g_raised[slot].devices |= bit;
+  return DSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+dsa_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------ argument checks
+
+bool indexer_shape_ok(const dsa_dims_t& d, int mode) {
+  if (d.h_idx == 64 && d.d_idx == 128) return true;
+  return mode == DSA_PREFILL && d.h_idx == 4 && d.d_idx == 32;
+}
+
+bool mla_shape_ok(const dsa_dims_t& d) {
+  return (d.h == 128 && d.d_qk == 576 && d.d_v == 512) ||
+         (d.h == 16 && d.d_qk == 160 && d.d_v == 128);
+}
+
+dsa_status_t check_common(const dsa_dims_t* dims, const dsa_seqs_t* seqs) {
+  if (dims == nullptr || seqs == nullptr) return DSA_ERR_INVALID_ARG;
+  const dsa_seqs_t& s = *seqs;
+  if (s.mode != DSA_PREFILL && s.mode != DSA_DECODE) return DSA_ERR_INVALID_ARG;
+  if (s.batch <= 0 || s.total_rows < 0 || s.max_seqlen <= 0 || s.num_kv_rows <= 0)
+    return DSA_ERR_INVALID_ARG;
+  if (dims->topk < 64 || dims->topk > 2048 || dims->topk % 64 != 0)
+    return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (s.mode == DSA_PREFILL) {
+    if (s.cu_seqlens == nullptr || s.cu_seqlens_host == nullptr) return DSA_ERR_INVALID_ARG;
+    const int32_t* cu = s.cu_seqlens_host;
+    if (cu[0] != 0 || cu[s.batch] != s.total_rows) return DSA_ERR_INVALID_ARG;
+    for (int b = 0; b < s.batch; ++b) {
+      const int L = cu[b + 1] - cu[b];
+      if (L < 0 || L > s.max_seqlen) return DSA_ERR_INVALID_ARG;
+    }
+    if (s.total_rows > s.num_kv_rows) return DSA_ERR_INVALID_ARG;
+  } else {
+    if (s.seq_lens == nullptr || s.total_rows != s.batch) return DSA_ERR_INVALID_ARG;
+    if (dims->block_size != 64) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (s.block_table != nullptr) {
+      if (s.max_blocks < ceil_div(s.max_seqlen, 64)) return DSA_ERR_INVALID_ARG;
+    } else if (static_cast<int64_t>(s.batch) * s.max_seqlen > s.num_kv_rows) {
+      return DSA_ERR_INVALID_ARG;
+    }
+  }
+  return DSA_OK;
+}
+
+dsa_status_t check_rows(const dsa_seqs_t* s, int32_t row_begin, int32_t row_count) {
+  if (row_begin < 0 || row_count < 0 || row_begin + int64_t(row_count) > s->total_rows)
+    return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+// Largest key count (pos + 1) among rows [row_begin, row_begin + row_count).
+int64_t max_keys(const dsa_seqs_t* s, int32_t row_begin, int32_t row_count) {
+  if (s->mode == DSA_DECODE) return s->max_seqlen;
+  const int32_t* cu = s->cu_seqlens_host;
+  int64_t m = 0;
+  for (int b = 0; b < s->batch; ++b) {
+    const int64_t lo = std::max<int64_t>(cu[b], row_begin);
+    const int64_t hi = std::min<int64_t>(cu[b + 1], int64_t(row_begin) + row_count);
+    if (lo < hi) m = std::max<int64_t>(m, hi - cu[b]);
+  }
+  return m;
+}
+
+// ------------------------------------------------------------------------ TMA maps
+
+dsa_status_t make_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
+                      uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (encoder(&enc) != DSA_OK) return DSA_ERR_CUDA;
+  std::memset(map, 0, sizeof(*map));
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {row_bytes, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                   strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------ stage 1
+
+template <int H_I, int D_I, int QPG>
+dsa_status_t run_indexer_kernel(const CUtensorMap& kmap, const CUtensorMap& qmap,
+                                const IndexerParams& prm, dim3 grid, cudaStream_t st) {
+  using C = IndexerCfg<H_I, D_I, QPG>;
+  int smem = C::SMEM_BYTES;
+  if (C::TMEM_COLS == 512) smem = std::max(smem, 120 * 1024);   // one CTA per SM
+  auto k = dsa_indexer_kernel<H_I, D_I, QPG>;
+  if (prepare_kernel(k, smem) != DSA_OK) return DSA_ERR_CUDA;
+  k<<<grid, C::THREADS, smem, st>>>(kmap, qmap, prm);
+  return launch_status();
+}
+
+template <int H_I, int D_I, int QPG>
+dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
+                          const float* q_scale, const float* w, const uint8_t* k_idx,
+                          const float* k_scale, int32_t row_begin, int32_t row_count,
+                          float* scores, int64_t ld, int32_t* status, cudaStream_t st) {
+  using C = IndexerCfg<H_I, D_I, QPG>;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  CUtensorMap kmap, qmap;
+  if (make_map(&kmap, k_idx, s.num_kv_rows, D_I, 64) != DSA_OK) return DSA_ERR_CUDA;
+  if (make_map(&qmap, q_idx, uint64_t(s.total_rows) * H_I, D_I, C::N) != DSA_OK)
+    return DSA_ERR_CUDA;
+  IndexerParams prm{};
+  prm.q_scale = q_scale;
+  prm.w = w;
+  prm.k_scale = k_scale;
+  prm.scores = scores;
+  prm.ld = ld;
+  prm.status = status;
+  prm.seq_lens = s.seq_lens;
+  prm.block_table = s.block_table;
+  prm.max_blocks = s.max_blocks;
+  prm.kv_stride = s.max_seqlen;
+  prm.max_seqlen = s.max_seqlen;
+  prm.num_kv_rows = s.num_kv_rows;
+  const int ctas_per_sm = C::TMEM_COLS == 512 ? 1 : 2;
+  const int64_t target = int64_t(info.sm_count) * ctas_per_sm * 4;
+  if (s.mode == DSA_DECODE) {
+    const int64_t tiles = ceil_div(s.max_seqlen, 128);
+    int64_t splits = std::min<int64_t>(tiles, std::max<int64_t>(1, ceil_div(target, row_count)));
+    const int64_t tps = ceil_div(tiles, splits);
+    splits = ceil_div(tiles, tps);
+    prm.decode = 1;
+    prm.row0 = row_begin;
+    prm.nrows = row_count;
+    prm.out_row0 = 0;
+    prm.tiles_per_split = static_cast<int32_t>(tps);
+    return run_indexer_kernel<H_I, D_I, QPG>(kmap, qmap, prm, dim3(row_count, splits), st);
+  }
+  // prefill: one launch per sequence segment of the row range
+  const int32_t* cu = s.cu_seqlens_host;
+  for (int b = 0; b < s.batch; ++b) {
+    const int64_t lo = std::max<int64_t>(cu[b], row_begin);
+    const int64_t hi = std::min<int64_t>(cu[b + 1], int64_t(row_begin) + row_count);
+    if (lo >= hi) continue;
+    const int64_t nrows = hi - lo;
+    const int64_t groups = ceil_div(nrows, QPG);
+    const int64_t tiles = ceil_div(hi - cu[b], 128);
+    int64_t splits = std::min<int64_t>(tiles, std::max<int64_t>(1, ceil_div(target, groups)));
+    const int64_t tps = std::max<int64_t>(ceil_div(tiles, splits), std::min<int64_t>(tiles, 8));
+    splits = ceil_div(tiles, tps);
+    prm.decode = 0;
+    prm.row0 = static_cast<int32_t>(lo);
+    prm.nrows = static_cast<int32_t>(nrows);
+    prm.pos0 = static_cast<int32_t>(lo - cu[b]);
+    prm.key0 = cu[b];
+    prm.out_row0 = static_cast<int32_t>(lo - row_begin);
+    prm.tiles_per_split = static_cast<int32_t>(tps);
+    dsa_status_t e = run_indexer_kernel<H_I, D_I, QPG>(kmap, qmap, prm, dim3(groups, splits), st);
+    if (e != DSA_OK) return e;
+  }
+  return DSA_OK;
+}
+
+dsa_status_t indexer_dispatch(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
+                              const float* q_scale, const float* w, const uint8_t* k_idx,
+                              const float* k_scale, int32_t row_begin, int32_t row_count,
+                              float* scores, int64_t ld, int32_t* status, cudaStream_t st) {
+  if (row_count == 0) return DSA_OK;
+  if (d.h_idx == 64 && d.d_idx == 128) {
+    if (s.mode == DSA_DECODE)
+      return indexer_impl<64, 128, 1>(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin,
+                                      row_count, scores, ld, status, st);
+    return indexer_impl<64, 128, 4>(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin,
+                                    row_count, scores, ld, status, st);
+  }
+  return indexer_impl<4, 32, 64>(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
+                                 scores, ld, status, st);
+}
+
+// ------------------------------------------------------------------------ stage 2
+
+dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* scores, int64_t ld,
+                         int32_t row_begin, int32_t row_count, int32_t* idx, int32_t* status,
+                         cudaStream_t st) {
+  if (row_count == 0) return DSA_OK;
+  TopkParams prm{};
+  prm.scores = scores;
+  prm.ld = ld;
+  prm.idx = idx;
+  prm.topk = d.topk;
+  prm.decode = s.mode == DSA_DECODE;
+  prm.row_begin = row_begin;
+  prm.batch = s.batch;
+  prm.cu_seqlens = s.cu_seqlens;
+  prm.seq_lens = s.seq_lens;
+  prm.max_seqlen = s.max_seqlen;
+  prm.status = status;
+  dsa_topk_kernel<<<row_count, kTopkThreads, 0, st>>>(prm);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------------ stage 3
+
+int mla_splits(const dsa_dims_t& d, const dsa_seqs_t& s, int32_t row_count, int sm_count) {
+  if (s.mode != DSA_DECODE || row_count <= 0) return 1;
+  const int clusters = std::max(1, sm_count / 2);
+  int splits = std::max(1, clusters / row_count);
+  splits = std::min(splits, std::max(1, d.topk / 64 / 4));   // >= 4 tiles per split
+  return std::min(splits, 16);
+}
+
+size_t mla_ws_bytes(const dsa_dims_t& d, int splits, int32_t row_count) {
+  if (splits <= 1) return 0;
+  return size_t(splits) * row_count * d.h * (d.d_v + 1) * sizeof(float) + 256;
+}
+
+template <int D_QK, int D_V>
+dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
+                      const uint16_t* kv, const int32_t* idx, int32_t row_begin, int32_t row_count,
+                      uint16_t* out, float* lse, void* ws, size_t ws_bytes, int32_t* status,
+                      cudaStream_t st, int splits) {
+  using C = MlaCfg<D_QK, D_V>;
+  MlaParams prm{};
+  prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  prm.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  prm.idx = idx;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.row_begin = row_begin;
+  prm.row_count = row_count;
+  prm.topk = d.topk;
+  prm.h = d.h;
+  prm.splits = splits;
+  prm.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  prm.decode = s.mode == DSA_DECODE;
+  prm.batch = s.batch;
+  prm.cu_seqlens = s.cu_seqlens;
+  prm.seq_lens = s.seq_lens;
+  prm.block_table = s.block_table;
+  prm.max_blocks = s.max_blocks;
+  prm.kv_stride = s.max_seqlen;
+  prm.max_seqlen = s.max_seqlen;
+  prm.block_size = d.block_size > 0 ? d.block_size : 64;
+  prm.num_kv_rows = s.num_kv_rows;
+  prm.status = status;
+  if (splits > 1) {
+    if (ws == nullptr || ws_bytes < mla_ws_bytes(d, splits, row_count))
+      return DSA_ERR_WORKSPACE_TOO_SMALL;
+    prm.part_o = static_cast<float*>(ws);
+    prm.part_lse = prm.part_o + size_t(splits) * row_count * d.h * D_V;
+  }
+  auto k = dsa_sparse_mla_kernel<D_QK, D_V>;
+  if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
+  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(prm);
+  if (launch_status() != DSA_OK) return DSA_ERR_CUDA;
+  if (splits > 1) {
+    dsa_mla_combine_kernel<D_V><<<dim3(row_count, d.h), 128, 0, st>>>(prm);
+    return launch_status();
+  }
+  return DSA_OK;
+}
+
+dsa_status_t mla_dispatch(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
+                          const uint16_t* kv, const int32_t* idx, int32_t row_begin,
+                          int32_t row_count, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                          int32_t* status, cudaStream_t st, int splits) {
+  if (row_count == 0) return DSA_OK;
+  if (d.d_qk == 576)
+    return mla_impl<576, 512>(d, s, q, kv, idx, row_begin, row_count, out, lse, ws, ws_bytes,
+                              status, st, splits);
+  return mla_impl<160, 128>(d, s, q, kv, idx, row_begin, row_count, out, lse, ws, ws_bytes,
+                            status, st, splits);
+}
+
+// ------------------------------------------------------------------------ dsa_forward plan
+
+struct ForwardPlan {
+  int64_t slab_floats = 0;   // score slab
+  int64_t idx_ints = 0;      // chunk indices when idx_out is null
+  int mla_splits = 1;
+  size_t mla_bytes = 0;
+  size_t total = 0;
+};
+
+int64_t round4(int64_t x) { return (x + 3) / 4 * 4; }
+
+int64_t chunk_rows_for(int64_t L) {
+  const int64_t ld = round4(L);
+  return std::max<int64_t>(1, std::min<int64_t>(L, int64_t(kSlabBudget / (ld * 4))));
+}
+
+ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count) {
+  ForwardPlan p;
+  if (s.mode == DSA_DECODE) {
+    p.slab_floats = int64_t(s.batch) * round4(s.max_seqlen);
+    p.idx_ints = int64_t(s.batch) * d.topk;
+    p.mla_splits = mla_splits(d, s, s.batch, sm_count);
+    p.mla_bytes = mla_ws_bytes(d, p.mla_splits, s.batch);
+  } else {
+    const int32_t* cu = s.cu_seqlens_host;
+    int64_t max_rows = 0;
+    for (int b = 0; b < s.batch; ++b) {
+      const int64_t L = cu[b + 1] - cu[b];
+      if (L <= 0) continue;
+      const int64_t rows = chunk_rows_for(L);
+      p.slab_floats = std::max(p.slab_floats, rows * round4(L));
+      max_rows = std::max(max_rows, rows);
+    }
+    p.idx_ints = max_rows * d.topk;
+  }
+  auto align = [](size_t x) { return (x + 255) / 256 * 256; };
+  p.total = align(p.slab_floats * 4) + align(p.idx_ints * 4) + align(p.mla_bytes);
+  return p;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+
+extern "C" {
+
+int32_t dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+const char* dsa_status_string(dsa_status_t st) {
+  switch (st) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DSA_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case DSA_ERR_BAD_INDEX: return "index outside the caches";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                const uint8_t* q_idx, const float* q_scale, const float* w,
+                                const uint8_t* k_idx, const float* k_scale, int32_t row_begin,
+                                int32_t row_count, float* scores, int64_t ld_scores,
+                                int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (!indexer_shape_ok(*dims, seqs->mode)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(scores) || ld_scores % 4 != 0)
+    return DSA_ERR_MISALIGNED;
+  if (ld_scores < max_keys(seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
+  return indexer_dispatch(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
+                          scores, ld_scores, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
+                      int64_t ld_scores, int32_t row_begin, int32_t row_count, int32_t* idx,
+                      int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx) || ld_scores % 4 != 0) return DSA_ERR_MISALIGNED;
+  if (ld_scores < max_keys(seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
+  return topk_launch(*dims, *seqs, scores, ld_scores, row_begin, row_count, idx, dev_status,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_sparse_mla_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                     int32_t row_count) {
+  if (check_common(dims, seqs) != DSA_OK) return 0;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return 0;
+  return mla_ws_bytes(*dims, mla_splits(*dims, *seqs, row_count, info.sm_count), row_count);
+}
+
+dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                int32_t row_begin, int32_t row_count, uint16_t* out, float* lse,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q || !kv || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(workspace))
+    return DSA_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  const int splits = mla_splits(*dims, *seqs, row_count, info.sm_count);
+  return mla_dispatch(*dims, *seqs, q, kv, idx, row_begin, row_count, out, lse, workspace,
+                      workspace_bytes, dev_status, reinterpret_cast<cudaStream_t>(stream), splits);
+}
+
+size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs) {
+  if (check_common(dims, seqs) != DSA_OK) return 0;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return 0;
+  return plan_forward(*dims, *seqs, info.sm_count).total;
+}
+
+dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
+                         const float* q_scale, const float* w, const uint8_t* k_idx,
+                         const float* k_scale, const uint16_t* q, const uint16_t* kv,
+                         int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  const dsa_dims_t& d = *dims;
+  const dsa_seqs_t& s = *seqs;
+  if (!indexer_shape_ok(d, s.mode) || !mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !q || !kv || !out || !lse)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(kv) ||
+      !aligned16(out) || !aligned16(lse) || !aligned16(idx_out) || !aligned16(workspace))
+    return DSA_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  const ForwardPlan plan = plan_forward(d, s, info.sm_count);
+  if (workspace == nullptr || workspace_bytes < plan.total) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto align = [](size_t x) { return (x + 255) / 256 * 256; };
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  float* slab = reinterpret_cast<float*>(wsb);
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(wsb + align(plan.slab_floats * 4));
+  void* mla_ws = wsb + align(plan.slab_floats * 4) + align(plan.idx_ints * 4);
+
+  if (s.mode == DSA_DECODE) {
+    const int64_t ld = round4(s.max_seqlen);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if ((e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, 0, s.batch, slab, ld,
+                              dev_status, st)) != DSA_OK)
+      return e;
+    if ((e = topk_launch(d, s, slab, ld, 0, s.batch, idx, dev_status, st)) != DSA_OK) return e;
+    return mla_dispatch(d, s, q, kv, idx, 0, s.batch, out, lse, mla_ws, plan.mla_bytes,
+                        dev_status, st, plan.mla_splits);
+  }
+  const int32_t* cu = s.cu_seqlens_host;
+  for (int b = 0; b < s.batch; ++b) {
+    const int64_t L = cu[b + 1] - cu[b];
+    if (L <= 0) continue;
+    const int64_t ld = round4(L);
+    const int64_t rows = chunk_rows_for(L);
+    for (int64_t r0 = 0; r0 < L; r0 += rows) {
+      const int32_t row_begin = static_cast<int32_t>(cu[b] + r0);
+      const int32_t row_count = static_cast<int32_t>(std::min(rows, L - r0));
+      int32_t* idx = idx_out ? idx_out + int64_t(row_begin) * d.topk : idx_ws;
+      if ((e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
+                                slab, ld, dev_status, st)) != DSA_OK)
+        return e;
+      if ((e = topk_launch(d, s, slab, ld, row_begin, row_count, idx, dev_status, st)) != DSA_OK)
+        return e;
+      if ((e = mla_dispatch(d, s, q, kv, idx, row_begin, row_count, out, lse, nullptr, 0,
+                            dev_status, st, 1)) != DSA_OK)
+        return e;
+    }
+  }
+  return DSA_OK;
+}
+
+dsa_status_t dsa_read_device_status(const int32_t* dev_status, dsa_stream_t stream,
+                                    int32_t* raw) {
+  if (dev_status == nullptr) return DSA_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, dev_status, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (raw) *raw = v;
+  if (v & DSA_DEVICE_TIMEOUT) return DSA_ERR_TIMEOUT;
+  if (v & DSA_DEVICE_BAD_INDEX) return DSA_ERR_BAD_INDEX;
+  return DSA_OK;
+}
+
+}  // extern "C"

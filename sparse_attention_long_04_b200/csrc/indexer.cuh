@@ -1,0 +1,305 @@
+// Lightning indexer (stage 1): FP8 e4m3 scores of query rows against their prior keys.
+//
+//   S[t,s] = k_scale[s] * sum_j c[t,j] * ReLU( q[t,j,:] . k[s,:] ),  c[t,j] = w[t,j] * q_scale[t,j]
+//
+// ("FP8 index -> top-k selection -> sparse core attention", "DeepSeek V3.2-Exp Cuts Long-Context
+// Costs with DeepSeek Sparse Attention (DSA)", pipeline summary; "Lightning Indexer", maplevalley
+// page, section 1.)
+//
+// One CTA (grid x = query group, y = key split) takes one query group (QPG rows of the same
+// sequence) and a contiguous range of 128-key tiles.  The contraction is swapped so that keys are the MMA's M dimension:
+//   D[key, (row, head)] = K_tile[128 x D_I] * Q_group[N x D_I]^T,   N = QPG * H_I
+// with e4m3 operands in 128-byte (or 32-byte for D_I = 32) swizzled shared memory and an fp32
+// accumulator in Tensor Memory (TMEM lane = key).  Each epilogue thread then owns one key and
+// reduces its row's heads with no cross-thread traffic: 2 ALU ops (max, fma) per head.
+//
+// Roles: warp 0 issues TMA (Q once, then two 64-row key boxes per tile), warp 1 issues the
+// tcgen05.mma, warp 2 owns the TMEM allocation, warp 3 computes c[t,j], warps 4.. run the
+// epilogue.  Key stages are a ring of STAGES buffers; accumulators are double-buffered in TMEM
+// so the epilogue of tile i overlaps the MMA of tile i+1 and the loads of later tiles.
+#pragma once
+#include "sm100.cuh"
+
+namespace dsa {
+
+struct IndexerParams {
+  const float* q_scale;   // [T, H_I]
+  const float* w;         // [T, H_I]
+  const float* k_scale;   // [num_kv_rows]
+  float* scores;          // row `out_row0` of the output slab
+  int64_t ld;
+  int32_t* status;
+  int32_t decode;         // 1: one query row per sequence (decode), 0: prefill segment
+  // prefill segment: rows [row0, row0 + nrows) of one sequence; row0 sits at position pos0;
+  // key s of the sequence is packed row key0 + s.
+  // decode: rows [row0, row0 + nrows) are sequences row0.. (one row each)
+  int32_t row0, nrows, pos0, key0;
+  int32_t out_row0;       // slab row of `row0`
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t kv_stride;      // decode without block table: sequence b starts at row b * kv_stride
+  int32_t max_seqlen;     // decode: a seq_lens entry above this is clamped and reported
+  int64_t num_kv_rows;
+  int32_t tiles_per_split;
+};
+
+template <int H_I, int D_I, int QPG>
+struct IndexerCfg {
+  static constexpr int N = H_I * QPG;                 // MMA N: (row, head) columns
+  static constexpr int STAGES = QPG == 1 ? 6 : 8;
+  static constexpr int EPI_WARPS = QPG == 1 ? 4 : 8;
+  static constexpr int THREADS = (4 + EPI_WARPS) * 32;
+  static constexpr int TILE_BYTES = 128 * D_I;        // 128 keys
+  static constexpr int Q_BYTES = N * D_I;
+  static constexpr int KSTEPS = D_I / 32;             // one e4m3 MMA consumes K = 32
+  static constexpr uint32_t LAYOUT = D_I == 128 ? kSwizzle128B : kSwizzle32B;
+  static constexpr uint32_t SBO = 8 * D_I;            // next 8-row group
+  static constexpr int TMEM_COLS = 2 * N;             // double-buffered accumulator
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * TILE_BYTES + N * 4 + 256;
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
+  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+  static_assert(Q_BYTES % 1024 == 0 && TILE_BYTES % 1024 == 0, "1024-byte aligned tiles");
+};
+
+template <int H_I, int D_I, int QPG>
+__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
+    dsa_indexer_kernel(const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap qmap, const IndexerParams p) {
+  using C = IndexerCfg<H_I, D_I, QPG>;
+  constexpr int N = C::N;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + C::Q_BYTES;
+  float* sC = reinterpret_cast<float*>(sK + C::STAGES * C::TILE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + N);
+  uint64_t* full = bars;                      // [STAGES] key tile landed
+  uint64_t* empty = bars + C::STAGES;         // [STAGES] key tile consumed by the MMA
+  uint64_t* tfull = empty + C::STAGES;        // [2] accumulator ready
+  uint64_t* tempty = tfull + 2;               // [2] accumulator drained by the epilogue
+  uint64_t* qbar = tempty + 2;                // Q group landed
+  uint64_t* done = qbar + 1;                  // every MMA of this CTA completed
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---- geometry of this CTA's group (uniform across the CTA)
+  int n_keys, grow0, rows_in_group, pos_first;
+  int64_t seq_base = 0;   // decode contiguous: first physical row of the sequence
+  int b = 0;
+  if (p.decode) {
+    b = p.row0 + blockIdx.x;
+    n_keys = p.seq_lens[b];
+    if (n_keys > p.max_seqlen) {
+      if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+      n_keys = p.max_seqlen;
+    }
+    grow0 = b;
+    rows_in_group = 1;
+    pos_first = n_keys - 1;
+    seq_base = static_cast<int64_t>(b) * p.kv_stride;
+    if (n_keys <= 0) return;
+  } else {
+    grow0 = p.row0 + blockIdx.x * QPG;
+    rows_in_group = min(QPG, p.row0 + p.nrows - grow0);
+    pos_first = p.pos0 + (grow0 - p.row0);
+    n_keys = pos_first + rows_in_group;       // keys 0 .. last row's position
+  }
+  const int n_tiles_all = (n_keys + 127) / 128;
+  const int t_begin = blockIdx.y * p.tiles_per_split;
+  const int t_end = min(t_begin + p.tiles_per_split, n_tiles_all);
+  if (t_begin >= t_end) return;
+  const int n_tiles = t_end - t_begin;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), C::EPI_WARPS);
+    }
+    mbar_init(smem_u32(qbar), 1);
+    mbar_init(smem_u32(done), 1);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
+  if (warp == 3) {
+    for (int i = lane; i < N; i += 32) {
+      int r = i / H_I, j = i % H_I;
+      float c = 0.f;
+      if (r < rows_in_group) {
+        int64_t row = grow0 + r;
+        c = p.w[row * H_I + j] * p.q_scale[row * H_I + j];
+      }
+      sC[i] = c;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&qmap);
+      mbar_arrive_expect_tx(smem_u32(qbar), C::Q_BYTES);
+      tma_load_2d(smem_u32(sQ), &qmap, smem_u32(qbar), 0, grow0 * H_I);
+      int issued = 0;
+      const int n_blocks = (n_keys + 63) / 64;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::STAGES;
+        if (it >= C::STAGES &&
+            !mbar_wait(smem_u32(&empty[s]), ((it / C::STAGES) - 1) & 1, &abort_s)) {
+          abort_s = 1;
+          if (p.status) atomicOr(p.status, kStatusTimeout);
+          break;
+        }
+        const int tile = t_begin + it;
+        int64_t y[2];
+        bool ok[2];
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int blk = tile * 2 + hlf;
+          ok[hlf] = blk < n_blocks;
+          if (!p.decode) {
+            y[hlf] = static_cast<int64_t>(p.key0) + blk * 64;
+          } else if (p.block_table != nullptr) {
+            int64_t id = ok[hlf] ? p.block_table[static_cast<int64_t>(b) * p.max_blocks + blk] : 0;
+            if (ok[hlf] && (id < 0 || (id + 1) * 64 > p.num_kv_rows)) {
+              if (p.status) atomicOr(p.status, kStatusBadIndex);
+              ok[hlf] = false;
+            }
+            y[hlf] = id * 64;
+          } else {
+            y[hlf] = seq_base + blk * 64;
+          }
+        }
+        const uint32_t bytes = (ok[0] ? 64 * D_I : 0) + (ok[1] ? 64 * D_I : 0);
+        mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
+        for (int hlf = 0; hlf < 2; ++hlf)
+          if (ok[hlf])
+            tma_load_2d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
+                        smem_u32(&full[s]), 0, static_cast<int32_t>(y[hlf]));
+        ++issued;
+      }
+      // drain: never leave a copy in flight into shared memory of an exiting CTA
+      for (int it = max(0, issued - C::STAGES); it < issued; ++it)
+        mbar_wait(smem_u32(&full[it % C::STAGES]), (it / C::STAGES) & 1, nullptr);
+      mbar_wait(smem_u32(qbar), 0, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f32acc(0 /* e4m3 */, 128, N, 0, 0);
+      bool ok = mbar_wait(smem_u32(qbar), 0, &abort_s);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int s = it % C::STAGES;
+        const int a = it & 1;
+        ok = mbar_wait(smem_u32(&full[s]), (it / C::STAGES) & 1, &abort_s);
+        if (ok && it >= 2) ok = mbar_wait(smem_u32(&tempty[a]), ((it >> 1) - 1) & 1, &abort_s);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(sK + s * C::TILE_BYTES);
+        const uint32_t qaddr = smem_u32(sQ);
+#pragma unroll
+        for (int k = 0; k < C::KSTEPS; ++k)
+          umma_e4m3(tmem + a * N, sdesc(kaddr + k * 32, 16, C::SBO, C::LAYOUT),
+                    sdesc(qaddr + k * 32, 16, C::SBO, C::LAYOUT), idesc, k > 0);
+        umma_commit(smem_u32(&empty[s]));
+        umma_commit(smem_u32(&tfull[a]));
+      }
+      if (!ok) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+      umma_commit(smem_u32(done));
+      mbar_wait(smem_u32(done), 0, nullptr);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ epilogue
+    constexpr int PARTS = C::EPI_WARPS / 4;
+    constexpr int COLS = N / PARTS;          // columns this warp reduces
+    const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
+    const int part = (warp - 4) / 4;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    for (int it = 0; it < n_tiles; ++it) {
+      const int a = it & 1;
+      if (!mbar_wait(smem_u32(&tfull[a]), (it >> 1) & 1, &abort_s)) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int key = (t_begin + it) * 128 + quad * 32 + lane;
+      float ks = 0.f;
+      if (key < n_keys) {
+        int64_t phys;
+        if (!p.decode) {
+          phys = static_cast<int64_t>(p.key0) + key;
+        } else if (p.block_table != nullptr) {
+          int64_t id = p.block_table[static_cast<int64_t>(b) * p.max_blocks + key / 64];
+          phys = (id < 0 || (id + 1) * 64 > p.num_kv_rows) ? -1 : id * 64 + key % 64;
+        } else {
+          phys = seq_base + key;
+        }
+        ks = phys >= 0 && phys < p.num_kv_rows ? __ldg(p.k_scale + phys) : 0.f;
+      }
+      float acc = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < COLS; c0 += 32) {
+        const int col = part * COLS + c0;
+        uint32_t r[32];
+        tmem_ld32(lane_addr + a * N + col, r);
+        tmem_wait_ld();
+        const float4* cc = reinterpret_cast<const float4*>(sC + col);
+        if constexpr (H_I >= 32) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 c4 = cc[j / 4];
+            acc = fmaf(c4.x, fmaxf(__uint_as_float(r[j + 0]), 0.f), acc);
+            acc = fmaf(c4.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), acc);
+            acc = fmaf(c4.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), acc);
+            acc = fmaf(c4.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), acc);
+          }
+          if ((col + 32) % H_I == 0) {       // a query row's heads are complete
+            const int rr = col / H_I;
+            if (rr < rows_in_group && key <= pos_first + rr)
+              p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] =
+                  ks * acc;
+            acc = 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32 / H_I; ++q) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < H_I; ++j)
+              s = fmaf(sC[col + q * H_I + j], fmaxf(__uint_as_float(r[q * H_I + j]), 0.f), s);
+            const int rr = col / H_I + q;
+            if (rr < rows_in_group && key <= pos_first + rr)
+              p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] =
+                  ks * s;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[a]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa

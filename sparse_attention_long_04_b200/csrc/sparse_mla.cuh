@@ -1,0 +1,509 @@
+// Sparse MLA attention in MQA mode (stage 3) and the split-KV combine.
+//
+// For query row t, head h, over the selected logical keys I_t (idx >= 0):
+//   l_s = sigma * q[t,h,:] . kv[s,:]            (all D_QK = latent + RoPE dims)
+//   O[t,h,:] = sum_s softmax(l)_s * kv[s, 0:D_V] (values = the first D_V latent dims)
+//   LSE[t,h] = log sum_s exp(l_s)
+// Every selected latent row is shared by all query heads ("MLA in MQA mode ... each latent KV
+// entry is shared across query heads", "DeepSeek V3.2-Exp Cuts Long-Context Costs with
+// DeepSeek Sparse Attention (DSA)", "Instantiation").
+//
+// Design (sm_100a).  O for 128 heads x 512 values in fp32 is 256 KB = all of one SM's TMEM,
+// and Q (128 x 576 bf16 = 144 KB) plus gathered tiles do not fit one CTA's shared memory, so
+// each query row runs on a 2-CTA cluster:
+//   CTA r holds Q dims D_r (r = 0: [0, D_V/2); r = 1: [D_V/2, D_QK)) and gathers the same dims
+//   of each selected latent row.  Per 64-key tile it computes the partial logits
+//   S_r = Q[:, D_r] K[:, D_r]^T (tcgen05 bf16, M = 128 heads, N = 64 keys) into TMEM, the two
+//   CTAs swap S_r through distributed shared memory, and both form S = S_0 + S_1 in the same
+//   order, so both run an identical online softmax.  CTA r then accumulates its half of the
+//   values, O_r += P V[:, r * D_V/2 : (r+1) * D_V/2] (M = 128, N = D_V/2, K = 64 keys; V is
+//   read MN-major straight out of the gathered tile).  No tensor work is duplicated.
+//   Rescaling of O is lazy: it happens only when a tile's max exceeds the running reference
+//   by more than 2^8, so P stays <= 256.
+// Warp roles per CTA: warp 0 issues QK, warp 2 issues PV, warp 1 owns TMEM, warps 4-7 run the
+// softmax (thread = head = TMEM lane) and the epilogue, warps 8-11 resolve indices and gather
+// rows with 16-byte cp.async into 128-byte-swizzled tiles (2 stages).
+// Grid: x = 2 * row (the cluster pair), y = split-KV slice.
+#pragma once
+#include "sm100.cuh"
+
+namespace dsa {
+
+struct MlaParams {
+  const __nv_bfloat16* q;      // [T, H, D_QK]
+  const __nv_bfloat16* kv;     // [R, D_QK]
+  const int32_t* idx;          // [row_count, topk], relative to row_begin
+  __nv_bfloat16* out;          // [T, H, D_V]
+  float* lse;                  // [T, H]
+  float* part_o;               // split-KV partials [splits, row_count, H, D_V] or null
+  float* part_lse;             // [splits, row_count, H]
+  int32_t row_begin, row_count, topk, h, splits;
+  float scale_log2;            // sigma * log2(e)
+  int32_t decode;
+  int32_t batch;
+  const int32_t* cu_seqlens;
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t kv_stride;
+  int32_t max_seqlen;
+  int32_t block_size;
+  int64_t num_kv_rows;
+  int32_t* status;
+};
+
+template <int D_QK, int D_V>
+struct MlaCfg {
+  static constexpr int KB_ALL = (D_QK + 63) / 64;     // 64-element k-blocks of a latent row
+  static constexpr int V_HALF = D_V / 2;
+  static constexpr int VKB = V_HALF / 64;             // value k-blocks per CTA
+  static constexpr int KBC = KB_ALL - VKB;            // k-blocks held by rank 1 (>= rank 0)
+  static constexpr int BN = 64;                       // keys per tile
+  static constexpr int STAGES = 2;
+  static constexpr int MAX_TOPK = 2048;
+  static constexpr int THREADS = 384;
+  static constexpr int Q_BYTES = KBC * 128 * 128;
+  static constexpr int KV_STAGE_BYTES = KBC * BN * 128;
+  static constexpr int P_BYTES = 128 * 128;
+  static constexpr int X_BYTES = 128 * BN * 4;        // received partial logits
+  static constexpr int S_COL0 = V_HALF;               // TMEM: O at [0, V_HALF), S at S_COL0
+  static constexpr int TMEM_COLS = (V_HALF + 2 * BN) <= 256 ? 256 : 512;
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_STAGE_BYTES + P_BYTES + X_BYTES +
+                                    MAX_TOPK * 4 + 64 * 4 + 256;
+  static_assert(KBC >= VKB, "rank 1 holds at least as many k-blocks as rank 0");
+  static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(SMEM_BYTES > 114 * 1024, "one CTA per SM (TMEM and cluster peers)");
+};
+
+template <int D_QK, int D_V>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+    dsa_sparse_mla_kernel(const MlaParams p) {
+  using C = MlaCfg<D_QK, D_V>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + C::Q_BYTES;
+  uint8_t* sP = sKV + C::STAGES * C::KV_STAGE_BYTES;
+  float* sX = reinterpret_cast<float*>(sP + C::P_BYTES);
+  int32_t* sPhys = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sX) + C::X_BYTES);
+  int32_t* sTiles = sPhys + C::MAX_TOPK;                 // [32] active tile ids, [32] count
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sTiles + 64);
+  uint64_t* kv_full = bars;          // [2] producers (128 arrivals)
+  uint64_t* kv_empty = bars + 2;     // [2] QK commit + PV commit
+  uint64_t* s_full = bars + 4;       // [2] QK commit
+  uint64_t* s_empty = bars + 6;      // [2] 4 softmax warps
+  uint64_t* p_full = bars + 8;       // 128 softmax threads
+  uint64_t* pv_done = bars + 9;      // PV commit
+  uint64_t* x_full = bars + 10;      // 128 remote arrivals: peer's partial logits are here
+  uint64_t* peer_free = bars + 11;   // 128 remote arrivals: peer consumed what we sent
+  uint64_t* qk_done = bars + 12;
+  uint64_t* pv_fin = bars + 13;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  __shared__ int n_act_s;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int split = blockIdx.y;
+  const int r = blockIdx.x >> 1;
+  const int row = p.row_begin + r;
+  const int kb_begin = rank == 0 ? 0 : C::VKB;
+  const int kb_count = rank == 0 ? C::VKB : C::KBC;
+
+  // ---- row geometry
+  int b, n_keys;
+  int64_t key_base = 0;
+  if (p.decode) {
+    b = row;
+    n_keys = min(p.seq_lens[b], p.max_seqlen);   // an entry above max_seqlen is a caller error
+    key_base = static_cast<int64_t>(b) * p.kv_stride;
+  } else {
+    int lo = 0, hi = p.batch;
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (p.cu_seqlens[mid] <= row) lo = mid; else hi = mid;
+    }
+    b = lo;
+    n_keys = row - p.cu_seqlens[lo] + 1;
+    key_base = p.cu_seqlens[lo];
+  }
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&kv_full[i]), 128);
+      mbar_init(smem_u32(&kv_empty[i]), 2);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_empty[i]), 4);
+    }
+    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(pv_done), 1);
+    mbar_init(smem_u32(x_full), 128);
+    mbar_init(smem_u32(peer_free), 128);
+    mbar_init(smem_u32(qk_done), 1);
+    mbar_init(smem_u32(pv_fin), 1);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
+
+  if (warp >= 8) {
+    // ---- resolve logical indices to physical rows; load this CTA's Q dims
+    const int tp = threadIdx.x - 256;
+    const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
+    for (int j = tp; j < p.topk; j += 128) {
+      const int v = irow[j];
+      int64_t phys = -1;
+      if (v >= 0) {
+        if (v < n_keys) {
+          if (!p.decode) {
+            phys = key_base + v;
+          } else if (p.block_table != nullptr) {
+            const int64_t id = p.block_table[static_cast<int64_t>(b) * p.max_blocks +
+                                             v / p.block_size];
+            phys = id * p.block_size + v % p.block_size;
+            if (id < 0) phys = -1;
+          } else {
+            phys = key_base + v;
+          }
+          if (phys >= p.num_kv_rows) phys = -1;
+        }
+        if (phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+      }
+      sPhys[j] = static_cast<int32_t>(phys);
+    }
+    const __nv_bfloat16* qrow = p.q + static_cast<int64_t>(row) * p.h * D_QK;
+    for (int c = tp; c < 128 * kb_count * 8; c += 128) {
+      const int hrow = c / (kb_count * 8);
+      const int rem = c % (kb_count * 8);
+      const int kbl = rem / 8, ch = rem % 8;
+      const int d = (kb_begin + kbl) * 64 + ch * 8;
+      const bool ok = hrow < p.h && d < D_QK;
+      cp_async_16(smem_u32(sQ + kbl * 16384 + sw128_offset(hrow, ch)),
+                  ok ? static_cast<const void*>(qrow + static_cast<int64_t>(hrow) * D_QK + d)
+                     : static_cast<const void*>(p.q),
+                  ok ? 16u : 0u);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // ---- active tiles (at least one valid key), identical in both CTAs
+  if (warp == 0) {
+    const int n_tiles_all = p.topk / C::BN;
+    int cnt = 0;
+    for (int t = 0; t < n_tiles_all; ++t) {
+      const int j = t * C::BN + lane * 2;
+      const bool any = __any_sync(0xffffffffu, sPhys[j] >= 0 || sPhys[j + 1] >= 0);
+      if (any) {
+        if (lane == 0) sTiles[cnt] = t;
+        ++cnt;
+      }
+    }
+    if (lane == 0) {
+      const int per = (cnt + p.splits - 1) / p.splits;
+      const int t0 = min(cnt, split * per);
+      const int t1 = min(cnt, t0 + per);
+      for (int i = t0; i < t1; ++i) sTiles[i - t0] = sTiles[i];
+      n_act_s = t1 - t0;
+    }
+  }
+  __syncthreads();
+  cluster_sync();   // peer barriers initialised before any remote arrive
+  const int n = n_act_s;
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ QK issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f32acc(1 /* bf16 */, 128, C::BN, 0, 0);
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        const int s = i & 1;
+        ok = mbar_wait(smem_u32(&kv_full[s]), (i >> 1) & 1, &abort_s);
+        if (ok && i >= 2) ok = mbar_wait(smem_u32(&s_empty[s]), ((i >> 1) - 1) & 1, &abort_s);
+        if (!ok) break;
+        tc_fence_after();
+        fence_proxy_async_smem();
+        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sKV + s * C::KV_STAGE_BYTES);
+        for (int kb = 0; kb < kb_count; ++kb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tmem + C::S_COL0 + s * C::BN,
+                      sdesc_sw128(qa + kb * 16384 + k * 32, 16, 1024),
+                      sdesc_sw128(ka + kb * (C::BN * 128) + k * 32, 16, 1024), idesc,
+                      (kb | k) != 0);
+        umma_commit(smem_u32(&s_full[s]));
+        umma_commit(smem_u32(&kv_empty[s]));
+      }
+      if (!ok) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+      umma_commit(smem_u32(qk_done));
+      mbar_wait(smem_u32(qk_done), 0, nullptr);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f32acc(1, 128, C::V_HALF, 0, 1);
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        const int s = i & 1;
+        ok = mbar_wait(smem_u32(p_full), i & 1, &abort_s);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sP), va = smem_u32(sKV + s * C::KV_STAGE_BYTES);
+#pragma unroll
+        for (int k = 0; k < C::BN / 16; ++k)
+          umma_bf16(tmem, sdesc_sw128(pa + k * 32, 16, 1024),
+                    sdesc_sw128(va + k * 16 * 128, C::BN * 128, 1024), idesc, (i | k) != 0);
+        umma_commit(smem_u32(&kv_empty[s]));
+        umma_commit(smem_u32(pv_done));
+      }
+      if (!ok) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+      umma_commit(smem_u32(pv_fin));
+      mbar_wait(smem_u32(pv_fin), 0, nullptr);
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ gather producers
+    const int tp = threadIdx.x - 256;
+    const int chunks = C::BN * kb_count * 8;
+    for (int i = 0; i < n; ++i) {
+      const int s = i & 1;
+      if (i >= 2 && !mbar_wait(smem_u32(&kv_empty[s]), ((i >> 1) - 1) & 1, &abort_s)) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+        break;
+      }
+      const int tile = sTiles[i];
+      uint8_t* dst = sKV + s * C::KV_STAGE_BYTES;
+      for (int c = tp; c < chunks; c += 128) {
+        const int kr = c / (kb_count * 8);
+        const int rem = c % (kb_count * 8);
+        const int kbl = rem / 8, ch = rem % 8;
+        const int d = (kb_begin + kbl) * 64 + ch * 8;
+        const int32_t phys = sPhys[tile * C::BN + kr];
+        const bool ok = phys >= 0 && d < D_QK;
+        cp_async_16(smem_u32(dst + kbl * (C::BN * 128) + sw128_offset(kr, ch)),
+                    ok ? static_cast<const void*>(p.kv + static_cast<int64_t>(phys) * D_QK + d)
+                       : static_cast<const void*>(p.kv),
+                    ok ? 16u : 0u);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&kv_full[s]));
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int hrow = threadIdx.x - 128;               // head = TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t x_local = smem_u32(sX) + hrow * (C::BN * 4);
+    const uint32_t x_remote = map_to_rank(x_local, peer);
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+      const int s = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_full[s]), (i >> 1) & 1, &abort_s));
+      if (!ok) break;
+      tc_fence_after();
+      float sv[C::BN];
+      {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(lane_addr + C::S_COL0 + s * C::BN, u0);
+        tmem_ld32(lane_addr + C::S_COL0 + s * C::BN + 32, u1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          sv[j] = __uint_as_float(u0[j]);
+          sv[32 + j] = __uint_as_float(u1[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_empty[s]));
+      // swap partial logits with the peer CTA
+      if (i >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(peer_free), (i - 1) & 1, &abort_s));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int c = 0; c < C::BN / 4; ++c)
+        st_cluster_v4(x_remote + ((c ^ (hrow & 7)) << 4), sv[4 * c], sv[4 * c + 1], sv[4 * c + 2],
+                      sv[4 * c + 3]);
+      mbar_arrive_cluster(smem_u32(x_full), peer);
+      ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(x_full), i & 1, &abort_s));
+      if (!ok) break;
+      const int tile = sTiles[i];
+      float m_tile = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < C::BN / 4; ++c) {
+        const float4 o = *reinterpret_cast<const float4*>(
+            reinterpret_cast<const uint8_t*>(sX) + hrow * (C::BN * 4) + ((c ^ (hrow & 7)) << 4));
+        const float ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * c + e;
+          // both CTAs add rank 0's partial to rank 1's: bit-identical logits in both
+          const float full_s = rank == 0 ? sv[j] + ov[e] : ov[e] + sv[j];
+          sv[j] = sPhys[tile * C::BN + j] >= 0 ? full_s * p.scale_log2 : -INFINITY;
+          m_tile = fmaxf(m_tile, sv[j]);
+        }
+      }
+      mbar_arrive_cluster(smem_u32(peer_free), peer);
+      // P and O are free once PV(i-1) has completed
+      if (i >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (i - 1) & 1, &abort_s));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      const bool need = m_tile > m_ref + 8.0f;
+      float alpha = 1.f;
+      if (need) {
+        alpha = exp2f(m_ref - m_tile);
+        l_sum *= alpha;
+        m_ref = m_tile;
+      }
+      if (i >= 1 && __any_sync(0xffffffffu, need)) {
+        for (int c0 = 0; c0 < C::V_HALF; c0 += 32) {
+          uint32_t u[32];
+          tmem_ld32(lane_addr + c0, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
+          tmem_st32(lane_addr + c0, u);
+        }
+        tmem_wait_st();
+      }
+      float rowsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < C::BN / 8; ++c) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // the denominator sums the fp32 probabilities; only the PV operand is rounded
+          const float p0 = exp2f(sv[8 * c + 2 * e] - m_ref);
+          const float p1 = exp2f(sv[8 * c + 2 * e + 1] - m_ref);
+          rowsum += p0 + p1;
+          const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&two);
+        }
+        *reinterpret_cast<uint4*>(sP + sw128_offset(hrow, c)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l_sum += rowsum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    if (!ok) {
+      abort_s = 1;
+      if (p.status) atomicOr(p.status, kStatusTimeout);
+    }
+    // ---- epilogue
+    const bool write = hrow < p.h;
+    const int64_t orow = static_cast<int64_t>(row) * p.h + hrow;
+    if (ok && n > 0)
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (n - 1) & 1, &abort_s));
+    tc_fence_after();
+    const float inv_l = (n > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+    const float lse_v = (n > 0 && l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f
+                                              : -INFINITY;
+    float* po = nullptr;
+    if (p.part_o != nullptr)
+      po = p.part_o + ((static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow) * D_V +
+           rank * C::V_HALF;
+    for (int c0 = 0; c0 < C::V_HALF; c0 += 32) {
+      float o[32];
+      if (ok && n > 0) {
+        uint32_t u[32];
+        tmem_ld32(lane_addr + c0, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(u[j]) * inv_l;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = 0.f;
+      }
+      if (!write) continue;
+      if (po != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(po + c0 + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
+      } else {
+        __nv_bfloat16* dst = p.out + orow * D_V + rank * C::V_HALF + c0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 two = __floats2bfloat162_rn(o[j + 2 * e], o[j + 2 * e + 1]);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&two);
+          }
+          *reinterpret_cast<uint4*>(dst + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    if (write && rank == 0) {
+      if (p.part_lse != nullptr)
+        p.part_lse[(static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow] = lse_v;
+      else
+        p.lse[orow] = lse_v;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // no remote access to this CTA's shared memory after this point
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Merge split-KV partials by their LSE: O = sum_i e^(LSE_i - LSE) O_i, LSE = log sum e^LSE_i.
+template <int D_V>
+__global__ void __launch_bounds__(128) dsa_mla_combine_kernel(const MlaParams p) {
+  const int r = blockIdx.x, hrow = blockIdx.y;
+  const int64_t stride = static_cast<int64_t>(p.row_count) * p.h;
+  const int64_t base = static_cast<int64_t>(r) * p.h + hrow;
+  float m = -INFINITY;
+  for (int s = 0; s < p.splits; ++s) m = fmaxf(m, p.part_lse[s * stride + base]);
+  float wsum = 0.f;
+  float wts[16];
+  for (int s = 0; s < p.splits; ++s) {
+    const float w = m == -INFINITY ? 0.f : expf(p.part_lse[s * stride + base] - m);
+    wts[s] = w;
+    wsum += w;
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const int64_t orow = static_cast<int64_t>(p.row_begin + r) * p.h + hrow;
+  for (int d = threadIdx.x * 4; d < D_V; d += 128 * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < p.splits; ++s) {
+      const float4 v = *reinterpret_cast<const float4*>(p.part_o + (s * stride + base) * D_V + d);
+      const float w = wts[s] * inv;
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    const __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
+    const __nv_bfloat162 c = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&a);
+    pk.y = *reinterpret_cast<const uint32_t*>(&c);
+    *reinterpret_cast<uint2*>(p.out + orow * D_V + d) = pk;
+  }
+  if (threadIdx.x == 0) p.lse[orow] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+}
+
+}  // namespace dsa

@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point that
+include/dsa.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    from sparse_attention_long_04_b200 import build as b
+    b.build()
+    import sparse_attention_long_04_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    return sorted(set(re.findall(r"^DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for n in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward",
+              "dsa_forward_workspace_size", "dsa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(dsa):
+    lib = ctypes.CDLL(dsa.LIB_PATH)
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+    assert set(dsa.EXPORTED) >= set(declared_symbols())
+    assert dsa.abi_version() == 1
+    assert dsa.status_string(0) == "ok"
+    assert "workspace" in dsa.status_string(3)
+
+
+FAKE = 0x10000   # a 16-byte-aligned address that is never dereferenced: validation fails first
+
+
+def _pb(dsa, **kw):
+    args = dict(mode="decode", h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512, topk=2048,
+                softmax_scale=0.04, num_kv_rows=1 << 20, seqlens=[4096, 100],
+                seq_lens=FAKE, block_table=None, max_seqlen=4096)
+    args.update(kw)
+    pb = dsa.make_problem(**{k: v for k, v in args.items() if k != "seq_lens"},
+                          seq_lens=None)
+    pb.seqs.seq_lens = args["seq_lens"]
+    return pb
+
+
+def test_null_pointers_rejected(dsa):
+    pb = _pb(dsa)
+    st = dsa.dsa_indexer_scores(pb, None, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE, 4096, None, 0)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    st = dsa.dsa_topk(pb, FAKE, 4096, 0, 2, None, None, 0)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    st = dsa.dsa_sparse_mla_fwd(pb, FAKE, FAKE, FAKE, 0, 2, FAKE, None, None, 0, None, 0)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    lib = dsa.lib
+    assert lib.dsa_forward(None, None, *([None] * 11), 0, None, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_bad_shapes_rejected(dsa):
+    assert dsa.dsa_indexer_scores(_pb(dsa, h_idx=32), FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE,
+                                  4096, None, 0) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert dsa.dsa_sparse_mla_fwd(_pb(dsa, d_qk=512), FAKE, FAKE, FAKE, 0, 2, FAKE, FAKE, None,
+                                  0, None, 0) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert dsa.dsa_topk(_pb(dsa, topk=100), FAKE, 4096, 0, 2, FAKE, None,
+                        0) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    # the tiny indexer shape is prefill-only
+    assert dsa.dsa_indexer_scores(_pb(dsa, h_idx=4, d_idx=32), FAKE, FAKE, FAKE, FAKE, FAKE, 0,
+                                  2, FAKE, 4096, None, 0) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_misaligned_and_bad_ld_rejected(dsa):
+    pb = _pb(dsa)
+    assert dsa.dsa_indexer_scores(pb, FAKE + 8, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE, 4096, None,
+                                  0) == dsa.DSA_ERR_MISALIGNED
+    assert dsa.dsa_topk(pb, FAKE, 4098, 0, 2, FAKE, None, 0) == dsa.DSA_ERR_MISALIGNED
+    assert dsa.dsa_sparse_mla_fwd(pb, FAKE, FAKE + 4, FAKE, 0, 2, FAKE, FAKE, None, 0, None,
+                                  0) == dsa.DSA_ERR_MISALIGNED
+    # ld below the longest row
+    assert dsa.dsa_topk(pb, FAKE, 1024, 0, 2, FAKE, None, 0) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_bad_geometry_rejected(dsa):
+    pb = _pb(dsa)
+    assert dsa.dsa_topk(pb, FAKE, 4096, 1, 2, FAKE, None, 0) == dsa.DSA_ERR_INVALID_ARG  # rows
+    pre = dsa.make_problem(mode="prefill", h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512,
+                           topk=2048, softmax_scale=0.04, num_kv_rows=100, seqlens=[60, 70],
+                           cu_seqlens=FAKE)
+    # more packed rows than cache rows
+    assert dsa.dsa_topk(pre, FAKE, 72, 0, 130, FAKE, None, 0) == dsa.DSA_ERR_INVALID_ARG
+    pre.seqs.cu_seqlens_host = None
+    assert dsa.dsa_topk(pre, FAKE, 72, 0, 1, FAKE, None, 0) == dsa.DSA_ERR_INVALID_ARG
+    # a block table narrower than the longest sequence
+    pb2 = _pb(dsa)
+    pb2.seqs.block_table = FAKE
+    pb2.seqs.max_blocks = 10
+    assert dsa.dsa_topk(pb2, FAKE, 4096, 0, 2, FAKE, None, 0) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_workspace_size_is_zero_on_bad_args(dsa):
+    pb = _pb(dsa, topk=7)
+    assert dsa.dsa_forward_workspace_size(pb) == 0
