@@ -137,7 +137,15 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     peaks = read_peaks()
     stream = torch.cuda.current_stream()
-    wl = make_config(DECODE_CFG, device=dev, seed=1000 + DECODE_CFG + 7919 * rank)
+    if args.decode_batch:
+        from dsa_workloads import make_decode
+        c = CONFIGS[DECODE_CFG]
+        wl = make_decode(DECODE_CFG, args.decode_batch, c["ctx"],
+                         {k: c[k] for k in ("h_idx", "d_idx", "topk", "h", "d_qk", "d_v")},
+                         c["boost"], c["paged"], dev, seed=1000 + DECODE_CFG + 7919 * rank,
+                         name=f"{c['name']}_B{args.decode_batch}")
+    else:
+        wl = make_config(DECODE_CFG, device=dev, seed=1000 + DECODE_CFG + 7919 * rank)
     d = wl.dims
     pb = dsa.problem_of(wl)
     B = wl.batch
@@ -253,7 +261,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e4m3+bf16",
         "data": "synthetic",
-        "config": {"workload": CONFIGS[DECODE_CFG]["name"], "batch": B,
+        "config": {"workload": wl.name, "batch": B,
                    "context": wl.max_seqlen, "page": 64, "topk": d["topk"],
                    "indexer": f"{d['h_idx']}x{d['d_idx']} e4m3", "heads": d["h"],
                    "latent": d["d_qk"], "d_v": d["d_v"],
@@ -327,11 +335,20 @@ def run_prefill(args, dsa, dev, stream, peaks, rank, world):
 
 
 def load_traffic(name):
+    """DRAM bytes per launch from the committed ncu summary, or None when the kernel source has
+    changed since the counters were taken."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        return json.load(f).get(name)
+        rec = json.load(f).get(name)
+    if rec is None:
+        return None
+    src = os.path.join(ROOT, "sparse_attention_long_04_b200", "csrc", "indexer.cuh")
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if h == rec.get("indexer_cuh_sha256_16") else None
 
 
 # ------------------------------------------------------------------------------ CPU oracle
@@ -413,6 +430,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="profiling only: decode sequences (default: the workload's 64)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

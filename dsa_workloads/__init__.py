@@ -138,8 +138,17 @@ def make_prefill(cfg_id: int, seqlens: List[int], dims: dict, needles: int, devi
     N(0,1) entries.  Latent KV and MLA queries stay pure N(0,1)."""
     seed = 1000 + cfg_id if seed is None else seed
     h_idx, d_idx, h, d_qk = dims["h_idx"], dims["d_idx"], dims["h"], dims["d_qk"]
-    qi_f, ki_f, w_l, q_l, kv_l = [], [], [], [], []
+    T = int(sum(seqlens))
+    q8 = torch.empty(T, h_idx, d_idx, dtype=torch.uint8, device=device)
+    qs = torch.empty(T, h_idx, dtype=torch.float32, device=device)
+    k8 = torch.empty(T, d_idx, dtype=torch.uint8, device=device)
+    ks = torch.empty(T, dtype=torch.float32, device=device)
+    w = torch.empty(T, h_idx, dtype=torch.float32, device=device)
+    q = torch.empty(T, h, d_qk, dtype=torch.bfloat16, device=device)
+    kv = torch.empty(T, d_qk, dtype=torch.bfloat16, device=device)
+    off = 0
     for b, L in enumerate(seqlens):
+        sl = slice(off, off + L)
         qi = torch.randn(L, h_idx, d_idx, generator=_gen(seed, 1, b, device), device=device)
         ki = torch.randn(L, d_idx, generator=_gen(seed, 2, b, device), device=device)
         if needles > 0 and L > 0:
@@ -153,26 +162,29 @@ def make_prefill(cfg_id: int, seqlens: List[int], dims: dict, needles: int, devi
                    * band_end.unsqueeze(1).float()).long().clamp_(max=L - 1)
             ki.index_add_(0, pos.reshape(-1),
                           (3.0 * math.sqrt(d_idx)) * u.repeat_interleave(needles, dim=0))
-        qi_f.append(qi)
-        ki_f.append(ki)
-        w_l.append(torch.rand(L, h_idx, generator=_gen(seed, 4, b, device), device=device))
-        q_l.append(torch.randn(L, h, d_qk, generator=_gen(seed, 5, b, device), device=device)
-                   .to(torch.bfloat16))
-        kv_l.append(torch.randn(L, d_qk, generator=_gen(seed, 6, b, device), device=device)
-                    .to(torch.bfloat16))
-    qi = torch.cat(qi_f)
-    ki = torch.cat(ki_f)
-    # literal per-token q scale: one amax over the token's h_idx x d_idx values, stored per head
-    q8, qs = quantize_e4m3_rows(qi, 2)
-    qs = qs.unsqueeze(1).expand(-1, h_idx).contiguous()
-    k8, ks = quantize_e4m3_rows(ki, 1)
+        # literal per-token q scale: one amax over the token's h_idx x d_idx values, stored per
+        # indexer head
+        q8[sl], s_tok = quantize_e4m3_rows(qi, 2)
+        qs[sl] = s_tok.unsqueeze(1)
+        k8[sl], ks[sl] = quantize_e4m3_rows(ki, 1)
+        del qi, ki
+        w[sl] = torch.rand(L, h_idx, generator=_gen(seed, 4, b, device), device=device)
+        gq, gkv = _gen(seed, 5, b, device), _gen(seed, 6, b, device)
+        step = max(1, (1 << 26) // (h * d_qk))          # bounded fp32 temporaries
+        for r0 in range(0, L, step):
+            r1 = min(L, r0 + step)
+            q[off + r0:off + r1] = torch.randn(r1 - r0, h, d_qk, generator=gq, device=device)
+        step = max(1, (1 << 26) // d_qk)
+        for r0 in range(0, L, step):
+            r1 = min(L, r0 + step)
+            kv[off + r0:off + r1] = torch.randn(r1 - r0, d_qk, generator=gkv, device=device)
+        off += L
     cu = torch.tensor([0] + list(torch.tensor(seqlens).cumsum(0).tolist()), dtype=torch.int32,
                       device=device)
     return Workload(cfg_id=cfg_id, name=name or f"prefill_{len(seqlens)}seq", mode="prefill",
                     dims=dict(dims), softmax_scale=softmax_scale or 1.0 / math.sqrt(d_qk),
-                    seqlens=list(seqlens), q_idx=q8, q_scale=qs, w=torch.cat(w_l).contiguous(),
-                    k_idx=k8, k_scale=ks, q=torch.cat(q_l).contiguous(),
-                    kv=torch.cat(kv_l).contiguous(), cu_seqlens=cu, max_seqlen=max(seqlens))
+                    seqlens=list(seqlens), q_idx=q8, q_scale=qs, w=w, k_idx=k8, k_scale=ks,
+                    q=q, kv=kv, cu_seqlens=cu, max_seqlen=max(seqlens))
 
 
 def make_decode(cfg_id: int, batch: int, ctx, dims: dict, boost: float, paged: bool, device,

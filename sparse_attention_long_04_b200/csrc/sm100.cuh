@@ -93,6 +93,35 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Non-suspending probe of phase `parity`, cluster-scope acquire.
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded spin (no suspension) for phases completed by another CTA of the cluster, whose
+// completion may not wake a thread suspended in try_wait promptly.
+__device__ __forceinline__ bool mbar_spin_cluster(uint32_t bar, uint32_t parity,
+                                                  const volatile int* abort) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_test_wait_cluster(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (abort != nullptr && *abort) return false;
+      uint64_t now = global_timer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
 // Bounded wait for phase `parity` of `bar`.  Returns false when the wall-clock limit passes
 // or when *abort becomes non-zero (another role of the CTA already gave up); the caller
 // then records the failure and unwinds instead of hanging.
@@ -139,6 +168,16 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
+}
+
+// Asynchronous 16-byte store into the shared memory of another CTA of the cluster; on arrival
+// it performs complete_tx(16) on the barrier `remote_bar` (also a cluster address).
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remote_bar, float a,
+                                            float b, float c, float d) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(remote_addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+      : "memory");
 }
 
 // ---------------------------------------------------------------------------- cp.async

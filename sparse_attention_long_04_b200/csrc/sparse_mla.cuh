@@ -69,7 +69,7 @@ struct MlaCfg {
   static constexpr int S_COL0 = V_HALF;               // TMEM: O at [0, V_HALF), S at S_COL0
   static constexpr int TMEM_COLS = (V_HALF + 2 * BN) <= 256 ? 256 : 512;
   static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_STAGE_BYTES + P_BYTES + X_BYTES +
-                                    MAX_TOPK * 4 + 64 * 4 + 256;
+                                    MAX_TOPK * 4 + 64 * 4 + 32 * 8 + 256;
   static_assert(KBC >= VKB, "rank 1 holds at least as many k-blocks as rank 0");
   static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -88,16 +88,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   uint8_t* sP = sKV + C::STAGES * C::KV_STAGE_BYTES;
   float* sX = reinterpret_cast<float*>(sP + C::P_BYTES);
   int32_t* sPhys = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sX) + C::X_BYTES);
-  int32_t* sTiles = sPhys + C::MAX_TOPK;                 // [32] active tile ids, [32] count
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sTiles + 64);
+  int32_t* sTiles = sPhys + C::MAX_TOPK;                 // [32] active tile ids (this split)
+  uint64_t* sMask = reinterpret_cast<uint64_t*>(sTiles + 64);   // [32] valid keys per tile
+  uint64_t* bars = sMask + 32;
   uint64_t* kv_full = bars;          // [2] producers (128 arrivals)
   uint64_t* kv_empty = bars + 2;     // [2] QK commit + PV commit
   uint64_t* s_full = bars + 4;       // [2] QK commit
   uint64_t* s_empty = bars + 6;      // [2] 4 softmax warps
   uint64_t* p_full = bars + 8;       // 128 softmax threads
   uint64_t* pv_done = bars + 9;      // PV commit
-  uint64_t* x_full = bars + 10;      // 128 remote arrivals: peer's partial logits are here
-  uint64_t* peer_free = bars + 11;   // 128 remote arrivals: peer consumed what we sent
+  uint64_t* x_full = bars + 10;      // 1 local arrive + 32 KB of the peer's st.async bytes
+  uint64_t* peer_free = bars + 11;   // 4 remote arrivals: the peer consumed what we sent
   uint64_t* qk_done = bars + 12;
   uint64_t* pv_fin = bars + 13;
   __shared__ uint32_t tmem_base_s;
@@ -140,8 +141,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     }
     mbar_init(smem_u32(p_full), 128);
     mbar_init(smem_u32(pv_done), 1);
-    mbar_init(smem_u32(x_full), 128);
-    mbar_init(smem_u32(peer_free), 128);
+    mbar_init(smem_u32(x_full), 1);
+    mbar_init(smem_u32(peer_free), 4);
     mbar_init(smem_u32(qk_done), 1);
     mbar_init(smem_u32(pv_fin), 1);
     abort_s = 0;
@@ -150,30 +151,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   if (warp == 1) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
 
   if (warp >= 8) {
-    // ---- resolve logical indices to physical rows; load this CTA's Q dims
+    // ---- resolve logical indices to physical rows (all loads of a round issued together);
+    //      load this CTA's Q dims
     const int tp = threadIdx.x - 256;
     const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
-    for (int j = tp; j < p.topk; j += 128) {
-      const int v = irow[j];
-      int64_t phys = -1;
-      if (v >= 0) {
-        if (v < n_keys) {
-          if (!p.decode) {
-            phys = key_base + v;
-          } else if (p.block_table != nullptr) {
-            const int64_t id = p.block_table[static_cast<int64_t>(b) * p.max_blocks +
-                                             v / p.block_size];
-            phys = id * p.block_size + v % p.block_size;
-            if (id < 0) phys = -1;
-          } else {
-            phys = key_base + v;
-          }
-          if (phys >= p.num_kv_rows) phys = -1;
-        }
-        if (phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
-      }
-      sPhys[j] = static_cast<int32_t>(phys);
-    }
     const __nv_bfloat16* qrow = p.q + static_cast<int64_t>(row) * p.h * D_QK;
     for (int c = tp; c < 128 * kb_count * 8; c += 128) {
       const int hrow = c / (kb_count * 8);
@@ -187,30 +168,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                   ok ? 16u : 0u);
     }
     cp_async_commit();
+    for (int j0 = 0; j0 < p.topk; j0 += 4 * 512) {
+      int4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + (u * 128 + tp) * 4;
+        v[u] = j < p.topk ? *reinterpret_cast<const int4*>(irow + j) : make_int4(-1, -1, -1, -1);
+      }
+      int64_t ph[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int vi = (&v[e / 4].x)[e % 4];
+        ph[e] = -1;
+        if (vi >= 0 && vi < n_keys) {
+          if (p.decode && p.block_table != nullptr)
+            ph[e] = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + vi / p.block_size);
+          else
+            ph[e] = key_base + vi;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int vi = (&v[e / 4].x)[e % 4];
+        int64_t phys = ph[e];
+        if (vi >= 0 && vi < n_keys && p.decode && p.block_table != nullptr)
+          phys = phys < 0 ? -1 : phys * p.block_size + vi % p.block_size;
+        if (phys >= p.num_kv_rows) phys = -1;
+        if (vi >= 0 && phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+        const int j = j0 + ((e / 4) * 128 + tp) * 4 + (e % 4);
+        if (j < p.topk) sPhys[j] = static_cast<int32_t>(phys);
+      }
+    }
     cp_async_wait<0>();
     fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // ---- active tiles (at least one valid key), identical in both CTAs
+  // ---- per-tile validity masks and the active tiles (>= 1 valid key), identical in both CTAs
   if (warp == 0) {
     const int n_tiles_all = p.topk / C::BN;
     int cnt = 0;
     for (int t = 0; t < n_tiles_all; ++t) {
-      const int j = t * C::BN + lane * 2;
-      const bool any = __any_sync(0xffffffffu, sPhys[j] >= 0 || sPhys[j + 1] >= 0);
-      if (any) {
-        if (lane == 0) sTiles[cnt] = t;
+      const uint32_t lo = __ballot_sync(0xffffffffu, sPhys[t * C::BN + lane] >= 0);
+      const uint32_t hi = __ballot_sync(0xffffffffu, sPhys[t * C::BN + 32 + lane] >= 0);
+      const uint64_t m = (static_cast<uint64_t>(hi) << 32) | lo;
+      if (m != 0) {
+        if (lane == 0) {
+          sTiles[cnt] = t;
+          sMask[cnt] = m;
+        }
         ++cnt;
       }
     }
+    __syncwarp();
     if (lane == 0) {
       const int per = (cnt + p.splits - 1) / p.splits;
       const int t0 = min(cnt, split * per);
       const int t1 = min(cnt, t0 + per);
-      for (int i = t0; i < t1; ++i) sTiles[i - t0] = sTiles[i];
+      for (int i = t0; i < t1; ++i) {
+        sTiles[i - t0] = sTiles[i];
+        sMask[i - t0] = sMask[i];
+      }
       n_act_s = t1 - t0;
+      if (t1 > t0) mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);   // arm tile 0
     }
   }
   __syncthreads();
@@ -309,6 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t x_local = smem_u32(sX) + hrow * (C::BN * 4);
     const uint32_t x_remote = map_to_rank(x_local, peer);
+    const uint32_t x_full_remote = map_to_rank(smem_u32(x_full), peer);
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
@@ -331,19 +353,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&s_empty[s]));
-      // swap partial logits with the peer CTA
+      // swap partial logits with the peer CTA: st.async lands in the peer's buffer and
+      // counts its bytes on the peer's x_full
       if (i >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(peer_free), (i - 1) & 1, &abort_s));
         if (!ok) break;
       }
 #pragma unroll
       for (int c = 0; c < C::BN / 4; ++c)
-        st_cluster_v4(x_remote + ((c ^ (hrow & 7)) << 4), sv[4 * c], sv[4 * c + 1], sv[4 * c + 2],
-                      sv[4 * c + 3]);
-      mbar_arrive_cluster(smem_u32(x_full), peer);
+        st_async_v4(x_remote + ((c ^ (hrow & 7)) << 4), x_full_remote, sv[4 * c], sv[4 * c + 1],
+                    sv[4 * c + 2], sv[4 * c + 3]);
       ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(x_full), i & 1, &abort_s));
       if (!ok) break;
-      const int tile = sTiles[i];
+      if (hrow == 0 && i + 1 < n) mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);  // arm i+1
+      const uint64_t vmask = sMask[i];
       float m_tile = -INFINITY;
 #pragma unroll
       for (int c = 0; c < C::BN / 4; ++c) {
@@ -355,11 +378,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           const int j = 4 * c + e;
           // both CTAs add rank 0's partial to rank 1's: bit-identical logits in both
           const float full_s = rank == 0 ? sv[j] + ov[e] : ov[e] + sv[j];
-          sv[j] = sPhys[tile * C::BN + j] >= 0 ? full_s * p.scale_log2 : -INFINITY;
+          sv[j] = ((vmask >> j) & 1ull) ? full_s * p.scale_log2 : -INFINITY;
           m_tile = fmaxf(m_tile, sv[j]);
         }
       }
-      mbar_arrive_cluster(smem_u32(peer_free), peer);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(smem_u32(peer_free), peer);
       // P and O are free once PV(i-1) has completed
       if (i >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (i - 1) & 1, &abort_s));
