@@ -155,6 +155,31 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t
                                 float* lse, void* workspace, size_t workspace_bytes,
                                 int32_t* dev_status, dsa_stream_t stream);
 
+/* Sparse MLA forward for callers that cannot allocate device memory.  No counterpart on the
+ * pages: it is a packaging of dsa_sparse_mla_fwd, not a step of the method.
+ *
+ * Some callers may not call cudaMalloc or any allocator at all: code recorded into a CUDA graph,
+ * where an allocation would break the capture; runtimes that hand out every byte of device memory
+ * from their own fixed pool; plugins whose host framework forbids allocator calls on the hot
+ * path.  This entry point computes exactly what dsa_sparse_mla_fwd computes (same arguments
+ * minus the workspace) and keeps its split-KV partials in a scratch array built into the
+ * library: DSA_NOALLOC_SCRATCH_BYTES (20 MiB) of device memory that every GPU loading the
+ * library holds until the process exits.
+ *   - The first call on a device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with that device current).  Make that first call before any stream
+ *     capture.
+ *   - A call whose split-KV partials would not fit the array returns
+ *     DSA_ERR_WORKSPACE_TOO_SMALL before launching (on a 148-SM B200 every row count fits).
+ *   - Every call shares the one array and each call overwrites the parts it uses, so nothing has
+ *     to start at zero; two calls that overlap on the GPU (different streams, no ordering) race
+ *     on it and give undefined results.  Calls on one stream are safe. */
+#define DSA_NOALLOC_SCRATCH_BYTES (20u << 20)
+DSA_API dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                                const uint16_t* q, const uint16_t* kv,
+                                                const int32_t* idx, int32_t row_begin,
+                                                int32_t row_count, uint16_t* out, float* lse,
+                                                int32_t* dev_status, dsa_stream_t stream);
+
 /* Bytes of workspace dsa_forward needs (score slab for one row chunk, chunk indices when
  * idx_out is NULL, split-KV partials).  Larger workspaces allow larger prefill chunks. */
 DSA_API size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs);

@@ -36,7 +36,9 @@ DSA_DECODE = 1
 
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_fwd", "dsa_forward_workspace_size", "dsa_forward",
-            "dsa_read_device_status", "dsa_status_string", "dsa_abi_version")
+            "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
+            "dsa_sparse_mla_fwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
 class DsaError(RuntimeError):
@@ -78,6 +80,7 @@ def _load():
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_status_string": (ctypes.c_char_p, [I32]),
         "dsa_abi_version": (I32, []),
+        "dsa_sparse_mla_fwd_noalloc": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -201,6 +204,15 @@ def dsa_sparse_mla_fwd(pb: Problem, q, kv, idx, row_begin: int, row_count: int, 
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q), _ptr(kv), _ptr(idx), row_begin,
         row_count, _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes, _ptr(dev_status),
         _stream(stream)))
+
+
+def dsa_sparse_mla_fwd_noalloc(pb: Problem, q, kv, idx, row_begin: int, row_count: int, out, lse,
+                               dev_status=None, stream=None) -> int:
+    """dsa_sparse_mla_fwd without a workspace, for callers that may not allocate device memory
+    (its scratch is an array built into the library; see include/dsa.h)."""
+    return int(lib.dsa_sparse_mla_fwd_noalloc(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q), _ptr(kv), _ptr(idx), row_begin,
+        row_count, _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
 
 
 def dsa_forward_workspace_size(pb: Problem) -> int:

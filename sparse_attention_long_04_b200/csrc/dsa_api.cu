@@ -569,4 +569,51 @@ dsa_status_t dsa_read_device_status(const int32_t* dev_status, dsa_stream_t stre
   return DSA_OK;
 }
 
+// ---------------------------------------------------------------------------- no allocation
+// Scratch for dsa_sparse_mla_fwd_noalloc: a device array built into the library.  In host code
+// `g_noalloc_scratch` is only a stand-in symbol, never a device address; the address of each
+// device's copy comes from cudaGetSymbolAddress with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+
+dsa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return DSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+}  // namespace
+
+dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                        const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                        int32_t row_begin, int32_t row_count, uint16_t* out,
+                                        float* lse, int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q || !kv || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || !aligned16(lse))
+    return DSA_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  const int splits = mla_splits(*dims, *seqs, row_count, info.sm_count);
+  const size_t need = mla_ws_bytes(*dims, splits, row_count);
+  if (need > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  if (need > 0 && (e = noalloc_scratch(&scratch)) != DSA_OK) return e;
+  return mla_dispatch(*dims, *seqs, q, kv, idx, row_begin, row_count, out, lse, scratch,
+                      need > 0 ? DSA_NOALLOC_SCRATCH_BYTES : 0, dev_status,
+                      reinterpret_cast<cudaStream_t>(stream), splits);
+}
+
 }  // extern "C"
