@@ -11,19 +11,21 @@
 // Design (sm_100a).  O for 128 heads x 512 values in fp32 is 256 KB = all of one SM's TMEM,
 // and Q (128 x 576 bf16 = 144 KB) plus gathered tiles do not fit one CTA's shared memory, so
 // each query row runs on a 2-CTA cluster:
-//   CTA r holds Q dims D_r (r = 0: [0, D_V/2); r = 1: [D_V/2, D_QK)) and gathers the same dims
-//   of each selected latent row.  Per 64-key tile it computes the partial logits
-//   S_r = Q[:, D_r] K[:, D_r]^T (tcgen05 bf16, M = 128 heads, N = 64 keys) into TMEM, the two
-//   CTAs swap S_r through distributed shared memory, and both form S = S_0 + S_1 in the same
-//   order, so both run an identical online softmax.  CTA r then accumulates its half of the
-//   values, O_r += P V[:, r * D_V/2 : (r+1) * D_V/2] (M = 128, N = D_V/2, K = 64 keys; V is
-//   read MN-major straight out of the gathered tile).  No tensor work is duplicated.
-//   Rescaling of O is lazy: it happens only when a tile's max exceeds the running reference
-//   by more than 2^8, so P stays <= 256.
-// Warp roles per CTA: warp 0 issues QK, warp 2 issues PV, warp 1 owns TMEM, warps 4-7 run the
-// softmax (thread = head = TMEM lane) and the epilogue, warps 8-11 resolve indices and gather
-// rows with 16-byte cp.async into 128-byte-swizzled tiles (2 stages).
-// Grid: x = 2 * row (the cluster pair), y = split-KV slice.
+//   CTA r owns the QK dims D_r (r = 0: [0, D_V/2); r = 1: [D_V/2, D_QK)) and the value dims
+//   [r D_V/2, (r+1) D_V/2).  Its slice of Q lives in Tensor Memory as the A operand of the QK
+//   MMA; the selected latent rows are gathered (their D_r dims) into 128-byte-swizzled shared
+//   memory tiles of 64 keys.  Per tile: S_r = Q_r K_r^T (tcgen05 bf16, A from TMEM, M = 128
+//   heads, N = 64 keys); the two CTAs swap S_r with bulk shared-to-shared copies into each
+//   other's memory and both form S = S_0 + S_1 in the same order, so both run an identical
+//   online softmax; P goes to TMEM and CTA r accumulates O_r += P V_r (A = P from TMEM,
+//   N = D_V/2, K = 64 keys, V read MN-major straight out of the gathered tile).  No tensor
+//   work is duplicated.  Rescaling of O is lazy (only when a tile's max beats the running
+//   reference by more than 2^8, so P <= 256).
+// TMEM columns: O [0, V_HALF) | S [V_HALF, +64) | P [+64, +32) | Q (kb_count x 32 columns).
+// Warp roles per CTA (512 threads): warp 0 issues QK, warp 2 issues PV, warp 1 owns TMEM,
+// warps 4-11 run the softmax (thread = head = TMEM lane; warps 4-7 take keys 0-31 of a tile,
+// warps 8-11 keys 32-63) and the epilogue, warps 12-15 resolve indices and gather rows with
+// 16-byte cp.async (3 stages).  Grid: x = 2 * row (the cluster pair), y = split-KV slice.
 #pragma once
 #include "sm100.cuh"
 
@@ -59,48 +61,57 @@ struct MlaCfg {
   static constexpr int VKB = V_HALF / 64;             // value k-blocks per CTA
   static constexpr int KBC = KB_ALL - VKB;            // k-blocks held by rank 1 (>= rank 0)
   static constexpr int BN = 64;                       // keys per tile
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = 3;
   static constexpr int MAX_TOPK = 2048;
-  static constexpr int THREADS = 384;
-  static constexpr int Q_BYTES = KBC * 128 * 128;
+  static constexpr int THREADS = 512;
   static constexpr int KV_STAGE_BYTES = KBC * BN * 128;
-  static constexpr int P_BYTES = 128 * 128;
-  static constexpr int X_BYTES = 128 * BN * 4;        // received partial logits
-  static constexpr int S_COL0 = V_HALF;               // TMEM: O at [0, V_HALF), S at S_COL0
-  static constexpr int TMEM_COLS = (V_HALF + 2 * BN) <= 256 ? 256 : 512;
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_STAGE_BYTES + P_BYTES + X_BYTES +
-                                    MAX_TOPK * 4 + 64 * 4 + 32 * 8 + 256;
+  static constexpr int X_BYTES = 128 * BN * 4;        // partial logits of one tile
+  static constexpr int S_COL = V_HALF;
+  static constexpr int P_COL = S_COL + BN;
+  static constexpr int Q_COL = P_COL + BN / 2;
+  static constexpr int TMEM_NEED = Q_COL + KBC * 32;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * KV_STAGE_BYTES + 2 * X_BYTES +
+                                    MAX_TOPK * 4 + 32 * 4 + 32 * 8 + 2 * 2 * 128 * 4 +
+                                    2 * 128 * 4 + 256;   // barriers: 19 x 8 bytes
   static_assert(KBC >= VKB, "rank 1 holds at least as many k-blocks as rank 0");
   static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
+  static_assert(TMEM_NEED <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(SMEM_BYTES > 114 * 1024, "one CTA per SM (TMEM and cluster peers)");
 };
 
 template <int D_QK, int D_V>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     dsa_sparse_mla_kernel(const MlaParams p) {
   using C = MlaCfg<D_QK, D_V>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::Q_BYTES;
-  uint8_t* sP = sKV + C::STAGES * C::KV_STAGE_BYTES;
-  float* sX = reinterpret_cast<float*>(sP + C::P_BYTES);
-  int32_t* sPhys = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sX) + C::X_BYTES);
-  int32_t* sTiles = sPhys + C::MAX_TOPK;                 // [32] active tile ids (this split)
-  uint64_t* sMask = reinterpret_cast<uint64_t*>(sTiles + 64);   // [32] valid keys per tile
-  uint64_t* bars = sMask + 32;
-  uint64_t* kv_full = bars;          // [2] producers (128 arrivals)
-  uint64_t* kv_empty = bars + 2;     // [2] QK commit + PV commit
-  uint64_t* s_full = bars + 4;       // [2] QK commit
-  uint64_t* s_empty = bars + 6;      // [2] 4 softmax warps
-  uint64_t* p_full = bars + 8;       // 128 softmax threads
+  uint8_t* sKV = smem;                                          // [STAGES] gathered tiles
+  uint8_t* sXin = sKV + C::STAGES * C::KV_STAGE_BYTES;          // peer's partial logits
+  uint8_t* sXout = sXin + C::X_BYTES;                           // ours, staged for the copy
+  int32_t* sPhys = reinterpret_cast<int32_t*>(sXout + C::X_BYTES);
+  int32_t* sTiles = sPhys + C::MAX_TOPK;                        // [32] active tiles (split)
+  uint64_t* sMask = reinterpret_cast<uint64_t*>(sTiles + 32);   // [32] valid keys per tile
+  float* sRed = reinterpret_cast<float*>(sMask + 32);           // [2 tiles][2 halves][128]
+  float* sLsum = sRed + 2 * 2 * 128;                            // [2 halves][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sLsum + 2 * 128);
+  uint64_t* kv_full = bars;          // [3] 128 producer arrivals
+  uint64_t* kv_empty = bars + 3;     // [3] QK commit + PV commit
+  uint64_t* s_full = bars + 6;       // QK commit
+  uint64_t* s_empty = bars + 7;      // 8 softmax warps
+  uint64_t* p_full = bars + 8;       // 256 softmax threads
   uint64_t* pv_done = bars + 9;      // PV commit
-  uint64_t* x_full = bars + 10;      // 1 local arrive + 32 KB of the peer's st.async bytes
-  uint64_t* peer_free = bars + 11;   // 4 remote arrivals: the peer consumed what we sent
-  uint64_t* qk_done = bars + 12;
-  uint64_t* pv_fin = bars + 13;
+  uint64_t* x_full = bars + 10;      // 1 local arrive + X_BYTES from the peer's copies
+  uint64_t* peer_free = bars + 11;   // 1 remote arrival: the peer read what we sent
+  uint64_t* mx_bar = bars + 12;      // 256 arrivals per tile: both halves' partial max written
+  uint64_t* fin_bar = bars + 13;     // 256 arrivals: both halves' partial sums written
+  uint64_t* qk_fin = bars + 14;
+  uint64_t* pv_fin = bars + 15;
+  uint64_t* staged = bars + 16;      // 256 arrivals: our partial logits are in the staging area
+  uint64_t* stage_free = bars + 17;  // 1 arrival: the copy out of the staging area is done
+  uint64_t* xin_read = bars + 18;    // 256 arrivals: the peer's partial logits were read
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int n_act_s;
@@ -133,41 +144,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(smem_u32(&kv_full[i]), 128);
       mbar_init(smem_u32(&kv_empty[i]), 2);
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_empty[i]), 4);
     }
-    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(s_empty), 8);
+    mbar_init(smem_u32(p_full), 256);
     mbar_init(smem_u32(pv_done), 1);
     mbar_init(smem_u32(x_full), 1);
-    mbar_init(smem_u32(peer_free), 4);
-    mbar_init(smem_u32(qk_done), 1);
+    mbar_init(smem_u32(peer_free), 1);
+    mbar_init(smem_u32(staged), 256);
+    mbar_init(smem_u32(stage_free), 1);
+    mbar_init(smem_u32(xin_read), 256);
+    mbar_init(smem_u32(mx_bar), 256);
+    mbar_init(smem_u32(fin_bar), 256);
+    mbar_init(smem_u32(qk_fin), 1);
     mbar_init(smem_u32(pv_fin), 1);
     abort_s = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
 
-  if (warp >= 8) {
-    // ---- resolve logical indices to physical rows (all loads of a round issued together);
-    //      load this CTA's Q dims
-    const int tp = threadIdx.x - 256;
+  if (warp >= 12) {
+    // ---- resolve logical indices to physical rows (all loads of a round issued together)
+    const int tp = threadIdx.x - 384;
     const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
-    const __nv_bfloat16* qrow = p.q + static_cast<int64_t>(row) * p.h * D_QK;
-    for (int c = tp; c < 128 * kb_count * 8; c += 128) {
-      const int hrow = c / (kb_count * 8);
-      const int rem = c % (kb_count * 8);
-      const int kbl = rem / 8, ch = rem % 8;
-      const int d = (kb_begin + kbl) * 64 + ch * 8;
-      const bool ok = hrow < p.h && d < D_QK;
-      cp_async_16(smem_u32(sQ + kbl * 16384 + sw128_offset(hrow, ch)),
-                  ok ? static_cast<const void*>(qrow + static_cast<int64_t>(hrow) * D_QK + d)
-                     : static_cast<const void*>(p.q),
-                  ok ? 16u : 0u);
-    }
-    cp_async_commit();
     for (int j0 = 0; j0 < p.topk; j0 += 4 * 512) {
       int4 v[4];
 #pragma unroll
@@ -182,7 +184,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         ph[e] = -1;
         if (vi >= 0 && vi < n_keys) {
           if (p.decode && p.block_table != nullptr)
-            ph[e] = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + vi / p.block_size);
+            ph[e] = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
+                          vi / p.block_size);
           else
             ph[e] = key_base + vi;
         }
@@ -199,12 +202,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         if (j < p.topk) sPhys[j] = static_cast<int32_t>(phys);
       }
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  if (warp >= 4 && warp < 12) {
+    // ---- this CTA's slice of Q into TMEM (the QK A operand): head = lane, 2 bf16 per column
+    const int hrow = (warp & 3) * 32 + lane;
+    const int half = (warp - 4) >> 2;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int d0 = kb_begin * 64 + half * kb_count * 32;        // first dim of this half
+    const __nv_bfloat16* qrow = p.q + (static_cast<int64_t>(row) * p.h + hrow) * D_QK;
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint32_t u[16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int d = d0 + kb * 32 + c * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (hrow < p.h && d < D_QK) v = *reinterpret_cast<const uint4*>(qrow + d);
+        u[4 * c + 0] = v.x;
+        u[4 * c + 1] = v.y;
+        u[4 * c + 2] = v.z;
+        u[4 * c + 3] = v.w;
+      }
+      tmem_st16(lane_addr + C::Q_COL + half * kb_count * 16 + kb * 16, u);
+    }
+    tmem_wait_st();
+  }
   // ---- per-tile validity masks and the active tiles (>= 1 valid key), identical in both CTAs
   if (warp == 0) {
     const int n_tiles_all = p.topk / C::BN;
@@ -234,10 +259,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (t1 > t0) mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);   // arm tile 0
     }
   }
+  tc_fence_before();
   __syncthreads();
-  cluster_sync();   // peer barriers initialised before any remote arrive
+  tc_fence_after();
+  cluster_sync();   // peer barriers initialised before any remote access
   const int n = n_act_s;
-  const uint32_t tmem = tmem_base_s;
 
   if (warp == 0) {
     // ------------------------------------------------------------ QK issuer
@@ -245,29 +271,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       constexpr uint32_t idesc = idesc_f32acc(1 /* bf16 */, 128, C::BN, 0, 0);
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
-        const int s = i & 1;
-        ok = mbar_wait(smem_u32(&kv_full[s]), (i >> 1) & 1, &abort_s);
-        if (ok && i >= 2) ok = mbar_wait(smem_u32(&s_empty[s]), ((i >> 1) - 1) & 1, &abort_s);
+        const int s = i % C::STAGES;
+        ok = mbar_wait(smem_u32(&kv_full[s]), (i / C::STAGES) & 1, &abort_s);
+        if (ok && i >= 1) ok = mbar_wait(smem_u32(s_empty), (i - 1) & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
         fence_proxy_async_smem();
-        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sKV + s * C::KV_STAGE_BYTES);
+        const uint32_t ka = smem_u32(sKV + s * C::KV_STAGE_BYTES);
         for (int kb = 0; kb < kb_count; ++kb)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem + C::S_COL0 + s * C::BN,
-                      sdesc_sw128(qa + kb * 16384 + k * 32, 16, 1024),
-                      sdesc_sw128(ka + kb * (C::BN * 128) + k * 32, 16, 1024), idesc,
-                      (kb | k) != 0);
-        umma_commit(smem_u32(&s_full[s]));
+            umma_bf16_ts(tmem + C::S_COL, tmem + C::Q_COL + kb * 32 + k * 8,
+                         sdesc_sw128(ka + kb * (C::BN * 128) + k * 32, 16, 1024), idesc,
+                         (kb | k) != 0);
+        umma_commit(smem_u32(s_full));
         umma_commit(smem_u32(&kv_empty[s]));
       }
       if (!ok) {
         abort_s = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
       }
-      umma_commit(smem_u32(qk_done));
-      mbar_wait(smem_u32(qk_done), 0, nullptr);
+      umma_commit(smem_u32(qk_fin));
+      mbar_wait(smem_u32(qk_fin), 0, nullptr);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ PV issuer
@@ -275,15 +300,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       constexpr uint32_t idesc = idesc_f32acc(1, 128, C::V_HALF, 0, 1);
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
-        const int s = i & 1;
+        const int s = i % C::STAGES;
         ok = mbar_wait(smem_u32(p_full), i & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sP), va = smem_u32(sKV + s * C::KV_STAGE_BYTES);
+        const uint32_t va = smem_u32(sKV + s * C::KV_STAGE_BYTES);
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k)
-          umma_bf16(tmem, sdesc_sw128(pa + k * 32, 16, 1024),
-                    sdesc_sw128(va + k * 16 * 128, C::BN * 128, 1024), idesc, (i | k) != 0);
+          umma_bf16_ts(tmem, tmem + C::P_COL + k * 8,
+                       sdesc_sw128(va + k * 16 * 128, C::BN * 128, 1024), idesc, (i | k) != 0);
         umma_commit(smem_u32(&kv_empty[s]));
         umma_commit(smem_u32(pv_done));
       }
@@ -294,13 +319,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       umma_commit(smem_u32(pv_fin));
       mbar_wait(smem_u32(pv_fin), 0, nullptr);
     }
-  } else if (warp >= 8) {
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ exchange helper
+    // Copies our staged partial logits into the peer's buffer and tells the peer when its
+    // partials have been read here: the cluster-scope release of that signal is slow, so it is
+    // kept off the softmax warps.
+    if (lane == 0) {
+      const uint32_t xin_remote = map_to_rank(smem_u32(sXin), peer);
+      const uint32_t x_full_remote = map_to_rank(smem_u32(x_full), peer);
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        ok = mbar_wait(smem_u32(staged), i & 1, &abort_s);
+        if (ok && i >= 1) ok = mbar_wait<true>(smem_u32(peer_free), (i - 1) & 1, &abort_s);
+        if (!ok) break;
+        bulk_copy_to_peer(xin_remote, smem_u32(sXout), C::X_BYTES, x_full_remote);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(smem_u32(stage_free));
+        ok = mbar_wait(smem_u32(xin_read), i & 1, &abort_s);
+        if (!ok) break;
+        mbar_arrive_cluster(smem_u32(peer_free), peer);
+      }
+      if (!ok) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+      bulk_wait_read_all();
+    }
+  } else if (warp >= 12) {
     // ------------------------------------------------------------ gather producers
-    const int tp = threadIdx.x - 256;
+    const int tp = threadIdx.x - 384;
     const int chunks = C::BN * kb_count * 8;
     for (int i = 0; i < n; ++i) {
-      const int s = i & 1;
-      if (i >= 2 && !mbar_wait(smem_u32(&kv_empty[s]), ((i >> 1) - 1) & 1, &abort_s)) {
+      const int s = i % C::STAGES;
+      if (i >= C::STAGES &&
+          !mbar_wait(smem_u32(&kv_empty[s]), ((i / C::STAGES) - 1) & 1, &abort_s)) {
         abort_s = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
         break;
@@ -326,64 +379,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int hrow = threadIdx.x - 128;               // head = TMEM lane
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t x_local = smem_u32(sX) + hrow * (C::BN * 4);
-    const uint32_t x_remote = map_to_rank(x_local, peer);
-    const uint32_t x_full_remote = map_to_rank(smem_u32(x_full), peer);
+    const int quad = warp & 3;
+    const int half = (warp - 4) >> 2;           // keys [32 half, 32 half + 32) of each tile
+    const int hrow = quad * 32 + lane;          // head = TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    // row `hrow`, this half, 16-byte chunk c (0..7) of the staged / received partial logits
+    const uint32_t x_row = half * (128 * 128) + hrow * 128;
+    constexpr int OC = C::V_HALF / 2;           // O columns this half rescales / stores
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
-      const int s = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_full[s]), (i >> 1) & 1, &abort_s));
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(s_full), i & 1, &abort_s));
       if (!ok) break;
       tc_fence_after();
-      float sv[C::BN];
+      float sv[32];
       {
-        uint32_t u0[32], u1[32];
-        tmem_ld32(lane_addr + C::S_COL0 + s * C::BN, u0);
-        tmem_ld32(lane_addr + C::S_COL0 + s * C::BN + 32, u1);
+        uint32_t u[32];
+        tmem_ld32(lane_addr + C::S_COL + half * 32, u);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          sv[j] = __uint_as_float(u0[j]);
-          sv[32 + j] = __uint_as_float(u1[j]);
-        }
+        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(u[j]);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s_empty[s]));
-      // swap partial logits with the peer CTA: st.async lands in the peer's buffer and
-      // counts its bytes on the peer's x_full
+      if (lane == 0) mbar_arrive(smem_u32(s_empty));
+      // stage our partial logits; the helper copies them into the peer's buffer
       if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(peer_free), (i - 1) & 1, &abort_s));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(stage_free), (i - 1) & 1, &abort_s));
         if (!ok) break;
       }
 #pragma unroll
-      for (int c = 0; c < C::BN / 4; ++c)
-        st_async_v4(x_remote + ((c ^ (hrow & 7)) << 4), x_full_remote, sv[4 * c], sv[4 * c + 1],
-                    sv[4 * c + 2], sv[4 * c + 3]);
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(sXout + x_row + ((c ^ (hrow & 7)) << 4)) =
+            make_float4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(staged));
       ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(x_full), i & 1, &abort_s));
       if (!ok) break;
-      if (hrow == 0 && i + 1 < n) mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);  // arm i+1
-      const uint64_t vmask = sMask[i];
-      float m_tile = -INFINITY;
+      if (warp == 4 && lane == 0 && i + 1 < n)
+        mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);   // arm tile i+1
+      const uint32_t vbits = static_cast<uint32_t>(sMask[i] >> (32 * half));
+      float m_half = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < C::BN / 4; ++c) {
-        const float4 o = *reinterpret_cast<const float4*>(
-            reinterpret_cast<const uint8_t*>(sX) + hrow * (C::BN * 4) + ((c ^ (hrow & 7)) << 4));
+      for (int c = 0; c < 8; ++c) {
+        const float4 o = *reinterpret_cast<const float4*>(sXin + x_row + ((c ^ (hrow & 7)) << 4));
         const float ov[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = 4 * c + e;
           // both CTAs add rank 0's partial to rank 1's: bit-identical logits in both
           const float full_s = rank == 0 ? sv[j] + ov[e] : ov[e] + sv[j];
-          sv[j] = ((vmask >> j) & 1ull) ? full_s * p.scale_log2 : -INFINITY;
-          m_tile = fmaxf(m_tile, sv[j]);
+          sv[j] = ((vbits >> j) & 1u) ? full_s * p.scale_log2 : -INFINITY;
+          m_half = fmaxf(m_half, sv[j]);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(smem_u32(peer_free), peer);
+      mbar_arrive(smem_u32(xin_read));
+      // row max over both halves (double-buffered by tile parity)
+      float* red = sRed + (i & 1) * 256;
+      red[half * 128 + hrow] = m_half;
+      mbar_arrive(smem_u32(mx_bar));
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(mx_bar), i & 1, &abort_s));
+      if (!ok) break;
+      const float m_tile = fmaxf(red[hrow], red[128 + hrow]);
       // P and O are free once PV(i-1) has completed
       if (i >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (i - 1) & 1, &abort_s));
@@ -398,7 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         m_ref = m_tile;
       }
       if (i >= 1 && __any_sync(0xffffffffu, need)) {
-        for (int c0 = 0; c0 < C::V_HALF; c0 += 32) {
+        for (int c0 = half * OC; c0 < (half + 1) * OC; c0 += 32) {
           uint32_t u[32];
           tmem_ld32(lane_addr + c0, u);
           tmem_wait_ld();
@@ -406,26 +463,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
           tmem_st32(lane_addr + c0, u);
         }
-        tmem_wait_st();
       }
+      uint32_t pk[16];
       float rowsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < C::BN / 8; ++c) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          // the denominator sums the fp32 probabilities; only the PV operand is rounded
-          const float p0 = exp2f(sv[8 * c + 2 * e] - m_ref);
-          const float p1 = exp2f(sv[8 * c + 2 * e + 1] - m_ref);
-          rowsum += p0 + p1;
-          const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<const uint32_t*>(&two);
-        }
-        *reinterpret_cast<uint4*>(sP + sw128_offset(hrow, c)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int e = 0; e < 16; ++e) {
+        // the denominator sums the fp32 probabilities; only the PV operand is rounded
+        const float p0 = exp2f(sv[2 * e] - m_ref);
+        const float p1 = exp2f(sv[2 * e + 1] - m_ref);
+        rowsum += p0 + p1;
+        const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&two);
       }
       l_sum += rowsum;
-      fence_proxy_async_smem();
+      tmem_st16(lane_addr + C::P_COL + half * 16, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
     }
@@ -433,20 +485,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       abort_s = 1;
       if (p.status) atomicOr(p.status, kStatusTimeout);
     }
-    // ---- epilogue
+    // ---- epilogue: l = l(keys 0-31) + l(keys 32-63), the same order in both halves
+    sLsum[half * 128 + hrow] = l_sum;
+    mbar_arrive(smem_u32(fin_bar));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(fin_bar), 0, &abort_s));
+    const float l_tot = ok ? sLsum[hrow] + sLsum[128 + hrow] : 0.f;
     const bool write = hrow < p.h;
     const int64_t orow = static_cast<int64_t>(row) * p.h + hrow;
     if (ok && n > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (n - 1) & 1, &abort_s));
     tc_fence_after();
-    const float inv_l = (n > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
-    const float lse_v = (n > 0 && l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f
-                                              : -INFINITY;
+    const float inv_l = (n > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+    const float lse_v =
+        (n > 0 && l_tot > 0.f) ? (m_ref + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
     float* po = nullptr;
     if (p.part_o != nullptr)
       po = p.part_o + ((static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow) * D_V +
            rank * C::V_HALF;
-    for (int c0 = 0; c0 < C::V_HALF; c0 += 32) {
+    for (int c0 = half * OC; c0 < (half + 1) * OC; c0 += 32) {
       float o[32];
       if (ok && n > 0) {
         uint32_t u[32];
@@ -477,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
       }
     }
-    if (write && rank == 0) {
+    if (write && rank == 0 && half == 0) {
       if (p.part_lse != nullptr)
         p.part_lse[(static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow] = lse_v;
       else
