@@ -430,6 +430,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--prefill-only", type=int, default=0, choices=[0, 1, 4, 5],
+                    help="profiling only: time just the prefill of this workload (4 or 5)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="profiling only: decode sequences (default: the workload's 64)")
     args = ap.parse_args()
@@ -448,6 +450,17 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
+        if args.prefill_only:
+            import sparse_attention_long_04_b200 as dsa
+            global PREFILL_CFG
+            PREFILL_CFG = args.prefill_only
+            dev = torch.device("cuda", local_rank)
+            torch.cuda.set_device(dev)
+            line = run_prefill(args, dsa, dev, torch.cuda.current_stream(), read_peaks(), rank,
+                               world)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            return
         line = run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -90,6 +90,17 @@ def _np(t, dtype=None) -> np.ndarray:
     return a.astype(dtype) if dtype is not None and a.dtype != dtype else a
 
 
+def _take(t, rows, dtype=None) -> np.ndarray:
+    """Rows ``rows`` of a torch tensor (gathered where it lives, then copied to the host) or of
+    a numpy array; bf16 comes back as uint16 bit patterns."""
+    rows = np.asarray(rows, dtype=np.int64)
+    if hasattr(t, "detach"):
+        import torch
+        idx = torch.as_tensor(rows, device=t.device)
+        return _np(t.index_select(0, idx), dtype)
+    return _np(np.asarray(t)[rows], dtype)
+
+
 def e4m3_to_f64(byte: int) -> float:
     return float(lib().dsa_oracle_e4m3_to_f64(int(byte)))
 
@@ -147,11 +158,6 @@ def indexer_rows(wl, rows: Sequence[int], fp32: bool = False) -> Dict[int, np.nd
     geo = Geometry.of(wl)
     d = wl.dims
     h_idx, d_idx = d["h_idx"], d["d_idx"]
-    q8 = _np(wl.q_idx, np.uint8)
-    qs = _np(wl.q_scale, np.float32)
-    w = _np(wl.w, np.float32)
-    k8 = _np(wl.k_idx, np.uint8)
-    ks = _np(wl.k_scale, np.float32)
     by_seq: Dict[int, List[int]] = {}
     for r in rows:
         b, _ = geo.row_seq_pos(r)
@@ -161,11 +167,11 @@ def indexer_rows(wl, rows: Sequence[int], fp32: bool = False) -> Dict[int, np.nd
         pos = np.array([geo.row_seq_pos(r)[1] for r in rs], dtype=np.int32)
         n_keys = int(pos.max()) + 1
         phys = geo.phys(b, np.arange(n_keys))
-        kseq = np.ascontiguousarray(k8[phys])
-        kss = np.ascontiguousarray(ks[phys])
-        qq = np.ascontiguousarray(q8[rs])
-        qsc = np.ascontiguousarray(qs[rs])
-        ww = np.ascontiguousarray(w[rs])
+        kseq = _take(wl.k_idx, phys, np.uint8)
+        kss = _take(wl.k_scale, phys, np.float32)
+        qq = _take(wl.q_idx, rs, np.uint8)
+        qsc = _take(wl.q_scale, rs, np.float32)
+        ww = _take(wl.w, rs, np.float32)
         res = np.full((len(rs), n_keys), np.nan, dtype=np.float64)
         lib().dsa_oracle_indexer_seq(len(rs), h_idx, d_idx, _ptr(qq), _ptr(qsc), _ptr(ww),
                                      _ptr(pos), n_keys, _ptr(kseq), _ptr(kss), n_keys,
@@ -203,9 +209,13 @@ def sparse_mla_rows(wl, rows: Sequence[int], idx: np.ndarray):
         b, _ = geo.row_seq_pos(r)
         sel = idx[i] >= 0
         phys[i, sel] = geo.phys(b, idx[i, sel])
-    q = _np(wl.q)
-    qq = np.ascontiguousarray(q[list(rows)])
-    kv = _np(wl.kv)
+    qq = _take(wl.q, list(rows))
+    # only the selected latent rows travel: remap physical rows to a compact host array
+    used = np.unique(phys[phys >= 0])
+    kv = _take(wl.kv, used) if len(used) else np.zeros((1, d_qk), np.uint16)
+    compact = np.full(phys.shape, -1, dtype=np.int64)
+    compact[phys >= 0] = np.searchsorted(used, phys[phys >= 0])
+    phys = compact
     out = np.empty((len(rows), h, d_v), dtype=np.float64)
     lse = np.empty((len(rows), h), dtype=np.float64)
     lib().dsa_oracle_sparse_mla(len(rows), h, d_qk, d_v, float(wl.softmax_scale), _ptr(qq),

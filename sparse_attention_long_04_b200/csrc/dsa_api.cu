@@ -291,7 +291,25 @@ dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* 
   prm.seq_lens = s.seq_lens;
   prm.max_seqlen = s.max_seqlen;
   prm.status = status;
-  dsa_topk_kernel<<<row_count, kTopkThreads, 0, st>>>(prm);
+  // CTAs per row: enough that a row's slices fit shared memory (up to 8, the portable limit)
+  const int64_t longest = std::min<int64_t>(max_keys(&s, row_begin, row_count), ld);
+  int csize = 1;
+  while (csize < 8 && int64_t(csize) * kTopkSlice < longest) csize *= 2;
+  prm.csize = csize;
+  if (prepare_kernel(dsa_topk_kernel, kTopkSmem) != DSA_OK) return DSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(int64_t(row_count) * csize));
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = kTopkSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dsa_topk_kernel, prm) != cudaSuccess) return DSA_ERR_CUDA;
   return launch_status();
 }
 
@@ -441,7 +459,8 @@ dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
   if (!indexer_shape_ok(*dims, seqs->mode)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
   if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(scores) || ld_scores % 4 != 0)
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(scores) ||
+      ld_scores % 4 != 0)
     return DSA_ERR_MISALIGNED;
   if (ld_scores < max_keys(seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
   return indexer_dispatch(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
@@ -508,7 +527,8 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
   if (!indexer_shape_ok(d, s.mode) || !mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !q || !kv || !out || !lse)
     return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(kv) ||
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(q) ||
+      !aligned16(kv) ||
       !aligned16(out) || !aligned16(lse) || !aligned16(idx_out) || !aligned16(workspace))
     return DSA_ERR_MISALIGNED;
   DeviceInfo info;

@@ -13,10 +13,12 @@
 // accumulator in Tensor Memory (TMEM lane = key).  Each epilogue thread then owns one key and
 // reduces its row's heads with no cross-thread traffic: 2 ALU ops (max, fma) per head.
 //
-// Roles: warp 0 issues TMA (Q once, then two 64-row key boxes per tile), warp 1 issues the
-// tcgen05.mma, warp 2 owns the TMEM allocation, warp 3 computes c[t,j], warps 4.. run the
-// epilogue.  Key stages are a ring of STAGES buffers; accumulators are double-buffered in TMEM
-// so the epilogue of tile i overlaps the MMA of tile i+1 and the loads of later tiles.
+// Roles: warp 0 issues TMA (Q once, then per tile two 64-row key boxes plus a bulk copy of each
+// box's k_scale), warp 1 issues the tcgen05.mma, warp 2 owns the TMEM allocation, warp 3
+// computes c[t,j], warps 4.. run the epilogue.  Key stages are a ring of STAGES buffers; the
+// accumulators are a ring of ACC buffers in TMEM so the epilogue of tile i overlaps the MMA of
+// later tiles.  Decode (one query row, N = 64) runs two epilogue warpgroups on alternate tiles;
+// prefill (N = 256) splits each tile's columns over two warpgroups.
 #pragma once
 #include "sm100.cuh"
 
@@ -48,22 +50,28 @@ template <int H_I, int D_I, int QPG>
 struct IndexerCfg {
   static constexpr int N = H_I * QPG;                 // MMA N: (row, head) columns
   static constexpr int STAGES = QPG == 1 ? 6 : 8;
-  static constexpr int EPI_WARPS = QPG == 1 ? 4 : 8;
+  static constexpr int ACC = QPG == 1 ? 4 : 2;        // TMEM accumulator ring
+  static constexpr int EPI_WARPS = 8;
+  static constexpr bool TILE_SPLIT = QPG == 1;        // warpgroups take alternate tiles
+  static constexpr int EPI_PER_TILE = TILE_SPLIT ? 4 : EPI_WARPS;   // warps reading one tile
   static constexpr int THREADS = (4 + EPI_WARPS) * 32;
   static constexpr int TILE_BYTES = 128 * D_I;        // 128 keys
   static constexpr int Q_BYTES = N * D_I;
   static constexpr int KSTEPS = D_I / 32;             // one e4m3 MMA consumes K = 32
   static constexpr uint32_t LAYOUT = D_I == 128 ? kSwizzle128B : kSwizzle32B;
   static constexpr uint32_t SBO = 8 * D_I;            // next 8-row group
-  static constexpr int TMEM_COLS = 2 * N;             // double-buffered accumulator
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * TILE_BYTES + N * 4 + 256;
+  static constexpr int TMEM_COLS = ACC * N;
+  static constexpr int SCALE_FLOATS = 2 * 80;         // per stage: 2 boxes x (64 + slack)
+  static constexpr int SMEM_BYTES =
+      1024 + Q_BYTES + STAGES * TILE_BYTES + STAGES * SCALE_FLOATS * 4 + STAGES * 2 * 16 +
+      N * 4 + 512;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   static_assert(Q_BYTES % 1024 == 0 && TILE_BYTES % 1024 == 0, "1024-byte aligned tiles");
 };
 
 template <int H_I, int D_I, int QPG>
-__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
+__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ? 2 : 1)
     dsa_indexer_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap qmap, const IndexerParams p) {
   using C = IndexerCfg<H_I, D_I, QPG>;
@@ -73,13 +81,18 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::Q_BYTES;
-  float* sC = reinterpret_cast<float*>(sK + C::STAGES * C::TILE_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + N);
-  uint64_t* full = bars;                      // [STAGES] key tile landed
-  uint64_t* empty = bars + C::STAGES;         // [STAGES] key tile consumed by the MMA
-  uint64_t* tfull = empty + C::STAGES;        // [2] accumulator ready
-  uint64_t* tempty = tfull + 2;               // [2] accumulator drained by the epilogue
-  uint64_t* qbar = tempty + 2;                // Q group landed
+  float* sScale = reinterpret_cast<float*>(sK + C::STAGES * C::TILE_BYTES);  // [STAGES][2][80]
+  int64_t* sA0 = reinterpret_cast<int64_t*>(sScale + C::STAGES * C::SCALE_FLOATS);  // [STAGES][2]
+  int32_t* sOff = reinterpret_cast<int32_t*>(sA0 + C::STAGES * 2);   // [STAGES][2]
+  int32_t* sCnt = sOff + C::STAGES * 2;                               // [STAGES][2]
+  float* sC = reinterpret_cast<float*>(sCnt + C::STAGES * 2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(sC + N) + 7) & ~uintptr_t(7));
+  uint64_t* full = bars;                      // [STAGES] key tile (and its scales) landed
+  uint64_t* empty = bars + C::STAGES;         // [STAGES] tile consumed: MMA + epilogue (scales)
+  uint64_t* tfull = empty + C::STAGES;        // [ACC] accumulator ready
+  uint64_t* tempty = tfull + C::ACC;          // [ACC] accumulator drained by the epilogue
+  uint64_t* qbar = tempty + C::ACC;           // Q group landed
   uint64_t* done = qbar + 1;                  // every MMA of this CTA completed
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
@@ -117,11 +130,11 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&empty[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1 + C::EPI_PER_TILE);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::ACC; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), C::EPI_WARPS);
+      mbar_init(smem_u32(&tempty[i]), C::TILE_SPLIT ? 4 : C::EPI_WARPS);
     }
     mbar_init(smem_u32(qbar), 1);
     mbar_init(smem_u32(done), 1);
@@ -181,12 +194,27 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
             y[hlf] = seq_base + blk * 64;
           }
         }
-        const uint32_t bytes = (ok[0] ? 64 * D_I : 0) + (ok[1] ? 64 * D_I : 0);
+        // each box's 64 scales: a 16-byte-aligned superset of the rows, inside the cache
+        int64_t a0[2];
+        uint32_t sb[2];
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          a0[hlf] = y[hlf] & ~int64_t(3);
+          const int64_t avail = p.num_kv_rows - a0[hlf];
+          sb[hlf] = ok[hlf] ? static_cast<uint32_t>((avail < 68 ? avail : int64_t(68)) / 4 * 16) : 0u;
+          sOff[s * 2 + hlf] = static_cast<int32_t>(y[hlf] - a0[hlf]);
+          sCnt[s * 2 + hlf] = static_cast<int32_t>(sb[hlf] / 4);
+          sA0[s * 2 + hlf] = a0[hlf];
+        }
+        const uint32_t bytes = (ok[0] ? 64 * D_I : 0) + (ok[1] ? 64 * D_I : 0) + sb[0] + sb[1];
         mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
-        for (int hlf = 0; hlf < 2; ++hlf)
+        for (int hlf = 0; hlf < 2; ++hlf) {
           if (ok[hlf])
             tma_load_2d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
                         smem_u32(&full[s]), 0, static_cast<int32_t>(y[hlf]));
+          if (sb[hlf] > 0)
+            bulk_load_g2s(smem_u32(sScale + s * C::SCALE_FLOATS + hlf * 80),
+                          p.k_scale + a0[hlf], sb[hlf], smem_u32(&full[s]));
+        }
         ++issued;
       }
       // drain: never leave a copy in flight into shared memory of an exiting CTA
@@ -201,9 +229,10 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
       bool ok = mbar_wait(smem_u32(qbar), 0, &abort_s);
       for (int it = 0; ok && it < n_tiles; ++it) {
         const int s = it % C::STAGES;
-        const int a = it & 1;
+        const int a = it % C::ACC;
         ok = mbar_wait(smem_u32(&full[s]), (it / C::STAGES) & 1, &abort_s);
-        if (ok && it >= 2) ok = mbar_wait(smem_u32(&tempty[a]), ((it >> 1) - 1) & 1, &abort_s);
+        if (ok && it >= C::ACC)
+          ok = mbar_wait(smem_u32(&tempty[a]), ((it / C::ACC) - 1) & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
         const uint32_t kaddr = smem_u32(sK + s * C::TILE_BYTES);
@@ -224,33 +253,43 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    constexpr int PARTS = C::EPI_WARPS / 4;
+    constexpr int PARTS = C::TILE_SPLIT ? 1 : C::EPI_WARPS / 4;
     constexpr int COLS = N / PARTS;          // columns this warp reduces
     const int quad = warp & 3;               // TMEM lanes 32*quad .. 32*quad+31
-    const int part = (warp - 4) / 4;
+    const int grp = (warp - 4) / 4;          // warpgroup
+    const int part = C::TILE_SPLIT ? 0 : grp;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    for (int it = 0; it < n_tiles; ++it) {
-      const int a = it & 1;
-      if (!mbar_wait(smem_u32(&tfull[a]), (it >> 1) & 1, &abort_s)) {
+    for (int it = C::TILE_SPLIT ? grp : 0; it < n_tiles; it += C::TILE_SPLIT ? 2 : 1) {
+      const int a = it % C::ACC;
+      const int s = it % C::STAGES;
+      if (!mbar_wait(smem_u32(&tfull[a]), (it / C::ACC) & 1, &abort_s)) {
         abort_s = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
         break;
       }
       tc_fence_after();
-      const int key = (t_begin + it) * 128 + quad * 32 + lane;
+      // the tile's scales came with its keys: observe that phase of full[s] (the stage is not
+      // refilled before this warp releases it below)
+      if (!mbar_wait(smem_u32(&full[s]), (it / C::STAGES) & 1, &abort_s)) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+        break;
+      }
+      const int kin = quad * 32 + lane;        // key within the tile
+      const int key = (t_begin + it) * 128 + kin;
+      const int hb = kin >> 6;
+      const int j = sOff[s * 2 + hb] + (kin & 63);
       float ks = 0.f;
       if (key < n_keys) {
-        int64_t phys;
-        if (!p.decode) {
-          phys = static_cast<int64_t>(p.key0) + key;
-        } else if (p.block_table != nullptr) {
-          int64_t id = p.block_table[static_cast<int64_t>(b) * p.max_blocks + key / 64];
-          phys = (id < 0 || (id + 1) * 64 > p.num_kv_rows) ? -1 : id * 64 + key % 64;
-        } else {
-          phys = seq_base + key;
+        if (j < sCnt[s * 2 + hb]) {
+          ks = sScale[s * C::SCALE_FLOATS + hb * 80 + j];
+        } else {                               // the last rows of the cache: not bulk-copied
+          const int64_t row = sA0[s * 2 + hb] + j;
+          ks = row < p.num_kv_rows ? __ldg(p.k_scale + row) : 0.f;
         }
-        ks = phys >= 0 && phys < p.num_kv_rows ? __ldg(p.k_scale + phys) : 0.f;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
       float acc = 0.f;
 #pragma unroll 1
       for (int c0 = 0; c0 < COLS; c0 += 32) {
@@ -278,14 +317,14 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, 1)
         } else {
 #pragma unroll
           for (int q = 0; q < 32 / H_I; ++q) {
-            float s = 0.f;
+            float sacc = 0.f;
 #pragma unroll
             for (int j = 0; j < H_I; ++j)
-              s = fmaf(sC[col + q * H_I + j], fmaxf(__uint_as_float(r[q * H_I + j]), 0.f), s);
+              sacc = fmaf(sC[col + q * H_I + j], fmaxf(__uint_as_float(r[q * H_I + j]), 0.f), sacc);
             const int rr = col / H_I + q;
             if (rr < rows_in_group && key <= pos_first + rr)
               p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] =
-                  ks * s;
+                  ks * sacc;
           }
         }
       }

@@ -207,6 +207,16 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remot
       : "memory");
 }
 
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global memory into
+// this CTA's shared memory; completion is counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to the shared memory of a
 // CTA of the cluster; on arrival it performs complete_tx(bytes) on `remote_bar`.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src,

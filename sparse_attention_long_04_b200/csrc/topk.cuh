@@ -4,14 +4,18 @@
 // DeepSeek Sparse Attention (DSA)", "Training signal"; "Top-k Token Selection", maplevalley
 // page, section 1.)
 //
-// Radix select, no sort: each score maps to a 32-bit key whose unsigned order is the float
-// order (-0 folded onto +0).  Three histogram passes over the row (digits of 11, 11 and 10
-// bits, most significant first, each restricted to the keys that match the digits fixed so
-// far) pin the exact k-th key tau and how many keys equal to tau are still needed.  A final
-// pass walks the row in index order with block-wide scans: every key > tau is taken, and the
-// first `need` keys == tau (the smallest indices) are taken.  Output: the selected indices in
-// increasing order, then -1 padding.  One CTA of 1024 threads per row; rows are read with
-// 16-byte vector loads (the score slab stays in L2 between the indexer and this kernel).
+// Radix select, no sort.  Each score maps to a 32-bit key whose unsigned order is the float
+// order (-0 folded onto +0).  A row is split over a cluster of C CTAs (C = 1..8); CTA c reads
+// its slice of the row from global memory once and keeps the keys in shared memory, building
+// the histogram of the first digit (the top 11 bits) while it loads.  Three digits (11, 11 and
+// 10 bits, most significant first) are resolved in turn: each CTA histograms the keys that
+// match the digits fixed so far (warp-aggregated shared atomics), the C histograms are summed
+// through distributed shared memory, and every CTA picks the same bin.  After the first digit
+// the keys of the chosen bin are compacted into a short candidate list, so the later digits
+// scan only those.  After the last digit the exact k-th key tau and the number of keys == tau
+// still needed are known.  The output pass takes every key > tau and the first `need` keys == tau in index
+// order (the smallest indices): per-warp counts give each warp's output offset (an exclusive
+// scan over the cluster in index order), and the indices come out in increasing order.
 #pragma once
 #include "sm100.cuh"
 
@@ -29,9 +33,15 @@ struct TopkParams {
   const int32_t* seq_lens;
   int32_t max_seqlen;
   int32_t* status;
+  int32_t csize;           // CTAs per row (the cluster size)
 };
 
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkSlice = 16384;          // keys a CTA keeps in shared memory
+constexpr int kTopkBins = 2048;
+constexpr int kTopkCand = 4096;           // candidates kept after the first digit
+constexpr int kTopkSmem = kTopkSlice * 4 + kTopkCand * 4 + 2 * kTopkBins * 4 + 1024;
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -39,54 +49,103 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block scan of one value per thread; returns the prefix, *total gets the sum.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tmp,
-                                                    uint32_t* total) {
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_u4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Exclusive scan over the CTA's threads (one value each); *total receives the sum.
+__device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tmp[warp] = x;
+  if (lane == 31) tmp[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    uint32_t w = warp_tmp[lane];
+    const uint32_t w = lane < kTopkWarps ? tmp[lane] : 0u;
     uint32_t t = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
       if (lane >= o) t += y;
     }
-    warp_tmp[lane] = t - w;                       // exclusive prefix of warp sums
-    if (lane == 31) warp_tmp[32] = t;
+    if (lane < kTopkWarps) tmp[lane] = t - w;
+    if (lane == 31) tmp[32] = t;
   }
   __syncthreads();
-  const uint32_t res = warp_tmp[warp] + x - v;
-  *total = warp_tmp[32];
-  __syncthreads();                                // warp_tmp reusable afterwards
+  const uint32_t res = tmp[warp] + x - v;
+  *total = tmp[32];
+  __syncthreads();
   return res;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const TopkParams p) {
-  __shared__ uint32_t hist[2048];
-  __shared__ uint32_t warp_tmp[33];
-  __shared__ uint32_t s_bin, s_above;
-  const int tid = threadIdx.x;
-  const int r = blockIdx.x;
+__device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Sums the cluster's histograms (nb bins) into every CTA's hsum, which the caller zeroed before
+// the histogram was built: every CTA adds its non-zero bins into every CTA's hsum.
+__device__ __forceinline__ void cluster_hist_sum(uint32_t* hist, uint32_t* hsum, uint32_t nb,
+                                                 int C) {
+  if (C > 1) {
+    cluster_sync();   // every hist complete, every hsum zeroed
+    for (uint32_t i = threadIdx.x; i < nb; i += kTopkThreads) {
+      const uint32_t v = hist[i];
+      if (v != 0)
+        for (int c = 0; c < C; ++c) red_cluster_add(map_to_rank(smem_u32(hsum + i), c), v);
+    }
+    cluster_sync();
+  } else {
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < nb; i += kTopkThreads) hsum[i] = hist[i];
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t topk_smem[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(topk_smem);           // [kTopkSlice]
+  uint32_t* cand = keys + kTopkSlice;                                // [kTopkCand] keys
+  uint32_t* hist = cand + kTopkCand;                                 // [kTopkBins] this CTA
+  uint32_t* hsum = hist + kTopkBins;                                 // [kTopkBins] cluster sum
+  uint32_t* tmp = hsum + kTopkBins;                                  // [40] scan scratch
+  uint32_t* wgt = tmp + 40;                                          // [16] per-warp > tau
+  uint32_t* weq = wgt + 16;                                          // [16] per-warp == tau
+  uint32_t* cnt = weq + 16;                                          // [16] per-CTA (gt, eq)
+  __shared__ uint32_t s_bin, s_above, s_ncand;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = p.csize;
+  const int crank = static_cast<int>(blockIdx.x) % C;
+  const int r = blockIdx.x / C;
   const int row = p.row_begin + r;
   int n;
   if (p.decode) {
     n = p.seq_lens[row];
     if (n > p.max_seqlen || n > p.ld) {     // caller error: clamp to the slab and report
-      if (tid == 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+      if (tid == 0 && crank == 0 && p.status) atomicOr(p.status, kStatusBadIndex);
       n = static_cast<int>(min(static_cast<int64_t>(min(n, p.max_seqlen)), p.ld));
     }
   } else {
     int lo = 0, hi = p.batch;                     // largest b with cu[b] <= row
     while (hi - lo > 1) {
-      int mid = (lo + hi) >> 1;
+      const int mid = (lo + hi) >> 1;
       if (p.cu_seqlens[mid] <= row) lo = mid; else hi = mid;
     }
     n = row - p.cu_seqlens[lo] + 1;
@@ -94,50 +153,109 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const TopkPar
   const float* srow = p.scores + static_cast<int64_t>(r) * p.ld;
   int32_t* out = p.idx + static_cast<int64_t>(r) * p.topk;
   const int K = p.topk;
-  if (n <= K) {
-    for (int j = tid; j < K; j += kTopkThreads) out[j] = j < n ? j : -1;
+  if (n <= K) {                                    // uniform over the cluster: no barrier used
+    for (int j = crank * kTopkThreads + tid; j < K; j += C * kTopkThreads)
+      out[j] = j < n ? j : -1;
     return;
   }
-  const int n4 = (n + 3) / 4;
-  const float4* srow4 = reinterpret_cast<const float4*>(srow);
+  // this CTA's slice [s0, s1); a multiple of 4 long so every slice starts 16-byte aligned
+  const int per = ((n + C - 1) / C + 3) / 4 * 4;
+  const int s0 = min(n, crank * per);
+  const int s1 = min(n, s0 + per);
+  const int m = s1 - s0;
+  const bool cached = m <= kTopkSlice;
+  auto key_at = [&](int i) -> uint32_t {
+    return cached ? keys[i] : score_key(srow[s0 + i]);
+  };
+  // 4 consecutive keys (i multiple of 4; lanes past m read as 0 and are masked by callers)
+  auto key4_at = [&](int i) -> uint4 {
+    if (cached) return *reinterpret_cast<const uint4*>(keys + i);
+    uint4 k = make_uint4(0, 0, 0, 0);
+    if (i + 0 < m) k.x = score_key(srow[s0 + i + 0]);
+    if (i + 1 < m) k.y = score_key(srow[s0 + i + 1]);
+    if (i + 2 < m) k.z = score_key(srow[s0 + i + 2]);
+    if (i + 3 < m) k.w = score_key(srow[s0 + i + 3]);
+    return k;
+  };
+
+  // ---- digit 1 (top 11 bits): load + histogram in one pass
+  for (int i = tid; i < kTopkBins; i += kTopkThreads) {
+    hist[i] = 0;
+    hsum[i] = 0;
+  }
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
+  // all of a thread's loads are issued before any is used (one latency, not one per round)
+  if (cached) {
+    constexpr int kVec = kTopkSlice / 4 / kTopkThreads;   // float4 per thread (8)
+    float4 v[kVec];
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int i4 = (u * kTopkThreads + tid) * 4;
+      v[u] = i4 < m ? *reinterpret_cast<const float4*>(srow + s0 + i4)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int i4 = (u * kTopkThreads + tid) * 4;
+      if (i4 < m) {
+        const uint4 k = make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z),
+                                   score_key(v[u].w));
+        *reinterpret_cast<uint4*>(keys + i4) = k;
+        atomicAdd(&hist[k.x >> 21], 1u);
+        if (i4 + 1 < m) atomicAdd(&hist[k.y >> 21], 1u);
+        if (i4 + 2 < m) atomicAdd(&hist[k.z >> 21], 1u);
+        if (i4 + 3 < m) atomicAdd(&hist[k.w >> 21], 1u);
+      }
+    }
+  } else {
+    for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&hist[key_at(i) >> 21], 1u);
+  }
 
   uint32_t prefix = 0, mask = 0, need = K;
+  bool use_cand = false;
+  uint32_t ncand = 0;
   constexpr int kShift[3] = {21, 10, 0};
   constexpr int kBits[3] = {11, 11, 10};
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = kShift[pass];
     const uint32_t nb = 1u << kBits[pass];
-    for (uint32_t i = tid; i < nb; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i4 = tid; i4 < n4; i4 += kTopkThreads) {
-      const float4 v = srow4[i4];
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (i4 * 4 + e < n) {
-          const uint32_t key = score_key(vv[e]);
-          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    if (pass > 0) {
+      for (uint32_t i = tid; i < nb; i += kTopkThreads) {
+        hist[i] = 0;
+        hsum[i] = 0;
+      }
+      __syncthreads();
+      if (use_cand) {
+        for (uint32_t i = tid; i < ncand; i += kTopkThreads) {
+          const uint32_t k = cand[i];
+          if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
+        }
+      } else {
+        for (int i = tid; i < m; i += kTopkThreads) {
+          const uint32_t k = key_at(i);
+          if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
         }
       }
     }
-    __syncthreads();
-    // Descending cumulative count: thread t owns bins in descending order.
-    const uint32_t per = nb / kTopkThreads;       // 2 or 1 bins per thread
+    cluster_hist_sum(hist, hsum, nb, C);
+    // the bin holding the need-th largest key: descending cumulative counts
+    const uint32_t bpt = nb / kTopkThreads;         // 4 or 2 bins per thread
     uint32_t mine = 0;
-    for (uint32_t j = 0; j < per; ++j) mine += hist[nb - 1 - (tid * per + j)];
+    for (uint32_t j = 0; j < bpt; ++j) mine += hsum[nb - 1 - (tid * bpt + j)];
     uint32_t tot;
-    const uint32_t before = block_excl_scan(mine, warp_tmp, &tot);
+    const uint32_t before = cta_excl_scan(mine, tmp, &tot);
     if (before < need && before + mine >= need) {
       uint32_t c = before;
-      for (uint32_t j = 0; j < per; ++j) {
-        const uint32_t bin = nb - 1 - (tid * per + j);
-        if (c + hist[bin] >= need) {
+      for (uint32_t j = 0; j < bpt; ++j) {
+        const uint32_t bin = nb - 1 - (tid * bpt + j);
+        if (c + hsum[bin] >= need) {
           s_bin = bin;
           s_above = c;
           break;
         }
-        c += hist[bin];
+        c += hsum[bin];
       }
     }
     __syncthreads();
@@ -145,53 +263,151 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const TopkPar
     need -= s_above;
     prefix |= bin << shift;
     mask |= (nb - 1) << shift;
-    const bool exact = hist[bin] == need;         // every key of this bucket is taken
+    const bool exact = hsum[bin] == need;           // every key of this bucket is taken
+    const uint32_t local_in_bin = hist[bin];        // this CTA's keys in the chosen bin
     __syncthreads();
     if (exact) break;
+    if (pass == 0) {
+      // compact this CTA's keys of the chosen bin (order is irrelevant for histograms)
+      use_cand = local_in_bin <= kTopkCand;
+      if (use_cand) {
+        for (int base = warp * 128; base < m; base += kTopkThreads * 4) {   // warp-uniform
+          const int i4 = base + lane * 4;
+          const uint4 k = i4 < m ? key4_at(i4) : make_uint4(0, 0, 0, 0);
+          const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
+          uint32_t hit = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (i4 + e < m && (kk[e] & mask) == prefix) hit |= 1u << e;
+          const uint32_t nh = __popc(hit);
+          uint32_t inc = nh;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+          }
+          uint32_t wbase = 0;
+          if (lane == 31 && inc > 0) wbase = atomicAdd(&s_ncand, inc);
+          wbase = __shfl_sync(0xffffffffu, wbase, 31);
+          uint32_t slot = wbase + inc - nh;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if ((hit >> e) & 1u) cand[slot++] = kk[e];
+        }
+        __syncthreads();
+        ncand = s_ncand;
+      }
+    }
   }
 
-  // Ordered pass: keys > prefix (under mask) are taken; keys == prefix are taken while the
-  // running count of such keys (in index order) is below `need`.
-  uint32_t eq_seen = 0, out_pos = 0;
-  const int chunk = kTopkThreads * 4;
-#pragma unroll 1
-  for (int base = 0; base < n; base += chunk) {
-    const int i0 = base + tid * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i0 < n) v = srow4[i0 / 4];
-    const float vv[4] = {v.x, v.y, v.z, v.w};
-    uint32_t gt = 0, eq = 0;
+  // ---- output: keys > tau, then the first `need` keys == tau in index order
+  const int wn = ((m + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;   // per warp, x128
+  const int w0 = min(m, warp * wn), w1 = min(m, w0 + wn);
+  uint32_t gt = 0, eq = 0;
+  for (int i4 = w0 + lane * 4; i4 < w1; i4 += 128) {
+    const uint4 k = key4_at(i4);
+    const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (i0 + e < n) {
-        const uint32_t km = score_key(vv[e]) & mask;
-        gt |= (km > prefix ? 1u : 0u) << e;
-        eq |= (km == prefix ? 1u : 0u) << e;
+      if (i4 + e < w1) {
+        const uint32_t km = kk[e] & mask;
+        gt += km > prefix;
+        eq += km == prefix;
       }
     }
-    uint32_t eq_total;
-    const uint32_t eq_before = eq_seen + block_excl_scan(__popc(eq), warp_tmp, &eq_total);
-    uint32_t take = gt;
-    uint32_t e_rank = eq_before;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+  if (lane == 0) {
+    wgt[warp] = gt;
+    weq[warp] = eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t g = 0, e = 0;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      g += wgt[w];
+      e += weq[w];
+    }
+    if (C > 1) {
+      for (int c = 0; c < C; ++c) {
+        st_cluster_u32(map_to_rank(smem_u32(cnt + crank), c), g);
+        st_cluster_u32(map_to_rank(smem_u32(cnt + 8 + crank), c), e);
+      }
+    } else {
+      cnt[0] = g;
+      cnt[8] = e;
+    }
+  }
+  if (C > 1) cluster_sync(); else __syncthreads();
+  // every key == tau is taken when the cluster holds exactly `need` of them (the usual case)
+  uint32_t eq_all = 0;
+  for (int c = 0; c < C; ++c) eq_all += cnt[8 + c];
+  const bool all_eq = eq_all == need;
+  // offsets: keys taken by the CTAs, then the warps, before this one (index order)
+  uint32_t w_out = 0, w_eq = 0;
+  for (int c = 0; c < crank; ++c) {
+    w_out += cnt[c] + (need > w_eq ? min(need - w_eq, cnt[8 + c]) : 0u);
+    w_eq += cnt[8 + c];
+  }
+  for (int w = 0; w < warp; ++w) {
+    w_out += wgt[w] + (need > w_eq ? min(need - w_eq, weq[w]) : 0u);
+    w_eq += weq[w];
+  }
+  // 128 keys per round: lane j holds keys 4j..4j+3 of the round (index order = lane order)
+  for (int b0 = w0; b0 < w1; b0 += 128) {
+    const int i4 = b0 + lane * 4;
+    const uint4 k = key4_at(i4);
+    const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
+    uint32_t gtm = 0, eqm = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if ((eq >> e) & 1u) {
-        if (e_rank < need) take |= 1u << e;
-        ++e_rank;
+      if (i4 + e < w1) {
+        const uint32_t km = kk[e] & mask;
+        gtm |= (km > prefix ? 1u : 0u) << e;
+        eqm |= (km == prefix ? 1u : 0u) << e;
       }
     }
-    uint32_t take_total;
-    uint32_t pos = out_pos + block_excl_scan(__popc(take), warp_tmp, &take_total);
+    uint32_t take = gtm | eqm;
+    uint32_t inc = 0;
+    if (!all_eq) {
+      // eq rank of this lane's first key: exclusive scan of eq counts over lanes
+      const uint32_t neq = __popc(eqm);
+      inc = neq;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      uint32_t eq_rank = w_eq + inc - neq;
+      take = gtm;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((eqm >> e) & 1u) {
+          if (eq_rank < need) take |= 1u << e;
+          ++eq_rank;
+        }
+    }
+    const uint32_t ntake = __popc(take);
+    uint32_t tinc = ntake;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, tinc, o);
+      if (lane >= o) tinc += y;
+    }
+    uint32_t pos = w_out + tinc - ntake;
 #pragma unroll
     for (int e = 0; e < 4; ++e)
       if ((take >> e) & 1u) {
-        if (pos < static_cast<uint32_t>(K)) out[pos] = i0 + e;
+        if (pos < static_cast<uint32_t>(K)) out[pos] = s0 + i4 + e;
         ++pos;
       }
-    eq_seen += eq_total;
-    out_pos += take_total;
+    w_out += __shfl_sync(0xffffffffu, tinc, 31);
+    if (!all_eq) w_eq += __shfl_sync(0xffffffffu, inc, 31);
   }
-  for (int j = out_pos + tid; j < K; j += kTopkThreads) out[j] = -1;
 }
 
 }  // namespace dsa
