@@ -22,7 +22,8 @@
 //   work is duplicated.  Rescaling of O is lazy (only when a tile's max beats the running
 //   reference by more than 2^8, so P <= 256).
 // TMEM columns: O [0, V_HALF) | S [V_HALF, +64) | P [+64, +32) | Q (kb_count x 32 columns).
-// Warp roles per CTA (512 threads): warp 0 issues QK, warp 2 issues PV, warp 1 owns TMEM,
+// Warp roles per CTA (512 threads): warp 0 issues QK, warp 2 issues PV, warp 1 owns TMEM and
+// forwards read signals to the peer, warp 3 copies our partial logits to the peer,
 // warps 4-11 run the softmax (thread = head = TMEM lane; warps 4-7 take keys 0-31 of a tile,
 // warps 8-11 keys 32-63) and the epilogue, warps 12-15 resolve indices and gather rows with
 // 16-byte cp.async (3 stages).  Grid: x = 2 * row (the cluster pair), y = split-KV slice.
@@ -62,7 +63,7 @@ struct MlaCfg {
   static constexpr int KBC = KB_ALL - VKB;            // k-blocks held by rank 1 (>= rank 0)
   static constexpr int BN = 64;                       // keys per tile
   static constexpr int STAGES = 3;
-  static constexpr int MAX_TOPK = 2048;
+  static constexpr int MAX_TILES = 32;                // topk <= 2048
   static constexpr int THREADS = 512;
   static constexpr int KV_STAGE_BYTES = KBC * BN * 128;
   static constexpr int X_BYTES = 128 * BN * 4;        // partial logits of one tile
@@ -71,9 +72,9 @@ struct MlaCfg {
   static constexpr int Q_COL = P_COL + BN / 2;
   static constexpr int TMEM_NEED = Q_COL + KBC * 32;
   static constexpr int TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * KV_STAGE_BYTES + 2 * X_BYTES +
-                                    MAX_TOPK * 4 + 32 * 4 + 32 * 8 + 2 * 2 * 128 * 4 +
-                                    2 * 128 * 4 + 256;   // barriers: 19 x 8 bytes
+  static constexpr int SMEM_BYTES = 1024 + STAGES * KV_STAGE_BYTES + 3 * X_BYTES +
+                                    STAGES * 8 + MAX_TILES * 12 +
+                                    2 * 2 * 128 * 4 + 2 * 128 * 4 + 512;
   static_assert(KBC >= VKB, "rank 1 holds at least as many k-blocks as rank 0");
   static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
   static_assert(TMEM_NEED <= 512, "TMEM columns");
@@ -89,13 +90,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sKV = smem;                                          // [STAGES] gathered tiles
-  uint8_t* sXin = sKV + C::STAGES * C::KV_STAGE_BYTES;          // peer's partial logits
-  uint8_t* sXout = sXin + C::X_BYTES;                           // ours, staged for the copy
-  int32_t* sPhys = reinterpret_cast<int32_t*>(sXout + C::X_BYTES);
-  int32_t* sTiles = sPhys + C::MAX_TOPK;                        // [32] active tiles (split)
-  uint64_t* sMask = reinterpret_cast<uint64_t*>(sTiles + 32);   // [32] valid keys per tile
-  float* sRed = reinterpret_cast<float*>(sMask + 32);           // [2 tiles][2 halves][128]
-  float* sLsum = sRed + 2 * 2 * 128;                            // [2 halves][128]
+  uint8_t* sXin = sKV + C::STAGES * C::KV_STAGE_BYTES;          // [2] peer's partial logits
+  uint8_t* sXout = sXin + 2 * C::X_BYTES;                       // ours, staged for the copy
+  // [STAGES][4]: per producer warp, its 16 rows whose cache location was invalid
+  uint16_t* sBad = reinterpret_cast<uint16_t*>(sXout + C::X_BYTES);
+  uint64_t* sMask = reinterpret_cast<uint64_t*>(sBad + C::STAGES * 4);   // [32] valid keys
+
+  int32_t* sTiles = reinterpret_cast<int32_t*>(sMask + C::MAX_TILES);   // [32] active tiles
+  float* sRed = reinterpret_cast<float*>(sTiles + C::MAX_TILES);        // [2][2][128]
+  float* sLsum = sRed + 2 * 2 * 128;                            // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sLsum + 2 * 128);
   uint64_t* kv_full = bars;          // [3] 128 producer arrivals
   uint64_t* kv_empty = bars + 3;     // [3] QK commit + PV commit
@@ -103,15 +106,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   uint64_t* s_empty = bars + 7;      // 8 softmax warps
   uint64_t* p_full = bars + 8;       // 256 softmax threads
   uint64_t* pv_done = bars + 9;      // PV commit
-  uint64_t* x_full = bars + 10;      // 1 local arrive + X_BYTES from the peer's copies
-  uint64_t* peer_free = bars + 11;   // 1 remote arrival: the peer read what we sent
-  uint64_t* mx_bar = bars + 12;      // 256 arrivals per tile: both halves' partial max written
-  uint64_t* fin_bar = bars + 13;     // 256 arrivals: both halves' partial sums written
-  uint64_t* qk_fin = bars + 14;
-  uint64_t* pv_fin = bars + 15;
-  uint64_t* staged = bars + 16;      // 256 arrivals: our partial logits are in the staging area
-  uint64_t* stage_free = bars + 17;  // 1 arrival: the copy out of the staging area is done
-  uint64_t* xin_read = bars + 18;    // 256 arrivals: the peer's partial logits were read
+  uint64_t* x_full = bars + 10;      // [2] 1 local arrive + X_BYTES from the peer's copy
+  uint64_t* peer_free = bars + 12;   // [2] 1 remote arrival: the peer read that buffer
+  uint64_t* mx_bar = bars + 14;      // 256 arrivals per tile: both halves' partial max
+  uint64_t* fin_bar = bars + 15;     // 256 arrivals: both halves' partial sums
+  uint64_t* qk_fin = bars + 16;
+  uint64_t* pv_fin = bars + 17;
+  uint64_t* staged = bars + 18;      // 256 arrivals: our partial logits are staged
+  uint64_t* stage_free = bars + 19;  // 1 arrival: the copy out of the staging area is done
+  uint64_t* xin_read = bars + 20;    // [2] per buffer, 256 arrivals: the peer's partials read
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int n_act_s;
@@ -124,6 +127,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   const int row = p.row_begin + r;
   const int kb_begin = rank == 0 ? 0 : C::VKB;
   const int kb_count = rank == 0 ? C::VKB : C::KBC;
+  const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
 
   // ---- row geometry
   int b, n_keys;
@@ -152,55 +156,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     mbar_init(smem_u32(s_empty), 8);
     mbar_init(smem_u32(p_full), 256);
     mbar_init(smem_u32(pv_done), 1);
-    mbar_init(smem_u32(x_full), 1);
-    mbar_init(smem_u32(peer_free), 1);
-    mbar_init(smem_u32(staged), 256);
-    mbar_init(smem_u32(stage_free), 1);
-    mbar_init(smem_u32(xin_read), 256);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&x_full[i]), 1);
+      mbar_init(smem_u32(&peer_free[i]), 1);
+    }
     mbar_init(smem_u32(mx_bar), 256);
     mbar_init(smem_u32(fin_bar), 256);
     mbar_init(smem_u32(qk_fin), 1);
     mbar_init(smem_u32(pv_fin), 1);
+    mbar_init(smem_u32(staged), 256);
+    mbar_init(smem_u32(stage_free), 1);
+    mbar_init(smem_u32(&xin_read[0]), 256);
+    mbar_init(smem_u32(&xin_read[1]), 256);
     abort_s = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
-
   if (warp >= 12) {
-    // ---- resolve logical indices to physical rows (all loads of a round issued together)
-    const int tp = threadIdx.x - 384;
-    const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
-    for (int j0 = 0; j0 < p.topk; j0 += 4 * 512) {
-      int4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j0 + (u * 128 + tp) * 4;
-        v[u] = j < p.topk ? *reinterpret_cast<const int4*>(irow + j) : make_int4(-1, -1, -1, -1);
-      }
-      int64_t ph[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int vi = (&v[e / 4].x)[e % 4];
-        ph[e] = -1;
-        if (vi >= 0 && vi < n_keys) {
-          if (p.decode && p.block_table != nullptr)
-            ph[e] = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
-                          vi / p.block_size);
-          else
-            ph[e] = key_base + vi;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int vi = (&v[e / 4].x)[e % 4];
-        int64_t phys = ph[e];
-        if (vi >= 0 && vi < n_keys && p.decode && p.block_table != nullptr)
-          phys = phys < 0 ? -1 : phys * p.block_size + vi % p.block_size;
-        if (phys >= p.num_kv_rows) phys = -1;
-        if (vi >= 0 && phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
-        const int j = j0 + ((e / 4) * 128 + tp) * 4 + (e % 4);
-        if (j < p.topk) sPhys[j] = static_cast<int32_t>(phys);
-      }
+    // ---- which tiles hold a valid key (index in [0, n_keys)); warp w takes tiles w, w+4, ..
+    const int n_tiles_all = p.topk / C::BN;
+    for (int t = warp - 12; t < n_tiles_all; t += 4) {
+      const int v0 = irow[t * C::BN + lane], v1 = irow[t * C::BN + 32 + lane];
+      if ((v0 >= n_keys || v1 >= n_keys) && p.status) atomicOr(p.status, kStatusBadIndex);
+      const uint32_t lo = __ballot_sync(0xffffffffu, v0 >= 0 && v0 < n_keys);
+      const uint32_t hi = __ballot_sync(0xffffffffu, v1 >= 0 && v1 < n_keys);
+      if (lane == 0) sMask[t] = (static_cast<uint64_t>(hi) << 32) | lo;
     }
   }
   tc_fence_before();
@@ -230,34 +210,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     }
     tmem_wait_st();
   }
-  // ---- per-tile validity masks and the active tiles (>= 1 valid key), identical in both CTAs
-  if (warp == 0) {
+  if (warp == 0 && lane == 0) {
+    // ---- the active tiles of this split, identical in both CTAs
     const int n_tiles_all = p.topk / C::BN;
     int cnt = 0;
-    for (int t = 0; t < n_tiles_all; ++t) {
-      const uint32_t lo = __ballot_sync(0xffffffffu, sPhys[t * C::BN + lane] >= 0);
-      const uint32_t hi = __ballot_sync(0xffffffffu, sPhys[t * C::BN + 32 + lane] >= 0);
-      const uint64_t m = (static_cast<uint64_t>(hi) << 32) | lo;
-      if (m != 0) {
-        if (lane == 0) {
-          sTiles[cnt] = t;
-          sMask[cnt] = m;
-        }
+    for (int t = 0; t < n_tiles_all; ++t)
+      if (sMask[t] != 0) {
+        sTiles[cnt] = t;
         ++cnt;
       }
-    }
-    __syncwarp();
-    if (lane == 0) {
-      const int per = (cnt + p.splits - 1) / p.splits;
-      const int t0 = min(cnt, split * per);
-      const int t1 = min(cnt, t0 + per);
-      for (int i = t0; i < t1; ++i) {
-        sTiles[i - t0] = sTiles[i];
-        sMask[i - t0] = sMask[i];
-      }
-      n_act_s = t1 - t0;
-      if (t1 > t0) mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);   // arm tile 0
-    }
+    const int per = (cnt + p.splits - 1) / p.splits;
+    const int t0 = min(cnt, split * per);
+    const int t1 = min(cnt, t0 + per);
+    for (int i = t0; i < t1; ++i) sTiles[i - t0] = sTiles[i];
+    n_act_s = t1 - t0;
+    if (t1 - t0 > 0) mbar_arrive_expect_tx(smem_u32(&x_full[0]), C::X_BYTES);   // arm tile 0
+    if (t1 - t0 > 1) mbar_arrive_expect_tx(smem_u32(&x_full[1]), C::X_BYTES);   // arm tile 1
   }
   tc_fence_before();
   __syncthreads();
@@ -265,7 +233,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   cluster_sync();   // peer barriers initialised before any remote access
   const int n = n_act_s;
 
-  if (warp == 0) {
+  if (warp == 1) {
+    // ------------------------------------------------------------ read-signal forwarder
+    // Tells the peer, as soon as our softmax has read its partial logits of tile i, that buffer
+    // i % 2 may take tile i + 2 (per-buffer barriers: a buffer's reads cannot run two phases
+    // ahead of this wait).
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        ok = mbar_wait(smem_u32(&xin_read[i & 1]), (i >> 1) & 1, &abort_s);
+        if (ok) mbar_arrive_cluster(smem_u32(&peer_free[i & 1]), peer);
+      }
+      if (!ok) {
+        abort_s = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ QK issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f32acc(1 /* bf16 */, 128, C::BN, 0, 0);
@@ -320,25 +304,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
       mbar_wait(smem_u32(pv_fin), 0, nullptr);
     }
   } else if (warp == 3) {
-    // ------------------------------------------------------------ exchange helper
-    // Copies our staged partial logits into the peer's buffer and tells the peer when its
-    // partials have been read here: the cluster-scope release of that signal is slow, so it is
-    // kept off the softmax warps.
+    // ------------------------------------------------------------ exchange copier
+    // Copies our staged partial logits of tile i into the peer's buffer (i % 2) once the peer
+    // has read tile i - 2 from it; cross-CTA signalling stays off the softmax warps.
     if (lane == 0) {
       const uint32_t xin_remote = map_to_rank(smem_u32(sXin), peer);
       const uint32_t x_full_remote = map_to_rank(smem_u32(x_full), peer);
       bool ok = true;
       for (int i = 0; i < n && ok; ++i) {
         ok = mbar_wait(smem_u32(staged), i & 1, &abort_s);
-        if (ok && i >= 1) ok = mbar_wait<true>(smem_u32(peer_free), (i - 1) & 1, &abort_s);
+        if (ok && i >= 2) ok = mbar_wait<true>(smem_u32(&peer_free[i & 1]), ((i >> 1) - 1) & 1,
+                                               &abort_s);
         if (!ok) break;
-        bulk_copy_to_peer(xin_remote, smem_u32(sXout), C::X_BYTES, x_full_remote);
+        bulk_copy_to_peer(xin_remote + (i & 1) * C::X_BYTES, smem_u32(sXout), C::X_BYTES,
+                          x_full_remote + (i & 1) * 8);
         bulk_commit();
         bulk_wait_read_all();
         mbar_arrive(smem_u32(stage_free));
-        ok = mbar_wait(smem_u32(xin_read), i & 1, &abort_s);
-        if (!ok) break;
-        mbar_arrive_cluster(smem_u32(peer_free), peer);
       }
       if (!ok) {
         abort_s = 1;
@@ -348,27 +330,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------ gather producers
-    const int tp = threadIdx.x - 384;
-    const int chunks = C::BN * kb_count * 8;
+    // Producer warp w owns rows [16w, 16w + 16) of every tile: lanes 0..15 resolve their
+    // logical key to a physical row (the next tile's index is loaded a tile ahead), then the
+    // warp gathers this CTA's dims of its rows with 16-byte cp.async.  No cross-warp barrier.
+    const int pw = warp - 12;
+    const int chunks = 16 * kb_count * 8;
+    int32_t v_next = -1;
+    if (n > 0 && lane < 16) v_next = irow[sTiles[0] * C::BN + pw * 16 + lane];
     for (int i = 0; i < n; ++i) {
       const int s = i % C::STAGES;
       if (i >= C::STAGES &&
-          !mbar_wait(smem_u32(&kv_empty[s]), ((i / C::STAGES) - 1) & 1, &abort_s)) {
+          !__all_sync(0xffffffffu, mbar_wait(smem_u32(&kv_empty[s]), ((i / C::STAGES) - 1) & 1,
+                                             &abort_s))) {
         abort_s = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
         break;
       }
-      const int tile = sTiles[i];
+      const int v = v_next;
+      if (i + 1 < n && lane < 16) v_next = irow[sTiles[i + 1] * C::BN + pw * 16 + lane];
+      int64_t phys = -1;
+      if (lane < 16 && v >= 0 && v < n_keys) {
+        if (p.decode && p.block_table != nullptr) {
+          const int64_t id = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
+                                   v / p.block_size);
+          phys = id < 0 ? -1 : id * p.block_size + v % p.block_size;
+        } else {
+          phys = key_base + v;
+        }
+        if (phys >= p.num_kv_rows) phys = -1;
+        if (phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+      }
+      const uint32_t bad = __ballot_sync(0xffffffffu, lane < 16 && v >= 0 && v < n_keys && phys < 0);
+      if (lane == 0) sBad[s * 4 + pw] = static_cast<uint16_t>(bad & 0xFFFFu);
+      const int32_t my_row = static_cast<int32_t>(phys);
       uint8_t* dst = sKV + s * C::KV_STAGE_BYTES;
-      for (int c = tp; c < chunks; c += 128) {
-        const int kr = c / (kb_count * 8);
+      for (int c = lane; c < chunks; c += 32) {
+        const int rw = c / (kb_count * 8);          // row within this warp's 16
         const int rem = c % (kb_count * 8);
         const int kbl = rem / 8, ch = rem % 8;
         const int d = (kb_begin + kbl) * 64 + ch * 8;
-        const int32_t phys = sPhys[tile * C::BN + kr];
-        const bool ok = phys >= 0 && d < D_QK;
+        const int kr = pw * 16 + rw;                // row within the tile
+        const int32_t prow = __shfl_sync(0xffffffffu, my_row, rw);
+        const bool ok = prow >= 0 && d < D_QK;
         cp_async_16(smem_u32(dst + kbl * (C::BN * 128) + sw128_offset(kr, ch)),
-                    ok ? static_cast<const void*>(p.kv + static_cast<int64_t>(phys) * D_QK + d)
+                    ok ? static_cast<const void*>(p.kv + static_cast<int64_t>(prow) * D_QK + d)
                        : static_cast<const void*>(p.kv),
                     ok ? 16u : 0u);
       }
@@ -387,42 +392,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     const uint32_t x_row = half * (128 * 128) + hrow * 128;
     constexpr int OC = C::V_HALF / 2;           // O columns this half rescales / stores
     float m_ref = -INFINITY, l_sum = 0.f;
+    float own[32];                              // our partial logits of the tile in flight
     bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(s_full), i & 1, &abort_s));
-      if (!ok) break;
+    // Loads S(j) from TMEM, frees it for the next QK, stages it for the peer; keeps our partial.
+    auto stage_tile = [&](int j) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s_full), j & 1, &abort_s))) return false;
       tc_fence_after();
-      float sv[32];
-      {
-        uint32_t u[32];
-        tmem_ld32(lane_addr + C::S_COL + half * 32, u);
-        tmem_wait_ld();
+      uint32_t u[32];
+      tmem_ld32(lane_addr + C::S_COL + half * 32, u);
+      tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(u[j]);
-      }
+      for (int e = 0; e < 32; ++e) own[e] = __uint_as_float(u[e]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_empty));
-      // stage our partial logits; the helper copies them into the peer's buffer
-      if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(stage_free), (i - 1) & 1, &abort_s));
-        if (!ok) break;
-      }
+      if (j >= 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(smem_u32(stage_free), (j - 1) & 1, &abort_s)))
+        return false;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<float4*>(sXout + x_row + ((c ^ (hrow & 7)) << 4)) =
-            make_float4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
+            make_float4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(staged));
-      ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(x_full), i & 1, &abort_s));
+      return true;
+    };
+    if (n > 0) ok = stage_tile(0);
+    for (int i = 0; i < n && ok; ++i) {
+      float sv[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sv[e] = own[e];
+      // start the swap of the next tile before working on this one
+      if (i + 1 < n) {
+        ok = stage_tile(i + 1);
+        if (!ok) break;
+      }
+      const int xb = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(&x_full[xb]), (i >> 1) & 1, &abort_s));
       if (!ok) break;
-      if (warp == 4 && lane == 0 && i + 1 < n)
-        mbar_arrive_expect_tx(smem_u32(x_full), C::X_BYTES);   // arm tile i+1
-      const uint32_t vbits = static_cast<uint32_t>(sMask[i] >> (32 * half));
+      if (warp == 4 && lane == 0 && i + 2 < n)
+        mbar_arrive_expect_tx(smem_u32(&x_full[xb]), C::X_BYTES);   // arm tile i+2
+      // the producers' invalid-row bits of this tile: observe its kv_full phase first (the
+      // stage is not refilled before PV(i), which needs this tile's P)
+      const int st = i % C::STAGES;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&kv_full[st]), (i / C::STAGES) & 1, &abort_s));
+      if (!ok) break;
+      const uint64_t bad = static_cast<uint64_t>(sBad[st * 4 + 0]) |
+                           (static_cast<uint64_t>(sBad[st * 4 + 1]) << 16) |
+                           (static_cast<uint64_t>(sBad[st * 4 + 2]) << 32) |
+                           (static_cast<uint64_t>(sBad[st * 4 + 3]) << 48);
+      const uint64_t vmask = sMask[sTiles[i]] & ~bad;
+      const uint32_t vbits = static_cast<uint32_t>(vmask >> (32 * half));
+      const uint8_t* xin = sXin + xb * C::X_BYTES;
       float m_half = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float4 o = *reinterpret_cast<const float4*>(sXin + x_row + ((c ^ (hrow & 7)) << 4));
+        const float4 o = *reinterpret_cast<const float4*>(xin + x_row + ((c ^ (hrow & 7)) << 4));
         const float ov[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -433,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           m_half = fmaxf(m_half, sv[j]);
         }
       }
-      mbar_arrive(smem_u32(xin_read));
+      mbar_arrive(smem_u32(&xin_read[xb]));
       // row max over both halves (double-buffered by tile parity)
       float* red = sRed + (i & 1) * 256;
       red[half * 128 + hrow] = m_half;
