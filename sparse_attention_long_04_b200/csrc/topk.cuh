@@ -7,13 +7,14 @@
 // Radix select, no sort.  Each score maps to a 32-bit key whose unsigned order is the float
 // order (-0 folded onto +0).  A row is split over a cluster of C CTAs (C = 1..8); CTA c reads
 // its slice of the row from global memory once and keeps the keys in shared memory, building
-// the histogram of the first digit (the top 11 bits) while it loads.  Three digits (11, 11 and
-// 10 bits, most significant first) are resolved in turn: each CTA histograms the keys that
-// match the digits fixed so far (warp-aggregated shared atomics), the C histograms are summed
-// through distributed shared memory, and every CTA picks the same bin.  After the first digit
-// the keys of the chosen bin are compacted into a short candidate list, so the later digits
-// scan only those.  After the last digit the exact k-th key tau and the number of keys == tau
-// still needed are known.  The output pass takes every key > tau and the first `need` keys == tau in index
+// the histogram of the first digit (the top 11 bits) while it loads.  The C histograms are
+// summed through distributed shared memory (each CTA adds its non-zero bins into every CTA)
+// and every CTA picks the bin holding the k-th largest key.  The keys of that bin are few:
+// every CTA appends its own into CTA 0's candidate buffer, CTA 0 resolves the remaining 21
+// bits (digits of 11 and 10 bits) locally and broadcasts the exact k-th key tau and the count
+// of keys == tau still needed.  (If the bin is too crowded for the buffer, e.g. mass ties, the
+// CTAs resolve the remaining digits together with filtered scans and cluster-summed
+// histograms instead.)  The output pass takes every key > tau and the first `need` keys == tau in index
 // order (the smallest indices): per-warp counts give each warp's output offset (an exclusive
 // scan over the cluster in index order), and the indices come out in increasing order.
 #pragma once
@@ -40,8 +41,9 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkSlice = 16384;          // keys a CTA keeps in shared memory
 constexpr int kTopkBins = 2048;
-constexpr int kTopkCand = 4096;           // candidates kept after the first digit
-constexpr int kTopkSmem = kTopkSlice * 4 + kTopkCand * 4 + 2 * kTopkBins * 4 + 1024;
+constexpr int kTopkCand = 8192;           // candidate keys CTA 0 gathers after the first digit
+// 112.5 KiB: two CTAs still fit on one SM
+constexpr int kTopkSmem = kTopkSlice * 4 + kTopkCand * 4 + 2 * kTopkBins * 4 + 512;
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -118,17 +120,54 @@ __device__ __forceinline__ void cluster_hist_sum(uint32_t* hist, uint32_t* hsum,
   }
 }
 
+__device__ __forceinline__ uint32_t atom_cluster_add(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v)
+               : "memory");
+  return old;
+}
+
+// Bin holding the need-th largest key of hsum (nb bins, descending cumulative counts); all
+// threads of the CTA call it and all get the same (bin, count above the bin).
+__device__ __forceinline__ void find_bin(const uint32_t* hsum, uint32_t nb, uint32_t need,
+                                         uint32_t* tmp, uint32_t* s_bin, uint32_t* s_above,
+                                         uint32_t* bin, uint32_t* above) {
+  const int tid = threadIdx.x;
+  const uint32_t bpt = nb / kTopkThreads;         // 4 or 2 bins per thread
+  uint32_t mine = 0;
+  for (uint32_t j = 0; j < bpt; ++j) mine += hsum[nb - 1 - (tid * bpt + j)];
+  uint32_t tot;
+  const uint32_t before = cta_excl_scan(mine, tmp, &tot);
+  if (before < need && before + mine >= need) {
+    uint32_t c = before;
+    for (uint32_t j = 0; j < bpt; ++j) {
+      const uint32_t b = nb - 1 - (tid * bpt + j);
+      if (c + hsum[b] >= need) {
+        *s_bin = b;
+        *s_above = c;
+        break;
+      }
+      c += hsum[b];
+    }
+  }
+  __syncthreads();
+  *bin = *s_bin;
+  *above = *s_above;
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(topk_smem);           // [kTopkSlice]
-  uint32_t* cand = keys + kTopkSlice;                                // [kTopkCand] keys
+  uint32_t* cand = keys + kTopkSlice;                                // [kTopkCand] (CTA 0)
   uint32_t* hist = cand + kTopkCand;                                 // [kTopkBins] this CTA
   uint32_t* hsum = hist + kTopkBins;                                 // [kTopkBins] cluster sum
   uint32_t* tmp = hsum + kTopkBins;                                  // [40] scan scratch
   uint32_t* wgt = tmp + 40;                                          // [16] per-warp > tau
   uint32_t* weq = wgt + 16;                                          // [16] per-warp == tau
   uint32_t* cnt = weq + 16;                                          // [16] per-CTA (gt, eq)
-  __shared__ uint32_t s_bin, s_above, s_ncand;
+  uint32_t* bc = cnt + 16;                                           // [4] broadcast result
+  __shared__ uint32_t s_bin, s_above, s_ncand, s_base;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = p.csize;
@@ -167,8 +206,7 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   auto key_at = [&](int i) -> uint32_t {
     return cached ? keys[i] : score_key(srow[s0 + i]);
   };
-  // 4 consecutive keys (i multiple of 4; lanes past m read as 0 and are masked by callers)
-  auto key4_at = [&](int i) -> uint4 {
+  auto key4_at = [&](int i) -> uint4 {            // i multiple of 4, i < m
     if (cached) return *reinterpret_cast<const uint4*>(keys + i);
     uint4 k = make_uint4(0, 0, 0, 0);
     if (i + 0 < m) k.x = score_key(srow[s0 + i + 0]);
@@ -185,7 +223,6 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   }
   if (tid == 0) s_ncand = 0;
   __syncthreads();
-  // all of a thread's loads are issued before any is used (one latency, not one per round)
   if (cached) {
     constexpr int kVec = kTopkSlice / 4 / kTopkThreads;   // float4 per thread (8)
     float4 v[kVec];
@@ -211,91 +248,118 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   } else {
     for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&hist[key_at(i) >> 21], 1u);
   }
+  cluster_hist_sum(hist, hsum, kTopkBins, C);
+  uint32_t bin, above;
+  find_bin(hsum, kTopkBins, K, tmp, &s_bin, &s_above, &bin, &above);
+  uint32_t need = K - above;
+  uint32_t prefix = bin << 21, mask = 0xFFE00000u;
+  const uint32_t in_bin_total = hsum[bin];
+  const uint32_t in_bin_local = hist[bin];
+  __syncthreads();
 
-  uint32_t prefix = 0, mask = 0, need = K;
-  bool use_cand = false;
-  uint32_t ncand = 0;
-  constexpr int kShift[3] = {21, 10, 0};
-  constexpr int kBits[3] = {11, 11, 10};
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = kShift[pass];
-    const uint32_t nb = 1u << kBits[pass];
-    if (pass > 0) {
-      for (uint32_t i = tid; i < nb; i += kTopkThreads) {
-        hist[i] = 0;
-        hsum[i] = 0;
-      }
-      __syncthreads();
-      if (use_cand) {
-        for (uint32_t i = tid; i < ncand; i += kTopkThreads) {
-          const uint32_t k = cand[i];
-          if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
-        }
-      } else {
-        for (int i = tid; i < m; i += kTopkThreads) {
-          const uint32_t k = key_at(i);
-          if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
+  if (in_bin_total != need) {                     // else: every key of the bin is taken
+    if (in_bin_total <= static_cast<uint32_t>(kTopkCand)) {
+      // ---- gather the bin's keys into CTA 0 and resolve the last 21 bits there
+      if (tid == 0)
+        s_base = in_bin_local ? (C > 1 ? atom_cluster_add(map_to_rank(smem_u32(&s_ncand), 0),
+                                                           in_bin_local)
+                                       : atomicAdd(&s_ncand, in_bin_local))
+                              : 0u;
+      if (C > 1) cluster_sync(); else __syncthreads();   // reservations done (CTA 0's count)
+      uint32_t mine = 0;                           // this thread's matches, in its 4-key groups
+      const int nrounds = (m + kTopkThreads * 4 - 1) / (kTopkThreads * 4);
+      for (int u = 0; u < nrounds; ++u) {
+        const int i4 = (u * kTopkThreads + tid) * 4;
+        if (i4 < m) {
+          const uint4 k = key4_at(i4);
+          mine += (k.x & mask) == prefix;
+          mine += i4 + 1 < m && (k.y & mask) == prefix;
+          mine += i4 + 2 < m && (k.z & mask) == prefix;
+          mine += i4 + 3 < m && (k.w & mask) == prefix;
         }
       }
-    }
-    cluster_hist_sum(hist, hsum, nb, C);
-    // the bin holding the need-th largest key: descending cumulative counts
-    const uint32_t bpt = nb / kTopkThreads;         // 4 or 2 bins per thread
-    uint32_t mine = 0;
-    for (uint32_t j = 0; j < bpt; ++j) mine += hsum[nb - 1 - (tid * bpt + j)];
-    uint32_t tot;
-    const uint32_t before = cta_excl_scan(mine, tmp, &tot);
-    if (before < need && before + mine >= need) {
-      uint32_t c = before;
-      for (uint32_t j = 0; j < bpt; ++j) {
-        const uint32_t bin = nb - 1 - (tid * bpt + j);
-        if (c + hsum[bin] >= need) {
-          s_bin = bin;
-          s_above = c;
-          break;
-        }
-        c += hsum[bin];
-      }
-    }
-    __syncthreads();
-    const uint32_t bin = s_bin;
-    need -= s_above;
-    prefix |= bin << shift;
-    mask |= (nb - 1) << shift;
-    const bool exact = hsum[bin] == need;           // every key of this bucket is taken
-    const uint32_t local_in_bin = hist[bin];        // this CTA's keys in the chosen bin
-    __syncthreads();
-    if (exact) break;
-    if (pass == 0) {
-      // compact this CTA's keys of the chosen bin (order is irrelevant for histograms)
-      use_cand = local_in_bin <= kTopkCand;
-      if (use_cand) {
-        for (int base = warp * 128; base < m; base += kTopkThreads * 4) {   // warp-uniform
-          const int i4 = base + lane * 4;
-          const uint4 k = i4 < m ? key4_at(i4) : make_uint4(0, 0, 0, 0);
+      uint32_t tot;
+      uint32_t slot = s_base + cta_excl_scan(mine, tmp, &tot);
+      const uint32_t dst0 = C > 1 ? map_to_rank(smem_u32(cand), 0) : smem_u32(cand);
+      for (int u = 0; u < nrounds && mine; ++u) {
+        const int i4 = (u * kTopkThreads + tid) * 4;
+        if (i4 < m) {
+          const uint4 k = key4_at(i4);
           const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
-          uint32_t hit = 0;
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (i4 + e < m && (kk[e] & mask) == prefix) hit |= 1u << e;
-          const uint32_t nh = __popc(hit);
-          uint32_t inc = nh;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
+            if (i4 + e < m && (kk[e] & mask) == prefix) {
+              if (C > 1) st_cluster_u32(dst0 + slot * 4, kk[e]);
+              else cand[slot] = kk[e];
+              ++slot;
+            }
+        }
+      }
+      if (C > 1) cluster_sync(); else __syncthreads();   // CTA 0 holds every candidate
+      if (crank == 0) {
+        // digits 2 and 3 over the candidates, locally
+        constexpr int kShift[2] = {10, 0};
+        constexpr int kBits[2] = {11, 10};
+        for (int pass = 0; pass < 2; ++pass) {
+          const uint32_t nb = 1u << kBits[pass];
+          for (uint32_t i = tid; i < nb; i += kTopkThreads) hsum[i] = 0;
+          __syncthreads();
+          for (uint32_t i = tid; i < in_bin_total; i += kTopkThreads) {
+            const uint32_t k = cand[i];
+            if ((k & mask) == prefix) atomicAdd(&hsum[(k >> kShift[pass]) & (nb - 1)], 1u);
           }
-          uint32_t wbase = 0;
-          if (lane == 31 && inc > 0) wbase = atomicAdd(&s_ncand, inc);
-          wbase = __shfl_sync(0xffffffffu, wbase, 31);
-          uint32_t slot = wbase + inc - nh;
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if ((hit >> e) & 1u) cand[slot++] = kk[e];
+          __syncthreads();
+          uint32_t b2, ab2;
+          find_bin(hsum, nb, need, tmp, &s_bin, &s_above, &b2, &ab2);
+          need -= ab2;
+          prefix |= b2 << kShift[pass];
+          mask |= (nb - 1) << kShift[pass];
+          const bool exact = hsum[b2] == need;
+          __syncthreads();
+          if (exact) break;
+        }
+        if (tid == 0)
+          for (int c = 0; c < C; ++c) {
+            const uint32_t base = C > 1 ? map_to_rank(smem_u32(bc), c) : smem_u32(bc);
+            if (C > 1) {
+              st_cluster_u32(base + 0, prefix);
+              st_cluster_u32(base + 4, mask);
+              st_cluster_u32(base + 8, need);
+            } else {
+              bc[0] = prefix;
+              bc[1] = mask;
+              bc[2] = need;
+            }
+          }
+      }
+      if (C > 1) cluster_sync(); else __syncthreads();   // the broadcast has landed
+      prefix = bc[0];
+      mask = bc[1];
+      need = bc[2];
+    } else {
+      // ---- crowded bin: the remaining digits with filtered scans and cluster sums
+      constexpr int kShift[2] = {10, 0};
+      constexpr int kBits[2] = {11, 10};
+      for (int pass = 0; pass < 2; ++pass) {
+        const uint32_t nb = 1u << kBits[pass];
+        for (uint32_t i = tid; i < nb; i += kTopkThreads) {
+          hist[i] = 0;
+          hsum[i] = 0;
         }
         __syncthreads();
-        ncand = s_ncand;
+        for (int i = tid; i < m; i += kTopkThreads) {
+          const uint32_t k = key_at(i);
+          if ((k & mask) == prefix) atomicAdd(&hist[(k >> kShift[pass]) & (nb - 1)], 1u);
+        }
+        cluster_hist_sum(hist, hsum, nb, C);
+        uint32_t b2, ab2;
+        find_bin(hsum, nb, need, tmp, &s_bin, &s_above, &b2, &ab2);
+        need -= ab2;
+        prefix |= b2 << kShift[pass];
+        mask |= (nb - 1) << kShift[pass];
+        const bool exact = hsum[b2] == need;
+        __syncthreads();
+        if (exact) break;
       }
     }
   }
@@ -360,7 +424,7 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   // 128 keys per round: lane j holds keys 4j..4j+3 of the round (index order = lane order)
   for (int b0 = w0; b0 < w1; b0 += 128) {
     const int i4 = b0 + lane * 4;
-    const uint4 k = key4_at(i4);
+    const uint4 k = i4 < w1 ? key4_at(i4) : make_uint4(0, 0, 0, 0);
     const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
     uint32_t gtm = 0, eqm = 0;
 #pragma unroll

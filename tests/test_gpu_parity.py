@@ -148,6 +148,37 @@ def test_topk_exact_synthetic(dsa, k):
         check_topk_exact(ix[i], sc[i, :n], k, f"row {i} n={n} kind={kinds[i]}")
 
 
+def test_topk_cluster_paths(dsa):
+    """Rows long enough to split over a cluster of CTAs: a resolvable first-digit bin (its keys
+    gathered into one CTA), a crowded bin (every key in one bin: the digits are resolved by the
+    whole cluster), ties across slice boundaries, ragged lengths, signed scores."""
+    k = 2048
+    g = torch.Generator(device="cuda").manual_seed(77)
+    rows = [
+        torch.randn(131072, generator=g, device="cuda").abs(),
+        torch.randn(100003, generator=g, device="cuda"),
+        1.0 + 0.25 * torch.rand(60000, generator=g, device="cuda"),
+        torch.randint(0, 31, (50001,), generator=g, device="cuda").float(),
+        1.0 + torch.randint(0, 4096, (70002,), generator=g, device="cuda").float() / 16384.0,
+        torch.randn(16385, generator=g, device="cuda") * 1e-30,
+        torch.full((32768,), 2.5, device="cuda"),
+    ]
+    lens = [len(r) for r in rows]
+    ld = _ld(max(lens))
+    scores = torch.zeros(len(rows), ld, device="cuda")
+    for i, r in enumerate(rows):
+        scores[i, :len(r)] = r
+    pb = dsa.make_problem(mode="decode", h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512, topk=k,
+                          softmax_scale=1.0, num_kv_rows=len(rows) * max(lens), seqlens=lens,
+                          seq_lens=torch.tensor(lens, dtype=torch.int32, device="cuda"))
+    idx = torch.empty(len(rows), k, dtype=torch.int32, device="cuda")
+    assert dsa.dsa_topk(pb, scores, ld, 0, len(rows), idx) == 0
+    torch.cuda.synchronize()
+    sc, ix = to_np(scores), to_np(idx)
+    for i, n in enumerate(lens):
+        check_topk_exact(ix[i], sc[i, :n], k, f"row {i} n={n}")
+
+
 def test_topk_negative_and_signed_zero(dsa):
     k = 64
     g = torch.Generator(device="cuda").manual_seed(9)
