@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -179,6 +180,22 @@ dsa_status_t make_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Rows of `row_bytes` bytes (a multiple of 16), boxes of box_bytes x box_rows, 128-byte swizzle.
+dsa_status_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
+                          uint32_t box_bytes, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (encoder(&enc) != DSA_OK) return DSA_ERR_CUDA;
+  std::memset(map, 0, sizeof(*map));
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_bytes, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                   strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------------ stage 1
 
 template <int H_I, int D_I, int QPG>
@@ -317,10 +334,22 @@ dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* 
 
 int mla_splits(const dsa_dims_t& d, const dsa_seqs_t& s, int32_t row_count, int sm_count) {
   if (s.mode != DSA_DECODE || row_count <= 0) return 1;
-  const int clusters = std::max(1, sm_count / 2);
-  int splits = std::max(1, clusters / row_count);
-  splits = std::min(splits, std::max(1, d.topk / 64 / 4));   // >= 4 tiles per split
-  return std::min(splits, 16);
+  // Two CTAs (one per value half) per row and split; one CTA per SM.  Pick the split count
+  // with the smallest estimated makespan: waves x (prologue + tiles per split), in tile units
+  // (prologue ~3 tiles; a combine pass costs ~2 more).
+  const int tiles = std::max(1, (std::min(d.topk, std::max(1, s.max_seqlen)) + 63) / 64);
+  const int sms = std::max(1, sm_count);
+  int best = 1;
+  double best_t = 1e30;
+  for (int sp = 1; sp <= std::min(16, std::max(1, tiles / 4)); ++sp) {
+    const double waves = std::ceil(2.0 * row_count * sp / sms);
+    const double t = waves * (3.0 + std::ceil(double(tiles) / sp)) + (sp > 1 ? 2.0 : 0.0);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = sp;
+    }
+  }
+  return best;
 }
 
 size_t mla_ws_bytes(const dsa_dims_t& d, int splits, int32_t row_count) {
@@ -363,9 +392,14 @@ dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* 
     prm.part_o = static_cast<float*>(ws);
     prm.part_lse = prm.part_o + size_t(splits) * row_count * d.h * D_V;
   }
+  // latent rows gathered four at a time (64 dims x 1 row boxes); Q in 64-dim x 128-head boxes
+  CUtensorMap kv_map, q_map;
+  if (make_row_map(&kv_map, kv, uint64_t(s.num_kv_rows), D_QK * 2, 128, 1) != DSA_OK ||
+      make_row_map(&q_map, q, uint64_t(s.total_rows) * d.h, D_QK * 2, 128, 128) != DSA_OK)
+    return DSA_ERR_CUDA;
   auto k = dsa_sparse_mla_kernel<D_QK, D_V>;
   if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
-  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(prm);
+  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(kv_map, q_map, prm);
   if (launch_status() != DSA_OK) return DSA_ERR_CUDA;
   if (splits > 1) {
     dsa_mla_combine_kernel<D_V><<<dim3(row_count, d.h), 128, 0, st>>>(prm);

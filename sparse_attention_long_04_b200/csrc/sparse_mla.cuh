@@ -4,29 +4,30 @@
 //   l_s = sigma * q[t,h,:] . kv[s,:]            (all D_QK = latent + RoPE dims)
 //   O[t,h,:] = sum_s softmax(l)_s * kv[s, 0:D_V] (values = the first D_V latent dims)
 //   LSE[t,h] = log sum_s exp(l_s)
-// Every selected latent row is shared by all query heads ("MLA in MQA mode ... each latent KV
-// entry is shared across query heads", "DeepSeek V3.2-Exp Cuts Long-Context Costs with
-// DeepSeek Sparse Attention (DSA)", "Instantiation").
+// Every selected latent row serves all query heads: MLA run in its multi-query form
+// ("DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention (DSA)",
+// "Instantiation").
 //
 // Design (sm_100a).  O for 128 heads x 512 values in fp32 is 256 KB = all of one SM's TMEM,
-// and Q (128 x 576 bf16 = 144 KB) plus gathered tiles do not fit one CTA's shared memory, so
-// each query row runs on a 2-CTA cluster:
-//   CTA r owns the QK dims D_r (r = 0: [0, D_V/2); r = 1: [D_V/2, D_QK)) and the value dims
-//   [r D_V/2, (r+1) D_V/2).  Its slice of Q lives in Tensor Memory as the A operand of the QK
-//   MMA; the selected latent rows are gathered (their D_r dims) into 128-byte-swizzled shared
-//   memory tiles of 64 keys.  Per tile: S_r = Q_r K_r^T (tcgen05 bf16, A from TMEM, M = 128
-//   heads, N = 64 keys); the two CTAs swap S_r with bulk shared-to-shared copies into each
-//   other's memory and both form S = S_0 + S_1 in the same order, so both run an identical
-//   online softmax; P goes to TMEM and CTA r accumulates O_r += P V_r (A = P from TMEM,
-//   N = D_V/2, K = 64 keys, V read MN-major straight out of the gathered tile).  No tensor
-//   work is duplicated.  Rescaling of O is lazy (only when a tile's max beats the running
-//   reference by more than 2^8, so P <= 256).
-// TMEM columns: O [0, V_HALF) | S [V_HALF, +64) | P [+64, +32) | Q (kb_count x 32 columns).
-// Warp roles per CTA (512 threads): warp 0 issues QK, warp 2 issues PV, warp 1 owns TMEM and
-// forwards read signals to the peer, warp 3 copies our partial logits to the peer,
-// warps 4-11 run the softmax (thread = head = TMEM lane; warps 4-7 take keys 0-31 of a tile,
-// warps 8-11 keys 32-63) and the epilogue, warps 12-15 resolve indices and gather rows with
-// 16-byte cp.async (3 stages).  Grid: x = 2 * row (the cluster pair), y = split-KV slice.
+// so each query row runs on two CTAs: CTA v (v = 0, 1) accumulates the value dims
+// [v D_V/2, (v+1) D_V/2) and, to need nothing from its partner, computes the full logits of
+// every tile itself (the QK product is done twice; the two CTAs exchange no data).  Both run
+// the same instructions on the same inputs, so their logits, softmax and LSE agree bit for bit.
+//   Q (128 heads x 576 bf16) is the QK A operand: TMA brings it in as 128-byte-swizzled 64-dim
+//   blocks; the first KBT blocks move on into Tensor Memory (2 bf16 per column), the rest stay
+//   in shared memory.  Every selected key is resolved to its physical cache row once, up front
+//   (invalid keys borrow a valid row of their tile and are masked out of the softmax); the rows
+//   of each 64-key tile (all dims) are then gathered by TMA, four rows per instruction, into a
+//   2-stage ring.  Per tile: S = Q K^T (tcgen05 bf16, M = 128 heads, N = 64 keys, fp32 in
+//   TMEM), an online softmax (thread = head = TMEM lane), P (bf16) back into TMEM, and
+//   O_v += P V_v (A = P from TMEM, N = D_V/2, V read MN-major straight out of the gathered
+//   tile).  Rescaling of O is lazy (only when a tile's max beats the running reference by more
+//   than 2^8, so P <= 256).
+// TMEM columns: O [0, D_V/2) | S [+64) | P [+32) | Q (KBT x 32 columns).
+// Warp roles per CTA (512 threads): warp 0 loads Q and issues QK, warp 2 issues PV, warp 1
+// owns TMEM, warps 4-11 move Q into TMEM and run the softmax (warps 4-7 take keys 0-31 of a
+// tile, warps 8-11 keys 32-63) and the epilogue, warps 12-15 resolve the keys and gather (warp
+// w: rows [16w, 16w + 16) of every tile).  Grid: x = 2 * row + v, y = split-KV slice.
 #pragma once
 #include "sm100.cuh"
 
@@ -58,76 +59,73 @@ struct MlaParams {
 template <int D_QK, int D_V>
 struct MlaCfg {
   static constexpr int KB_ALL = (D_QK + 63) / 64;     // 64-element k-blocks of a latent row
-  static constexpr int V_HALF = D_V / 2;
+  static constexpr int V_HALF = D_V / 2;              // value dims per CTA
   static constexpr int VKB = V_HALF / 64;             // value k-blocks per CTA
-  static constexpr int KBC = KB_ALL - VKB;            // k-blocks held by rank 1 (>= rank 0)
   static constexpr int BN = 64;                       // keys per tile
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 2;
   static constexpr int MAX_TILES = 32;                // topk <= 2048
   static constexpr int THREADS = 512;
-  static constexpr int KV_STAGE_BYTES = KBC * BN * 128;
-  static constexpr int X_BYTES = 128 * BN * 4;        // partial logits of one tile
   static constexpr int S_COL = V_HALF;
   static constexpr int P_COL = S_COL + BN;
   static constexpr int Q_COL = P_COL + BN / 2;
-  static constexpr int TMEM_NEED = Q_COL + KBC * 32;
-  static constexpr int TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * KV_STAGE_BYTES + 3 * X_BYTES +
-                                    STAGES * 8 + MAX_TILES * 12 +
-                                    2 * 2 * 128 * 4 + 2 * 128 * 4 + 512;
-  static_assert(KBC >= VKB, "rank 1 holds at least as many k-blocks as rank 0");
+  static constexpr int KBT_MAX = (512 - Q_COL) / 32;
+  static constexpr int KBT = KB_ALL < KBT_MAX ? KB_ALL : KBT_MAX;   // Q k-blocks in TMEM
+  static constexpr int KBS = KB_ALL - KBT;                            // Q k-blocks in smem
+  static constexpr int TMEM_COLS = Q_COL + KBT * 32 <= 256 ? 256 : 512;
+  static constexpr int KB_BYTES = BN * 128;                           // one k-block of a tile
+  static constexpr int KV_STAGE_BYTES = KB_ALL * KB_BYTES;
+  static constexpr int Q_KB_BYTES = 128 * 128;                        // one k-block of Q
+  static constexpr int Q_SMEM_BYTES = KBS * Q_KB_BYTES;
+  static constexpr int ROWS_PER_WARP_TX = 16 * KB_ALL * 128;          // gather bytes per warp
+  static constexpr int SMEM_USED = 1024 + Q_SMEM_BYTES + STAGES * KV_STAGE_BYTES +
+                                   MAX_TILES * BN * 4 + MAX_TILES * 12 + 2 * 2 * 128 * 4 +
+                                   2 * 128 * 4 + 256;
+  // at least 116 KB, so that one CTA runs per SM (its TMEM allocation never waits)
+  static constexpr int SMEM_BYTES = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
   static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
-  static_assert(TMEM_NEED <= 512, "TMEM columns");
+  static_assert(Q_COL + KBT * 32 <= 512, "TMEM columns");
+  static_assert(KBT * Q_KB_BYTES <= STAGES * KV_STAGE_BYTES, "Q staging fits the gather ring");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-  static_assert(SMEM_BYTES > 114 * 1024, "one CTA per SM (TMEM and cluster peers)");
 };
 
 template <int D_QK, int D_V>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
-    dsa_sparse_mla_kernel(const MlaParams p) {
+__global__ void __launch_bounds__(512, 1)
+    dsa_sparse_mla_kernel(const __grid_constant__ CUtensorMap kv_map,
+                          const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
   using C = MlaCfg<D_QK, D_V>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sKV = smem;                                          // [STAGES] gathered tiles
-  uint8_t* sXin = sKV + C::STAGES * C::KV_STAGE_BYTES;          // [2] peer's partial logits
-  uint8_t* sXout = sXin + 2 * C::X_BYTES;                       // ours, staged for the copy
-  // [STAGES][4]: per producer warp, its 16 rows whose cache location was invalid
-  uint16_t* sBad = reinterpret_cast<uint16_t*>(sXout + C::X_BYTES);
-  uint64_t* sMask = reinterpret_cast<uint64_t*>(sBad + C::STAGES * 4);   // [32] valid keys
-
-  int32_t* sTiles = reinterpret_cast<int32_t*>(sMask + C::MAX_TILES);   // [32] active tiles
+  uint8_t* sQ = smem;                                           // [KBS][128 heads][128 B]
+  uint8_t* sKV = sQ + C::Q_SMEM_BYTES;                          // [STAGES] gathered tiles
+  int32_t* sPhys = reinterpret_cast<int32_t*>(sKV + C::STAGES * C::KV_STAGE_BYTES);  // [topk]
+  uint64_t* sMask = reinterpret_cast<uint64_t*>(sPhys + C::MAX_TILES * C::BN);   // [32]
+  int32_t* sTiles = reinterpret_cast<int32_t*>(sMask + C::MAX_TILES);            // [32]
   float* sRed = reinterpret_cast<float*>(sTiles + C::MAX_TILES);        // [2][2][128]
   float* sLsum = sRed + 2 * 2 * 128;                            // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sLsum + 2 * 128);
-  uint64_t* kv_full = bars;          // [3] 128 producer arrivals
-  uint64_t* kv_empty = bars + 3;     // [3] QK commit + PV commit
-  uint64_t* s_full = bars + 6;       // QK commit
-  uint64_t* s_empty = bars + 7;      // 8 softmax warps
-  uint64_t* p_full = bars + 8;       // 256 softmax threads
-  uint64_t* pv_done = bars + 9;      // PV commit
-  uint64_t* x_full = bars + 10;      // [2] 1 local arrive + X_BYTES from the peer's copy
-  uint64_t* peer_free = bars + 12;   // [2] 1 remote arrival: the peer read that buffer
-  uint64_t* mx_bar = bars + 14;      // 256 arrivals per tile: both halves' partial max
-  uint64_t* fin_bar = bars + 15;     // 256 arrivals: both halves' partial sums
-  uint64_t* qk_fin = bars + 16;
-  uint64_t* pv_fin = bars + 17;
-  uint64_t* staged = bars + 18;      // 256 arrivals: our partial logits are staged
-  uint64_t* stage_free = bars + 19;  // 1 arrival: the copy out of the staging area is done
-  uint64_t* xin_read = bars + 20;    // [2] per buffer, 256 arrivals: the peer's partials read
+  uint64_t* kv_full = bars;          // [2] 4 producer arrivals + gathered bytes
+  uint64_t* kv_empty = bars + 2;     // [2] PV commit
+  uint64_t* s_full = bars + 4;       // QK commit
+  uint64_t* s_empty = bars + 5;      // 8 softmax warps
+  uint64_t* p_full = bars + 6;       // 256 softmax threads
+  uint64_t* pv_done = bars + 7;      // PV commit
+  uint64_t* mx_bar = bars + 8;       // 256 arrivals per tile: both halves' partial max
+  uint64_t* fin_bar = bars + 9;      // 256 arrivals: both halves' partial sums
+  uint64_t* qk_fin = bars + 10;
+  uint64_t* pv_fin = bars + 11;
+  uint64_t* q_bar = bars + 12;       // 1 arrival + Q bytes
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int n_act_s;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
+  const int vh = static_cast<int>(blockIdx.x & 1u);   // value half
   const int split = blockIdx.y;
   const int r = blockIdx.x >> 1;
   const int row = p.row_begin + r;
-  const int kb_begin = rank == 0 ? 0 : C::VKB;
-  const int kb_count = rank == 0 ? C::VKB : C::KBC;
   const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
+  const int n_tiles_all = p.topk / C::BN;
 
   // ---- row geometry
   int b, n_keys;
@@ -149,70 +147,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(smem_u32(&kv_full[i]), 128);
-      mbar_init(smem_u32(&kv_empty[i]), 2);
+      mbar_init(smem_u32(&kv_full[i]), 4);
+      mbar_init(smem_u32(&kv_empty[i]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
     mbar_init(smem_u32(s_empty), 8);
     mbar_init(smem_u32(p_full), 256);
     mbar_init(smem_u32(pv_done), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&x_full[i]), 1);
-      mbar_init(smem_u32(&peer_free[i]), 1);
-    }
     mbar_init(smem_u32(mx_bar), 256);
     mbar_init(smem_u32(fin_bar), 256);
     mbar_init(smem_u32(qk_fin), 1);
     mbar_init(smem_u32(pv_fin), 1);
-    mbar_init(smem_u32(staged), 256);
-    mbar_init(smem_u32(stage_free), 1);
-    mbar_init(smem_u32(&xin_read[0]), 256);
-    mbar_init(smem_u32(&xin_read[1]), 256);
+    mbar_init(smem_u32(q_bar), 1);
     abort_s = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
-  if (warp >= 12) {
-    // ---- which tiles hold a valid key (index in [0, n_keys)); warp w takes tiles w, w+4, ..
-    const int n_tiles_all = p.topk / C::BN;
-    for (int t = warp - 12; t < n_tiles_all; t += 4) {
-      const int v0 = irow[t * C::BN + lane], v1 = irow[t * C::BN + 32 + lane];
-      if ((v0 >= n_keys || v1 >= n_keys) && p.status) atomicOr(p.status, kStatusBadIndex);
-      const uint32_t lo = __ballot_sync(0xffffffffu, v0 >= 0 && v0 < n_keys);
-      const uint32_t hi = __ballot_sync(0xffffffffu, v1 >= 0 && v1 < n_keys);
-      if (lane == 0) sMask[t] = (static_cast<uint64_t>(hi) << 32) | lo;
-    }
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
-  if (warp >= 4 && warp < 12) {
-    // ---- this CTA's slice of Q into TMEM (the QK A operand): head = lane, 2 bf16 per column
-    const int hrow = (warp & 3) * 32 + lane;
-    const int half = (warp - 4) >> 2;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int d0 = kb_begin * 64 + half * kb_count * 32;        // first dim of this half
-    const __nv_bfloat16* qrow = p.q + (static_cast<int64_t>(row) * p.h + hrow) * D_QK;
-    for (int kb = 0; kb < kb_count; ++kb) {
-      uint32_t u[16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int d = d0 + kb * 32 + c * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (hrow < p.h && d < D_QK) v = *reinterpret_cast<const uint4*>(qrow + d);
-        u[4 * c + 0] = v.x;
-        u[4 * c + 1] = v.y;
-        u[4 * c + 2] = v.z;
-        u[4 * c + 3] = v.w;
-      }
-      tmem_st16(lane_addr + C::Q_COL + half * kb_count * 16 + kb * 16, u);
+  if (threadIdx.x == 0) {
+    // ---- Q: blocks [0, KBT) into the (still idle) gather ring, the rest into sQ
+    tma_prefetch_desc(&kv_map);
+    tma_prefetch_desc(&q_map);
+    mbar_arrive_expect_tx(smem_u32(q_bar), C::KB_ALL * C::Q_KB_BYTES);
+    for (int kb = 0; kb < C::KB_ALL; ++kb) {
+      uint8_t* dst = kb < C::KBT ? sKV + kb * C::Q_KB_BYTES : sQ + (kb - C::KBT) * C::Q_KB_BYTES;
+      tma_load_2d(smem_u32(dst), &q_map, smem_u32(q_bar), kb * 128, row * p.h);
     }
-    tmem_wait_st();
   }
+  if (warp >= 12) {
+    // ---- every selected key -> physical row (or -1), 16 keys per thread, loads in flight
+    const int t = threadIdx.x - 384;
+    for (int e = t; e < p.topk; e += 128) {
+      const int v = irow[e];
+      int64_t phys = -1;
+      if (v >= 0 && v < n_keys) {
+        if (p.decode && p.block_table != nullptr) {
+          const int64_t id = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
+                                   v / p.block_size);
+          phys = id < 0 ? -1 : id * p.block_size + v % p.block_size;
+        } else {
+          phys = key_base + v;
+        }
+        if (phys >= p.num_kv_rows) phys = -1;
+        if (phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+      } else if (v >= n_keys && p.status) {
+        atomicOr(p.status, kStatusBadIndex);
+      }
+      sPhys[e] = static_cast<int32_t>(phys);
+    }
+  }
+  __syncthreads();
+  if (warp >= 12) {
+    // ---- per tile: the valid-key mask; invalid keys borrow the tile's first valid row
+    for (int tt = warp - 12; tt < n_tiles_all; tt += 4) {
+      int32_t* ph = sPhys + tt * C::BN;
+      const int32_t a0 = ph[lane], a1 = ph[32 + lane];
+      const uint32_t lo = __ballot_sync(0xffffffffu, a0 >= 0);
+      const uint32_t hi = __ballot_sync(0xffffffffu, a1 >= 0);
+      const uint64_t m = (static_cast<uint64_t>(hi) << 32) | lo;
+      if (m != 0) {
+        const int first = __ffsll(static_cast<long long>(m)) - 1;
+        const int32_t fb = ph[first];
+        __syncwarp();
+        if (a0 < 0) ph[lane] = fb;
+        if (a1 < 0) ph[32 + lane] = fb;
+      }
+      if (lane == 0) sMask[tt] = m;
+    }
+  }
+  __syncthreads();
   if (warp == 0 && lane == 0) {
-    // ---- the active tiles of this split, identical in both CTAs
-    const int n_tiles_all = p.topk / C::BN;
+    // ---- the active tiles of this split, identical in both CTAs of the row
     int cnt = 0;
     for (int t = 0; t < n_tiles_all; ++t)
       if (sMask[t] != 0) {
@@ -224,52 +229,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     const int t1 = min(cnt, t0 + per);
     for (int i = t0; i < t1; ++i) sTiles[i - t0] = sTiles[i];
     n_act_s = t1 - t0;
-    if (t1 - t0 > 0) mbar_arrive_expect_tx(smem_u32(&x_full[0]), C::X_BYTES);   // arm tile 0
-    if (t1 - t0 > 1) mbar_arrive_expect_tx(smem_u32(&x_full[1]), C::X_BYTES);   // arm tile 1
+  }
+  if (warp >= 4 && warp < 12) {
+    // ---- Q blocks [0, KBT) from the staging area into TMEM: head = lane, dim d in column
+    // Q_COL + d / 2 (half h of the warps takes blocks h, h + 2, ...)
+    const int hrow = (warp & 3) * 32 + lane;
+    const int half = (warp - 4) >> 2;
+    const uint32_t lane_addr = tmem_base_s + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(q_bar), 0, &abort_s))) {
+      abort_s = 1;
+      if (p.status) atomicOr(p.status, kStatusTimeout);
+    } else {
+      for (int kb = half; kb < C::KBT; kb += 2) {
+        uint32_t u[32];
+        const uint8_t* src = sKV + kb * C::Q_KB_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + sw128_offset(hrow, ch));
+          u[4 * ch + 0] = v.x;
+          u[4 * ch + 1] = v.y;
+          u[4 * ch + 2] = v.z;
+          u[4 * ch + 3] = v.w;
+        }
+        tmem_st32(lane_addr + C::Q_COL + kb * 32, u);
+      }
+      tmem_wait_st();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();   // the staging area is free for the gather ring from here on
   tc_fence_after();
-  cluster_sync();   // peer barriers initialised before any remote access
-  const int n = n_act_s;
+  const uint32_t tmem = tmem_base_s;
+  const int n = abort_s ? 0 : n_act_s;
 
-  if (warp == 1) {
-    // ------------------------------------------------------------ read-signal forwarder
-    // Tells the peer, as soon as our softmax has read its partial logits of tile i, that buffer
-    // i % 2 may take tile i + 2 (per-buffer barriers: a buffer's reads cannot run two phases
-    // ahead of this wait).
-    if (lane == 0) {
-      bool ok = true;
-      for (int i = 0; i < n && ok; ++i) {
-        ok = mbar_wait(smem_u32(&xin_read[i & 1]), (i >> 1) & 1, &abort_s);
-        if (ok) mbar_arrive_cluster(smem_u32(&peer_free[i & 1]), peer);
-      }
-      if (!ok) {
-        abort_s = 1;
-        if (p.status) atomicOr(p.status, kStatusTimeout);
-      }
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ QK issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f32acc(1 /* bf16 */, 128, C::BN, 0, 0);
-      bool ok = true;
+      const uint32_t qa = smem_u32(sQ);
+      bool ok = n == 0 || mbar_wait(smem_u32(q_bar), 0, &abort_s);
       for (int i = 0; i < n && ok; ++i) {
         const int s = i % C::STAGES;
         ok = mbar_wait(smem_u32(&kv_full[s]), (i / C::STAGES) & 1, &abort_s);
         if (ok && i >= 1) ok = mbar_wait(smem_u32(s_empty), (i - 1) & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
-        fence_proxy_async_smem();
         const uint32_t ka = smem_u32(sKV + s * C::KV_STAGE_BYTES);
-        for (int kb = 0; kb < kb_count; ++kb)
+        for (int kb = 0; kb < C::KBT; ++kb)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_bf16_ts(tmem + C::S_COL, tmem + C::Q_COL + kb * 32 + k * 8,
-                         sdesc_sw128(ka + kb * (C::BN * 128) + k * 32, 16, 1024), idesc,
+                         sdesc_sw128(ka + kb * C::KB_BYTES + k * 32, 16, 1024), idesc,
                          (kb | k) != 0);
+        for (int kb = C::KBT; kb < C::KB_ALL; ++kb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tmem + C::S_COL,
+                      sdesc_sw128(qa + (kb - C::KBT) * C::Q_KB_BYTES + k * 32, 16, 1024),
+                      sdesc_sw128(ka + kb * C::KB_BYTES + k * 32, 16, 1024), idesc, 1u);
         umma_commit(smem_u32(s_full));
-        umma_commit(smem_u32(&kv_empty[s]));
       }
       if (!ok) {
         abort_s = 1;
@@ -288,11 +306,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
         ok = mbar_wait(smem_u32(p_full), i & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t va = smem_u32(sKV + s * C::KV_STAGE_BYTES);
+        const uint32_t va = smem_u32(sKV + s * C::KV_STAGE_BYTES) + vh * C::VKB * C::KB_BYTES;
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k)
           umma_bf16_ts(tmem, tmem + C::P_COL + k * 8,
-                       sdesc_sw128(va + k * 16 * 128, C::BN * 128, 1024), idesc, (i | k) != 0);
+                       sdesc_sw128(va + k * 16 * 128, C::KB_BYTES, 1024), idesc, (i | k) != 0);
         umma_commit(smem_u32(&kv_empty[s]));
         umma_commit(smem_u32(pv_done));
       }
@@ -303,84 +321,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
       umma_commit(smem_u32(pv_fin));
       mbar_wait(smem_u32(pv_fin), 0, nullptr);
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ exchange copier
-    // Copies our staged partial logits of tile i into the peer's buffer (i % 2) once the peer
-    // has read tile i - 2 from it; cross-CTA signalling stays off the softmax warps.
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ gather producers
+    // Lane 0 of producer warp w gathers rows [16w, 16w + 16) of each tile: 4 rows x 64 dims
+    // per TMA instruction, KB_ALL k-blocks.
     if (lane == 0) {
-      const uint32_t xin_remote = map_to_rank(smem_u32(sXin), peer);
-      const uint32_t x_full_remote = map_to_rank(smem_u32(x_full), peer);
+      const int pw = warp - 12;
       bool ok = true;
+      int issued = 0;
       for (int i = 0; i < n && ok; ++i) {
-        ok = mbar_wait(smem_u32(staged), i & 1, &abort_s);
-        if (ok && i >= 2) ok = mbar_wait<true>(smem_u32(&peer_free[i & 1]), ((i >> 1) - 1) & 1,
-                                               &abort_s);
+        const int s = i % C::STAGES;
+        if (i >= C::STAGES)
+          ok = mbar_wait(smem_u32(&kv_empty[s]), ((i / C::STAGES) - 1) & 1, &abort_s);
         if (!ok) break;
-        bulk_copy_to_peer(xin_remote + (i & 1) * C::X_BYTES, smem_u32(sXout), C::X_BYTES,
-                          x_full_remote + (i & 1) * 8);
-        bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(smem_u32(stage_free));
+        const uint32_t bar = smem_u32(&kv_full[s]);
+        mbar_arrive_expect_tx(bar, C::ROWS_PER_WARP_TX);
+        const int32_t* ph = sPhys + sTiles[i] * C::BN + pw * 16;
+        const uint32_t dst0 = smem_u32(sKV + s * C::KV_STAGE_BYTES) + pw * 16 * 128;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int4 rr = *reinterpret_cast<const int4*>(ph + 4 * g);
+          for (int kb = 0; kb < C::KB_ALL; ++kb)
+            tma_gather4(dst0 + kb * C::KB_BYTES + g * 512, &kv_map, bar, kb * 128, rr.x, rr.y,
+                        rr.z, rr.w);
+        }
+        ++issued;
       }
       if (!ok) {
         abort_s = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
       }
-      bulk_wait_read_all();
-    }
-  } else if (warp >= 12) {
-    // ------------------------------------------------------------ gather producers
-    // Producer warp w owns rows [16w, 16w + 16) of every tile: lanes 0..15 resolve their
-    // logical key to a physical row (the next tile's index is loaded a tile ahead), then the
-    // warp gathers this CTA's dims of its rows with 16-byte cp.async.  No cross-warp barrier.
-    const int pw = warp - 12;
-    const int chunks = 16 * kb_count * 8;
-    int32_t v_next = -1;
-    if (n > 0 && lane < 16) v_next = irow[sTiles[0] * C::BN + pw * 16 + lane];
-    for (int i = 0; i < n; ++i) {
-      const int s = i % C::STAGES;
-      if (i >= C::STAGES &&
-          !__all_sync(0xffffffffu, mbar_wait(smem_u32(&kv_empty[s]), ((i / C::STAGES) - 1) & 1,
-                                             &abort_s))) {
-        abort_s = 1;
-        if (p.status) atomicOr(p.status, kStatusTimeout);
-        break;
-      }
-      const int v = v_next;
-      if (i + 1 < n && lane < 16) v_next = irow[sTiles[i + 1] * C::BN + pw * 16 + lane];
-      int64_t phys = -1;
-      if (lane < 16 && v >= 0 && v < n_keys) {
-        if (p.decode && p.block_table != nullptr) {
-          const int64_t id = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
-                                   v / p.block_size);
-          phys = id < 0 ? -1 : id * p.block_size + v % p.block_size;
-        } else {
-          phys = key_base + v;
-        }
-        if (phys >= p.num_kv_rows) phys = -1;
-        if (phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
-      }
-      const uint32_t bad = __ballot_sync(0xffffffffu, lane < 16 && v >= 0 && v < n_keys && phys < 0);
-      if (lane == 0) sBad[s * 4 + pw] = static_cast<uint16_t>(bad & 0xFFFFu);
-      const int32_t my_row = static_cast<int32_t>(phys);
-      uint8_t* dst = sKV + s * C::KV_STAGE_BYTES;
-      for (int c = lane; c < chunks; c += 32) {
-        const int rw = c / (kb_count * 8);          // row within this warp's 16
-        const int rem = c % (kb_count * 8);
-        const int kbl = rem / 8, ch = rem % 8;
-        const int d = (kb_begin + kbl) * 64 + ch * 8;
-        const int kr = pw * 16 + rw;                // row within the tile
-        const int32_t prow = __shfl_sync(0xffffffffu, my_row, rw);
-        const bool ok = prow >= 0 && d < D_QK;
-        cp_async_16(smem_u32(dst + kbl * (C::BN * 128) + sw128_offset(kr, ch)),
-                    ok ? static_cast<const void*>(p.kv + static_cast<int64_t>(prow) * D_QK + d)
-                       : static_cast<const void*>(p.kv),
-                    ok ? 16u : 0u);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&kv_full[s]));
+      // no gather may still be writing this CTA's shared memory when it exits (immediate
+      // unless the loop above was cut short)
+      for (int i = max(0, issued - C::STAGES); i < issued; ++i)
+        mbar_wait(smem_u32(&kv_full[i % C::STAGES]), (i / C::STAGES) & 1, nullptr);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
@@ -388,77 +362,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     const int half = (warp - 4) >> 2;           // keys [32 half, 32 half + 32) of each tile
     const int hrow = quad * 32 + lane;          // head = TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    // row `hrow`, this half, 16-byte chunk c (0..7) of the staged / received partial logits
-    const uint32_t x_row = half * (128 * 128) + hrow * 128;
     constexpr int OC = C::V_HALF / 2;           // O columns this half rescales / stores
     float m_ref = -INFINITY, l_sum = 0.f;
-    float own[32];                              // our partial logits of the tile in flight
-    bool ok = true;
-    // Loads S(j) from TMEM, frees it for the next QK, stages it for the peer; keeps our partial.
-    auto stage_tile = [&](int j) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(s_full), j & 1, &abort_s))) return false;
+    bool ok = !abort_s;
+    for (int i = 0; i < n && ok; ++i) {
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(s_full), i & 1, &abort_s));
+      if (!ok) break;
       tc_fence_after();
-      uint32_t u[32];
-      tmem_ld32(lane_addr + C::S_COL + half * 32, u);
-      tmem_wait_ld();
+      float sv[32];
+      {
+        uint32_t u[32];
+        tmem_ld32(lane_addr + C::S_COL + half * 32, u);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) own[e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(u[e]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_empty));
-      if (j >= 1 &&
-          !__all_sync(0xffffffffu, mbar_wait(smem_u32(stage_free), (j - 1) & 1, &abort_s)))
-        return false;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<float4*>(sXout + x_row + ((c ^ (hrow & 7)) << 4)) =
-            make_float4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(staged));
-      return true;
-    };
-    if (n > 0) ok = stage_tile(0);
-    for (int i = 0; i < n && ok; ++i) {
-      float sv[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) sv[e] = own[e];
-      // start the swap of the next tile before working on this one
-      if (i + 1 < n) {
-        ok = stage_tile(i + 1);
-        if (!ok) break;
-      }
-      const int xb = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait<true>(smem_u32(&x_full[xb]), (i >> 1) & 1, &abort_s));
-      if (!ok) break;
-      if (warp == 4 && lane == 0 && i + 2 < n)
-        mbar_arrive_expect_tx(smem_u32(&x_full[xb]), C::X_BYTES);   // arm tile i+2
-      // the producers' invalid-row bits of this tile: observe its kv_full phase first (the
-      // stage is not refilled before PV(i), which needs this tile's P)
-      const int st = i % C::STAGES;
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&kv_full[st]), (i / C::STAGES) & 1, &abort_s));
-      if (!ok) break;
-      const uint64_t bad = static_cast<uint64_t>(sBad[st * 4 + 0]) |
-                           (static_cast<uint64_t>(sBad[st * 4 + 1]) << 16) |
-                           (static_cast<uint64_t>(sBad[st * 4 + 2]) << 32) |
-                           (static_cast<uint64_t>(sBad[st * 4 + 3]) << 48);
-      const uint64_t vmask = sMask[sTiles[i]] & ~bad;
-      const uint32_t vbits = static_cast<uint32_t>(vmask >> (32 * half));
-      const uint8_t* xin = sXin + xb * C::X_BYTES;
+      const uint32_t vbits = static_cast<uint32_t>(sMask[sTiles[i]] >> (32 * half));
       float m_half = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float4 o = *reinterpret_cast<const float4*>(xin + x_row + ((c ^ (hrow & 7)) << 4));
-        const float ov[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 4 * c + e;
-          // both CTAs add rank 0's partial to rank 1's: bit-identical logits in both
-          const float full_s = rank == 0 ? sv[j] + ov[e] : ov[e] + sv[j];
-          sv[j] = ((vbits >> j) & 1u) ? full_s * p.scale_log2 : -INFINITY;
-          m_half = fmaxf(m_half, sv[j]);
-        }
+      for (int j = 0; j < 32; ++j) {
+        sv[j] = ((vbits >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
+        m_half = fmaxf(m_half, sv[j]);
       }
-      mbar_arrive(smem_u32(&xin_read[xb]));
       // row max over both halves (double-buffered by tile parity)
       float* red = sRed + (i & 1) * 256;
       red[half * 128 + hrow] = m_half;
@@ -526,7 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     float* po = nullptr;
     if (p.part_o != nullptr)
       po = p.part_o + ((static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow) * D_V +
-           rank * C::V_HALF;
+           vh * C::V_HALF;
     for (int c0 = half * OC; c0 < (half + 1) * OC; c0 += 32) {
       float o[32];
       if (ok && n > 0) {
@@ -545,7 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
         for (int j = 0; j < 32; j += 4)
           *reinterpret_cast<float4*>(po + c0 + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
       } else {
-        __nv_bfloat16* dst = p.out + orow * D_V + rank * C::V_HALF + c0;
+        __nv_bfloat16* dst = p.out + orow * D_V + vh * C::V_HALF + c0;
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
           uint32_t pk[4];
@@ -558,16 +486,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
         }
       }
     }
-    if (write && rank == 0 && half == 0) {
+    if (write && vh == 0 && half == 0) {
       if (p.part_lse != nullptr)
         p.part_lse[(static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow] = lse_v;
       else
         p.lse[orow] = lse_v;
     }
   }
+  if (threadIdx.x == 0) mbar_wait(smem_u32(q_bar), 0, nullptr);   // Q has landed
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // no remote access to this CTA's shared memory after this point
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
