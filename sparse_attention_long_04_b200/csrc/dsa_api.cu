@@ -392,14 +392,13 @@ dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* 
     prm.part_o = static_cast<float*>(ws);
     prm.part_lse = prm.part_o + size_t(splits) * row_count * d.h * D_V;
   }
-  // latent rows gathered four at a time (64 dims x 1 row boxes); Q in 64-dim x 128-head boxes
-  CUtensorMap kv_map, q_map;
-  if (make_row_map(&kv_map, kv, uint64_t(s.num_kv_rows), D_QK * 2, 128, 1) != DSA_OK ||
-      make_row_map(&q_map, q, uint64_t(s.total_rows) * d.h, D_QK * 2, 128, 128) != DSA_OK)
+  // Q in 64-dim x 128-head boxes
+  CUtensorMap q_map;
+  if (make_row_map(&q_map, q, uint64_t(s.total_rows) * d.h, D_QK * 2, 128, 128) != DSA_OK)
     return DSA_ERR_CUDA;
   auto k = dsa_sparse_mla_kernel<D_QK, D_V>;
   if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
-  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(kv_map, q_map, prm);
+  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(q_map, prm);
   if (launch_status() != DSA_OK) return DSA_ERR_CUDA;
   if (splits > 1) {
     dsa_mla_combine_kernel<D_V><<<dim3(row_count, d.h), 128, 0, st>>>(prm);

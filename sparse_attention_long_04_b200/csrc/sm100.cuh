@@ -167,6 +167,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Whole-warp wait: lane 0 alone polls (one shared-memory request per poll instead of 32), then
+// the warp synchronises; all lanes return the same result.
+template <bool kCluster = false>
+__device__ __forceinline__ bool warp_mbar_wait(uint32_t bar, uint32_t parity,
+                                               const volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31u) == 0) ok = mbar_wait<kCluster>(bar, parity, abort) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();   // orders the other lanes after lane 0's acquire
+  return ok != 0;
+}
+
 // ---------------------------------------------------------------------------- proxies, cluster
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -239,6 +251,11 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(src_bytes)
                : "memory");
+}
+// Arrives on the mbarrier once all of this thread's earlier cp.async copies have landed (the
+// arrival is one of the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
 template <int N>

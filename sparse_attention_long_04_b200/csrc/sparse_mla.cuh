@@ -16,19 +16,24 @@
 //   Q (128 heads x 576 bf16) is the QK A operand: TMA brings it in as 128-byte-swizzled 64-dim
 //   blocks; the first KBT blocks move on into Tensor Memory (2 bf16 per column), the rest stay
 //   in shared memory.  Every selected key is resolved to its physical cache row once, up front
-//   (invalid keys borrow a valid row of their tile and are masked out of the softmax); the rows
-//   of each 64-key tile (all dims) are then gathered by TMA, four rows per instruction, into a
-//   2-stage ring.  Per tile: S = Q K^T (tcgen05 bf16, M = 128 heads, N = 64 keys, fp32 in
-//   TMEM), an online softmax (thread = head = TMEM lane), P (bf16) back into TMEM, and
-//   O_v += P V_v (A = P from TMEM, N = D_V/2, V read MN-major straight out of the gathered
-//   tile).  Rescaling of O is lazy (only when a tile's max beats the running reference by more
-//   than 2^8, so P <= 256).
+//   (invalid keys borrow a valid row of their tile and are masked out of the softmax).  The
+//   rows of each 64-key tile are gathered with 16-byte cp.async in two parts with their own
+//   2-slot rings: the value dims of this CTA (needed until PV) and the other dims (needed only
+//   by QK, so refilled as soon as QK is done); each copying thread's arrival on the slot's
+//   barrier fires when its copies land, so no producer waits on memory.  Per tile:
+//   S = Q K^T (tcgen05 bf16, M = 128 heads, N = 64 keys, fp32 in TMEM), an online softmax
+//   (thread = head = TMEM lane, all 64 keys), P (bf16) back into TMEM, and O_v += P V_v
+//   (A = P from TMEM, N = D_V/2, V read MN-major straight out of the gathered tile).  Rescaling
+//   of O is lazy (only when a tile's max beats the running reference by more than 2^8, so
+//   P <= 256).
 // TMEM columns: O [0, D_V/2) | S [+64) | P [+32) | Q (KBT x 32 columns).
 // Warp roles per CTA (512 threads): warp 0 loads Q and issues QK, warp 2 issues PV, warp 1
-// owns TMEM, warps 4-11 move Q into TMEM and run the softmax (warps 4-7 take keys 0-31 of a
-// tile, warps 8-11 keys 32-63) and the epilogue, warps 12-15 resolve the keys and gather (warp
-// w: rows [16w, 16w + 16) of every tile).  Grid: x = 2 * row + v, y = split-KV slice.
+// owns TMEM, warps 4-7 move Q into TMEM, run the softmax and the epilogue, warps 8-15 resolve
+// the keys, then gather rows [16w, 16w + 16) of every tile: warps 8-11 the QK-only dims,
+// warps 12-15 the value dims.  Grid: x = 2 * row + v, y = split-KV slice.
 #pragma once
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace dsa {
@@ -61,6 +66,7 @@ struct MlaCfg {
   static constexpr int KB_ALL = (D_QK + 63) / 64;     // 64-element k-blocks of a latent row
   static constexpr int V_HALF = D_V / 2;              // value dims per CTA
   static constexpr int VKB = V_HALF / 64;             // value k-blocks per CTA
+  static constexpr int KK = KB_ALL - VKB;             // QK-only k-blocks
   static constexpr int BN = 64;                       // keys per tile
   static constexpr int STAGES = 2;
   static constexpr int MAX_TILES = 32;                // topk <= 2048
@@ -73,48 +79,47 @@ struct MlaCfg {
   static constexpr int KBS = KB_ALL - KBT;                            // Q k-blocks in smem
   static constexpr int TMEM_COLS = Q_COL + KBT * 32 <= 256 ? 256 : 512;
   static constexpr int KB_BYTES = BN * 128;                           // one k-block of a tile
-  static constexpr int KV_STAGE_BYTES = KB_ALL * KB_BYTES;
+  static constexpr int K_SLOT_BYTES = KK * KB_BYTES;
+  static constexpr int V_SLOT_BYTES = VKB * KB_BYTES;
+  static constexpr int RING_BYTES = STAGES * (K_SLOT_BYTES + V_SLOT_BYTES);
   static constexpr int Q_KB_BYTES = 128 * 128;                        // one k-block of Q
   static constexpr int Q_SMEM_BYTES = KBS * Q_KB_BYTES;
-  static constexpr int ROWS_PER_WARP_TX = 16 * KB_ALL * 128;          // gather bytes per warp
-  static constexpr int SMEM_USED = 1024 + Q_SMEM_BYTES + STAGES * KV_STAGE_BYTES +
-                                   MAX_TILES * BN * 4 + MAX_TILES * 12 + 2 * 2 * 128 * 4 +
-                                   2 * 128 * 4 + 256;
+  static constexpr int SMEM_USED = 1024 + Q_SMEM_BYTES + RING_BYTES + MAX_TILES * BN * 4 +
+                                   MAX_TILES * 12 + 256;
   // at least 116 KB, so that one CTA runs per SM (its TMEM allocation never waits)
   static constexpr int SMEM_BYTES = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
   static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
   static_assert(Q_COL + KBT * 32 <= 512, "TMEM columns");
-  static_assert(KBT * Q_KB_BYTES <= STAGES * KV_STAGE_BYTES, "Q staging fits the gather ring");
+  static_assert(KBT * Q_KB_BYTES <= RING_BYTES, "Q staging fits the gather rings");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 template <int D_QK, int D_V>
 __global__ void __launch_bounds__(512, 1)
-    dsa_sparse_mla_kernel(const __grid_constant__ CUtensorMap kv_map,
-                          const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
+    dsa_sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
   using C = MlaCfg<D_QK, D_V>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;                                           // [KBS][128 heads][128 B]
-  uint8_t* sKV = sQ + C::Q_SMEM_BYTES;                          // [STAGES] gathered tiles
-  int32_t* sPhys = reinterpret_cast<int32_t*>(sKV + C::STAGES * C::KV_STAGE_BYTES);  // [topk]
+  uint8_t* sRing = sQ + C::Q_SMEM_BYTES;                        // gather rings (Q staging first)
+  uint8_t* sK = sRing;                                          // [STAGES][KK k-blocks]
+  uint8_t* sV = sRing + C::STAGES * C::K_SLOT_BYTES;            // [STAGES][VKB k-blocks]
+  int32_t* sPhys = reinterpret_cast<int32_t*>(sRing + C::RING_BYTES);             // [topk]
   uint64_t* sMask = reinterpret_cast<uint64_t*>(sPhys + C::MAX_TILES * C::BN);   // [32]
   int32_t* sTiles = reinterpret_cast<int32_t*>(sMask + C::MAX_TILES);            // [32]
-  float* sRed = reinterpret_cast<float*>(sTiles + C::MAX_TILES);        // [2][2][128]
-  float* sLsum = sRed + 2 * 2 * 128;                            // [2][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sLsum + 2 * 128);
-  uint64_t* kv_full = bars;          // [2] 4 producer arrivals + gathered bytes
-  uint64_t* kv_empty = bars + 2;     // [2] PV commit
-  uint64_t* s_full = bars + 4;       // QK commit
-  uint64_t* s_empty = bars + 5;      // 8 softmax warps
-  uint64_t* p_full = bars + 6;       // 256 softmax threads
-  uint64_t* pv_done = bars + 7;      // PV commit
-  uint64_t* mx_bar = bars + 8;       // 256 arrivals per tile: both halves' partial max
-  uint64_t* fin_bar = bars + 9;      // 256 arrivals: both halves' partial sums
-  uint64_t* qk_fin = bars + 10;
-  uint64_t* pv_fin = bars + 11;
-  uint64_t* q_bar = bars + 12;       // 1 arrival + Q bytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sTiles + C::MAX_TILES);
+  uint64_t* k_full = bars;           // [2] 128 K-part threads (each when its copies land)
+  uint64_t* k_empty = bars + 2;      // [2] QK commit
+  uint64_t* v_full = bars + 4;       // [2] 128 V-part threads (each when its copies land)
+  uint64_t* v_empty = bars + 6;      // [2] PV commit
+  uint64_t* s_full = bars + 8;       // QK commit
+  uint64_t* s_empty = bars + 9;      // 4 softmax warps
+  uint64_t* p_full = bars + 10;      // 128 softmax threads
+  uint64_t* pv_done = bars + 11;     // PV commit
+  uint64_t* qk_fin = bars + 12;
+  uint64_t* pv_fin = bars + 13;
+  uint64_t* q_bar = bars + 14;       // 1 arrival + Q bytes
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int n_act_s;
@@ -147,15 +152,15 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(smem_u32(&kv_full[i]), 4);
-      mbar_init(smem_u32(&kv_empty[i]), 1);
+      mbar_init(smem_u32(&k_full[i]), 128);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 128);
+      mbar_init(smem_u32(&v_empty[i]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(s_empty), 8);
-    mbar_init(smem_u32(p_full), 256);
+    mbar_init(smem_u32(s_empty), 4);
+    mbar_init(smem_u32(p_full), 128);
     mbar_init(smem_u32(pv_done), 1);
-    mbar_init(smem_u32(mx_bar), 256);
-    mbar_init(smem_u32(fin_bar), 256);
     mbar_init(smem_u32(qk_fin), 1);
     mbar_init(smem_u32(pv_fin), 1);
     mbar_init(smem_u32(q_bar), 1);
@@ -165,41 +170,57 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 1) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
   __syncthreads();
   if (threadIdx.x == 0) {
-    // ---- Q: blocks [0, KBT) into the (still idle) gather ring, the rest into sQ
-    tma_prefetch_desc(&kv_map);
+    // ---- Q: blocks [0, KBT) into the (still idle) gather rings, the rest into sQ
     tma_prefetch_desc(&q_map);
     mbar_arrive_expect_tx(smem_u32(q_bar), C::KB_ALL * C::Q_KB_BYTES);
     for (int kb = 0; kb < C::KB_ALL; ++kb) {
-      uint8_t* dst = kb < C::KBT ? sKV + kb * C::Q_KB_BYTES : sQ + (kb - C::KBT) * C::Q_KB_BYTES;
+      uint8_t* dst = kb < C::KBT ? sRing + kb * C::Q_KB_BYTES : sQ + (kb - C::KBT) * C::Q_KB_BYTES;
       tma_load_2d(smem_u32(dst), &q_map, smem_u32(q_bar), kb * 128, row * p.h);
     }
   }
-  if (warp >= 12) {
-    // ---- every selected key -> physical row (or -1), 16 keys per thread, loads in flight
-    const int t = threadIdx.x - 384;
-    for (int e = t; e < p.topk; e += 128) {
-      const int v = irow[e];
-      int64_t phys = -1;
-      if (v >= 0 && v < n_keys) {
-        if (p.decode && p.block_table != nullptr) {
-          const int64_t id = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
-                                   v / p.block_size);
-          phys = id < 0 ? -1 : id * p.block_size + v % p.block_size;
-        } else {
-          phys = key_base + v;
-        }
-        if (phys >= p.num_kv_rows) phys = -1;
-        if (phys < 0 && p.status) atomicOr(p.status, kStatusBadIndex);
-      } else if (v >= n_keys && p.status) {
-        atomicOr(p.status, kStatusBadIndex);
-      }
-      sPhys[e] = static_cast<int32_t>(phys);
+  if (warp >= 8) {
+    // ---- every selected key -> physical row (or -1): 8 keys per thread, all index loads in
+    // flight together, then all block-table loads
+    const int t = threadIdx.x - 256;
+    constexpr int KPT = C::MAX_TILES * C::BN / 256;
+    int v[KPT];
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int e = t + 256 * j;
+      v[j] = e < p.topk ? irow[e] : -1;
     }
+    int64_t phys[KPT];
+    bool bad_idx = false;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      phys[j] = -1;
+      if (v[j] >= n_keys) bad_idx = true;
+      if (v[j] >= 0 && v[j] < n_keys) {
+        if (p.decode && p.block_table != nullptr)
+          phys[j] = __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks +
+                          v[j] / p.block_size);
+        else
+          phys[j] = key_base + v[j];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      int64_t ph = phys[j];
+      if (v[j] >= 0 && v[j] < n_keys) {
+        if (p.decode && p.block_table != nullptr)
+          ph = ph < 0 ? -1 : ph * p.block_size + v[j] % p.block_size;
+        if (ph >= p.num_kv_rows) ph = -1;
+        if (ph < 0) bad_idx = true;
+      }
+      const int e = t + 256 * j;
+      if (e < p.topk) sPhys[e] = static_cast<int32_t>(ph);
+    }
+    if (bad_idx && p.status) atomicOr(p.status, kStatusBadIndex);
   }
   __syncthreads();
-  if (warp >= 12) {
+  if (warp >= 8) {
     // ---- per tile: the valid-key mask; invalid keys borrow the tile's first valid row
-    for (int tt = warp - 12; tt < n_tiles_all; tt += 4) {
+    for (int tt = warp - 8; tt < n_tiles_all; tt += 8) {
       int32_t* ph = sPhys + tt * C::BN;
       const int32_t a0 = ph[lane], a1 = ph[32 + lane];
       const uint32_t lo = __ballot_sync(0xffffffffu, a0 >= 0);
@@ -230,26 +251,25 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = t0; i < t1; ++i) sTiles[i - t0] = sTiles[i];
     n_act_s = t1 - t0;
   }
-  if (warp >= 4 && warp < 12) {
+  if (warp >= 4 && warp < 8) {
     // ---- Q blocks [0, KBT) from the staging area into TMEM: head = lane, dim d in column
-    // Q_COL + d / 2 (half h of the warps takes blocks h, h + 2, ...)
+    // Q_COL + d / 2
     const int hrow = (warp & 3) * 32 + lane;
-    const int half = (warp - 4) >> 2;
     const uint32_t lane_addr = tmem_base_s + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(q_bar), 0, &abort_s))) {
+    if (!(warp_mbar_wait(smem_u32(q_bar), 0, &abort_s))) {
       abort_s = 1;
       if (p.status) atomicOr(p.status, kStatusTimeout);
     } else {
-      for (int kb = half; kb < C::KBT; kb += 2) {
+      for (int kb = 0; kb < C::KBT; ++kb) {
         uint32_t u[32];
-        const uint8_t* src = sKV + kb * C::Q_KB_BYTES;
+        const uint8_t* src = sRing + kb * C::Q_KB_BYTES;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src + sw128_offset(hrow, ch));
-          u[4 * ch + 0] = v.x;
-          u[4 * ch + 1] = v.y;
-          u[4 * ch + 2] = v.z;
-          u[4 * ch + 3] = v.w;
+          const uint4 q4 = *reinterpret_cast<const uint4*>(src + sw128_offset(hrow, ch));
+          u[4 * ch + 0] = q4.x;
+          u[4 * ch + 1] = q4.y;
+          u[4 * ch + 2] = q4.z;
+          u[4 * ch + 3] = q4.w;
         }
         tmem_st32(lane_addr + C::Q_COL + kb * 32, u);
       }
@@ -257,7 +277,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();   // the staging area is free for the gather ring from here on
+  __syncthreads();   // the staging area is free for the gather rings from here on
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
   const int n = abort_s ? 0 : n_act_s;
@@ -267,27 +287,41 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f32acc(1 /* bf16 */, 128, C::BN, 0, 0);
       const uint32_t qa = smem_u32(sQ);
+      const int v0 = vh * C::VKB;                 // first value k-block of this CTA
       bool ok = n == 0 || mbar_wait(smem_u32(q_bar), 0, &abort_s);
       for (int i = 0; i < n && ok; ++i) {
         const int s = i % C::STAGES;
-        ok = mbar_wait(smem_u32(&kv_full[s]), (i / C::STAGES) & 1, &abort_s);
+        const uint32_t ph = (i / C::STAGES) & 1;
+        ok = mbar_wait(smem_u32(&k_full[s]), ph, &abort_s) &&
+             mbar_wait(smem_u32(&v_full[s]), ph, &abort_s);
         if (ok && i >= 1) ok = mbar_wait(smem_u32(s_empty), (i - 1) & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t ka = smem_u32(sKV + s * C::KV_STAGE_BYTES);
-        for (int kb = 0; kb < C::KBT; ++kb)
+        fence_proxy_async_smem();   // the gathered rows were written by cp.async
+        const uint32_t ka = smem_u32(sK + s * C::K_SLOT_BYTES);
+        const uint32_t va = smem_u32(sV + s * C::V_SLOT_BYTES);
+        // k-block kb of the tile: a value block of this CTA in the V slot, else the K slot
+        auto kb_addr = [&](int kb) -> uint32_t {
+          if (kb >= v0 && kb < v0 + C::VKB) return va + (kb - v0) * C::KB_BYTES;
+          return ka + (kb < v0 ? kb : kb - C::VKB) * C::KB_BYTES;
+        };
+        for (int kb = 0; kb < C::KBT; ++kb) {
+          const uint32_t ba = kb_addr(kb);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_bf16_ts(tmem + C::S_COL, tmem + C::Q_COL + kb * 32 + k * 8,
-                         sdesc_sw128(ka + kb * C::KB_BYTES + k * 32, 16, 1024), idesc,
-                         (kb | k) != 0);
-        for (int kb = C::KBT; kb < C::KB_ALL; ++kb)
+                         sdesc_sw128(ba + k * 32, 16, 1024), idesc, (kb | k) != 0);
+        }
+        for (int kb = C::KBT; kb < C::KB_ALL; ++kb) {
+          const uint32_t ba = kb_addr(kb);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_bf16(tmem + C::S_COL,
                       sdesc_sw128(qa + (kb - C::KBT) * C::Q_KB_BYTES + k * 32, 16, 1024),
-                      sdesc_sw128(ka + kb * C::KB_BYTES + k * 32, 16, 1024), idesc, 1u);
+                      sdesc_sw128(ba + k * 32, 16, 1024), idesc, 1u);
+        }
         umma_commit(smem_u32(s_full));
+        umma_commit(smem_u32(&k_empty[s]));
       }
       if (!ok) {
         abort_s = 1;
@@ -306,12 +340,12 @@ __global__ void __launch_bounds__(512, 1)
         ok = mbar_wait(smem_u32(p_full), i & 1, &abort_s);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t va = smem_u32(sKV + s * C::KV_STAGE_BYTES) + vh * C::VKB * C::KB_BYTES;
+        const uint32_t va = smem_u32(sV + s * C::V_SLOT_BYTES);
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k)
           umma_bf16_ts(tmem, tmem + C::P_COL + k * 8,
                        sdesc_sw128(va + k * 16 * 128, C::KB_BYTES, 1024), idesc, (i | k) != 0);
-        umma_commit(smem_u32(&kv_empty[s]));
+        umma_commit(smem_u32(&v_empty[s]));
         umma_commit(smem_u32(pv_done));
       }
       if (!ok) {
@@ -321,82 +355,90 @@ __global__ void __launch_bounds__(512, 1)
       umma_commit(smem_u32(pv_fin));
       mbar_wait(smem_u32(pv_fin), 0, nullptr);
     }
-  } else if (warp >= 12) {
+  } else if (warp >= 8) {
     // ------------------------------------------------------------ gather producers
-    // Lane 0 of producer warp w gathers rows [16w, 16w + 16) of each tile: 4 rows x 64 dims
-    // per TMA instruction, KB_ALL k-blocks.
-    if (lane == 0) {
-      const int pw = warp - 12;
-      bool ok = true;
-      int issued = 0;
-      for (int i = 0; i < n && ok; ++i) {
-        const int s = i % C::STAGES;
-        if (i >= C::STAGES)
-          ok = mbar_wait(smem_u32(&kv_empty[s]), ((i / C::STAGES) - 1) & 1, &abort_s);
-        if (!ok) break;
-        const uint32_t bar = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(bar, C::ROWS_PER_WARP_TX);
-        const int32_t* ph = sPhys + sTiles[i] * C::BN + pw * 16;
-        const uint32_t dst0 = smem_u32(sKV + s * C::KV_STAGE_BYTES) + pw * 16 * 128;
+    // Warp 8 + 4 part + w copies rows [16w, 16w + 16) of each tile: part 0 the QK-only k-blocks
+    // (K slot), part 1 this CTA's value k-blocks (V slot), 16-byte cp.async per lane; each lane
+    // then arrives on the slot's full barrier once its copies have landed.
+    const int part = (warp - 8) >> 2;
+    const int pw = (warp - 8) & 3;
+    const int ch = lane & 7;                    // 16-byte chunk of a 128-byte row block
+    const int rsub = lane >> 3;                 // rows rsub, rsub + 4, rsub + 8, rsub + 12
+    uint64_t* full = part == 0 ? k_full : v_full;
+    uint64_t* empty = part == 0 ? k_empty : v_empty;
+    // one tile's part: rows [16 pw, 16 pw + 16), NKB k-blocks (latent-row block kb_of(ks))
+    auto copy_part = [&](auto nkb_c, uint8_t* dst, const int32_t* ph, auto kb_of) {
+      constexpr int NKB = decltype(nkb_c)::value;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int4 rr = *reinterpret_cast<const int4*>(ph + 4 * g);
-          for (int kb = 0; kb < C::KB_ALL; ++kb)
-            tma_gather4(dst0 + kb * C::KB_BYTES + g * 512, &kv_map, bar, kb * 128, rr.x, rr.y,
-                        rr.z, rr.w);
+      for (int j = 0; j < 4; ++j) {
+        const int rr = rsub + 4 * j;
+        const __nv_bfloat16* src = p.kv + static_cast<int64_t>(ph[rr]) * D_QK + ch * 8;
+        const uint32_t drow = smem_u32(dst) + sw128_offset(pw * 16 + rr, ch);
+#pragma unroll
+        for (int ks = 0; ks < NKB; ++ks) {
+          const int kb = kb_of(ks);
+          const bool in = kb * 64 + ch * 8 < D_QK;
+          cp_async_16(drow + ks * C::KB_BYTES, in ? static_cast<const void*>(src + kb * 64)
+                                                  : static_cast<const void*>(p.kv),
+                      in ? 16u : 0u);
         }
-        ++issued;
       }
-      if (!ok) {
-        abort_s = 1;
-        if (p.status) atomicOr(p.status, kStatusTimeout);
+    };
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int s = i % C::STAGES;
+      if (i >= C::STAGES &&
+          !(warp_mbar_wait(smem_u32(&empty[s]), ((i / C::STAGES) - 1) & 1,
+                                             &abort_s))) {
+        ok = false;
+        break;
       }
-      // no gather may still be writing this CTA's shared memory when it exits (immediate
-      // unless the loop above was cut short)
-      for (int i = max(0, issued - C::STAGES); i < issued; ++i)
-        mbar_wait(smem_u32(&kv_full[i % C::STAGES]), (i / C::STAGES) & 1, nullptr);
+      const int32_t* ph = sPhys + sTiles[i] * C::BN + pw * 16;
+      if (part == 0)   // the QK-only k-blocks: all but this CTA's value blocks
+        copy_part(std::integral_constant<int, C::KK>{}, sK + s * C::K_SLOT_BYTES, ph,
+                  [&](int ks) { return ks < vh * C::VKB ? ks : ks + C::VKB; });
+      else             // this CTA's value k-blocks
+        copy_part(std::integral_constant<int, C::VKB>{}, sV + s * C::V_SLOT_BYTES, ph,
+                  [&](int ks) { return vh * C::VKB + ks; });
+      cp_async_arrive_noinc(smem_u32(&full[s]));
     }
+    if (!ok) {
+      abort_s = 1;
+      if (p.status) atomicOr(p.status, kStatusTimeout);
+    }
+    cp_async_wait<0>();   // nothing may still be writing this CTA's shared memory at exit
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int quad = warp & 3;
-    const int half = (warp - 4) >> 2;           // keys [32 half, 32 half + 32) of each tile
-    const int hrow = quad * 32 + lane;          // head = TMEM lane
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    constexpr int OC = C::V_HALF / 2;           // O columns this half rescales / stores
+    const int hrow = (warp & 3) * 32 + lane;    // head = TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = !abort_s;
     for (int i = 0; i < n && ok; ++i) {
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(s_full), i & 1, &abort_s));
+      ok = (warp_mbar_wait(smem_u32(s_full), i & 1, &abort_s));
       if (!ok) break;
       tc_fence_after();
-      float sv[32];
-      {
-        uint32_t u[32];
-        tmem_ld32(lane_addr + C::S_COL + half * 32, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(u[e]);
-      }
+      uint32_t su[2][32];                       // S of keys [32 hh, 32 hh + 32)
+      tmem_ld32(lane_addr + C::S_COL, su[0]);
+      tmem_ld32(lane_addr + C::S_COL + 32, su[1]);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_empty));
-      const uint32_t vbits = static_cast<uint32_t>(sMask[sTiles[i]] >> (32 * half));
-      float m_half = -INFINITY;
+      const uint64_t vmask = sMask[sTiles[i]];
+      float m_tile = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        sv[j] = ((vbits >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
-        m_half = fmaxf(m_half, sv[j]);
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t vb = static_cast<uint32_t>(vmask >> (32 * hh));
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float x = ((vb >> j) & 1u) ? __uint_as_float(su[hh][j]) * p.scale_log2 : -INFINITY;
+          su[hh][j] = __float_as_uint(x);
+          m_tile = fmaxf(m_tile, x);
+        }
       }
-      // row max over both halves (double-buffered by tile parity)
-      float* red = sRed + (i & 1) * 256;
-      red[half * 128 + hrow] = m_half;
-      mbar_arrive(smem_u32(mx_bar));
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(mx_bar), i & 1, &abort_s));
-      if (!ok) break;
-      const float m_tile = fmaxf(red[hrow], red[128 + hrow]);
       // P and O are free once PV(i-1) has completed
       if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (i - 1) & 1, &abort_s));
+        ok = (warp_mbar_wait(smem_u32(pv_done), (i - 1) & 1, &abort_s));
         if (!ok) break;
         tc_fence_after();
       }
@@ -407,8 +449,25 @@ __global__ void __launch_bounds__(512, 1)
         l_sum *= alpha;
         m_ref = m_tile;
       }
+      float rowsum = 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          // the denominator sums the fp32 probabilities; only the PV operand is rounded
+          const float p0 = exp2f(__uint_as_float(su[hh][2 * e]) - m_ref);
+          const float p1 = exp2f(__uint_as_float(su[hh][2 * e + 1]) - m_ref);
+          rowsum += p0 + p1;
+          const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&two);
+        }
+        tmem_st16(lane_addr + C::P_COL + hh * 16, pk);
+      }
+      l_sum += rowsum;
+      // O to the new reference (after P, so the logits are no longer live; before PV(i))
       if (i >= 1 && __any_sync(0xffffffffu, need)) {
-        for (int c0 = half * OC; c0 < (half + 1) * OC; c0 += 32) {
+        for (int c0 = 0; c0 < C::V_HALF; c0 += 32) {
           uint32_t u[32];
           tmem_ld32(lane_addr + c0, u);
           tmem_wait_ld();
@@ -417,19 +476,6 @@ __global__ void __launch_bounds__(512, 1)
           tmem_st32(lane_addr + c0, u);
         }
       }
-      uint32_t pk[16];
-      float rowsum = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        // the denominator sums the fp32 probabilities; only the PV operand is rounded
-        const float p0 = exp2f(sv[2 * e] - m_ref);
-        const float p1 = exp2f(sv[2 * e + 1] - m_ref);
-        rowsum += p0 + p1;
-        const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
-        pk[e] = *reinterpret_cast<const uint32_t*>(&two);
-      }
-      l_sum += rowsum;
-      tmem_st16(lane_addr + C::P_COL + half * 16, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
@@ -438,24 +484,20 @@ __global__ void __launch_bounds__(512, 1)
       abort_s = 1;
       if (p.status) atomicOr(p.status, kStatusTimeout);
     }
-    // ---- epilogue: l = l(keys 0-31) + l(keys 32-63), the same order in both halves
-    sLsum[half * 128 + hrow] = l_sum;
-    mbar_arrive(smem_u32(fin_bar));
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(fin_bar), 0, &abort_s));
-    const float l_tot = ok ? sLsum[hrow] + sLsum[128 + hrow] : 0.f;
+    // ---- epilogue
     const bool write = hrow < p.h;
     const int64_t orow = static_cast<int64_t>(row) * p.h + hrow;
     if (ok && n > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(pv_done), (n - 1) & 1, &abort_s));
+      ok = (warp_mbar_wait(smem_u32(pv_done), (n - 1) & 1, &abort_s));
     tc_fence_after();
-    const float inv_l = (n > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+    const float inv_l = (ok && n > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
     const float lse_v =
-        (n > 0 && l_tot > 0.f) ? (m_ref + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        (ok && n > 0 && l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
     float* po = nullptr;
     if (p.part_o != nullptr)
       po = p.part_o + ((static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow) * D_V +
            vh * C::V_HALF;
-    for (int c0 = half * OC; c0 < (half + 1) * OC; c0 += 32) {
+    for (int c0 = 0; c0 < C::V_HALF; c0 += 32) {
       float o[32];
       if (ok && n > 0) {
         uint32_t u[32];
@@ -486,7 +528,7 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    if (write && vh == 0 && half == 0) {
+    if (write && vh == 0) {
       if (p.part_lse != nullptr)
         p.part_lse[(static_cast<int64_t>(split) * p.row_count + r) * p.h + hrow] = lse_v;
       else
