@@ -18,7 +18,7 @@ namespace {
 using namespace dsa;
 
 constexpr int kMaxDevices = 64;
-constexpr size_t kSlabBudget = size_t(96) << 20;   // prefill score slab per row chunk
+constexpr size_t kSlabBudget = size_t(256) << 20;  // prefill score slab per row chunk
 
 struct DeviceInfo {
   int sm_count = 0;
@@ -431,9 +431,15 @@ struct ForwardPlan {
 
 int64_t round4(int64_t x) { return (x + 3) / 4 * 4; }
 
-int64_t chunk_rows_for(int64_t L) {
+// Prefill rows per chunk of a sequence of L rows: as many as the slab budget allows; when the
+// sequence needs several chunks, a multiple of sm_count / 2 rows, so that each chunk's attention
+// launch (two CTAs per row, one per SM) fills whole waves.
+int64_t chunk_rows_for(int64_t L, int sm_count) {
   const int64_t ld = round4(L);
-  return std::max<int64_t>(1, std::min<int64_t>(L, int64_t(kSlabBudget / (ld * 4))));
+  const int64_t cap = std::max<int64_t>(1, int64_t(kSlabBudget / (ld * 4)));
+  if (cap >= L) return L;
+  const int64_t wave = std::max(1, sm_count / 2);
+  return cap >= wave ? cap / wave * wave : cap;
 }
 
 ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count) {
@@ -449,7 +455,7 @@ ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count)
     for (int b = 0; b < s.batch; ++b) {
       const int64_t L = cu[b + 1] - cu[b];
       if (L <= 0) continue;
-      const int64_t rows = chunk_rows_for(L);
+      const int64_t rows = chunk_rows_for(L, sm_count);
       p.slab_floats = std::max(p.slab_floats, rows * round4(L));
       max_rows = std::max(max_rows, rows);
     }
@@ -590,7 +596,7 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
     const int64_t L = cu[b + 1] - cu[b];
     if (L <= 0) continue;
     const int64_t ld = round4(L);
-    const int64_t rows = chunk_rows_for(L);
+    const int64_t rows = chunk_rows_for(L, info.sm_count);
     for (int64_t r0 = 0; r0 < L; r0 += rows) {
       const int32_t row_begin = static_cast<int32_t>(cu[b] + r0);
       const int32_t row_count = static_cast<int32_t>(std::min(rows, L - r0));

@@ -290,6 +290,40 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+      if constexpr (!C::TILE_SPLIT && H_I >= 32 && H_I % 32 == 0) {
+        // all of this warp's columns in one TMEM round trip; the accumulator is free again
+        // before the arithmetic starts
+        constexpr int NCH = COLS / 32;
+        uint32_t r[NCH][32];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) tmem_ld32(lane_addr + a * N + part * COLS + c * 32, r[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[a]));
+        constexpr int CPR = H_I / 32;          // chunks per query row
+#pragma unroll
+        for (int q = 0; q < NCH / CPR; ++q) {
+          float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = q * CPR; c < (q + 1) * CPR; ++c) {
+            const float4* cc = reinterpret_cast<const float4*>(sC + part * COLS + c * 32);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 c4 = cc[j / 4];
+              acc4[0] = fmaf(c4.x, fmaxf(__uint_as_float(r[c][j + 0]), 0.f), acc4[0]);
+              acc4[1] = fmaf(c4.y, fmaxf(__uint_as_float(r[c][j + 1]), 0.f), acc4[1]);
+              acc4[2] = fmaf(c4.z, fmaxf(__uint_as_float(r[c][j + 2]), 0.f), acc4[2]);
+              acc4[3] = fmaf(c4.w, fmaxf(__uint_as_float(r[c][j + 3]), 0.f), acc4[3]);
+            }
+          }
+          const int rr = (part * COLS) / H_I + q;
+          if (rr < rows_in_group && key <= pos_first + rr)
+            p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] =
+                ks * ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
+        }
+        continue;
+      }
       float acc = 0.f;
 #pragma unroll 1
       for (int c0 = 0; c0 < COLS; c0 += 32) {
