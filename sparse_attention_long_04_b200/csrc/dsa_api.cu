@@ -219,7 +219,9 @@ dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_
   DeviceInfo info;
   if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
   CUtensorMap kmap, qmap;
-  if (make_map(&kmap, k_idx, s.num_kv_rows, D_I, 64) != DSA_OK) return DSA_ERR_CUDA;
+  // prefill keys are contiguous: one 128-row box per tile; decode: 64-row (paged) boxes
+  if (make_map(&kmap, k_idx, s.num_kv_rows, D_I, s.mode == DSA_DECODE ? 64 : 128) != DSA_OK)
+    return DSA_ERR_CUDA;
   if (make_map(&qmap, q_idx, uint64_t(s.total_rows) * H_I, D_I, C::N) != DSA_OK)
     return DSA_ERR_CUDA;
   IndexerParams prm{};

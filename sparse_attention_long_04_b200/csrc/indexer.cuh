@@ -18,7 +18,7 @@
 // computes c[t,j], warps 4.. run the epilogue.  Key stages are a ring of STAGES buffers; the
 // accumulators are a ring of ACC buffers in TMEM so the epilogue of tile i overlaps the MMA of
 // later tiles.  Decode (one query row, N = 64) runs two epilogue warpgroups on alternate tiles;
-// prefill (N = 256) splits each tile's columns over two warpgroups.
+// prefill (N = 256) splits each tile's columns over four warpgroups, one query row each.
 #pragma once
 #include "sm100.cuh"
 
@@ -51,7 +51,7 @@ struct IndexerCfg {
   static constexpr int N = H_I * QPG;                 // MMA N: (row, head) columns
   static constexpr int STAGES = QPG == 1 ? 6 : 8;
   static constexpr int ACC = QPG == 1 ? 4 : 2;        // TMEM accumulator ring
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARPS = QPG == 1 ? 8 : 16;    // prefill: one query row per warpgroup
   static constexpr bool TILE_SPLIT = QPG == 1;        // warpgroups take alternate tiles
   static constexpr int EPI_PER_TILE = TILE_SPLIT ? 4 : EPI_WARPS;   // warps reading one tile
   static constexpr int THREADS = (4 + EPI_WARPS) * 32;
@@ -82,10 +82,12 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::Q_BYTES;
   float* sScale = reinterpret_cast<float*>(sK + C::STAGES * C::TILE_BYTES);  // [STAGES][2][80]
-  int64_t* sA0 = reinterpret_cast<int64_t*>(sScale + C::STAGES * C::SCALE_FLOATS);  // [STAGES][2]
-  int32_t* sOff = reinterpret_cast<int32_t*>(sA0 + C::STAGES * 2);   // [STAGES][2]
-  int32_t* sCnt = sOff + C::STAGES * 2;                               // [STAGES][2]
-  float* sC = reinterpret_cast<float*>(sCnt + C::STAGES * 2);
+  // per stage and 64-key half: the cache row of the half's first key, where its scale sits in
+  // the stage's scale buffer, and how many of the half's scales were copied there
+  int64_t* sRow0 = reinterpret_cast<int64_t*>(sScale + C::STAGES * C::SCALE_FLOATS);  // [STAGES][2]
+  int32_t* sFirst = reinterpret_cast<int32_t*>(sRow0 + C::STAGES * 2);   // [STAGES][2]
+  int32_t* sValid = sFirst + C::STAGES * 2;                               // [STAGES][2]
+  float* sC = reinterpret_cast<float*>(sValid + C::STAGES * 2);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(sC + N) + 7) & ~uintptr_t(7));
   uint64_t* full = bars;                      // [STAGES] key tile (and its scales) landed
@@ -176,44 +178,64 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
           break;
         }
         const int tile = t_begin + it;
-        int64_t y[2];
-        bool ok[2];
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          const int blk = tile * 2 + hlf;
-          ok[hlf] = blk < n_blocks;
-          if (!p.decode) {
-            y[hlf] = static_cast<int64_t>(p.key0) + blk * 64;
-          } else if (p.block_table != nullptr) {
-            int64_t id = ok[hlf] ? p.block_table[static_cast<int64_t>(b) * p.max_blocks + blk] : 0;
-            if (ok[hlf] && (id < 0 || (id + 1) * 64 > p.num_kv_rows)) {
-              if (p.status) atomicOr(p.status, kStatusBadIndex);
-              ok[hlf] = false;
-            }
-            y[hlf] = id * 64;
-          } else {
-            y[hlf] = seq_base + blk * 64;
+        float* sbuf = sScale + s * C::SCALE_FLOATS;
+        uint32_t bytes;
+        if (!p.decode) {
+          // prefill: the tile's 128 keys are contiguous rows; one box and one scale copy
+          const int64_t y = static_cast<int64_t>(p.key0) + tile * 128;
+          const int64_t a0 = y & ~int64_t(3);
+          const int64_t avail = p.num_kv_rows - a0;
+          const uint32_t sb = static_cast<uint32_t>((avail < 132 ? avail : int64_t(132)) / 4 * 16);
+          const int lead = static_cast<int>(y - a0);
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            sRow0[s * 2 + hlf] = y + hlf * 64;
+            sFirst[s * 2 + hlf] = lead + hlf * 64;
+            sValid[s * 2 + hlf] = static_cast<int32_t>(sb / 4) - lead - hlf * 64;
           }
-        }
-        // each box's 64 scales: a 16-byte-aligned superset of the rows, inside the cache
-        int64_t a0[2];
-        uint32_t sb[2];
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          a0[hlf] = y[hlf] & ~int64_t(3);
-          const int64_t avail = p.num_kv_rows - a0[hlf];
-          sb[hlf] = ok[hlf] ? static_cast<uint32_t>((avail < 68 ? avail : int64_t(68)) / 4 * 16) : 0u;
-          sOff[s * 2 + hlf] = static_cast<int32_t>(y[hlf] - a0[hlf]);
-          sCnt[s * 2 + hlf] = static_cast<int32_t>(sb[hlf] / 4);
-          sA0[s * 2 + hlf] = a0[hlf];
-        }
-        const uint32_t bytes = (ok[0] ? 64 * D_I : 0) + (ok[1] ? 64 * D_I : 0) + sb[0] + sb[1];
-        mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          if (ok[hlf])
-            tma_load_2d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
-                        smem_u32(&full[s]), 0, static_cast<int32_t>(y[hlf]));
-          if (sb[hlf] > 0)
-            bulk_load_g2s(smem_u32(sScale + s * C::SCALE_FLOATS + hlf * 80),
-                          p.k_scale + a0[hlf], sb[hlf], smem_u32(&full[s]));
+          bytes = 128 * D_I + sb;
+          mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
+          tma_load_2d(smem_u32(sK + s * C::TILE_BYTES), &kmap, smem_u32(&full[s]), 0,
+                      static_cast<int32_t>(y));
+          if (sb > 0) bulk_load_g2s(smem_u32(sbuf), p.k_scale + a0, sb, smem_u32(&full[s]));
+        } else {
+          int64_t y[2];
+          bool ok[2];
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            const int blk = tile * 2 + hlf;
+            ok[hlf] = blk < n_blocks;
+            if (p.block_table != nullptr) {
+              int64_t id = ok[hlf] ? p.block_table[static_cast<int64_t>(b) * p.max_blocks + blk] : 0;
+              if (ok[hlf] && (id < 0 || (id + 1) * 64 > p.num_kv_rows)) {
+                if (p.status) atomicOr(p.status, kStatusBadIndex);
+                ok[hlf] = false;
+              }
+              y[hlf] = ok[hlf] ? id * 64 : 0;
+            } else {
+              y[hlf] = seq_base + blk * 64;
+            }
+          }
+          // each box's 64 scales: a 16-byte-aligned superset of the rows, inside the cache
+          uint32_t sb[2];
+          int64_t a0[2];
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            a0[hlf] = y[hlf] & ~int64_t(3);
+            const int64_t avail = p.num_kv_rows - a0[hlf];
+            sb[hlf] = ok[hlf] ? static_cast<uint32_t>((avail < 68 ? avail : int64_t(68)) / 4 * 16) : 0u;
+            const int lead = static_cast<int>(y[hlf] - a0[hlf]);
+            sRow0[s * 2 + hlf] = y[hlf];
+            sFirst[s * 2 + hlf] = hlf * 80 + lead;
+            sValid[s * 2 + hlf] = static_cast<int32_t>(sb[hlf] / 4) - lead;
+          }
+          bytes = (ok[0] ? 64 * D_I : 0) + (ok[1] ? 64 * D_I : 0) + sb[0] + sb[1];
+          mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            if (ok[hlf])
+              tma_load_2d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
+                          smem_u32(&full[s]), 0, static_cast<int32_t>(y[hlf]));
+            if (sb[hlf] > 0)
+              bulk_load_g2s(smem_u32(sbuf + hlf * 80), p.k_scale + a0[hlf], sb[hlf],
+                            smem_u32(&full[s]));
+          }
         }
         ++issued;
       }
@@ -278,14 +300,14 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
       const int kin = quad * 32 + lane;        // key within the tile
       const int key = (t_begin + it) * 128 + kin;
       const int hb = kin >> 6;
-      const int j = sOff[s * 2 + hb] + (kin & 63);
+      const int j = kin & 63;
       float ks = 0.f;
       if (key < n_keys) {
-        if (j < sCnt[s * 2 + hb]) {
-          ks = sScale[s * C::SCALE_FLOATS + hb * 80 + j];
+        if (j < sValid[s * 2 + hb]) {
+          ks = sScale[s * C::SCALE_FLOATS + sFirst[s * 2 + hb] + j];
         } else {                               // the last rows of the cache: not bulk-copied
-          const int64_t row = sA0[s * 2 + hb] + j;
-          ks = row < p.num_kv_rows ? __ldg(p.k_scale + row) : 0.f;
+          const int64_t row = sRow0[s * 2 + hb] + j;
+          ks = row >= 0 && row < p.num_kv_rows ? __ldg(p.k_scale + row) : 0.f;
         }
       }
       __syncwarp();

@@ -26,6 +26,9 @@ enum : int32_t {
 
 // Wall-clock limit of every wait on an mbarrier or on a peer CTA.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+// mbarrier try_wait suspend-time hint: a waiting thread sleeps until the phase completes or
+// this much time has passed, instead of spinning on issue slots
+constexpr uint32_t kSuspendHintNs = 100000u;       // 100 us
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -72,10 +75,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }

@@ -102,6 +102,27 @@ def test_indexer_decode_paged_ragged(dsa):
     _indexer_case(dsa, wl, [0, 1, 2, 3])
 
 
+def test_indexer_bad_block_reported(dsa):
+    """A block-table entry that is negative or past the cache is skipped and reported as
+    DSA_DEVICE_BAD_INDEX; the other sequences' scores are unaffected."""
+    wl = make_decode(16, 3, [700, 300, 130], FULL, boost=0.01, paged=True, device="cuda",
+                     total_blocks=40)
+    good = oracle.indexer_rows(wl, [1, 2])
+    wl.block_table[0, 3] = -1
+    wl.block_table[0, 5] = 40          # one past the last physical block
+    pb = dsa.problem_of(wl)
+    ld = _ld(wl.max_seqlen)
+    scores = torch.full((3, ld), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert dsa.dsa_indexer_scores(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx, wl.k_scale, 0, 3,
+                                  scores, ld, status) == 0
+    torch.cuda.synchronize()
+    assert int(status.item()) & dsa.DSA_DEVICE_BAD_INDEX
+    sc = to_np(scores)
+    for r in (1, 2):
+        check_scores(sc[r, :len(good[r])], good[r], f"row {r}")
+
+
 def test_indexer_row_subrange(dsa):
     wl = make_prefill(14, [300, 400], FULL, needles=8, device="cuda")
     scores = run_indexer(dsa, wl, rows_begin=250, rows_count=200)
