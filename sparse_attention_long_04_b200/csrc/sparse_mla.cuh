@@ -425,17 +425,30 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_empty));
       const uint64_t vmask = sMask[sTiles[i]];
-      float m_tile = -INFINITY;
+      // the tile max of the unscaled logits (sigma log2 e > 0), as 8 independent partial maxima
+      float mm[8];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t vb = static_cast<uint32_t>(vmask >> (32 * hh));
+      for (int q = 0; q < 8; ++q) mm[q] = -INFINITY;
+      if (vmask == ~0ull) {                     // every key of the tile is valid (the usual case)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float x = ((vb >> j) & 1u) ? __uint_as_float(su[hh][j]) * p.scale_log2 : -INFINITY;
-          su[hh][j] = __float_as_uint(x);
-          m_tile = fmaxf(m_tile, x);
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mm[j & 7] = fmaxf(mm[j & 7], __uint_as_float(su[hh][j]));
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t vb = static_cast<uint32_t>(vmask >> (32 * hh));
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = ((vb >> j) & 1u) ? __uint_as_float(su[hh][j]) : -INFINITY;
+            su[hh][j] = __float_as_uint(x);    // invalid keys: -inf, so p = 0 below
+            mm[j & 7] = fmaxf(mm[j & 7], x);
+          }
         }
       }
+      const float m_tile =
+          fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])),
+                fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7]))) * p.scale_log2;
       // P and O are free once PV(i-1) has completed
       if (i >= 1) {
         ok = (warp_mbar_wait(smem_u32(pv_done), (i - 1) & 1, &abort_s));
@@ -449,21 +462,27 @@ __global__ void __launch_bounds__(512, 1)
         l_sum *= alpha;
         m_ref = m_tile;
       }
-      float rowsum = 0.f;
+      // p = 2^(sigma log2e s - m_ref) (0 for invalid keys); 8 independent partial sums
+      float rs[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) rs[q] = 0.f;
+      const float sc = p.scale_log2, nm = -m_ref;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           // the denominator sums the fp32 probabilities; only the PV operand is rounded
-          const float p0 = exp2f(__uint_as_float(su[hh][2 * e]) - m_ref);
-          const float p1 = exp2f(__uint_as_float(su[hh][2 * e + 1]) - m_ref);
-          rowsum += p0 + p1;
+          const float p0 = exp2f(fmaf(__uint_as_float(su[hh][2 * e]), sc, nm));
+          const float p1 = exp2f(fmaf(__uint_as_float(su[hh][2 * e + 1]), sc, nm));
+          rs[(2 * e) & 7] += p0;
+          rs[(2 * e + 1) & 7] += p1;
           const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
           pk[e] = *reinterpret_cast<const uint32_t*>(&two);
         }
         tmem_st16(lane_addr + C::P_COL + hh * 16, pk);
       }
+      const float rowsum = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       l_sum += rowsum;
       // O to the new reference (after P, so the logits are no longer live; before PV(i))
       if (i >= 1 && __any_sync(0xffffffffu, need)) {
