@@ -42,6 +42,28 @@ def read_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+# ------------------------------------------------------------------------------ ranks
+
+def rank_seed(cfg: int, rank: int) -> int:
+    """Seed of rank `rank`'s own synthetic batch (weak scaling: every rank draws a different
+    batch of the same shape)."""
+    return 1000 + cfg + 7919 * rank
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (the job's time); no collective when world == 1."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the units all ranks processed per second of the slowest rank."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -142,10 +164,10 @@ def run_ours(args, rank, world, local_rank):
         c = CONFIGS[DECODE_CFG]
         wl = make_decode(DECODE_CFG, args.decode_batch, c["ctx"],
                          {k: c[k] for k in ("h_idx", "d_idx", "topk", "h", "d_qk", "d_v")},
-                         c["boost"], c["paged"], dev, seed=1000 + DECODE_CFG + 7919 * rank,
+                         c["boost"], c["paged"], dev, seed=rank_seed(DECODE_CFG, rank),
                          name=f"{c['name']}_B{args.decode_batch}")
     else:
-        wl = make_config(DECODE_CFG, device=dev, seed=1000 + DECODE_CFG + 7919 * rank)
+        wl = make_config(DECODE_CFG, device=dev, seed=rank_seed(DECODE_CFG, rank))
     d = wl.dims
     pb = dsa.problem_of(wl)
     B = wl.batch
@@ -200,13 +222,8 @@ def run_ours(args, rank, world, local_rank):
     k_ms = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
             for e in evs]
     per_kernel = [sum(x[j] for x in k_ms) / len(k_ms) for j in range(3)]
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
-    ms_step = ms_max / args.steps
-    value = world * B / (ms_step / 1e3)
+    ms_step = max_over_ranks(ms, world, dev) / args.steps
+    value = weak_value(world, B, ms_step)
 
     # ---- end to end through the public call, host buffers, copies inside the timed region
     fwd = dsa.Forward(wl, keep_idx=False)
@@ -235,12 +252,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * B / (e2e_ms / args.steps / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = weak_value(world, B, e2e_ms / args.steps)
     st, raw = dsa.dsa_read_device_status(status, stream)
     dsa.check(st, "device status after timing")
 
@@ -296,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
 
 def run_prefill(args, dsa, dev, stream, peaks, rank, world):
     from dsa_workloads import make_config, CONFIGS
-    wl = make_config(PREFILL_CFG, device=dev, seed=1000 + PREFILL_CFG + 7919 * rank)
+    wl = make_config(PREFILL_CFG, device=dev, seed=rank_seed(PREFILL_CFG, rank))
     fwd = dsa.Forward(wl, keep_idx=False)
     steps = max(1, min(args.steps, args.prefill_steps))
     for _ in range(max(1, min(args.warmup, 3))):
@@ -310,19 +323,14 @@ def run_prefill(args, dsa, dev, stream, peaks, rank, world):
         dsa.check(fwd(stream), "prefill forward")
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    ms_step = ms / steps
+    ms_step = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
     st, raw = dsa.dsa_read_device_status(fwd.status, stream)
     dsa.check(st, "prefill device status")
     f8, f16 = prefill_flops(wl.seqlens, wl.dims)
     p8 = 2.0 * peaks["bf16_sustained"]
     ideal_ms = (f8 / (p8 * 1e12) + f16 / (peaks["bf16_sustained"] * 1e12)) * 1e3
     T = wl.total_rows
-    res = {"workload": CONFIGS[PREFILL_CFG]["name"], "value": round(world * T / (ms_step / 1e3), 1),
+    res = {"workload": CONFIGS[PREFILL_CFG]["name"], "value": round(weak_value(world, T, ms_step), 1),
            "unit": "tokens/s", "ms_per_step": round(ms_step, 3), "steps": steps,
            "roofline": {"bound": "tensor", "frac": round(ideal_ms / ms_step, 4),
                         "ideal_ms": round(ideal_ms, 3), "flops_fp8": f8, "flops_bf16": f16,
