@@ -12,6 +12,8 @@ summary):
   indexer_rows      S[t,s] = s_k[s] sum_j w[t,j] s_q[t,j] ReLU(q[t,j].k[s]),  s <= pos(t)
   topk_rows         k largest S per row, ties -> smaller index, all keys if fewer than k
   sparse_mla_rows   MQA-mode attention over the selected latent rows, fp64, with LSE
+  quantize_e4m3     per-row e4m3 quantisation (scale = amax / 448), the decode cache append's
+  cache_append      arithmetic; cache_append writes a decode step's new token into the caches
 
 The C library ``dsa_oracle.c`` does the arithmetic (OpenMP over rows); this module only
 resolves which physical cache row holds logical key s of a sequence and moves bytes.
@@ -56,6 +58,9 @@ def lib():
         L.dsa_oracle_sparse_mla.argtypes = [
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, f64p, f64p]
+        L.dsa_oracle_quantize_e4m3.restype = None
+        L.dsa_oracle_quantize_e4m3.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p]
         L.dsa_oracle_num_threads.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -229,3 +234,53 @@ def forward_rows(wl, rows: Sequence[int]):
     idx = topk_rows([sc[r] for r in rows], wl.dims["topk"])
     o, lse = sparse_mla_rows(wl, rows, idx)
     return sc, idx, o, lse
+
+
+# ---- decode cache append ---------------------------------------------------------------------
+
+def quantize_e4m3(x) -> tuple:
+    """Per-row e4m3 codes and fp32 scales of fp32 rows ``x`` [n, d] (the "FP8 index" input
+    format: one scale per token).  Returns (uint8 [n, d], float32 [n])."""
+    x = np.ascontiguousarray(_np(x), dtype=np.float32)
+    n, d = x.shape
+    codes = np.empty((n, d), dtype=np.uint8)
+    scales = np.empty(n, dtype=np.float32)
+    lib().dsa_oracle_quantize_e4m3(n, d, _ptr(x), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def cache_append(k_cache, k_scale, kv_cache, seq_lens, block_table, max_seqlen: int,
+                 k_new, kv_new, block_size: int = 64):
+    """One decode step's append: for each sequence b the new token sits at position
+    p = seq_lens[b] - 1; its indexer key k_new[b] (fp32) is quantised per token and written
+    with its scale, and its latent row kv_new[b] (bf16 bits) is copied, at the physical row
+    block_table[b, p // bs] * bs + p % bs (b * max_seqlen + p without a table).  Entries
+    whose position or block is outside the caches are skipped.  Returns copies of the three
+    caches and a bool [B] of the skipped entries."""
+    kc, ks, kv = _np(k_cache).copy(), _np(k_scale).copy(), _np(kv_cache).copy()
+    lens = _np(seq_lens).astype(np.int64)
+    bt = _np(block_table)
+    codes, scales = quantize_e4m3(k_new)
+    kvn = _np(kv_new)
+    rows = kc.shape[0]
+    bad = np.zeros(len(lens), dtype=bool)
+    for b, n in enumerate(lens):
+        p = int(n) - 1
+        if p < 0 or p >= max_seqlen:
+            bad[b] = True
+            continue
+        if bt is not None:
+            blk = int(bt[b, p // block_size])
+            phys = blk * block_size + p % block_size
+            if blk < 0 or (blk + 1) * block_size > rows:
+                bad[b] = True
+                continue
+        else:
+            phys = b * max_seqlen + p
+            if phys >= rows:
+                bad[b] = True
+                continue
+        kc[phys] = codes[b]
+        ks[phys] = scales[b]
+        kv[phys] = kvn[b]
+    return kc, ks, kv, bad

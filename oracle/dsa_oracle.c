@@ -22,7 +22,9 @@
  *             weighted sum of the first d_v latent dims, LSE = log sum exp(l_s)
  *
  * Floating point: e4m3 and bf16 inputs are decoded exactly; the indexer runs in fp64 (or
- * in fp32 with index-ordered accumulation when asked), attention runs in fp64.
+ * in fp32 with index-ordered accumulation when asked), attention runs in fp64.  The decode
+ * cache append quantises the new token's indexer key per token to e4m3 ("FP8 index", same
+ * page, pipeline summary) in fp32, the precision the kernel uses for that decision.
  */
 #include <math.h>
 #include <stdint.h>
@@ -197,6 +199,54 @@ void dsa_oracle_sparse_mla(int n_rows, int h, int d_qk, int d_v, double scale,
 }
 
 /* Threads the OpenMP runtime will use (reported beside CPU timings). */
+/* ---- per-token e4m3 quantisation (the decode cache append) --------------------------------- */
+
+/* Round-to-nearest-even of a finite |y| <= 448 onto the E4M3 grid, from the format's
+ * definition: below 2^-6 the grid is m * 2^-9 (m = 0..8, and m = 8 is the first normal value
+ * 2^-6); from 2^e to 2^(e+1) (e = -6..8) it is (1 + m/8) * 2^e, m = 0..7.  Returns the code. */
+static uint8_t e4m3_round(float yf) {
+  double y = (double)yf;                  /* exact */
+  uint8_t sign = 0;
+  if (y < 0) { sign = 0x80; y = -y; }
+  if (y >= 448.0) return sign | 0x7E;    /* saturate (the caller clamps already) */
+  if (y < ldexp(1.0, -6)) {
+    double q = y / ldexp(1.0, -9);        /* exact: division by a power of two */
+    double f = floor(q);
+    double r = q - f;
+    double m = (r > 0.5 || (r == 0.5 && fmod(f, 2.0) != 0.0)) ? f + 1.0 : f;
+    return sign | (uint8_t)m;             /* m = 8 encodes exponent field 1, mantissa 0 */
+  }
+  int e;
+  frexp(y, &e);                           /* y = fr * 2^e, fr in [0.5, 1) */
+  e -= 1;                                 /* y in [2^e, 2^(e+1)) */
+  double q = (y / ldexp(1.0, e) - 1.0) * 8.0;   /* exact */
+  double f = floor(q);
+  double r = q - f;
+  int m = (int)f + ((r > 0.5 || (r == 0.5 && ((int)f & 1))) ? 1 : 0);
+  if (m == 8) { m = 0; e += 1; }
+  return sign | (uint8_t)(((e + 7) << 3) | m);
+}
+
+/* Quantise n_rows rows of d fp32 values, each with its own scale: amax = max |x| over the
+ * row, scale = amax / 448 in fp32 (1 when amax = 0), y = x / scale in fp32, clamped to
+ * [-448, 448], then rounded to the nearest E4M3 value (ties to even).  codes [n_rows, d],
+ * scales [n_rows]. */
+void dsa_oracle_quantize_e4m3(int n_rows, int d, const float* x, uint8_t* codes, float* scales) {
+  for (int r = 0; r < n_rows; ++r) {
+    const float* xr = x + (int64_t)r * d;
+    float amax = 0.0f;
+    for (int i = 0; i < d; ++i) amax = fmaxf(amax, fabsf(xr[i]));
+    const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    scales[r] = scale;
+    for (int i = 0; i < d; ++i) {
+      float y = xr[i] / scale;
+      if (y > 448.0f) y = 448.0f;
+      if (y < -448.0f) y = -448.0f;
+      codes[(int64_t)r * d + i] = e4m3_round(y);
+    }
+  }
+}
+
 int dsa_oracle_num_threads(void) {
 #ifdef _OPENMP
   extern int omp_get_max_threads(void);

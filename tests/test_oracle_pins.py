@@ -307,3 +307,96 @@ def test_workload_quantiser_roundtrip_bound():
     amax = x.abs().amax(dim=(1, 2)).double()
     assert bool((err <= torch.maximum(x.double().abs() * 2 ** -4,
                                       (amax / 448 * 2 ** -9)[:, None, None] * 1.0001)).all())
+
+
+# ---------------------------------------------------------------- decode cache append (e4m3)
+
+def test_quantize_matches_torch_cast_and_generator():
+    """Per-token e4m3 quantisation against an independent implementation: the generator's
+    torch path (amax / 448, torch's round-to-nearest-even float8_e4m3fn cast)."""
+    from dsa_workloads import quantize_e4m3_rows
+    g = torch.Generator().manual_seed(31)
+    rows = [torch.randn(64, 128, generator=g),
+            torch.randn(64, 128, generator=g) ** 3 * 50,          # heavy tails
+            torch.randn(8, 128, generator=g) * 1e-6,              # subnormal codes after scaling
+            torch.full((2, 128), 3.25)]                            # constant rows
+    for x in rows:
+        ref_c, ref_s = quantize_e4m3_rows(x, 1)
+        c, s = oracle.quantize_e4m3(x.numpy())
+        assert np.array_equal(c, ref_c.numpy())
+        assert np.array_equal(s, ref_s.numpy())
+
+
+def test_quantize_ties_round_to_even():
+    """Every midpoint between consecutive positive e4m3 values (exact in fp32) rounds to the
+    neighbour with the even mantissa, like torch's cast; a 448 entry pins the scale to 1."""
+    vals = sorted({oracle.e4m3_to_f64(b) for b in range(0x7F) if b != 0x7F})
+    mids = [(a + b) / 2 for a, b in zip(vals[:-1], vals[1:])]
+    x = np.array(mids + [448.0], dtype=np.float32)
+    c, s = oracle.quantize_e4m3(x[None, :])
+    assert s[0] == 1.0
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(c[0], ref)
+    assert all(int(v) & 1 == 0 for v in c[0, :-1])    # ties land on even mantissas
+
+
+def test_quantize_error_bound_and_zero_row():
+    """|x - e4m3(x / s) * s| <= half the e4m3 spacing at that magnitude (times s); an all-zero
+    row has scale 1 and zero codes; the largest magnitude maps to +-448."""
+    g = np.random.default_rng(5)
+    x = g.standard_normal((16, 128)).astype(np.float32)
+    c, s = oracle.quantize_e4m3(x)
+    for r in range(16):
+        dq = np.array([oracle.e4m3_to_f64(b) for b in c[r]]) * s[r]
+        y = np.abs(x[r] / s[r]).astype(np.float64)
+        spacing = np.where(y < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(y, 1e-30))) - 3))
+        assert np.all(np.abs(dq - x[r]) <= 0.5 * spacing * s[r] * (1 + 1e-6))
+        assert abs(oracle.e4m3_to_f64(c[r][np.argmax(np.abs(x[r]))])) == 448.0
+    c0, s0 = oracle.quantize_e4m3(np.zeros((1, 128), np.float32))
+    assert s0[0] == 1.0 and not c0.any()
+
+
+def test_cache_append_paged_equals_contiguous():
+    """The append writes each sequence's new token at position seq_len - 1 through its block
+    table, touches nothing else, and reads back the same through a paged or a contiguous
+    layout; entries whose position or block is outside the caches are skipped."""
+    from dsa_workloads import make_decode, TINY
+    dims = dict(TINY, h_idx=64, d_idx=128)
+    lens = [130, 64, 1, 200]
+    wl = make_decode(21, 4, lens, dims, boost=0.0, paged=True, device="cpu", total_blocks=20)
+    g = np.random.default_rng(9)
+    k_new = g.standard_normal((4, 128)).astype(np.float32)
+    kv_new = (g.standard_normal((4, dims["d_qk"])).astype(np.float32).view(np.uint32) >> 16
+              ).astype(np.uint16)
+    kc, ks, kv, bad = oracle.cache_append(wl.k_idx, wl.k_scale, wl.kv, wl.seq_lens,
+                                          wl.block_table, wl.max_seqlen, k_new, kv_new)
+    assert not bad.any()
+    codes, scales = oracle.quantize_e4m3(k_new)
+    geo = oracle.Geometry.of(wl)
+    changed = set()
+    for b, n in enumerate(lens):
+        phys = int(geo.phys(b, np.array([n - 1]))[0])
+        changed.add(phys)
+        assert np.array_equal(kc[phys], codes[b]) and ks[phys] == scales[b]
+        assert np.array_equal(kv[phys], kv_new[b])
+    keep = np.array([r for r in range(kc.shape[0]) if r not in changed])
+    assert np.array_equal(kc[keep], oracle._np(wl.k_idx)[keep])
+    assert np.array_equal(kv[keep], oracle._np(wl.kv)[keep])
+    # contiguous layout: the same logical appends
+    R = 4 * wl.max_seqlen
+    z8, zs, z16 = (np.zeros((R, 128), np.uint8), np.ones(R, np.float32),
+                   np.zeros((R, dims["d_qk"]), np.uint16))
+    kc2, ks2, kv2, bad2 = oracle.cache_append(z8, zs, z16, wl.seq_lens, None, wl.max_seqlen,
+                                              k_new, kv_new)
+    for b, n in enumerate(lens):
+        pp = int(geo.phys(b, np.array([n - 1]))[0])
+        pc = b * wl.max_seqlen + n - 1
+        assert np.array_equal(kc2[pc], kc[pp]) and ks2[pc] == ks[pp]
+        assert np.array_equal(kv2[pc], kv[pp])
+    # out-of-range entries are skipped
+    bt = oracle._np(wl.block_table).copy()
+    bt[0, 2] = -1
+    lens_bad = np.array([130, 64, 0, 10_000], dtype=np.int32)
+    _, _, _, bad3 = oracle.cache_append(wl.k_idx, wl.k_scale, wl.kv, lens_bad, bt,
+                                        wl.max_seqlen, k_new, kv_new)
+    assert list(bad3) == [True, False, True, True]
