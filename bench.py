@@ -22,6 +22,7 @@ import sys
 import tempfile
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -299,6 +300,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
     }
     del fwd
+    line["cache_append"] = time_cache_append(args, dsa, wl, stream, peaks,
+                                             cpu_leg=rank == 0 and not args.no_cpu)
     if not args.no_prefill:
         del scores, idx, out, lse
         line["prefill"] = run_prefill(args, dsa, dev, stream, peaks, rank, world)
@@ -339,6 +342,62 @@ def run_prefill(args, dsa, dev, stream, peaks, rank, world):
                         "peak_note": "bf16 sustained measured; fp8 = 2x bf16 (nominal ratio)"}}
     del fwd, wl
     torch.cuda.empty_cache()
+    return res
+
+
+def time_cache_append(args, dsa, wl, stream, peaks, cpu_leg):
+    """The decode cache append (one new token per sequence quantised into the paged caches),
+    timed on its own after the decode step's numbers were taken: it rewrites each sequence's
+    last cache row.  Launch-bound by nature (189 KB at B = 64); reported beside the oracle doing
+    the same work per token on the host."""
+    import oracle
+    pb = dsa.problem_of(wl)
+    B, d = wl.batch, wl.dims
+    g = torch.Generator(device=wl.kv.device).manual_seed(77)
+    k_new = torch.randn(B, d["d_idx"], generator=g, device=wl.kv.device)
+    kv_new = torch.randn(B, d["d_qk"], generator=g, device=wl.kv.device).to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device=wl.kv.device)
+
+    def call():
+        dsa.check(dsa.dsa_cache_append(pb, k_new, kv_new, wl.k_idx, wl.k_scale, wl.kv, status,
+                                       stream), "cache_append")
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(20, args.steps)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / n
+    st, _ = dsa.dsa_read_device_status(status, stream)
+    dsa.check(st, "cache_append status")
+    per_tok = 4 * d["d_idx"] + 2 * d["d_qk"] + d["d_idx"] + 4 + 2 * d["d_qk"]
+    gbs = B * per_tok / (us / 1e6) / 1e9
+    res = {"us_per_call": round(us, 2), "batch": B, "bytes_per_call": B * per_tok,
+           "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm"],
+           "frac": round(gbs / peaks["hbm"], 5), "gpu_launches_per_call": 1,
+           "note": "one warp per sequence; launch latency, not bandwidth, sets the time"}
+    if cpu_leg:
+        # CPU baseline: the oracle doing the same work per token (quantise the keys, write the
+        # three rows into host caches)
+        import oracle
+        kn, kvn = k_new.cpu().numpy(), kv_new.view(torch.int16).cpu().numpy()
+        z8 = np.zeros((B, d["d_idx"]), np.uint8)
+        zs = np.zeros(B, np.float32)
+        z16 = np.zeros((B, d["d_qk"]), np.int16)
+        reps = 20
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            codes, scales = oracle.quantize_e4m3(kn)
+            z8[:] = codes
+            zs[:] = scales
+            z16[:] = kvn
+        res["cpu_baseline"] = {"us_per_call": round((time.perf_counter() - t0) / reps * 1e6, 1),
+                               "kind": "oracle", "cores": 1,
+                               "sample": f"the same {B} tokens, host caches"}
     return res
 
 

@@ -146,7 +146,11 @@ DSA_API size_t dsa_sparse_mla_workspace_size(const dsa_dims_t* dims, const dsa_s
 /* Stage 3.  Sparse MLA-MQA forward for rows [row_begin, row_begin + row_count).
  *   q    bf16 [total_rows, h, d_qk]   (indexed by absolute row)
  *   kv   bf16 [num_kv_rows, d_qk]
- *   idx  int32 [row_count, topk] logical key indices (-1 = unused), relative to row_begin
+ *   idx  int32 [row_count, topk] logical key indices (-1 = unused), relative to row_begin,
+ *        or NULL: every prior key of each row (dense causal attention), which is exactly the
+ *        top-k's selection when no row has more than topk prior keys; with NULL a row range
+ *        holding a row with more than topk prior keys (decode: max_seqlen > topk) returns
+ *        DSA_ERR_INVALID_ARG
  *   out  bf16 [total_rows, h, d_v] and lse fp32 [total_rows, h] (absolute rows); a row
  *        with no valid index gets out = 0 and lse = -inf. */
 DSA_API dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
@@ -185,13 +189,35 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const ds
 DSA_API size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs);
 
 /* The whole path for all seqs->total_rows query rows.  Inputs as for the three stages.
- *   idx_out  optional int32 [total_rows, topk]: the selected indices (NULL = not kept)
+ *   idx_out  optional int32 [total_rows, topk]: the selected indices (NULL = not kept).
+ *            When NULL, rows with at most topk prior keys (the first topk rows of each prefill
+ *            sequence; a decode batch whose max_seqlen <= topk) skip the indexer and the top-k,
+ *            whose selection would be all of their keys, and run dense attention.
  *   out, lse as for dsa_sparse_mla_fwd. */
 DSA_API dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
                          const float* q_scale, const float* w, const uint8_t* k_idx,
                          const float* k_scale, const uint16_t* q, const uint16_t* kv,
                          int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
                          size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream);
+
+/* Decode cache append, the step that fills the caches the path reads ("FP8 index -> top-k
+ * selection -> sparse core attention", "DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek
+ * Sparse Attention (DSA)", pipeline summary: the indexer reads keys in FP8).  DECODE mode only.
+ * For each sequence b the new token sits at position p = seq_lens[b] - 1 (the lengths already
+ * count it); it is written at physical row block_table[b][p / block_size] * block_size +
+ * p % block_size, or b * max_seqlen + p when block_table is NULL:
+ *   k_new     fp32 [batch, d_idx]: the new token's indexer key, quantised per token: scale =
+ *             amax / 448 in fp32 (1 when amax = 0), codes = the e4m3 value nearest to x / scale
+ *             (ties to even, saturating at +-448)
+ *   kv_new    bf16 [batch, d_qk]: the new token's latent row, copied unchanged
+ *   k_cache   e4m3 [num_kv_rows, d_idx], k_scale_cache fp32 [num_kv_rows], kv_cache bf16
+ *             [num_kv_rows, d_qk]: caller-owned caches, written at the one row per sequence
+ * All pointers 16-byte aligned.  An entry whose position or block falls outside the caches is
+ * skipped and sets DSA_DEVICE_BAD_INDEX in *dev_status. */
+DSA_API dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                      const float* k_new, const uint16_t* kv_new,
+                                      uint8_t* k_cache, float* k_scale_cache, uint16_t* kv_cache,
+                                      int32_t* dev_status, dsa_stream_t stream);
 
 /* Synchronises `stream`, reads the device status word and maps it: 0 -> DSA_OK,
  * DSA_DEVICE_TIMEOUT -> DSA_ERR_TIMEOUT, DSA_DEVICE_BAD_INDEX -> DSA_ERR_BAD_INDEX.

@@ -37,7 +37,7 @@ DSA_DECODE = 1
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_fwd", "dsa_forward_workspace_size", "dsa_forward",
             "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-            "dsa_sparse_mla_fwd_noalloc")
+            "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -81,6 +81,7 @@ def _load():
         "dsa_status_string": (ctypes.c_char_p, [I32]),
         "dsa_abi_version": (I32, []),
         "dsa_sparse_mla_fwd_noalloc": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, P]),
+        "dsa_cache_append": (I32, [DP, SP, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -225,6 +226,13 @@ def dsa_forward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, q, kv, idx_out, 
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
         _ptr(k_idx), _ptr(k_scale), _ptr(q), _ptr(kv), _ptr(idx_out), _ptr(out), _ptr(lse),
         _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def dsa_cache_append(pb: Problem, k_new, kv_new, k_cache, k_scale_cache, kv_cache,
+                     dev_status=None, stream=None) -> int:
+    return int(lib.dsa_cache_append(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(k_new), _ptr(kv_new), _ptr(k_cache),
+        _ptr(k_scale_cache), _ptr(kv_cache), _ptr(dev_status), _stream(stream)))
 
 
 def dsa_read_device_status(dev_status, stream=None):

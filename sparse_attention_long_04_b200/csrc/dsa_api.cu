@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "dsa.h"
+#include "cache_append.cuh"
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
@@ -159,6 +160,12 @@ int64_t max_keys(const dsa_seqs_t* s, int32_t row_begin, int32_t row_count) {
     if (lo < hi) m = std::max<int64_t>(m, hi - cu[b]);
   }
   return m;
+}
+
+// Without an index array sparse attention runs dense: every prior key of each row, which is only
+// the top-k's selection when no row has more than topk prior keys.
+bool dense_ok(const dsa_dims_t& d, const dsa_seqs_t* s, int32_t row_begin, int32_t row_count) {
+  return max_keys(s, row_begin, row_count) <= d.topk;
 }
 
 // ------------------------------------------------------------------------ TMA maps
@@ -538,7 +545,8 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
   if (e != DSA_OK) return e;
   if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
-  if (!q || !kv || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!q || !kv || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (idx == nullptr && !dense_ok(*dims, seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || !aligned16(lse) ||
       !aligned16(workspace))
     return DSA_ERR_MISALIGNED;
@@ -584,6 +592,9 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
   void* mla_ws = wsb + align(plan.slab_floats * 4) + align(plan.idx_ints * 4);
 
   if (s.mode == DSA_DECODE) {
+    if (idx_out == nullptr && s.max_seqlen <= d.topk)   // every context key is kept: dense
+      return mla_dispatch(d, s, q, kv, nullptr, 0, s.batch, out, lse, mla_ws, plan.mla_bytes,
+                          dev_status, st, plan.mla_splits);
     const int64_t ld = round4(s.max_seqlen);
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if ((e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, 0, s.batch, slab, ld,
@@ -599,7 +610,14 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
     if (L <= 0) continue;
     const int64_t ld = round4(L);
     const int64_t rows = chunk_rows_for(L, info.sm_count);
-    for (int64_t r0 = 0; r0 < L; r0 += rows) {
+    // rows with at most topk prior keys keep all of them: dense attention, no indexer or top-k
+    // (unless the caller wants the indices)
+    const int64_t n_dense = idx_out == nullptr ? std::min<int64_t>(L, d.topk) : 0;
+    if (n_dense > 0 &&
+        (e = mla_dispatch(d, s, q, kv, nullptr, cu[b], static_cast<int32_t>(n_dense), out, lse,
+                          nullptr, 0, dev_status, st, 1)) != DSA_OK)
+      return e;
+    for (int64_t r0 = n_dense; r0 < L; r0 += rows) {
       const int32_t row_begin = static_cast<int32_t>(cu[b] + r0);
       const int32_t row_count = static_cast<int32_t>(std::min(rows, L - r0));
       int32_t* idx = idx_out ? idx_out + int64_t(row_begin) * d.topk : idx_ws;
@@ -614,6 +632,44 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
     }
   }
   return DSA_OK;
+}
+
+dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* k_new,
+                              const uint16_t* kv_new, uint8_t* k_cache, float* k_scale_cache,
+                              uint16_t* kv_cache, int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  const dsa_dims_t& d = *dims;
+  const dsa_seqs_t& s = *seqs;
+  if (s.mode != DSA_DECODE) return DSA_ERR_INVALID_ARG;
+  const bool full = d.d_idx == 128 && d.d_qk == 576;
+  const bool tiny = d.d_idx == 32 && d.d_qk == 160;
+  if (!full && !tiny) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!k_new || !kv_new || !k_cache || !k_scale_cache || !kv_cache) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(kv_new) || !aligned16(k_cache) ||
+      !aligned16(k_scale_cache) || !aligned16(kv_cache))
+    return DSA_ERR_MISALIGNED;
+  AppendParams prm{};
+  prm.k_new = k_new;
+  prm.kv_new = reinterpret_cast<const uint4*>(kv_new);
+  prm.k_cache = k_cache;
+  prm.k_scale = k_scale_cache;
+  prm.kv_cache = reinterpret_cast<uint4*>(kv_cache);
+  prm.seq_lens = s.seq_lens;
+  prm.block_table = s.block_table;
+  prm.batch = s.batch;
+  prm.max_blocks = s.max_blocks;
+  prm.max_seqlen = s.max_seqlen;
+  prm.block_size = d.block_size;
+  prm.num_kv_rows = s.num_kv_rows;
+  prm.status = dev_status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(ceil_div(s.batch, 4)));
+  if (full)
+    dsa_cache_append_kernel<128, 576><<<grid, 128, 0, st>>>(prm);
+  else
+    dsa_cache_append_kernel<32, 160><<<grid, 128, 0, st>>>(prm);
+  return launch_status();
 }
 
 dsa_status_t dsa_read_device_status(const int32_t* dev_status, dsa_stream_t stream,
@@ -662,7 +718,8 @@ dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const dsa_seqs_t
   if (e != DSA_OK) return e;
   if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
-  if (!q || !kv || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!q || !kv || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (idx == nullptr && !dense_ok(*dims, seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || !aligned16(lse))
     return DSA_ERR_MISALIGNED;
   DeviceInfo info;

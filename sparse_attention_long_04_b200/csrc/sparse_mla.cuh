@@ -31,6 +31,8 @@
 // owns TMEM, warps 4-7 move Q into TMEM, run the softmax and the epilogue, warps 8-15 resolve
 // the keys, then gather rows [16w, 16w + 16) of every tile: warps 8-11 the QK-only dims,
 // warps 12-15 the value dims.  Grid: x = 2 * row + v, y = split-KV slice.
+// Without an index array the selection is every prior key (dense causal attention), which is
+// what the top-k keeps whenever a row has at most topk prior keys.
 #pragma once
 #include <type_traits>
 
@@ -41,7 +43,8 @@ namespace dsa {
 struct MlaParams {
   const __nv_bfloat16* q;      // [T, H, D_QK]
   const __nv_bfloat16* kv;     // [R, D_QK]
-  const int32_t* idx;          // [row_count, topk], relative to row_begin
+  const int32_t* idx;          // [row_count, topk], relative to row_begin; null: dense
+                               // (every prior key; the caller guarantees pos + 1 <= topk)
   __nv_bfloat16* out;          // [T, H, D_V]
   float* lse;                  // [T, H]
   float* part_o;               // split-KV partials [splits, row_count, H, D_V] or null
@@ -129,7 +132,8 @@ __global__ void __launch_bounds__(512, 1)
   const int split = blockIdx.y;
   const int r = blockIdx.x >> 1;
   const int row = p.row_begin + r;
-  const int32_t* irow = p.idx + static_cast<int64_t>(r) * p.topk;
+  const bool dense = p.idx == nullptr;
+  const int32_t* irow = dense ? nullptr : p.idx + static_cast<int64_t>(r) * p.topk;
   const int n_tiles_all = p.topk / C::BN;
 
   // ---- row geometry
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
     for (int j = 0; j < KPT; ++j) {
       const int e = t + 256 * j;
-      v[j] = e < p.topk ? irow[e] : -1;
+      v[j] = e >= p.topk ? -1 : dense ? (e < n_keys ? e : -1) : irow[e];
     }
     int64_t phys[KPT];
     bool bad_idx = false;

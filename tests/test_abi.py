@@ -108,3 +108,34 @@ def test_bad_geometry_rejected(dsa):
 def test_workspace_size_is_zero_on_bad_args(dsa):
     pb = _pb(dsa, topk=7)
     assert dsa.dsa_forward_workspace_size(pb) == 0
+
+
+def test_cache_append_argument_errors(dsa):
+    """The append is decode-only, needs its five buffers and 16-byte alignment, and supports
+    the two key/latent widths; all of this is rejected before any launch."""
+    pb = _pb(dsa)
+    ok = [FAKE] * 5
+    call = lambda p, bufs: dsa.dsa_cache_append(p, *bufs, None, 0)
+    assert call(pb, [None] + ok[1:]) == dsa.DSA_ERR_INVALID_ARG
+    assert call(pb, [FAKE + 4] + ok[1:]) == dsa.DSA_ERR_MISALIGNED
+    pre = dsa.make_problem(mode="prefill", h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512,
+                           topk=2048, softmax_scale=0.04, num_kv_rows=1 << 20, seqlens=[100],
+                           cu_seqlens=FAKE)
+    assert call(pre, ok) == dsa.DSA_ERR_INVALID_ARG
+    odd = _pb(dsa, d_qk=512)
+    assert call(odd, ok) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_dense_attention_needs_short_rows(dsa):
+    """Sparse attention without an index array means every prior key; a row range with a row
+    of more than topk prior keys is refused before any launch."""
+    pre = dsa.make_problem(mode="prefill", h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512,
+                           topk=2048, softmax_scale=0.04, num_kv_rows=1 << 20,
+                           seqlens=[5000], cu_seqlens=FAKE)
+    ws = [FAKE, FAKE]
+    # rows 0..2047 have at most 2048 prior keys; row 2048 has 2049
+    args = lambda rb, rc: (pre, FAKE, FAKE, None, rb, rc, FAKE, FAKE, None, 0, None, 0)
+    assert dsa.dsa_sparse_mla_fwd(*args(2000, 100)) == dsa.DSA_ERR_INVALID_ARG
+    dec = _pb(dsa, max_seqlen=4096)
+    assert dsa.dsa_sparse_mla_fwd(dec, FAKE, FAKE, None, 0, 2, FAKE, FAKE, None, 0, None,
+                                  0) == dsa.DSA_ERR_INVALID_ARG

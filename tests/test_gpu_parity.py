@@ -349,3 +349,70 @@ def test_forward_small_prefill_full_dims(dsa):
     f = _forward(dsa, wl)
     rows = [0, 1, 63, 2046, 2047, 2048, 2100, 2499, 2500, 2799]
     _check_forward(wl, f, rows)
+
+
+# --------------------------------------------------------------- dense (short-row) attention
+
+def test_sparse_mla_dense_equals_sparse_with_all_keys(dsa):
+    """Without an index array the attention takes every prior key; for rows with at most topk
+    prior keys that is exactly the top-k's selection, so the result is bit-identical to the
+    sparse call on the top-k's indices, and matches the oracle."""
+    wl = make_prefill(41, [2048, 700], FULL, needles=8, device="cuda")
+    T = wl.total_rows
+    scores = run_indexer(dsa, wl)
+    idx = run_topk(dsa, wl, scores)
+    o_s, l_s = run_mla(dsa, wl, idx)
+    pb = dsa.problem_of(wl)
+    d = wl.dims
+    o_d = torch.full((T, d["h"], d["d_v"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    l_d = torch.full((T, d["h"]), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, None, 0, T, o_d, l_d, None, 0, status) == 0
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(o_d.view(torch.int16), o_s.view(torch.int16))
+    assert torch.equal(l_d, l_s)
+    rows = list(range(0, T, 37)) + [2047, 2048, T - 1]
+    dense_idx = np.full((len(rows), d["topk"]), -1, dtype=np.int32)
+    for i, r in enumerate(rows):
+        n = n_valid_of(wl, r)
+        dense_idx[i, :n] = np.arange(n)
+    ro, rl = oracle.sparse_mla_rows(wl, rows, dense_idx)
+    o, l = to_np(o_d), to_np(l_d)
+    for i, r in enumerate(rows):
+        check_attention(o[r], l[r], ro[i], rl[i], d["h"], f"row {r}")
+
+
+def test_forward_without_indices_dense_first_rows(dsa):
+    """dsa_forward with no index output: the first topk rows of each sequence run dense (no
+    indexer, no top-k) and match the oracle (whose selection is every key there); the later
+    rows take the sparse path and equal, bit for bit, a run that keeps the indices."""
+    wl = make_config(1, device="cuda")                 # L = 1024, topk = 64
+    f = dsa.Forward(wl, keep_idx=False)
+    assert f() == 0
+    g = dsa.Forward(wl, keep_idx=True)
+    assert g() == 0
+    torch.cuda.synchronize()
+    assert int(f.status.item()) == 0 and int(g.status.item()) == 0
+    rows = list(range(0, 64))
+    _, _, o_ref, l_ref = oracle.forward_rows(wl, rows)
+    o, l = to_np(f.out), to_np(f.lse)
+    for i, r in enumerate(rows):
+        check_attention(o[r], l[r], o_ref[i], l_ref[i], wl.dims["h"], f"row {r}")
+    assert torch.equal(f.out[64:].view(torch.int16), g.out[64:].view(torch.int16))
+    assert torch.equal(f.lse[64:], g.lse[64:])
+
+
+def test_forward_short_decode_is_dense(dsa):
+    """A decode batch whose contexts all fit in topk keeps every key: dsa_forward skips the
+    indexer and the top-k and matches the oracle's whole pipeline."""
+    wl = make_decode(42, 4, [2048, 1, 900, 64], FULL, boost=0.01, paged=True, device="cuda")
+    f = dsa.Forward(wl, keep_idx=False)
+    assert f() == 0
+    torch.cuda.synchronize()
+    assert int(f.status.item()) == 0
+    rows = [0, 1, 2, 3]
+    _, idx_ref, o_ref, l_ref = oracle.forward_rows(wl, rows)
+    o, l = to_np(f.out), to_np(f.lse)
+    for i, r in enumerate(rows):
+        check_attention(o[r], l[r], o_ref[i], l_ref[i], wl.dims["h"], f"row {r}")
