@@ -208,6 +208,10 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   };
   auto key4_at = [&](int i) -> uint4 {            // i multiple of 4, i < m
     if (cached) return *reinterpret_cast<const uint4*>(keys + i);
+    if (i + 3 < m) {                              // a streamed slice: one 16-byte load
+      const float4 v = *reinterpret_cast<const float4*>(srow + s0 + i);
+      return make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+    }
     uint4 k = make_uint4(0, 0, 0, 0);
     if (i + 0 < m) k.x = score_key(srow[s0 + i + 0]);
     if (i + 1 < m) k.y = score_key(srow[s0 + i + 1]);
@@ -246,7 +250,23 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
       }
     }
   } else {
-    for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&hist[key_at(i) >> 21], 1u);
+    // a slice longer than shared memory holds: streamed with 16-byte loads, 4 in flight
+    for (int base = tid * 4; base < m; base += kTopkThreads * 16) {
+      uint4 k[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i4 = base + u * kTopkThreads * 4;
+        k[u] = i4 < m ? key4_at(i4) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i4 = base + u * kTopkThreads * 4;
+        if (i4 < m) atomicAdd(&hist[k[u].x >> 21], 1u);
+        if (i4 + 1 < m) atomicAdd(&hist[k[u].y >> 21], 1u);
+        if (i4 + 2 < m) atomicAdd(&hist[k[u].z >> 21], 1u);
+        if (i4 + 3 < m) atomicAdd(&hist[k[u].w >> 21], 1u);
+      }
+    }
   }
   cluster_hist_sum(hist, hsum, kTopkBins, C);
   uint32_t bin, above;
