@@ -166,7 +166,8 @@ def run_ours(args, rank, world, local_rank):
         wl = make_decode(DECODE_CFG, args.decode_batch, c["ctx"],
                          {k: c[k] for k in ("h_idx", "d_idx", "topk", "h", "d_qk", "d_v")},
                          c["boost"], c["paged"], dev, seed=rank_seed(DECODE_CFG, rank),
-                         name=f"{c['name']}_B{args.decode_batch}")
+                         name=f"{c['name']}_B{args.decode_batch}",
+                         scale_layout=c.get("scale_layout", "separate"))
     else:
         wl = make_config(DECODE_CFG, device=dev, seed=rank_seed(DECODE_CFG, rank))
     d = wl.dims
@@ -423,17 +424,19 @@ def load_traffic(name):
 def oracle_sample(wl, n_rows):
     """A decode workload holding only `n_rows` sequences of `wl`, laid out contiguously on the
     host (a gather of the inputs; no arithmetic), for timing the oracle."""
+    import oracle
     from dsa_workloads import Workload
     rows = list(range(n_rows))
     L = wl.max_seqlen
     bt = wl.block_table[:n_rows].long()
     phys = (bt[:, torch.arange(L, device=bt.device) // 64] * 64 +
             torch.arange(L, device=bt.device) % 64).reshape(-1)
+    codes, scales = oracle.key_rows(wl, phys.cpu().numpy())
     return Workload(cfg_id=wl.cfg_id, name=wl.name, mode="decode", dims=wl.dims,
                     softmax_scale=wl.softmax_scale, seqlens=wl.seqlens[:n_rows],
                     q_idx=wl.q_idx[rows].cpu(), q_scale=wl.q_scale[rows].cpu(),
-                    w=wl.w[rows].cpu(), k_idx=wl.k_idx[phys].cpu(),
-                    k_scale=wl.k_scale[phys].cpu(), q=wl.q[rows].cpu(), kv=wl.kv[phys].cpu(),
+                    w=wl.w[rows].cpu(), k_idx=torch.from_numpy(codes),
+                    k_scale=torch.from_numpy(scales), q=wl.q[rows].cpu(), kv=wl.kv[phys].cpu(),
                     seq_lens=wl.seq_lens[:n_rows].cpu(), block_table=None, max_seqlen=L)
 
 

@@ -13,7 +13,8 @@ Workload shapes follow the five DSA workloads this repository is measured on:
                              16 heads, latent 128+32, values 128, 8 needles per 128-row band
   decode_B32_N32k            32 sequences x 32768 context, full shapes, 1 % boosted keys
   decode_B64_N128k_paged     64 x 131072 context, 64-token pages, random block table,
-                             0.5 % planted keys
+                             0.5 % planted keys; each page of the indexer cache holds its 64
+                             key rows followed by their 64 scales
   prefill_L16k               1 causal sequence of 16384 tokens, needles
   prefill_varlen_T276480     8 packed sequences {4096, 8192, 16384, 16384, 32768, 65536,
                              131072, 2048}
@@ -43,7 +44,7 @@ CONFIGS: Dict[int, dict] = {
     2: dict(name="decode_B32_N32k", mode="decode", batch=32, ctx=32768, paged=False,
             boost=0.01, **FULL),
     3: dict(name="decode_B64_N128k_paged", mode="decode", batch=64, ctx=131072, paged=True,
-            boost=0.005, **FULL),
+            boost=0.005, scale_layout="interleaved", **FULL),
     4: dict(name="prefill_L16k", mode="prefill", seqlens=[16384], needles=8, **FULL),
     5: dict(name="prefill_varlen_T276480", mode="prefill",
             seqlens=[4096, 8192, 16384, 16384, 32768, 65536, 131072, 2048], needles=8, **FULL),
@@ -58,8 +59,10 @@ class Workload:
       q_idx      uint8 [T, h_idx, d_idx]   e4m3 bytes of the indexer queries
       q_scale    f32   [T, h_idx]          per-(token, indexer head) dequant scale
       w          f32   [T, h_idx]          indexer head weights
-      k_idx      uint8 [R, d_idx]          e4m3 bytes of the indexer keys (R physical rows)
-      k_scale    f32   [R]                 per-key dequant scale
+      k_idx      uint8 [R, d_idx]          e4m3 bytes of the indexer keys (R physical rows), or
+                                           with interleaved scales uint8 [R/64, 64*(d_idx+4)]:
+                                           each 64-row block's key rows, then its 64 fp32 scales
+      k_scale    f32   [R] or None         per-key dequant scale (None: inside k_idx's blocks)
       q          bf16  [T, h, d_qk]        absorbed MLA queries
       kv         bf16  [R, d_qk]           latent KV rows (values = first d_v dims)
     Prefill: T = R = total packed tokens; row r of sequence b sits at cu_seqlens[b] + pos.
@@ -77,7 +80,7 @@ class Workload:
     q_scale: torch.Tensor
     w: torch.Tensor
     k_idx: torch.Tensor
-    k_scale: torch.Tensor
+    k_scale: Optional[torch.Tensor]
     q: torch.Tensor
     kv: torch.Tensor
     cu_seqlens: Optional[torch.Tensor] = None     # int32 [batch+1] (prefill)
@@ -121,6 +124,16 @@ def quantize_e4m3_rows(x: torch.Tensor, group_dims: int):
     y = (flat / scale.unsqueeze(-1)).clamp_(-E4M3_MAX, E4M3_MAX)
     q8 = y.to(torch.float8_e4m3fn).view(torch.uint8).reshape(x.shape)
     return q8.contiguous(), scale.float().contiguous()
+
+
+def interleave_key_blocks(k8: torch.Tensor, ks: torch.Tensor, block: int = BLOCK_SIZE):
+    """The paged indexer cache with each block's scales stored right after its key rows:
+    uint8 [R / block, block * d + block * 4] (a layout change only; the bytes are the same)."""
+    R, d = k8.shape
+    nb = R // block
+    keys = k8.reshape(nb, block * d)
+    sc = ks.contiguous().view(torch.uint8).reshape(nb, block * 4)
+    return torch.cat([keys, sc], dim=1).contiguous()
 
 
 def _unit(v: torch.Tensor) -> torch.Tensor:
@@ -189,14 +202,15 @@ def make_prefill(cfg_id: int, seqlens: List[int], dims: dict, needles: int, devi
 
 def make_decode(cfg_id: int, batch: int, ctx, dims: dict, boost: float, paged: bool, device,
                 seed: Optional[int] = None, name: Optional[str] = None,
-                softmax_scale: Optional[float] = None, total_blocks: Optional[int] = None
-                ) -> Workload:
+                softmax_scale: Optional[float] = None, total_blocks: Optional[int] = None,
+                scale_layout: str = "separate") -> Workload:
     """Decode: one new token per sequence, whose k_I and latent KV are already in the cache
     (query position = seq_len - 1).  ``ctx`` is an int or a per-sequence list.
 
     Boost: u_b = unit(sum_j w_j q_I[b, j]); a seeded fraction ``boost`` of the context
     positions get k_I += 2 sqrt(d_idx) u_b.  Paged: 64-token blocks, the block table is a
-    seeded permutation of the physical blocks."""
+    seeded permutation of the physical blocks.  scale_layout "interleaved" (paged only) stores
+    each block's 64 key scales right after its 64 key rows (k_scale None)."""
     seed = 1000 + cfg_id if seed is None else seed
     h_idx, d_idx, h, d_qk = dims["h_idx"], dims["d_idx"], dims["h"], dims["d_qk"]
     lens = [int(ctx)] * batch if isinstance(ctx, int) else [int(c) for c in ctx]
@@ -230,6 +244,9 @@ def make_decode(cfg_id: int, batch: int, ctx, dims: dict, boost: float, paged: b
     qs = qs.unsqueeze(1).expand(-1, h_idx).contiguous()
     k8, ks = quantize_e4m3_rows(ki, 1)
     del ki
+    if scale_layout == "interleaved":
+        assert paged, "interleaved scales need the paged layout"
+        k8, ks = interleave_key_blocks(k8, ks), None
     q = torch.randn(batch, h, d_qk, generator=_gen(seed, 5, 0, device), device=device
                     ).to(torch.bfloat16)
     kv = torch.empty(rows, d_qk, dtype=torch.bfloat16, device=device)
@@ -253,7 +270,7 @@ def make_config(cfg_id: int, device="cpu", seed: Optional[int] = None) -> Worklo
         return make_prefill(cfg_id, c["seqlens"], dims, c["needles"], device, seed=seed,
                             name=c["name"])
     return make_decode(cfg_id, c["batch"], c["ctx"], dims, c["boost"], c["paged"], device,
-                       seed=seed, name=c["name"])
+                       seed=seed, name=c["name"], scale_layout=c.get("scale_layout", "separate"))
 
 
 def sample_rows(w: Workload, per_seq: int, first: int = 0, seed: Optional[int] = None

@@ -155,6 +155,24 @@ class Geometry:
         return b * self.max_seqlen + s
 
 
+def key_rows(wl, phys) -> tuple:
+    """e4m3 codes [n, d_idx] and fp32 scales [n] of the indexer keys at physical rows
+    ``phys``, from separate arrays or, when ``wl.k_scale`` is None, from 64-row blocks that
+    hold their key rows followed by their scales."""
+    phys = np.asarray(phys, dtype=np.int64)
+    if wl.k_scale is not None:
+        return _take(wl.k_idx, phys, np.uint8), _take(wl.k_scale, phys, np.float32)
+    d = wl.dims["d_idx"]
+    blk, j = phys // 64, phys % 64
+    ub, inv = np.unique(blk, return_inverse=True)
+    blocks = _take(wl.k_idx, ub, np.uint8)[inv]                  # [n, 64 * (d + 4)]
+    n = len(phys)
+    rows = np.arange(n)[:, None]
+    codes = blocks[rows, j[:, None] * d + np.arange(d)[None, :]]
+    sbytes = np.ascontiguousarray(blocks[rows, 64 * d + j[:, None] * 4 + np.arange(4)[None, :]])
+    return np.ascontiguousarray(codes), sbytes.view(np.float32).reshape(n)
+
+
 # ---- stages --------------------------------------------------------------------------------
 
 def indexer_rows(wl, rows: Sequence[int], fp32: bool = False) -> Dict[int, np.ndarray]:
@@ -172,8 +190,7 @@ def indexer_rows(wl, rows: Sequence[int], fp32: bool = False) -> Dict[int, np.nd
         pos = np.array([geo.row_seq_pos(r)[1] for r in rs], dtype=np.int32)
         n_keys = int(pos.max()) + 1
         phys = geo.phys(b, np.arange(n_keys))
-        kseq = _take(wl.k_idx, phys, np.uint8)
-        kss = _take(wl.k_scale, phys, np.float32)
+        kseq, kss = key_rows(wl, phys)
         qq = _take(wl.q_idx, rs, np.uint8)
         qsc = _take(wl.q_scale, rs, np.float32)
         ww = _take(wl.w, rs, np.float32)
@@ -255,14 +272,17 @@ def cache_append(k_cache, k_scale, kv_cache, seq_lens, block_table, max_seqlen: 
     p = seq_lens[b] - 1; its indexer key k_new[b] (fp32) is quantised per token and written
     with its scale, and its latent row kv_new[b] (bf16 bits) is copied, at the physical row
     block_table[b, p // bs] * bs + p % bs (b * max_seqlen + p without a table).  Entries
-    whose position or block is outside the caches are skipped.  Returns copies of the three
-    caches and a bool [B] of the skipped entries."""
-    kc, ks, kv = _np(k_cache).copy(), _np(k_scale).copy(), _np(kv_cache).copy()
+    whose position or block is outside the caches are skipped.  With ``k_scale`` None the key
+    cache is made of 64-row blocks holding their key rows then their fp32 scales.  Returns
+    copies of the three caches (the scales None in that layout) and a bool [B] of the skipped
+    entries."""
+    kc, kv = _np(k_cache).copy(), _np(kv_cache).copy()
+    ks = _np(k_scale).copy() if k_scale is not None else None    # None: scales in the blocks
     lens = _np(seq_lens).astype(np.int64)
     bt = _np(block_table)
     codes, scales = quantize_e4m3(k_new)
     kvn = _np(kv_new)
-    rows = kc.shape[0]
+    rows = kv.shape[0]
     bad = np.zeros(len(lens), dtype=bool)
     for b, n in enumerate(lens):
         p = int(n) - 1
@@ -280,7 +300,14 @@ def cache_append(k_cache, k_scale, kv_cache, seq_lens, block_table, max_seqlen: 
             if phys >= rows:
                 bad[b] = True
                 continue
-        kc[phys] = codes[b]
-        ks[phys] = scales[b]
+        if ks is not None:
+            kc[phys] = codes[b]
+            ks[phys] = scales[b]
+        else:                                   # block phys // 64: 64 key rows, then scales
+            d = codes.shape[1]
+            blk, j = phys // 64, phys % 64
+            kc[blk, j * d:(j + 1) * d] = codes[b]
+            kc[blk, 64 * d + 4 * j:64 * d + 4 * j + 4] = np.frombuffer(
+                scales[b:b + 1].tobytes(), dtype=np.uint8)
         kv[phys] = kvn[b]
     return kc, ks, kv, bad

@@ -10,7 +10,8 @@
 //
 // One warp per sequence: the key row is read with one float4 per lane (D_I = 128) and reduced
 // to its max with warp shuffles; the latent row moves as 16-byte chunks.  An entry whose
-// position or block falls outside the caches is skipped and reported.
+// position or block falls outside the caches is skipped and reported.  The key cache may hold
+// each 64-row block's scales right after its key rows (paged decode, no separate scale array).
 #pragma once
 #include <cuda_fp8.h>
 
@@ -21,8 +22,9 @@ namespace dsa {
 struct AppendParams {
   const float* k_new;          // [batch, D_I]
   const uint4* kv_new;         // [batch, D_QK] bf16, as 16-byte chunks
-  uint8_t* k_cache;            // [num_kv_rows, D_I] e4m3
-  float* k_scale;              // [num_kv_rows]
+  uint8_t* k_cache;            // [num_kv_rows, D_I] e4m3, or with k_scale null interleaved
+                               // blocks: [num_kv_rows / 64][64 * D_I bytes | 64 fp32 scales]
+  float* k_scale;              // [num_kv_rows] or null
   uint4* kv_cache;             // [num_kv_rows, D_QK] bf16, as 16-byte chunks
   const int32_t* seq_lens;     // [batch]
   const int32_t* block_table;  // [batch, max_blocks] or null
@@ -78,14 +80,21 @@ __global__ void __launch_bounds__(128) dsa_cache_append_kernel(const AppendParam
     const uint32_t c = __nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
     packed |= c << (8 * i);
   }
-  uint8_t* kdst = p.k_cache + row * D_I + lane * PER;
+  // the key row and its scale: separate arrays, or inside the row's 64-row block
+  const int64_t blk = row / 64, r64 = row % 64;
+  uint8_t* krow = p.k_scale != nullptr ? p.k_cache + row * D_I
+                                       : p.k_cache + blk * (64 * (D_I + 4)) + r64 * D_I;
+  float* sdst = p.k_scale != nullptr
+                    ? p.k_scale + row
+                    : reinterpret_cast<float*>(p.k_cache + blk * (64 * (D_I + 4)) + 64 * D_I) + r64;
+  uint8_t* kdst = krow + lane * PER;
   if constexpr (PER == 4) {
     *reinterpret_cast<uint32_t*>(kdst) = packed;
   } else {
 #pragma unroll
     for (int i = 0; i < PER; ++i) kdst[i] = static_cast<uint8_t>(packed >> (8 * i));
   }
-  if (lane == 0) p.k_scale[row] = scale;
+  if (lane == 0) *sdst = scale;
   // ---- latent row
   constexpr int CHUNKS = D_QK * 2 / 16;
   const uint4* ksrc = p.kv_new + static_cast<int64_t>(b) * CHUNKS;

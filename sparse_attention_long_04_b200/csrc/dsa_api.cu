@@ -187,6 +187,30 @@ dsa_status_t make_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Interleaved paged indexer cache: blocks of 64 key rows (row_bytes each) followed by their 64
+// fp32 scales; one box = one block's 64 key rows.
+dsa_status_t make_block_map(CUtensorMap* map, const void* base, uint64_t blocks,
+                            uint32_t row_bytes) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (encoder(&enc) != DSA_OK) return DSA_ERR_CUDA;
+  std::memset(map, 0, sizeof(*map));
+  cuuint64_t dims[3] = {row_bytes, 64, blocks};
+  cuuint64_t strides[2] = {row_bytes, uint64_t(64) * (row_bytes + 4)};
+  cuuint32_t box[3] = {row_bytes, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw =
+      row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                   strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// The indexer's scales may live inside the key blocks (k_scale NULL) only in paged decode.
+bool interleaved_ok(const dsa_seqs_t& s) {
+  return s.mode == DSA_DECODE && s.block_table != nullptr && s.num_kv_rows % 64 == 0;
+}
+
 // Rows of `row_bytes` bytes (a multiple of 16), boxes of box_bytes x box_rows, 128-byte swizzle.
 dsa_status_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
                           uint32_t box_bytes, uint32_t box_rows) {
@@ -226,15 +250,22 @@ dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_
   DeviceInfo info;
   if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
   CUtensorMap kmap, qmap;
-  // prefill keys are contiguous: one 128-row box per tile; decode: 64-row (paged) boxes
-  if (make_map(&kmap, k_idx, s.num_kv_rows, D_I, s.mode == DSA_DECODE ? 64 : 128) != DSA_OK)
+  // prefill keys are contiguous: one 128-row box per tile; decode: 64-row (paged) boxes; with
+  // the scales inside the blocks, one 3-D box per block
+  if (k_scale == nullptr) {
+    if (make_block_map(&kmap, k_idx, uint64_t(s.num_kv_rows / 64), D_I) != DSA_OK)
+      return DSA_ERR_CUDA;
+  } else if (make_map(&kmap, k_idx, s.num_kv_rows, D_I, s.mode == DSA_DECODE ? 64 : 128) !=
+             DSA_OK) {
     return DSA_ERR_CUDA;
+  }
   if (make_map(&qmap, q_idx, uint64_t(s.total_rows) * H_I, D_I, C::N) != DSA_OK)
     return DSA_ERR_CUDA;
   IndexerParams prm{};
   prm.q_scale = q_scale;
   prm.w = w;
   prm.k_scale = k_scale;
+  prm.k_blocks = k_idx;
   prm.scores = scores;
   prm.ld = ld;
   prm.status = status;
@@ -506,7 +537,8 @@ dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
   if (e != DSA_OK) return e;
   if (!indexer_shape_ok(*dims, seqs->mode)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
-  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
+  if (!q_idx || !q_scale || !w || !k_idx || !scores) return DSA_ERR_INVALID_ARG;
+  if (k_scale == nullptr && !interleaved_ok(*seqs)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(scores) ||
       ld_scores % 4 != 0)
     return DSA_ERR_MISALIGNED;
@@ -574,8 +606,9 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
   const dsa_dims_t& d = *dims;
   const dsa_seqs_t& s = *seqs;
   if (!indexer_shape_ok(d, s.mode) || !mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !q || !kv || !out || !lse)
+  if (!q_idx || !q_scale || !w || !k_idx || !q || !kv || !out || !lse)
     return DSA_ERR_INVALID_ARG;
+  if (k_scale == nullptr && !interleaved_ok(s)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(q) ||
       !aligned16(kv) ||
       !aligned16(out) || !aligned16(lse) || !aligned16(idx_out) || !aligned16(workspace))
@@ -645,7 +678,8 @@ dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs, co
   const bool full = d.d_idx == 128 && d.d_qk == 576;
   const bool tiny = d.d_idx == 32 && d.d_qk == 160;
   if (!full && !tiny) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (!k_new || !kv_new || !k_cache || !k_scale_cache || !kv_cache) return DSA_ERR_INVALID_ARG;
+  if (!k_new || !kv_new || !k_cache || !kv_cache) return DSA_ERR_INVALID_ARG;
+  if (k_scale_cache == nullptr && !interleaved_ok(s)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(kv_new) || !aligned16(k_cache) ||
       !aligned16(k_scale_cache) || !aligned16(kv_cache))
     return DSA_ERR_MISALIGNED;

@@ -27,7 +27,9 @@ namespace dsa {
 struct IndexerParams {
   const float* q_scale;   // [T, H_I]
   const float* w;         // [T, H_I]
-  const float* k_scale;   // [num_kv_rows]
+  const float* k_scale;   // [num_kv_rows], or null: paged decode with each block's 64 scales
+                          // stored right after its 64 key rows (k_blocks)
+  const uint8_t* k_blocks;  // interleaved layout: [num_kv_rows / 64][64 * D_I + 64 * 4] bytes
   float* scores;          // row `out_row0` of the output slab
   int64_t ld;
   int32_t* status;
@@ -214,6 +216,26 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
               y[hlf] = seq_base + blk * 64;
             }
           }
+          if (p.k_scale == nullptr) {
+            // interleaved blocks: 64 key rows (one 3-D box) and their 64 scales, contiguous
+            constexpr int64_t kBlockBytes = 64 * (D_I + 4);
+            bytes = 0;
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              sRow0[s * 2 + hlf] = y[hlf];
+              sFirst[s * 2 + hlf] = hlf * 80;
+              sValid[s * 2 + hlf] = ok[hlf] ? 64 : 0;
+              bytes += ok[hlf] ? 64 * D_I + 256 : 0;
+            }
+            mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              if (!ok[hlf]) continue;
+              const int64_t blk = y[hlf] / 64;
+              tma_load_3d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
+                          smem_u32(&full[s]), 0, 0, static_cast<int32_t>(blk));
+              bulk_load_g2s(smem_u32(sbuf + hlf * 80),
+                            p.k_blocks + blk * kBlockBytes + 64 * D_I, 256, smem_u32(&full[s]));
+            }
+          } else {
           // each box's 64 scales: a 16-byte-aligned superset of the rows, inside the cache
           uint32_t sb[2];
           int64_t a0[2];
@@ -235,6 +257,7 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
             if (sb[hlf] > 0)
               bulk_load_g2s(smem_u32(sbuf + hlf * 80), p.k_scale + a0[hlf], sb[hlf],
                             smem_u32(&full[s]));
+          }
           }
         }
         ++issued;
@@ -307,7 +330,8 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
           ks = sScale[s * C::SCALE_FLOATS + sFirst[s * 2 + hb] + j];
         } else {                               // the last rows of the cache: not bulk-copied
           const int64_t row = sRow0[s * 2 + hb] + j;
-          ks = row >= 0 && row < p.num_kv_rows ? __ldg(p.k_scale + row) : 0.f;
+          ks = p.k_scale != nullptr && row >= 0 && row < p.num_kv_rows ? __ldg(p.k_scale + row)
+                                                                          : 0.f;
         }
       }
       __syncwarp();

@@ -139,3 +139,13 @@ def test_dense_attention_needs_short_rows(dsa):
     dec = _pb(dsa, max_seqlen=4096)
     assert dsa.dsa_sparse_mla_fwd(dec, FAKE, FAKE, None, 0, 2, FAKE, FAKE, None, 0, None,
                                   0) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_scales_inside_key_blocks_only_for_paged_decode(dsa):
+    """k_scale NULL (scales stored inside the 64-row key blocks) is accepted only for paged
+    decode; elsewhere it is an argument error."""
+    dec = _pb(dsa)                                     # decode without a block table
+    assert dsa.dsa_indexer_scores(dec, FAKE, FAKE, FAKE, FAKE, None, 0, 2, FAKE, 4096, None,
+                                  0) == dsa.DSA_ERR_INVALID_ARG
+    assert dsa.dsa_cache_append(dec, FAKE, FAKE, FAKE, None, FAKE, None,
+                                0) == dsa.DSA_ERR_INVALID_ARG

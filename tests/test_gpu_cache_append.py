@@ -36,18 +36,21 @@ def _append(dsa, wl, k_new, kv_new):
     return int(status.item())
 
 
-@pytest.mark.parametrize("paged,dims", [(True, FULL), (False, dict(TINY))])
-def test_cache_append_whole_caches(dsa, paged, dims):
+@pytest.mark.parametrize("paged,dims,layout", [(True, FULL, "separate"),
+                                               (True, FULL, "interleaved"),
+                                               (False, dict(TINY), "separate")])
+def test_cache_append_whole_caches(dsa, paged, dims, layout):
     lens = [700, 64, 1, 130, 4096]
     wl = make_decode(31, len(lens), lens, dims, boost=0.0, paged=paged, device="cuda",
-                     total_blocks=400 if paged else None)
+                     total_blocks=400 if paged else None, scale_layout=layout)
     k_new, kv_new = _new_tokens(wl, 7)
     ref = oracle.cache_append(wl.k_idx, wl.k_scale, wl.kv, wl.seq_lens, wl.block_table,
                               wl.max_seqlen, k_new, kv_new)
     assert _append(dsa, wl, k_new, kv_new) == 0
     assert not ref[3].any()
     assert np.array_equal(to_np(wl.k_idx.view(torch.uint8)), ref[0])
-    assert np.array_equal(to_np(wl.k_scale), ref[1])
+    if wl.k_scale is not None:
+        assert np.array_equal(to_np(wl.k_scale), ref[1])
     assert np.array_equal(to_np(wl.kv.view(torch.int16)).view(np.uint16), ref[2])
 
 
@@ -77,14 +80,14 @@ def test_cache_append_full_size_decode_128k(dsa):
     g = np.random.default_rng(3)
     others = np.setdiff1d(g.integers(0, wl.kv.shape[0], 2000), rows)
     sel = torch.tensor(others, device="cuda")
-    before = (wl.k_idx.index_select(0, sel).clone(), wl.k_scale.index_select(0, sel).clone(),
-              wl.kv.index_select(0, sel).clone())
+    before_k = oracle.key_rows(wl, others)             # this workload's key blocks hold scales
+    before_kv = wl.kv.index_select(0, sel).clone()
     assert _append(dsa, wl, k_new, kv_new) == 0
     codes, scales = oracle.quantize_e4m3(k_new)
+    got_c, got_s = oracle.key_rows(wl, rows)
+    assert np.array_equal(got_c, codes) and np.array_equal(got_s, scales)
     r = torch.tensor(rows, device="cuda")
-    assert np.array_equal(to_np(wl.k_idx.index_select(0, r).view(torch.uint8)), codes)
-    assert np.array_equal(to_np(wl.k_scale.index_select(0, r)), scales)
     assert torch.equal(wl.kv.index_select(0, r), kv_new)
-    assert torch.equal(wl.k_idx.index_select(0, sel), before[0])
-    assert torch.equal(wl.k_scale.index_select(0, sel), before[1])
-    assert torch.equal(wl.kv.index_select(0, sel), before[2])
+    after_k = oracle.key_rows(wl, others)
+    assert np.array_equal(after_k[0], before_k[0]) and np.array_equal(after_k[1], before_k[1])
+    assert torch.equal(wl.kv.index_select(0, sel), before_kv)

@@ -102,6 +102,23 @@ def test_indexer_decode_paged_ragged(dsa):
     _indexer_case(dsa, wl, [0, 1, 2, 3])
 
 
+def test_indexer_decode_paged_interleaved_scales(dsa):
+    """The paged indexer cache with each block's scales after its key rows: scores equal,
+    bit for bit, those of the same keys in separate arrays, and the oracle's."""
+    lens = [3000, 64, 1, 200, 131]
+    a = make_decode(17, 5, lens, FULL, boost=0.01, paged=True, device="cuda")
+    b = make_decode(17, 5, lens, FULL, boost=0.01, paged=True, device="cuda",
+                    scale_layout="interleaved")
+    sa = run_indexer(dsa, a)
+    sb = run_indexer(dsa, b)
+    for r, n in enumerate(lens):
+        assert torch.equal(sa[r, :n], sb[r, :n]), r
+    ref = oracle.indexer_rows(b, list(range(5)))
+    sc = to_np(sb)
+    for r in range(5):
+        check_scores(sc[r, :len(ref[r])], ref[r], f"row {r}")
+
+
 def test_indexer_bad_block_reported(dsa):
     """A block-table entry that is negative or past the cache is skipped and reported as
     DSA_DEVICE_BAD_INDEX; the other sequences' scores are unaffected."""

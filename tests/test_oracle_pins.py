@@ -400,3 +400,31 @@ def test_cache_append_paged_equals_contiguous():
     _, _, _, bad3 = oracle.cache_append(wl.k_idx, wl.k_scale, wl.kv, lens_bad, bt,
                                         wl.max_seqlen, k_new, kv_new)
     assert list(bad3) == [True, False, True, True]
+
+
+def test_interleaved_key_blocks_hold_the_same_keys():
+    """A paged indexer cache whose 64-row blocks carry their own scales holds exactly the keys
+    and scales of the separate layout (same seed), and an append lands on the same bytes."""
+    from dsa_workloads import make_decode, FULL
+    a = make_decode(62, 3, [700, 64, 200], FULL, boost=0.01, paged=True, device="cpu")
+    b = make_decode(62, 3, [700, 64, 200], FULL, boost=0.01, paged=True, device="cpu",
+                    scale_layout="interleaved")
+    assert b.k_scale is None and b.k_idx.shape == (a.kv.shape[0] // 64, 64 * (128 + 4))
+    phys = np.arange(a.kv.shape[0])
+    ca, sa = oracle.key_rows(a, phys)
+    cb, sb = oracle.key_rows(b, phys)
+    assert np.array_equal(ca, cb) and np.array_equal(sa, sb)
+    g = np.random.default_rng(4)
+    k_new = g.standard_normal((3, 128)).astype(np.float32)
+    kv_new = np.zeros((3, 576), np.uint16)
+    ra = oracle.cache_append(a.k_idx, a.k_scale, a.kv, a.seq_lens, a.block_table,
+                             a.max_seqlen, k_new, kv_new)
+    rb = oracle.cache_append(b.k_idx, None, b.kv, b.seq_lens, b.block_table,
+                             b.max_seqlen, k_new, kv_new)
+    assert rb[1] is None
+    a2 = type(a)(**{**a.__dict__, "k_idx": torch.from_numpy(ra[0]),
+                    "k_scale": torch.from_numpy(ra[1])})
+    b2 = type(b)(**{**b.__dict__, "k_idx": torch.from_numpy(rb[0])})
+    c2a, s2a = oracle.key_rows(a2, phys)
+    c2b, s2b = oracle.key_rows(b2, phys)
+    assert np.array_equal(c2a, c2b) and np.array_equal(s2a, s2b)
