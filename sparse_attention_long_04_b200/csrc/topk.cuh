@@ -278,13 +278,16 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   __syncthreads();
 
   if (in_bin_total != need) {                     // else: every key of the bin is taken
-    if (in_bin_total <= static_cast<uint32_t>(kTopkCand)) {
-      // ---- gather the bin's keys into CTA 0 and resolve the last 21 bits there
+    if (in_bin_total + 3u * C <= static_cast<uint32_t>(kTopkCand)) {
+      // ---- gather the bin's keys into CTA 0 and resolve the last 21 bits there.  Each CTA
+      // reserves a multiple of 4 slots, compacts its keys locally (CTA 0: in place), pads with
+      // a key outside the bin and copies 16 bytes at a time into CTA 0's buffer.
+      const uint32_t n4 = (in_bin_local + 3u) & ~3u;
+      const uint32_t pad_key = bin == 0 ? 0xFFFFFFFFu : 0u;   // never matches the bin
       if (tid == 0)
-        s_base = in_bin_local ? (C > 1 ? atom_cluster_add(map_to_rank(smem_u32(&s_ncand), 0),
-                                                           in_bin_local)
-                                       : atomicAdd(&s_ncand, in_bin_local))
-                              : 0u;
+        s_base = n4 ? (C > 1 ? atom_cluster_add(map_to_rank(smem_u32(&s_ncand), 0), n4)
+                             : atomicAdd(&s_ncand, n4))
+                    : 0u;
       if (C > 1) cluster_sync(); else __syncthreads();   // reservations done (CTA 0's count)
       uint32_t mine = 0;                           // this thread's matches, in its 4-key groups
       const int nrounds = (m + kTopkThreads * 4 - 1) / (kTopkThreads * 4);
@@ -299,8 +302,8 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
         }
       }
       uint32_t tot;
-      uint32_t slot = s_base + cta_excl_scan(mine, tmp, &tot);
-      const uint32_t dst0 = C > 1 ? map_to_rank(smem_u32(cand), 0) : smem_u32(cand);
+      const uint32_t lbase = crank == 0 ? s_base : 0u;   // where this CTA compacts locally
+      uint32_t slot = lbase + cta_excl_scan(mine, tmp, &tot);
       for (int u = 0; u < nrounds && mine; ++u) {
         const int i4 = (u * kTopkThreads + tid) * 4;
         if (i4 < m) {
@@ -308,12 +311,15 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
           const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (i4 + e < m && (kk[e] & mask) == prefix) {
-              if (C > 1) st_cluster_u32(dst0 + slot * 4, kk[e]);
-              else cand[slot] = kk[e];
-              ++slot;
-            }
+            if (i4 + e < m && (kk[e] & mask) == prefix) cand[slot++] = kk[e];
         }
+      }
+      if (tid < static_cast<int>(n4 - in_bin_local)) cand[lbase + in_bin_local + tid] = pad_key;
+      __syncthreads();
+      if (C > 1 && crank != 0) {
+        const uint32_t dst0 = map_to_rank(smem_u32(cand), 0) + s_base * 4;
+        const uint4* src4 = reinterpret_cast<const uint4*>(cand);
+        for (uint32_t j = tid; j < n4 / 4; j += kTopkThreads) st_cluster_u4(dst0 + j * 16, src4[j]);
       }
       if (C > 1) cluster_sync(); else __syncthreads();   // CTA 0 holds every candidate
       if (crank == 0) {
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
           const uint32_t nb = 1u << kBits[pass];
           for (uint32_t i = tid; i < nb; i += kTopkThreads) hsum[i] = 0;
           __syncthreads();
-          for (uint32_t i = tid; i < in_bin_total; i += kTopkThreads) {
+          for (uint32_t i = tid; i < s_ncand; i += kTopkThreads) {
             const uint32_t k = cand[i];
             if ((k & mask) == prefix) atomicAdd(&hsum[(k >> kShift[pass]) & (nb - 1)], 1u);
           }
@@ -441,8 +447,11 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
     w_out += wgt[w] + (need > w_eq ? min(need - w_eq, weq[w]) : 0u);
     w_eq += weq[w];
   }
-  // 128 keys per round: lane j holds keys 4j..4j+3 of the round (index order = lane order)
-  for (int b0 = w0; b0 < w1; b0 += 128) {
+  // 128 keys per round: lane j holds keys 4j..4j+3 of the round (index order = lane order).
+  // Few keys are taken (topk of the row): a warp with none skips the loop, a round with none
+  // skips the scans.
+  const bool warp_has = wgt[warp] + weq[warp] != 0;
+  for (int b0 = w0; warp_has && b0 < w1; b0 += 128) {
     const int i4 = b0 + lane * 4;
     const uint4 k = i4 < w1 ? key4_at(i4) : make_uint4(0, 0, 0, 0);
     const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
@@ -455,18 +464,20 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
         eqm |= (km == prefix ? 1u : 0u) << e;
       }
     }
+    if (!__any_sync(0xffffffffu, (gtm | eqm) != 0)) continue;   // nothing here: offsets unchanged
+    // counts over the lanes before this one (index order) from one ballot per key slot
+    const uint32_t lt = (1u << lane) - 1u;
     uint32_t take = gtm | eqm;
-    uint32_t inc = 0;
+    uint32_t round_eq = 0;
     if (!all_eq) {
-      // eq rank of this lane's first key: exclusive scan of eq counts over lanes
-      const uint32_t neq = __popc(eqm);
-      inc = neq;
+      uint32_t eq_before = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t be = __ballot_sync(0xffffffffu, (eqm >> e) & 1u);
+        eq_before += __popc(be & lt);
+        round_eq += __popc(be);
       }
-      uint32_t eq_rank = w_eq + inc - neq;
+      uint32_t eq_rank = w_eq + eq_before;      // rank of this lane's first key == tau
       take = gtm;
 #pragma unroll
       for (int e = 0; e < 4; ++e)
@@ -475,22 +486,22 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
           ++eq_rank;
         }
     }
-    const uint32_t ntake = __popc(take);
-    uint32_t tinc = ntake;
+    uint32_t before = 0, round_take = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, tinc, o);
-      if (lane >= o) tinc += y;
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t bt = __ballot_sync(0xffffffffu, (take >> e) & 1u);
+      before += __popc(bt & lt);
+      round_take += __popc(bt);
     }
-    uint32_t pos = w_out + tinc - ntake;
+    uint32_t pos = w_out + before;
 #pragma unroll
     for (int e = 0; e < 4; ++e)
       if ((take >> e) & 1u) {
         if (pos < static_cast<uint32_t>(K)) out[pos] = s0 + i4 + e;
         ++pos;
       }
-    w_out += __shfl_sync(0xffffffffu, tinc, 31);
-    if (!all_eq) w_eq += __shfl_sync(0xffffffffu, inc, 31);
+    w_out += round_take;
+    if (!all_eq) w_eq += round_eq;
   }
 }
 
