@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(512, 1)
       abort_s = 1;
       if (p.status) atomicOr(p.status, kStatusTimeout);
     }
-    cp_async_wait<0>();   // nothing may still be writing this CTA's shared memory at exit
+    cp_async_wait_all();   // nothing may still be writing this CTA's shared memory at exit
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     const int hrow = (warp & 3) * 32 + lane;    // head = TMEM lane
