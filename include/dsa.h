@@ -225,6 +225,14 @@ DSA_API dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* 
 DSA_API dsa_status_t dsa_read_device_status(const int32_t* dev_status, dsa_stream_t stream,
                                     int32_t* raw);
 
+/* Diagnostics: checks that a wait which never completes ends instead of hanging.  Launches one
+ * CTA of two warps that wait, with the same bounded wait every kernel above uses (2 s limit), on
+ * an mbarrier nothing arrives at; each warp that gives up ORs DSA_DEVICE_TIMEOUT into
+ * *dev_status (device, 4-byte aligned, caller-owned) and the CTA then exits normally, leaving the
+ * context usable.  Asynchronous on `stream`, which stays busy for about 2 s; read the word with
+ * dsa_read_device_status, which then returns DSA_ERR_TIMEOUT. */
+DSA_API dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream);
+
 DSA_API const char* dsa_status_string(dsa_status_t status);
 DSA_API int32_t dsa_abi_version(void);
 

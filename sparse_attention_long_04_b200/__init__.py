@@ -37,7 +37,7 @@ DSA_DECODE = 1
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_fwd", "dsa_forward_workspace_size", "dsa_forward",
             "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-            "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append")
+            "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -78,6 +78,7 @@ def _load():
         "dsa_forward_workspace_size": (SZ, [DP, SP]),
         "dsa_forward": (I32, [DP, SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
+        "dsa_selftest_wait_timeout": (I32, [P, P]),
         "dsa_status_string": (ctypes.c_char_p, [I32]),
         "dsa_abi_version": (I32, []),
         "dsa_sparse_mla_fwd_noalloc": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, P]),
@@ -233,6 +234,10 @@ def dsa_cache_append(pb: Problem, k_new, kv_new, k_cache, k_scale_cache, kv_cach
     return int(lib.dsa_cache_append(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(k_new), _ptr(kv_new), _ptr(k_cache),
         _ptr(k_scale_cache), _ptr(kv_cache), _ptr(dev_status), _stream(stream)))
+
+
+def dsa_selftest_wait_timeout(dev_status, stream=None) -> int:
+    return int(lib.dsa_selftest_wait_timeout(_ptr(dev_status), _stream(stream)))
 
 
 def dsa_read_device_status(dev_status, stream=None):

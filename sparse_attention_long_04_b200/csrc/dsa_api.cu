@@ -506,6 +506,27 @@ ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count)
   return p;
 }
 
+// ---------------------------------------------------------------- bounded-wait self-test
+
+// One CTA waits on an mbarrier that nothing arrives at, with the wait every kernel here uses
+// (lane 0 polls, 2 s limit, then the whole warp gives up).  As in the kernels above, the first
+// warp to give up raises the CTA's abort flag so that the other ends its wait early; each warp
+// records a timeout in the status word and the CTA then exits normally.
+__global__ void __launch_bounds__(64) dsa_selftest_wait_kernel(int32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (!warp_mbar_wait(smem_u32(&bar), 0, &abort_flag) && (threadIdx.x & 31) == 0) {
+    abort_flag = 1;
+    atomicOr(status, kStatusTimeout);
+  }
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -703,6 +724,14 @@ dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs, co
     dsa_cache_append_kernel<128, 576><<<grid, 128, 0, st>>>(prm);
   else
     dsa_cache_append_kernel<32, 160><<<grid, 128, 0, st>>>(prm);
+  return launch_status();
+}
+
+dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream) {
+  if (dev_status == nullptr) return DSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return DSA_ERR_MISALIGNED;
+  dsa_selftest_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(dev_status);
   return launch_status();
 }
 

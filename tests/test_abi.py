@@ -149,3 +149,10 @@ def test_scales_inside_key_blocks_only_for_paged_decode(dsa):
                                   0) == dsa.DSA_ERR_INVALID_ARG
     assert dsa.dsa_cache_append(dec, FAKE, FAKE, FAKE, None, FAKE, None,
                                 0) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_wait_selftest_argument_errors(dsa):
+    """The bounded-wait self-test needs a 4-byte-aligned status word; both are checked before
+    any launch."""
+    assert dsa.dsa_selftest_wait_timeout(None, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert dsa.dsa_selftest_wait_timeout(FAKE + 2, 0) == dsa.DSA_ERR_MISALIGNED
