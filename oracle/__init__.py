@@ -14,6 +14,9 @@ summary):
   sparse_mla_rows   MQA-mode attention over the selected latent rows, fp64, with LSE
   quantize_e4m3     per-row e4m3 quantisation (scale = amax / 448), the decode cache append's
   cache_append      arithmetic; cache_append writes a decode step's new token into the caches
+  kl_target_rows    the indexer's training target: the main attention's head-summed distribution
+                    on the selected keys ("Training signal")
+  indexer_kl_rows   KL(target || softmax of the indexer scores) and its gradients for w, q, k
 
 The C library ``dsa_oracle.c`` does the arithmetic (OpenMP over rows); this module only
 resolves which physical cache row holds logical key s of a sequence and moves bytes.
@@ -61,6 +64,14 @@ def lib():
         L.dsa_oracle_quantize_e4m3.restype = None
         L.dsa_oracle_quantize_e4m3.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                                ctypes.c_void_p, ctypes.c_void_p]
+        L.dsa_oracle_attn_target.restype = None
+        L.dsa_oracle_attn_target.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, f64p]
+        L.dsa_oracle_indexer_kl.restype = None
+        L.dsa_oracle_indexer_kl.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, f64p, f64p, f64p,
+            ctypes.c_void_p, f64p, f64p, f64p, f64p, f64p, f64p]
         L.dsa_oracle_num_threads.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -251,6 +262,94 @@ def forward_rows(wl, rows: Sequence[int]):
     idx = topk_rows([sc[r] for r in rows], wl.dims["topk"])
     o, lse = sparse_mla_rows(wl, rows, idx)
     return sc, idx, o, lse
+
+
+# ---- indexer training signal -----------------------------------------------------------------
+
+def _selected_phys(geo, rows, idx):
+    """Physical cache rows of the selected logical keys (-1 where idx < 0)."""
+    phys = np.full(idx.shape, -1, dtype=np.int64)
+    for i, r in enumerate(rows):
+        b, _ = geo.row_seq_pos(r)
+        sel = idx[i] >= 0
+        phys[i, sel] = geo.phys(b, idx[i, sel])
+    return phys
+
+
+def kl_target_rows(wl, rows: Sequence[int], idx: np.ndarray) -> np.ndarray:
+    """The indexer's training target on the selected keys: the main attention's distribution
+    summed over heads and normalised (mean over heads of each head's softmax), float64
+    [n_rows, k]; 0 where idx < 0."""
+    geo = Geometry.of(wl)
+    d = wl.dims
+    idx = np.asarray(idx)
+    k = idx.shape[1]
+    phys = _selected_phys(geo, rows, idx)
+    qq = _take(wl.q, list(rows))
+    used = np.unique(phys[phys >= 0])
+    kv = _take(wl.kv, used) if len(used) else np.zeros((1, d["d_qk"]), np.uint16)
+    compact = np.full(phys.shape, -1, dtype=np.int64)
+    compact[phys >= 0] = np.searchsorted(used, phys[phys >= 0])
+    out = np.empty((len(rows), k), dtype=np.float64)
+    lib().dsa_oracle_attn_target(len(rows), d["h"], d["d_qk"], float(wl.softmax_scale),
+                                 _ptr(qq), _ptr(kv), _ptr(compact), k, _f64p(out))
+    return out
+
+
+def _e4m3_table() -> np.ndarray:
+    return np.array([e4m3_to_f64(b) for b in range(256)], dtype=np.float64)
+
+
+def indexer_kl_rows(wl, rows: Sequence[int], idx: np.ndarray, target: np.ndarray) -> dict:
+    """KL(target || softmax of the indexer scores) on the selected keys of each row, and its
+    gradients with respect to the indexer weights w, the real-valued indexer queries
+    (s_q * q-hat) and the real-valued indexer keys (s_k * k-hat).  Returns float64 arrays:
+    loss [n], scores [n, k], dw [n, h_idx], dq [n, h_idx, d_idx], and dk [u, d_idx] summed
+    over the given rows for the physical key rows dk_rows [u]."""
+    geo = Geometry.of(wl)
+    d = wl.dims
+    h_idx, d_idx = d["h_idx"], d["d_idx"]
+    idx = np.asarray(idx)
+    n, k = idx.shape
+    tab = _e4m3_table()
+    qc = _take(wl.q_idx, list(rows), np.uint8).reshape(n, h_idx, d_idx)
+    qs = _take(wl.q_scale, list(rows), np.float32).reshape(n, h_idx).astype(np.float64)
+    q = np.ascontiguousarray(tab[qc] * qs[:, :, None])
+    w = np.ascontiguousarray(_take(wl.w, list(rows), np.float32).reshape(n, h_idx), np.float64)
+    phys = _selected_phys(geo, rows, idx)
+    valid = (phys >= 0).astype(np.int32)
+    keys = np.zeros((n, k, d_idx), dtype=np.float64)
+    if valid.any():
+        codes, scales = key_rows(wl, phys[phys >= 0])
+        keys[phys >= 0] = tab[codes] * scales.astype(np.float64)[:, None]
+    res = indexer_kl_real(q, w, keys, valid, target)
+    dk_rows, inv = np.unique(phys[phys >= 0], return_inverse=True)
+    dk = np.zeros((len(dk_rows), d_idx))
+    np.add.at(dk, inv, res.pop("dk")[phys >= 0])
+    res.update(dk_rows=dk_rows, dk=dk)
+    return res
+
+
+def indexer_kl_real(q, w, keys, valid, target) -> dict:
+    """The same loss and gradients on real-valued inputs given directly (float64 q [n, h, d],
+    w [n, h], keys [n, k, d], valid [n, k], target [n, k]); dk is per selected entry,
+    [n, k, d]."""
+    q = np.ascontiguousarray(q, np.float64)
+    w = np.ascontiguousarray(w, np.float64)
+    keys = np.ascontiguousarray(keys, np.float64)
+    valid = np.ascontiguousarray(valid, np.int32)
+    tgt = np.ascontiguousarray(target, np.float64)
+    n, h_idx, d_idx = q.shape
+    k = keys.shape[1]
+    loss = np.empty(n)
+    scores = np.empty((n, k))
+    dw = np.empty((n, h_idx))
+    dq = np.empty((n, h_idx, d_idx))
+    dkeys = np.empty((n, k, d_idx))
+    lib().dsa_oracle_indexer_kl(n, h_idx, d_idx, k, _f64p(q), _f64p(w), _f64p(keys),
+                                _ptr(valid), _f64p(tgt), _f64p(loss), _f64p(scores),
+                                _f64p(dw), _f64p(dq), _f64p(dkeys))
+    return dict(loss=loss, scores=scores, dw=dw, dq=dq, dk=dkeys)
 
 
 # ---- decode cache append ---------------------------------------------------------------------

@@ -21,6 +21,10 @@
  *             (same page, "Instantiation"); logits l_s = sigma * q.kv[s], O = softmax-
  *             weighted sum of the first d_v latent dims, LSE = log sum exp(l_s)
  *
+ * The indexer's training signal (same page, "Training signal": the indexer imitates the main
+ * attention's head-summed distribution through a KL divergence) is written out too: the target
+ * distribution on the selected keys and the loss with its gradients for w, q and k.
+ *
  * Floating point: e4m3 and bf16 inputs are decoded exactly; the indexer runs in fp64 (or
  * in fp32 with index-ordered accumulation when asked), attention runs in fp64.  The decode
  * cache append quantises the new token's indexer key per token to e4m3 ("FP8 index", same
@@ -195,6 +199,140 @@ void dsa_oracle_sparse_mla(int n_rows, int h, int d_qk, int d_v, double scale,
     free(qd);
     free(logit);
     free(acc);
+  }
+}
+
+/* ---- indexer training signal --------------------------------------------------------------- */
+
+/* The indexer learns to imitate the main attention's head-summed distribution through a KL
+ * divergence ("DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention (DSA)",
+ * "Training signal").  In the sparse stage both distributions live on the selected keys.
+ *
+ * Target, for each row r over the physical latent rows rows[r, 0..k) that are >= 0:
+ *   l_{h,e} = scale * sum_{i<d_qk} q[r,h,i] * kv[rows[r,e], i]
+ *   LSE_h   = ln sum_e exp(l_{h,e})                         (over the selection)
+ *   t_e     = (1/h) sum_h exp(l_{h,e} - LSE_h)              (each head's distribution sums to 1,
+ *                                                            so t does too)
+ * Entries with rows < 0 get 0; a row with no valid entry is all 0.  q and kv are bf16 bit
+ * patterns; the arithmetic is binary64. */
+void dsa_oracle_attn_target(int n_rows, int h, int d_qk, double scale, const uint16_t* q,
+                            const uint16_t* kv, const int64_t* rows, int k, double* target) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int r = 0; r < n_rows; ++r) {
+    double* qd = (double*)malloc(sizeof(double) * (size_t)d_qk);
+    double* logit = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+    const int64_t* sel = rows + (int64_t)r * k;
+    double* t = target + (int64_t)r * k;
+    for (int e = 0; e < k; ++e) t[e] = 0.0;
+    for (int hh = 0; hh < h; ++hh) {
+      const uint16_t* qrow = q + ((int64_t)r * h + hh) * d_qk;
+      for (int i = 0; i < d_qk; ++i) qd[i] = dsa_oracle_bf16_to_f64(qrow[i]);
+      double m = -INFINITY;
+      for (int e = 0; e < k; ++e) {
+        if (sel[e] < 0) continue;
+        const uint16_t* kr = kv + sel[e] * (int64_t)d_qk;
+        double dot = 0.0;
+        for (int i = 0; i < d_qk; ++i) dot += qd[i] * dsa_oracle_bf16_to_f64(kr[i]);
+        logit[e] = scale * dot;
+        if (logit[e] > m) m = logit[e];
+      }
+      if (m == -INFINITY) continue;
+      double z = 0.0;
+      for (int e = 0; e < k; ++e)
+        if (sel[e] >= 0) z += exp(logit[e] - m);
+      const double lse = m + log(z);
+      for (int e = 0; e < k; ++e)
+        if (sel[e] >= 0) t[e] += exp(logit[e] - lse) / (double)h;
+    }
+    free(qd);
+    free(logit);
+  }
+}
+
+/* KL loss of the indexer against a target distribution, and its gradients.  Per row r, over
+ * the entries e < k with valid[r,e] != 0 (the selected keys), with real-valued inputs (the
+ * fp8 codes times their scales):
+ *   D_{j,e} = sum_{i<d} q[r,j,i] * keys[r,e,i]
+ *   S_e     = sum_j w[r,j] * max(D_{j,e}, 0)                 (the indexer score)
+ *   pi      = softmax_e(S)
+ *   loss_r  = sum_e p_e (ln p_e - ln pi_e)  with p = target[r, :] and 0 ln 0 = 0
+ *   g_e     = dloss/dS_e = pi_e * sum_f p_f - p_e
+ *   dw[r,j]      = sum_e g_e max(D_{j,e}, 0)
+ *   dq[r,j,:]    = sum_e g_e w[r,j] [D_{j,e} > 0] keys[r,e,:]
+ *   dkeys[r,e,:] = sum_j g_e w[r,j] [D_{j,e} > 0] q[r,j,:]
+ * (the derivative of max(x, 0) at x = 0 is taken as 0).  Invalid entries get S = -inf and
+ * zero gradients.  scores [n_rows, k] receives S.  Binary64 throughout. */
+void dsa_oracle_indexer_kl(int n_rows, int h_idx, int d, int k, const double* q,
+                           const double* w, const double* keys, const int32_t* valid,
+                           const double* target, double* loss, double* scores, double* dw,
+                           double* dq, double* dkeys) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int r = 0; r < n_rows; ++r) {
+    const double* qr = q + (int64_t)r * h_idx * d;
+    const double* wr = w + (int64_t)r * h_idx;
+    const double* kr = keys + (int64_t)r * k * d;
+    const int32_t* vr = valid + (int64_t)r * k;
+    const double* pr = target + (int64_t)r * k;
+    double* sr = scores + (int64_t)r * k;
+    double* dot = (double*)malloc(sizeof(double) * (size_t)h_idx * (size_t)(k > 0 ? k : 1));
+    double* g = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+    /* scores */
+    double m = -INFINITY;
+    for (int e = 0; e < k; ++e) {
+      sr[e] = -INFINITY;
+      if (!vr[e]) continue;
+      double acc = 0.0;
+      for (int j = 0; j < h_idx; ++j) {
+        double dd = 0.0;
+        for (int i = 0; i < d; ++i) dd += qr[j * d + i] * kr[(int64_t)e * d + i];
+        dot[(int64_t)j * k + e] = dd;
+        acc += wr[j] * (dd > 0.0 ? dd : 0.0);
+      }
+      sr[e] = acc;
+      if (acc > m) m = acc;
+    }
+    /* softmax, loss, dloss/dS */
+    double z = 0.0, psum = 0.0, l = 0.0;
+    for (int e = 0; e < k; ++e)
+      if (vr[e]) {
+        z += exp(sr[e] - m);
+        psum += pr[e];
+      }
+    const double logz = (m == -INFINITY) ? 0.0 : m + log(z);
+    for (int e = 0; e < k; ++e) {
+      g[e] = 0.0;
+      if (!vr[e]) continue;
+      const double logpi = sr[e] - logz;
+      if (pr[e] > 0.0) l += pr[e] * (log(pr[e]) - logpi);
+      g[e] = exp(logpi) * psum - pr[e];
+    }
+    loss[r] = l;
+    /* gradients */
+    for (int j = 0; j < h_idx; ++j) {
+      double a = 0.0;
+      for (int e = 0; e < k; ++e)
+        if (vr[e]) {
+          const double dd = dot[(int64_t)j * k + e];
+          a += g[e] * (dd > 0.0 ? dd : 0.0);
+        }
+      dw[(int64_t)r * h_idx + j] = a;
+      for (int i = 0; i < d; ++i) {
+        double b = 0.0;
+        for (int e = 0; e < k; ++e)
+          if (vr[e] && dot[(int64_t)j * k + e] > 0.0) b += g[e] * kr[(int64_t)e * d + i];
+        dq[((int64_t)r * h_idx + j) * d + i] = wr[j] * b;
+      }
+    }
+    for (int e = 0; e < k; ++e)
+      for (int i = 0; i < d; ++i) {
+        double c = 0.0;
+        if (vr[e])
+          for (int j = 0; j < h_idx; ++j)
+            if (dot[(int64_t)j * k + e] > 0.0) c += wr[j] * qr[j * d + i];
+        dkeys[((int64_t)r * k + e) * d + i] = g[e] * c;
+      }
+    free(dot);
+    free(g);
   }
 }
 

@@ -428,3 +428,124 @@ def test_interleaved_key_blocks_hold_the_same_keys():
     c2a, s2a = oracle.key_rows(a2, phys)
     c2b, s2b = oracle.key_rows(b2, phys)
     assert np.array_equal(c2a, c2b) and np.array_equal(s2a, s2b)
+
+
+# ---------------------------------------------------------------- indexer training signal
+
+def test_kl_target_is_the_head_mean_of_the_attention_weights():
+    """With no more selected keys than value dims, the head-mean of the attention outputs
+    (pinned against torch's SDPA above) determines the head-mean of the attention weights:
+    mean_h O[h] = sum_e t_e v_e.  The target must be that solution, sum to 1, and be 0 on
+    unused slots."""
+    wl = _tiny_attn_workload()
+    kvd = wl.kv.double().numpy()
+    rows = [30, 33, 39]
+    idx = np.array([[3, 11, 0, -1, 25, 7, 30, -1],
+                    [33, -1, 1, 2, 5, 8, 13, 21],
+                    [39, 38, 37, 4, -1, -1, -1, -1]], np.int32)
+    t = oracle.kl_target_rows(wl, rows, idx)
+    o, _ = oracle.sparse_mla_rows(wl, rows, idx)
+    for i in range(len(rows)):
+        sel = idx[i] >= 0
+        assert (t[i, ~sel] == 0).all()
+        assert t[i].sum() == pytest.approx(1.0, abs=1e-13)
+        v = kvd[idx[i, sel], :16]                        # [n_sel, d_v], independent rows
+        sol, *_ = np.linalg.lstsq(v.T, o[i].mean(axis=0), rcond=None)
+        np.testing.assert_allclose(t[i, sel], sol, rtol=1e-9, atol=1e-12)
+
+
+def test_kl_target_closed_forms():
+    wl = _tiny_attn_workload()
+    t = oracle.kl_target_rows(wl, [30, 30], np.array([[-1, 17, -1], [9, 9, 9]], np.int32))
+    assert list(t[0]) == [0.0, 1.0, 0.0]                # one key: all the mass
+    np.testing.assert_allclose(t[1], [1 / 3] * 3, rtol=1e-14)   # identical keys: uniform
+    assert not oracle.kl_target_rows(wl, [5], np.full((1, 4), -1, np.int32)).any()
+
+
+def _kl_workload():
+    dims = dict(h_idx=4, d_idx=32, topk=16, h=4, d_qk=24, d_v=16)
+    return make_prefill(95, [60], dims, needles=4, device="cpu", seed=5, softmax_scale=0.3)
+
+
+def test_indexer_kl_loss_is_scipy_kl_on_the_indexer_scores():
+    """The loss is scipy's relative entropy of the target against the softmax of the indexer
+    scores (those of the pinned indexer oracle) on each row's selected keys."""
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    wl = _kl_workload()
+    rows = [3, 17, 40, 59]
+    sc, idx, _, _ = oracle.forward_rows(wl, rows)
+    target = oracle.kl_target_rows(wl, rows, idx)
+    res = oracle.indexer_kl_rows(wl, rows, idx, target)
+    for i, r in enumerate(rows):
+        sel = idx[i] >= 0
+        assert (res["scores"][i, ~sel] == -np.inf).all()
+        np.testing.assert_allclose(res["scores"][i, sel], sc[r][idx[i, sel]], rtol=1e-12,
+                                   atol=1e-14)
+        ref = entropy(target[i, sel], softmax(sc[r][idx[i, sel]]))
+        assert res["loss"][i] == pytest.approx(ref, rel=1e-10, abs=1e-14)
+
+
+def _random_real_case(seed, n=2, h=3, d=5, k=7):
+    """Real-valued inputs whose dot products stay away from the ReLU kink."""
+    g = np.random.default_rng(seed)
+    while True:
+        q = g.standard_normal((n, h, d))
+        keys = g.standard_normal((n, k, d))
+        if np.abs(np.einsum("rjd,red->rje", q, keys)).min() > 0.05:
+            break
+    w = g.uniform(0.2, 1.5, (n, h))
+    valid = np.ones((n, k), np.int32)
+    valid[0, 2] = 0
+    target = g.uniform(0.1, 1.0, (n, k)) * valid
+    target[0] /= target[0].sum()
+    target[1] *= 0.7 / target[1].sum()                  # a target that does not sum to 1
+    return q, w, keys, valid, target
+
+
+def test_indexer_kl_gradients_match_finite_differences():
+    q, w, keys, valid, target = _random_real_case(11)
+    res = oracle.indexer_kl_real(q, w, keys, valid, target)
+    f = lambda q_, w_, k_: oracle.indexer_kl_real(q_, w_, k_, valid, target)["loss"].sum()
+    eps = 1e-6
+    for name, arr, grad in (("q", q, res["dq"]), ("w", w, res["dw"]), ("keys", keys, res["dk"])):
+        num = np.zeros_like(arr)
+        for ix in np.ndindex(arr.shape):
+            a, b = arr.copy(), arr.copy()
+            a[ix] += eps
+            b[ix] -= eps
+            args = {"q": (q, w, keys), "w": (q, w, keys), "keys": (q, w, keys)}[name]
+            fa = f(*(a if x is arr else x for x in args))
+            fb = f(*(b if x is arr else x for x in args))
+            num[ix] = (fa - fb) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+    assert not res["dk"][0, 2].any()                    # unused slot: no gradient
+
+
+def test_indexer_kl_vanishes_when_the_target_is_the_indexer_distribution():
+    from scipy.special import softmax
+    q, w, keys, valid, _ = _random_real_case(12)
+    s = np.maximum(np.einsum("rjd,red->rje", q, keys), 0.0)
+    scores = np.einsum("rj,rje->re", w, s)
+    target = np.where(valid > 0, softmax(np.where(valid > 0, scores, -np.inf), axis=1), 0.0)
+    res = oracle.indexer_kl_real(q, w, keys, valid, target)
+    assert np.abs(res["loss"]).max() < 1e-14
+    for key in ("dq", "dw", "dk"):
+        assert np.abs(res[key]).max() < 1e-13, key
+
+
+def test_indexer_kl_key_gradient_sums_over_rows():
+    """A physical key selected by several rows receives the sum of their gradients."""
+    wl = _kl_workload()
+    rows = [40, 41, 59]
+    _, idx, _, _ = oracle.forward_rows(wl, rows)
+    target = oracle.kl_target_rows(wl, rows, idx)
+    both = oracle.indexer_kl_rows(wl, rows, idx, target)
+    acc = {}
+    for i, r in enumerate(rows):
+        one = oracle.indexer_kl_rows(wl, [r], idx[i:i + 1], target[i:i + 1])
+        for p, g in zip(one["dk_rows"], one["dk"]):
+            acc[int(p)] = acc.get(int(p), 0.0) + g
+    assert sorted(acc) == both["dk_rows"].tolist()
+    for p, g in zip(both["dk_rows"], both["dk"]):
+        np.testing.assert_allclose(g, acc[int(p)], rtol=1e-12, atol=1e-15)
