@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DECODE_CFG, PREFILL_CFG = 3, 5
+TRAIN_CFG = 4   # the indexer's training step runs on prefill_L16k (one causal 16384-row sequence)
 METRIC = "DSA decode tokens/s and prefill tokens/s at 128k ctx; % of HBM/tensor roofline"
 
 
@@ -149,6 +150,18 @@ def prefill_flops(seqlens, d):
         m = min(L, K)
         sel += m * (m + 1) // 2 + (L - m) * K
     return (2 * d["h_idx"] * d["d_idx"] * pairs, 2 * d["h"] * (d["d_qk"] + d["d_v"]) * sel)
+
+
+def train_flops(seqlens, d):
+    """Algorithmic FLOPs of one indexer training step on the top-k selection: the target's
+    logits, 2*H*D_qk per (query, selected key) (bf16); the backward's three contractions (D,
+    dq, dk), 3 * 2*H_I*D_I per (query, selected key) (fp32)."""
+    K = d["topk"]
+    sel = 0
+    for L in seqlens:
+        m = min(L, K)
+        sel += m * (m + 1) // 2 + (L - m) * K
+    return 2 * d["h"] * d["d_qk"] * sel, 3 * 2 * d["h_idx"] * d["d_idx"] * sel
 
 
 # ------------------------------------------------------------------------------ our arm
@@ -339,6 +352,9 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_prefill:
         del scores, idx, out, lse
         line["prefill"] = run_prefill(args, dsa, dev, stream, peaks, rank, world)
+    if not args.no_train:
+        line["indexer_train"] = run_indexer_train(args, dsa, dev, stream, peaks, rank, world,
+                                                  clk, cpu_leg=rank == 0 and not args.no_cpu)
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     return line
@@ -375,6 +391,97 @@ def run_prefill(args, dsa, dev, stream, peaks, rank, world):
                         "peak_fp8_tflops": p8,
                         "peak_note": "bf16 sustained measured; fp8 = 2x bf16 (nominal ratio)"}}
     del fwd, wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, clk, cpu_leg):
+    """One training step of the indexer (sparse stage) on prefill_L16k: the KL target from the
+    main attention (bf16 tensor cores) and the KL loss with its gradients (CUDA cores, fp32),
+    after one forward pass that keeps the selection and the LSE.  dk is zeroed inside the
+    step (the backward adds into it)."""
+    from dsa_workloads import make_config, CONFIGS
+    wl = make_config(TRAIN_CFG, device=dev, seed=rank_seed(TRAIN_CFG, rank))
+    d = wl.dims
+    T, K = wl.total_rows, d["topk"]
+    fwd = dsa.Forward(wl, keep_idx=True)
+    dsa.check(fwd(stream), "forward for the training step")
+    pb = fwd.pb
+    target = torch.empty(T, K, dtype=torch.float32, device=dev)
+    loss = torch.empty(T, dtype=torch.float32, device=dev)
+    dw = torch.empty(T, d["h_idx"], dtype=torch.float32, device=dev)
+    dq = torch.empty(T, d["h_idx"], d["d_idx"], dtype=torch.float32, device=dev)
+    dk = torch.empty(wl.k_idx.shape[0], d["d_idx"], dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.check(dsa.dsa_indexer_kl_target(pb, wl.q, wl.kv, fwd.idx, fwd.lse, 0, T, target,
+                                            status, stream), "kl target")
+        if ev is not None:
+            ev[1].record(stream)
+        with torch.cuda.stream(stream):
+            dk.zero_()
+        dsa.check(dsa.dsa_indexer_kl_backward(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx,
+                                              wl.k_scale, fwd.idx, target, 0, T, loss, dw, dq,
+                                              dk, status, stream), "kl backward")
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, args.prefill_steps))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(evs[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_step = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    t_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    b_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    st, _ = dsa.dsa_read_device_status(status, stream)
+    dsa.check(st, "training step status")
+    f_t, f_b = train_flops(wl.seqlens, d)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = (clk or {}).get("sm_mhz") or 1965.0
+    fp32_peak = sms * 128 * 2 * mhz * 1e6 / 1e12      # FMA lanes x 2 FLOP x clock, TFLOP/s
+    b_tf = f_b / (b_ms / 1e3) / 1e12
+    t_tf = f_t / (t_ms / 1e3) / 1e12
+    res = {"workload": CONFIGS[TRAIN_CFG]["name"], "value": round(weak_value(world, T, ms_step), 1),
+           "unit": "tokens/s", "ms_per_step": round(ms_step, 3), "steps": steps,
+           "kernel_ms": {"kl_target": round(t_ms, 3), "kl_backward": round(b_ms, 3)},
+           "roofline": {"kernel": "dsa_indexer_kl_bwd_kernel", "bound": "alu",
+                        "achieved": round(b_tf, 2), "peak": round(fp32_peak, 1),
+                        "unit": "TFLOP/s", "frac": round(b_tf / fp32_peak, 4),
+                        "flops": f_b,
+                        "peak_note": f"fp32 FMA: {sms} SMs x 128 lanes x 2 FLOP x {mhz:.0f} MHz"},
+           "target_roofline": {"kernel": "dsa_sparse_mla_kernel (target mode)",
+                               "bound": "tensor", "achieved": round(t_tf, 1),
+                               "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                               "frac": round(t_tf / peaks["bf16_sustained"], 4), "flops": f_t},
+           "gpu_launches_per_step": 2,
+           "note": "after one forward that keeps the selection and LSE; per step: target, "
+                   "dk zeroed (a torch memset), backward"}
+    if cpu_leg:
+        import oracle
+        rows = [int(x) for x in np.linspace(T // 2, T - 1, 16)]
+        t0 = time.perf_counter()
+        sc = oracle.indexer_rows(wl, rows)
+        sel = oracle.topk_rows([sc[r] for r in rows], K)
+        tg = oracle.kl_target_rows(wl, rows, sel)
+        oracle.indexer_kl_rows(wl, rows, sel, tg)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": round(len(rows) / dt, 3), "unit": "tokens/s",
+                               "cores": oracle.num_threads(), "kind": "oracle",
+                               "sample": f"{len(rows)} rows of the second half (indexer, top-k, "
+                                         f"target, loss and gradients per row), {dt:.1f} s"}
+    del fwd, target, dq, dk
     torch.cuda.empty_cache()
     return res
 
@@ -531,6 +638,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-train", action="store_true",
+                    help="skip the indexer training step (prefill_L16k)")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--prefill-only", type=int, default=0, choices=[0, 1, 4, 5],

@@ -219,6 +219,57 @@ DSA_API dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* 
                                       uint8_t* k_cache, float* k_scale_cache, uint16_t* kv_cache,
                                       int32_t* dev_status, dsa_stream_t stream);
 
+/* ---- indexer training (sparse stage) ------------------------------------------------------
+ * The indexer is trained to imitate the main attention's head-summed distribution through a KL
+ * divergence ("DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention (DSA)",
+ * "Training signal"); in the sparse stage both distributions live on each row's selected keys.
+ * Two calls give one training step of the indexer after a forward pass that kept its indices
+ * and LSE: the target, then the loss with the gradients. */
+
+/* Target of rows [row_begin, row_begin + row_count):
+ *   target[t - row_begin, e] = (1/h) sum_h exp(sigma q[t,h,:] . kv[idx[t,e], :] - lse[t,h])
+ * (each head's attention distribution over the selection, averaged over heads; with the LSE
+ * of the forward pass over the same selection every row sums to 1).
+ *   q, kv, idx   as for dsa_sparse_mla_fwd (idx relative to row_begin; NULL = every prior key,
+ *                allowed only when no row has more than topk prior keys)
+ *   lse          fp32 [total_rows, h]: the forward's LSE (natural log, sigma applied)
+ *   target       fp32 [row_count, topk], caller-owned; entries with idx = -1 are set to 0
+ * Shapes as for dsa_sparse_mla_fwd.  All pointers 16-byte aligned.  Out-of-range indices are
+ * skipped (target 0) and set DSA_DEVICE_BAD_INDEX; timeouts set DSA_DEVICE_TIMEOUT. */
+DSA_API dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                           const uint16_t* q, const uint16_t* kv,
+                                           const int32_t* idx, const float* lse,
+                                           int32_t row_begin, int32_t row_count, float* target,
+                                           int32_t* dev_status, dsa_stream_t stream);
+
+/* KL loss of the indexer against `target` on the selected keys, and its gradients.  With the
+ * real-valued inputs q = q_scale * q_idx (per row and head) and k = k_scale * k_idx (per key),
+ * per row t over the entries e with idx[t,e] >= 0:
+ *   D[j,e] = q[t,j,:] . k[idx[t,e],:],  S_e = sum_j w[t,j] max(D[j,e], 0)  (the indexer score)
+ *   pi = softmax(S),  loss[t] = sum_e p_e (ln p_e - ln pi_e)  (p = target row, 0 ln 0 = 0)
+ *   g_e = pi_e sum_f p_f - p_e
+ *   dw[t,j]    = sum_e g_e max(D[j,e], 0)
+ *   dq[t,j,:]  = w[t,j] sum_e g_e [D[j,e] > 0] k[idx[t,e],:]
+ *   dk[row,:] += g_e sum_j w[t,j] [D[j,e] > 0] q[t,j,:]   for the physical row of idx[t,e]
+ * (d/dx max(x, 0) = 0 at x = 0; the gradients are those of the real values, so a caller that
+ * quantised q and k passes them straight through the rounding).
+ *   q_idx, q_scale, w, k_idx, k_scale   as for dsa_indexer_scores (k_scale must not be NULL)
+ *   idx      int32 [row_count, topk], relative to row_begin, -1 = unused (required)
+ *   target   fp32 [row_count, topk]
+ *   loss     fp32 [row_count];  dw fp32 [row_count, h_idx];  dq fp32 [row_count, h_idx, d_idx]
+ *   dk       fp32 [num_kv_rows, d_idx]: ADDED to (zero it first); the order of the atomic
+ *            additions is not fixed, so its last bits may vary from run to run
+ * Indexer shapes (h_idx, d_idx) = (64, 128) or (4, 32), both modes.  All pointers 16-byte
+ * aligned.  Out-of-range indices are skipped and set DSA_DEVICE_BAD_INDEX. */
+DSA_API dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                             const uint8_t* q_idx, const float* q_scale,
+                                             const float* w, const uint8_t* k_idx,
+                                             const float* k_scale, const int32_t* idx,
+                                             const float* target, int32_t row_begin,
+                                             int32_t row_count, float* loss, float* dw,
+                                             float* dq, float* dk, int32_t* dev_status,
+                                             dsa_stream_t stream);
+
 /* Synchronises `stream`, reads the device status word and maps it: 0 -> DSA_OK,
  * DSA_DEVICE_TIMEOUT -> DSA_ERR_TIMEOUT, DSA_DEVICE_BAD_INDEX -> DSA_ERR_BAD_INDEX.
  * *raw (optional, host) receives the word. */

@@ -37,7 +37,8 @@ DSA_DECODE = 1
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_fwd", "dsa_forward_workspace_size", "dsa_forward",
             "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-            "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout")
+            "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
+            "dsa_indexer_kl_target", "dsa_indexer_kl_backward")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -79,6 +80,9 @@ def _load():
         "dsa_forward": (I32, [DP, SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_selftest_wait_timeout": (I32, [P, P]),
+        "dsa_indexer_kl_target": (I32, [DP, SP, P, P, P, P, I32, I32, P, P, P]),
+        "dsa_indexer_kl_backward": (I32, [DP, SP, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P,
+                                          P]),
         "dsa_status_string": (ctypes.c_char_p, [I32]),
         "dsa_abi_version": (I32, []),
         "dsa_sparse_mla_fwd_noalloc": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, P]),
@@ -234,6 +238,22 @@ def dsa_cache_append(pb: Problem, k_new, kv_new, k_cache, k_scale_cache, kv_cach
     return int(lib.dsa_cache_append(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(k_new), _ptr(kv_new), _ptr(k_cache),
         _ptr(k_scale_cache), _ptr(kv_cache), _ptr(dev_status), _stream(stream)))
+
+
+def dsa_indexer_kl_target(pb: Problem, q, kv, idx, lse, row_begin: int, row_count: int, target,
+                          dev_status=None, stream=None) -> int:
+    return int(lib.dsa_indexer_kl_target(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q), _ptr(kv), _ptr(idx), _ptr(lse),
+        row_begin, row_count, _ptr(target), _ptr(dev_status), _stream(stream)))
+
+
+def dsa_indexer_kl_backward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, idx, target,
+                            row_begin: int, row_count: int, loss, dw, dq, dk, dev_status=None,
+                            stream=None) -> int:
+    return int(lib.dsa_indexer_kl_backward(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
+        _ptr(k_idx), _ptr(k_scale), _ptr(idx), _ptr(target), row_begin, row_count, _ptr(loss),
+        _ptr(dw), _ptr(dq), _ptr(dk), _ptr(dev_status), _stream(stream)))
 
 
 def dsa_selftest_wait_timeout(dev_status, stream=None) -> int:

@@ -11,6 +11,7 @@
 #include "dsa.h"
 #include "cache_append.cuh"
 #include "indexer.cuh"
+#include "indexer_bwd.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
@@ -397,18 +398,14 @@ size_t mla_ws_bytes(const dsa_dims_t& d, int splits, int32_t row_count) {
   return size_t(splits) * row_count * d.h * (d.d_v + 1) * sizeof(float) + 256;
 }
 
-template <int D_QK, int D_V>
-dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
-                      const uint16_t* kv, const int32_t* idx, int32_t row_begin, int32_t row_count,
-                      uint16_t* out, float* lse, void* ws, size_t ws_bytes, int32_t* status,
-                      cudaStream_t st, int splits) {
-  using C = MlaCfg<D_QK, D_V>;
+// The inputs and row geometry shared by the attention forward and the target pass.
+MlaParams mla_params(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
+                     const uint16_t* kv, const int32_t* idx, int32_t row_begin, int32_t row_count,
+                     int32_t splits, int32_t* status) {
   MlaParams prm{};
   prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
   prm.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
   prm.idx = idx;
-  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
-  prm.lse = lse;
   prm.row_begin = row_begin;
   prm.row_count = row_count;
   prm.topk = d.topk;
@@ -426,6 +423,18 @@ dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* 
   prm.block_size = d.block_size > 0 ? d.block_size : 64;
   prm.num_kv_rows = s.num_kv_rows;
   prm.status = status;
+  return prm;
+}
+
+template <int D_QK, int D_V>
+dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
+                      const uint16_t* kv, const int32_t* idx, int32_t row_begin, int32_t row_count,
+                      uint16_t* out, float* lse, void* ws, size_t ws_bytes, int32_t* status,
+                      cudaStream_t st, int splits) {
+  using C = MlaCfg<D_QK, D_V>;
+  MlaParams prm = mla_params(d, s, q, kv, idx, row_begin, row_count, splits, status);
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
   if (splits > 1) {
     if (ws == nullptr || ws_bytes < mla_ws_bytes(d, splits, row_count))
       return DSA_ERR_WORKSPACE_TOO_SMALL;
@@ -504,6 +513,43 @@ ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count)
   auto align = [](size_t x) { return (x + 255) / 256 * 256; };
   p.total = align(p.slab_floats * 4) + align(p.idx_ints * 4) + align(p.mla_bytes);
   return p;
+}
+
+// ------------------------------------------------------------------------ indexer training
+
+// Split count of the target pass: keys are independent there, so splits need no combine; fill
+// the SMs when the rows alone do not, keeping at least two tiles per CTA pair.
+int target_splits(const dsa_dims_t& d, int32_t row_count, int sm_count) {
+  const int tiles = d.topk / 64;
+  return std::max(1, std::min({16, tiles / 2, sm_count / std::max(1, 2 * row_count)}));
+}
+
+template <int D_QK, int D_V>
+dsa_status_t target_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
+                         const uint16_t* kv, const int32_t* idx, const float* lse,
+                         int32_t row_begin, int32_t row_count, float* target, int32_t* status,
+                         cudaStream_t st, int sm_count) {
+  using C = MlaCfg<D_QK, D_V>;
+  const int splits = target_splits(d, row_count, sm_count);
+  MlaParams prm = mla_params(d, s, q, kv, idx, row_begin, row_count, splits, status);
+  prm.lse_in = lse;
+  prm.target = target;
+  CUtensorMap q_map;
+  if (make_row_map(&q_map, q, uint64_t(s.total_rows) * d.h, D_QK * 2, 128, 128) != DSA_OK)
+    return DSA_ERR_CUDA;
+  auto k = dsa_sparse_mla_kernel<D_QK, D_V, true>;
+  if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
+  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(q_map, prm);
+  return launch_status();
+}
+
+template <int H_I, int D_I>
+dsa_status_t kl_backward_impl(const IdxBwdParams& prm, cudaStream_t st) {
+  using C = IdxBwdCfg<H_I, D_I>;
+  auto k = dsa_indexer_kl_bwd_kernel<H_I, D_I>;
+  if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
+  k<<<prm.row_count, C::THREADS, C::SMEM_BYTES, st>>>(prm);
+  return launch_status();
 }
 
 // ---------------------------------------------------------------- bounded-wait self-test
@@ -725,6 +771,81 @@ dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs, co
   else
     dsa_cache_append_kernel<32, 160><<<grid, 128, 0, st>>>(prm);
   return launch_status();
+}
+
+dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                   const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                   const float* lse, int32_t row_begin, int32_t row_count,
+                                   float* target, int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q || !kv || !lse || !target) return DSA_ERR_INVALID_ARG;
+  if (idx == nullptr && !dense_ok(*dims, seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(lse) || !aligned16(target))
+    return DSA_ERR_MISALIGNED;
+  if (row_count == 0) return DSA_OK;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->d_qk == 576)
+    return target_impl<576, 512>(*dims, *seqs, q, kv, idx, lse, row_begin, row_count, target,
+                                 dev_status, st, info.sm_count);
+  return target_impl<160, 128>(*dims, *seqs, q, kv, idx, lse, row_begin, row_count, target,
+                               dev_status, st, info.sm_count);
+}
+
+dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                     const uint8_t* q_idx, const float* q_scale, const float* w,
+                                     const uint8_t* k_idx, const float* k_scale,
+                                     const int32_t* idx, const float* target, int32_t row_begin,
+                                     int32_t row_count, float* loss, float* dw, float* dq,
+                                     float* dk, int32_t* dev_status, dsa_stream_t stream) {
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  const dsa_dims_t& d = *dims;
+  const dsa_seqs_t& s = *seqs;
+  const bool full = d.h_idx == 64 && d.d_idx == 128;
+  const bool tiny = d.h_idx == 4 && d.d_idx == 32;
+  if (!full && !tiny) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !idx || !target || !loss || !dw || !dq ||
+      !dk)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx) || !aligned16(target) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(q_scale) || !aligned16(w) ||
+      !aligned16(k_scale) || !aligned16(loss) || !aligned16(dw))
+    return DSA_ERR_MISALIGNED;
+  if (row_count == 0) return DSA_OK;
+  IdxBwdParams prm{};
+  prm.q_idx = q_idx;
+  prm.q_scale = q_scale;
+  prm.w = w;
+  prm.k_idx = k_idx;
+  prm.k_scale = k_scale;
+  prm.idx = idx;
+  prm.target = target;
+  prm.loss = loss;
+  prm.dw = dw;
+  prm.dq = dq;
+  prm.dk = dk;
+  prm.row_begin = row_begin;
+  prm.row_count = row_count;
+  prm.topk = d.topk;
+  prm.decode = s.mode == DSA_DECODE;
+  prm.batch = s.batch;
+  prm.cu_seqlens = s.cu_seqlens;
+  prm.seq_lens = s.seq_lens;
+  prm.block_table = s.block_table;
+  prm.max_blocks = s.max_blocks;
+  prm.kv_stride = s.max_seqlen;
+  prm.max_seqlen = s.max_seqlen;
+  prm.block_size = d.block_size > 0 ? d.block_size : 64;
+  prm.num_kv_rows = s.num_kv_rows;
+  prm.status = dev_status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return full ? kl_backward_impl<64, 128>(prm, st) : kl_backward_impl<4, 32>(prm, st);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream) {

@@ -33,6 +33,17 @@
 // warps 12-15 the value dims.  Grid: x = 2 * row + v, y = split-KV slice.
 // Without an index array the selection is every prior key (dense causal attention), which is
 // what the top-k keeps whenever a row has at most topk prior keys.
+//
+// Target mode (kTarget): the indexer's training target on the same selection, the main
+// attention's distribution summed over heads and normalised ("DeepSeek V3.2-Exp Cuts
+// Long-Context Costs with DeepSeek Sparse Attention (DSA)", "Training signal"):
+//   target[t, e] = (1/H) sum_h exp(sigma q[t,h,:] . kv[idx[t,e], :] - LSE[t,h])
+// with the LSE of the forward pass over the same selection.  The gathers and the QK product
+// are the forward's; there is no PV.  The two CTAs of a row take alternate tiles (each gathers
+// every dim of its tiles), the QK commit frees both parts of a slot, and the softmax warps
+// turn each logit into its probability (thread = head), sum the 128 heads of every key with a
+// butterfly across lanes and a 4-warp pass through shared memory, and write the 64 targets of
+// the tile.  Entries with idx = -1 get 0.
 #pragma once
 #include <type_traits>
 
@@ -62,6 +73,8 @@ struct MlaParams {
   int32_t block_size;
   int64_t num_kv_rows;
   int32_t* status;
+  const float* lse_in;         // target mode: the forward's LSE [T, H]
+  float* target;               // target mode: [row_count, topk], relative to row_begin
 };
 
 template <int D_QK, int D_V>
@@ -87,8 +100,9 @@ struct MlaCfg {
   static constexpr int RING_BYTES = STAGES * (K_SLOT_BYTES + V_SLOT_BYTES);
   static constexpr int Q_KB_BYTES = 128 * 128;                        // one k-block of Q
   static constexpr int Q_SMEM_BYTES = KBS * Q_KB_BYTES;
+  static constexpr int RED_BYTES = 2 * 4 * BN * 4;                    // target mode
   static constexpr int SMEM_USED = 1024 + Q_SMEM_BYTES + RING_BYTES + MAX_TILES * BN * 4 +
-                                   MAX_TILES * 12 + 256;
+                                   MAX_TILES * 12 + 256 + RED_BYTES;
   // at least 116 KB, so that one CTA runs per SM (its TMEM allocation never waits)
   static constexpr int SMEM_BYTES = SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024;
   static_assert(V_HALF % 64 == 0 && V_HALF <= 256, "PV MMA N");
@@ -97,7 +111,21 @@ struct MlaCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <int D_QK, int D_V>
+// One step of the head sum across a warp: each lane holds 2 LEN values (its partial sums of
+// 2 LEN keys); it keeps LEN of them (the upper half if lane bit LEN/2 is set), adds the partner
+// lane's copy of the same keys, and hands its other half to the partner.
+template <int LEN>
+__device__ __forceinline__ void head_sum_step(float (&v)[64], int lane) {
+  const bool up = (lane & (LEN / 2)) != 0;
+#pragma unroll
+  for (int j = 0; j < LEN; ++j) {
+    const float send = up ? v[j] : v[j + LEN];
+    const float keep = up ? v[j + LEN] : v[j];
+    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, LEN / 2);
+  }
+}
+
+template <int D_QK, int D_V, bool kTarget = false>
 __global__ void __launch_bounds__(512, 1)
     dsa_sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
   using C = MlaCfg<D_QK, D_V>;
@@ -123,6 +151,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* qk_fin = bars + 12;
   uint64_t* pv_fin = bars + 13;
   uint64_t* q_bar = bars + 14;       // 1 arrival + Q bytes
+  uint64_t* red_full = bars + 15;    // [2] target mode: 4 softmax warps
+  uint64_t* red_empty = bars + 17;   // [2] target mode: the writing warp
+  float* sRed = reinterpret_cast<float*>(bars + 32);   // target mode: [2][4 warps][BN]
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int n_act_s;
@@ -168,6 +199,10 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(smem_u32(qk_fin), 1);
     mbar_init(smem_u32(pv_fin), 1);
     mbar_init(smem_u32(q_bar), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&red_full[i]), 4);
+      mbar_init(smem_u32(&red_empty[i]), 1);
+    }
     abort_s = 0;
     fence_mbar_init();
   }
@@ -238,6 +273,11 @@ __global__ void __launch_bounds__(512, 1)
         if (a1 < 0) ph[32 + lane] = fb;
       }
       if (lane == 0) sMask[tt] = m;
+      if (kTarget && m == 0 && vh == 0 && split == 0) {   // no valid key: targets are 0
+        float* tg = p.target + static_cast<int64_t>(r) * p.topk + tt * C::BN;
+        tg[lane] = 0.f;
+        tg[32 + lane] = 0.f;
+      }
     }
   }
   __syncthreads();
@@ -252,8 +292,10 @@ __global__ void __launch_bounds__(512, 1)
     const int per = (cnt + p.splits - 1) / p.splits;
     const int t0 = min(cnt, split * per);
     const int t1 = min(cnt, t0 + per);
-    for (int i = t0; i < t1; ++i) sTiles[i - t0] = sTiles[i];
-    n_act_s = t1 - t0;
+    int m = 0;   // target mode: the two CTAs of a row take alternate tiles
+    for (int i = t0; i < t1; ++i)
+      if (!kTarget || ((i - t0) & 1) == vh) sTiles[m++] = sTiles[i];
+    n_act_s = m;
   }
   if (warp >= 4 && warp < 8) {
     // ---- Q blocks [0, KBT) from the staging area into TMEM: head = lane, dim d in column
@@ -326,6 +368,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         umma_commit(smem_u32(s_full));
         umma_commit(smem_u32(&k_empty[s]));
+        if (kTarget) umma_commit(smem_u32(&v_empty[s]));   // no PV reads the slot
       }
       if (!ok) {
         abort_s = 1;
@@ -334,7 +377,7 @@ __global__ void __launch_bounds__(512, 1)
       umma_commit(smem_u32(qk_fin));
       mbar_wait(smem_u32(qk_fin), 0, nullptr);
     }
-  } else if (warp == 2) {
+  } else if (warp == 2 && !kTarget) {
     // ------------------------------------------------------------ PV issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f32acc(1, 128, C::V_HALF, 0, 1);
@@ -411,6 +454,75 @@ __global__ void __launch_bounds__(512, 1)
       if (p.status) atomicOr(p.status, kStatusTimeout);
     }
     cp_async_wait_all();   // nothing may still be writing this CTA's shared memory at exit
+  } else if (kTarget && warp >= 4) {
+    // ------------------------------------------------------------ target: p per head, head sum
+    const int w4 = warp & 3;
+    const int hrow = w4 * 32 + lane;            // head = TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
+    // heads past H (the small shapes run 128 MMA rows for fewer heads) contribute nothing
+    const float lse2 =
+        hrow < p.h ? p.lse_in[static_cast<int64_t>(row) * p.h + hrow] * 1.4426950408889634f
+                   : INFINITY;
+    // after the butterfly this lane holds the head sums of keys key0 and key0 + 1
+    const int key0 = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
+                     ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+    const float inv_h = 1.f / static_cast<float>(p.h);
+    const float sc = p.scale_log2;
+    bool ok = !abort_s;
+    for (int i = 0; i < n && ok; ++i) {
+      ok = (warp_mbar_wait(smem_u32(s_full), i & 1, &abort_s));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t su[2][32];
+      tmem_ld32(lane_addr + C::S_COL, su[0]);
+      tmem_ld32(lane_addr + C::S_COL + 32, su[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(s_empty));
+      const uint64_t vmask = sMask[sTiles[i]];
+      float v[64];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t vb = static_cast<uint32_t>(vmask >> (32 * hh));
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float pr = exp2f(fmaf(__uint_as_float(su[hh][j]), sc, -lse2));
+          v[32 * hh + j] = ((vb >> j) & 1u) ? pr : 0.f;
+        }
+      }
+      head_sum_step<32>(v, lane);
+      head_sum_step<16>(v, lane);
+      head_sum_step<8>(v, lane);
+      head_sum_step<4>(v, lane);
+      head_sum_step<2>(v, lane);
+      // the 4 warps' sums meet in shared memory (double-buffered by tile parity)
+      const int buf = i & 1;
+      float* red = sRed + buf * 4 * C::BN;
+      if (i >= 2) {
+        ok = (warp_mbar_wait(smem_u32(&red_empty[buf]), ((i >> 1) - 1) & 1, &abort_s));
+        if (!ok) break;
+      }
+      *reinterpret_cast<float2*>(red + w4 * C::BN + key0) = make_float2(v[0], v[1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&red_full[buf]));
+      if (w4 == 0) {
+        ok = (warp_mbar_wait(smem_u32(&red_full[buf]), (i >> 1) & 1, &abort_s));
+        if (!ok) break;
+        float* tg = p.target + static_cast<int64_t>(r) * p.topk + sTiles[i] * C::BN;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int e = lane + 32 * c;
+          tg[e] = ((red[e] + red[C::BN + e]) + (red[2 * C::BN + e] + red[3 * C::BN + e])) * inv_h;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&red_empty[buf]));
+      }
+    }
+    if (!ok) {
+      abort_s = 1;
+      if (p.status) atomicOr(p.status, kStatusTimeout);
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     const int hrow = (warp & 3) * 32 + lane;    // head = TMEM lane

@@ -11,7 +11,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def dsa():
-    from sparse_attention_long_04_b200 import build as b
+    import importlib.util
+    # build.py by path: importing the package first would load a stale library
+    spec = importlib.util.spec_from_file_location(
+        "_dsa_lib_build", os.path.join(ROOT, "sparse_attention_long_04_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
     b.build()
     import sparse_attention_long_04_b200 as m
     return m
@@ -156,3 +161,30 @@ def test_wait_selftest_argument_errors(dsa):
     any launch."""
     assert dsa.dsa_selftest_wait_timeout(None, 0) == dsa.DSA_ERR_INVALID_ARG
     assert dsa.dsa_selftest_wait_timeout(FAKE + 2, 0) == dsa.DSA_ERR_MISALIGNED
+
+
+def test_indexer_training_argument_errors(dsa):
+    """The target and backward calls check their pointers, alignment, shapes and rows before
+    any launch."""
+    pb = _pb(dsa)
+
+    def target(p, q=FAKE, kv=FAKE, idx=FAKE, lse=FAKE, tgt=FAKE, rb=0, n=2):
+        return dsa.dsa_indexer_kl_target(p, q, kv, idx, lse, rb, n, tgt, None, 0)
+
+    assert target(pb, lse=None) == dsa.DSA_ERR_INVALID_ARG
+    assert target(pb, idx=None) == dsa.DSA_ERR_INVALID_ARG     # rows longer than topk
+    assert target(pb, tgt=FAKE + 4) == dsa.DSA_ERR_MISALIGNED
+    assert target(pb, rb=1) == dsa.DSA_ERR_INVALID_ARG          # past the last row
+    assert target(_pb(dsa, d_qk=512)) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+    ok = [FAKE] * 11   # q_idx, q_scale, w, k_idx, k_scale, idx, target | loss, dw, dq, dk
+
+    def backward(p, bufs, rb=0, n=2):
+        return dsa.dsa_indexer_kl_backward(p, *bufs[:7], rb, n, *bufs[7:], None, 0)
+
+    assert backward(pb, ok[:4] + [None] + ok[5:]) == dsa.DSA_ERR_INVALID_ARG   # k_scale
+    assert backward(pb, ok[:5] + [None] + ok[6:]) == dsa.DSA_ERR_INVALID_ARG   # idx
+    assert backward(pb, ok[:10] + [None]) == dsa.DSA_ERR_INVALID_ARG          # dk
+    assert backward(pb, [FAKE + 4] + ok[1:]) == dsa.DSA_ERR_MISALIGNED
+    assert backward(pb, ok, rb=1) == dsa.DSA_ERR_INVALID_ARG
+    assert backward(_pb(dsa, h_idx=32), ok) == dsa.DSA_ERR_UNSUPPORTED_SHAPE

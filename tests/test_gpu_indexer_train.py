@@ -1,0 +1,187 @@
+"""The indexer's training step on the GPU against the oracle: the KL target (the main attention's
+head-summed distribution on the selected keys) and the KL loss with its gradients for w, q, k.
+
+Every input the oracle sees comes from the seeded generators or from the oracle itself: the
+selection is the oracle's own top-k, the LSE the oracle's attention, the target the oracle's.
+The GPU gets the same values (the LSE and the target rounded to fp32).
+
+Tolerances (derived from the arithmetic):
+  target   |t_gpu - t_ref| <= 1e-4 t_ref + 1e-7: fp32 logits from exact bf16 products (relative
+           error ~1e-6 at logits of order 1), one exp2 and a 128-head fp32 sum
+  loss     |L_gpu - L_ref| <= 1e-3 |L_ref| + 1e-5: the fp32 indexer scores carry the indexer's
+           1e-3 relative tolerance into the softmax
+  grads    per row rel-L2 of dw and dq, and rel-L2 of dk over the touched keys, <= 2e-3: the
+           same score error plus fp32 accumulation over up to 2048 keys
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dsa_workloads import FULL, make_config, make_decode, make_prefill
+from tests.parity import to_np
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+T_REL, T_ABS = 1e-4, 1e-7
+L_REL, L_ABS = 1e-3, 1e-5
+G_REL_L2 = 2e-3
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import sparse_attention_long_04_b200 as m
+    return m
+
+
+def _oracle_selection(wl, rows):
+    """The oracle's own top-k of its own scores, and its attention LSE on that selection."""
+    sc = oracle.indexer_rows(wl, rows)
+    idx = oracle.topk_rows([sc[r] for r in rows], wl.dims["topk"])
+    _, lse = oracle.sparse_mla_rows(wl, rows, idx)
+    return sc, idx, lse
+
+
+def _gpu_target(dsa, wl, rb, idx, lse_rows):
+    n, k = idx.shape
+    lse = torch.zeros(wl.total_rows, wl.dims["h"], device="cuda")
+    lse[rb:rb + n] = torch.tensor(lse_rows, dtype=torch.float32, device="cuda")
+    idx_d = torch.tensor(idx, device="cuda")
+    tgt = torch.full((n, k), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = dsa.dsa_indexer_kl_target(dsa.problem_of(wl), wl.q, wl.kv, idx_d, lse, rb, n, tgt,
+                                   status, 0)
+    assert st == dsa.DSA_OK, dsa.status_string(st)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return to_np(tgt)
+
+
+def _check_target(got, ref, idx):
+    assert not np.isnan(got).any()
+    assert (got[idx < 0] == 0).all()
+    err = np.abs(got - ref)
+    bad = np.argwhere(err > T_REL * np.abs(ref) + T_ABS)
+    assert len(bad) == 0, (bad[:5], got[tuple(bad[0])], ref[tuple(bad[0])])
+
+
+def _rows_target(dsa, wl, rb, n):
+    rows = list(range(rb, rb + n))
+    _, idx, lse = _oracle_selection(wl, rows)
+    got = _gpu_target(dsa, wl, rb, idx, lse)
+    _check_target(got, oracle.kl_target_rows(wl, rows, idx), idx)
+    return rows, idx, got
+
+
+def test_kl_target_tiny_prefill(dsa):
+    wl = make_config(1, device="cuda")
+    _rows_target(dsa, wl, 0, 40)          # rows with fewer keys than k: holes in the selection
+    _rows_target(dsa, wl, 980, 44)
+
+
+def test_kl_target_full_dims_prefill_and_decode(dsa):
+    wl = make_prefill(22, [2500, 300], FULL, needles=8, device="cuda")
+    _rows_target(dsa, wl, 2040, 16)       # around pos + 1 = topk
+    _rows_target(dsa, wl, 2490, 20)       # the end of one sequence and the start of the next
+    wl = make_decode(21, 5, [7000, 2048, 2049, 100, 1], FULL, boost=0.01, paged=True,
+                     device="cuda")       # split across CTAs (few rows), paged keys
+    _rows_target(dsa, wl, 0, 5)
+
+
+def test_kl_target_dense_without_indices(dsa):
+    """No index array: every prior key, in position order (rows with at most k prior keys)."""
+    wl = make_config(1, device="cuda")
+    rows = list(range(0, 64))
+    idx = np.array([list(range(t + 1)) + [-1] * (63 - t) for t in rows], np.int32)
+    _, lse = oracle.sparse_mla_rows(wl, rows, idx)
+    lse_d = torch.zeros(wl.total_rows, wl.dims["h"], device="cuda")
+    lse_d[:64] = torch.tensor(lse, dtype=torch.float32, device="cuda")
+    tgt = torch.full((64, 64), float("nan"), device="cuda")
+    assert dsa.dsa_indexer_kl_target(dsa.problem_of(wl), wl.q, wl.kv, None, lse_d, 0, 64, tgt,
+                                     None, 0) == dsa.DSA_OK
+    torch.cuda.synchronize()
+    _check_target(to_np(tgt), oracle.kl_target_rows(wl, rows, idx), idx)
+
+
+def _gpu_backward(dsa, wl, rb, idx, target):
+    n, k = idx.shape
+    d = wl.dims
+    dev = "cuda"
+    idx_d = torch.tensor(idx, device=dev)
+    tgt = torch.tensor(target, dtype=torch.float32, device=dev)
+    loss = torch.full((n,), float("nan"), device=dev)
+    dw = torch.full((n, d["h_idx"]), float("nan"), device=dev)
+    dq = torch.full((n, d["h_idx"], d["d_idx"]), float("nan"), device=dev)
+    dk = torch.zeros(wl.kv.shape[0], d["d_idx"], device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = dsa.dsa_indexer_kl_backward(dsa.problem_of(wl), wl.q_idx, wl.q_scale, wl.w, wl.k_idx,
+                                     wl.k_scale, idx_d, tgt, rb, n, loss, dw, dq, dk, status, 0)
+    assert st == dsa.DSA_OK, dsa.status_string(st)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return to_np(loss), to_np(dw), to_np(dq), to_np(dk)
+
+
+def _rel_l2(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / nb if nb > 0 else np.linalg.norm(a)
+
+
+def _check_backward(dsa, wl, rb, n):
+    rows = list(range(rb, rb + n))
+    _, idx, _ = _oracle_selection(wl, rows)
+    target = oracle.kl_target_rows(wl, rows, idx).astype(np.float32)
+    ref = oracle.indexer_kl_rows(wl, rows, idx, target.astype(np.float64))
+    loss, dw, dq, dk = _gpu_backward(dsa, wl, rb, idx, target)
+    np.testing.assert_allclose(loss, ref["loss"], rtol=L_REL, atol=L_ABS)
+    for i in range(n):
+        assert _rel_l2(dw[i], ref["dw"][i]) <= G_REL_L2, ("dw", rows[i])
+        assert _rel_l2(dq[i], ref["dq"][i]) <= G_REL_L2, ("dq", rows[i])
+    assert _rel_l2(dk[ref["dk_rows"]], ref["dk"]) <= G_REL_L2
+    untouched = np.setdiff1d(np.arange(dk.shape[0]), ref["dk_rows"])
+    assert not dk[untouched].any()
+
+
+def test_kl_backward_tiny_prefill(dsa):
+    wl = make_config(1, device="cuda")
+    _check_backward(dsa, wl, 0, 40)
+    _check_backward(dsa, wl, 980, 44)
+
+
+def test_kl_backward_full_dims_prefill(dsa):
+    wl = make_prefill(22, [2500, 300], FULL, needles=8, device="cuda")
+    _check_backward(dsa, wl, 2040, 16)
+    _check_backward(dsa, wl, 2490, 20)
+
+
+def test_kl_backward_full_dims_paged_decode(dsa):
+    wl = make_decode(21, 5, [7000, 2048, 2049, 100, 1], FULL, boost=0.01, paged=True,
+                     device="cuda")
+    _check_backward(dsa, wl, 0, 5)
+
+
+def test_kl_backward_bad_index_reported(dsa):
+    wl = make_config(1, device="cuda")
+    rows = list(range(100, 104))
+    _, idx, _ = _oracle_selection(wl, rows)
+    target = oracle.kl_target_rows(wl, rows, idx)
+    bad = idx.copy()
+    bad[1, 3] = 5000                       # past the row's keys: skipped and reported
+    ref_idx = bad.copy()
+    ref_idx[1, 3] = -1
+    ref = oracle.indexer_kl_rows(wl, rows, ref_idx, target)
+    n, k = idx.shape
+    loss = torch.zeros(n, device="cuda")
+    dw = torch.zeros(n, 4, device="cuda")
+    dq = torch.zeros(n, 4, 32, device="cuda")
+    dk = torch.zeros(wl.kv.shape[0], 32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = dsa.dsa_indexer_kl_backward(dsa.problem_of(wl), wl.q_idx, wl.q_scale, wl.w, wl.k_idx,
+                                     wl.k_scale, torch.tensor(bad, device="cuda"),
+                                     torch.tensor(target, dtype=torch.float32, device="cuda"),
+                                     100, n, loss, dw, dq, dk, status, 0)
+    assert st == dsa.DSA_OK
+    torch.cuda.synchronize()
+    assert int(status.item()) & dsa.DSA_DEVICE_BAD_INDEX
+    np.testing.assert_allclose(to_np(loss), ref["loss"], rtol=L_REL, atol=L_ABS)
