@@ -400,8 +400,15 @@ def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, clk, cpu_leg):
     main attention (bf16 tensor cores) and the KL loss with its gradients (CUDA cores, fp32),
     after one forward pass that keeps the selection and the LSE.  dk is zeroed inside the
     step (the backward adds into it)."""
-    from dsa_workloads import make_config, CONFIGS
-    wl = make_config(TRAIN_CFG, device=dev, seed=rank_seed(TRAIN_CFG, rank))
+    from dsa_workloads import make_config, make_prefill, CONFIGS, FULL
+    if args.train_len == CONFIGS[TRAIN_CFG]["seqlens"][0]:
+        wl = make_config(TRAIN_CFG, device=dev, seed=rank_seed(TRAIN_CFG, rank))
+        name = CONFIGS[TRAIN_CFG]["name"]
+    else:   # profiling only: a shorter sequence of the same kind
+        c = CONFIGS[TRAIN_CFG]
+        name = f"prefill_L{args.train_len}"
+        wl = make_prefill(TRAIN_CFG, [args.train_len], FULL, c["needles"], dev,
+                          seed=rank_seed(TRAIN_CFG, rank), name=name)
     d = wl.dims
     T, K = wl.total_rows, d["topk"]
     fwd = dsa.Forward(wl, keep_idx=True)
@@ -453,7 +460,7 @@ def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, clk, cpu_leg):
     fp32_peak = sms * 128 * 2 * mhz * 1e6 / 1e12      # FMA lanes x 2 FLOP x clock, TFLOP/s
     b_tf = f_b / (b_ms / 1e3) / 1e12
     t_tf = f_t / (t_ms / 1e3) / 1e12
-    res = {"workload": CONFIGS[TRAIN_CFG]["name"], "value": round(weak_value(world, T, ms_step), 1),
+    res = {"workload": name, "value": round(weak_value(world, T, ms_step), 1),
            "unit": "tokens/s", "ms_per_step": round(ms_step, 3), "steps": steps,
            "kernel_ms": {"kl_target": round(t_ms, 3), "kl_backward": round(b_ms, 3)},
            "roofline": {"kernel": "dsa_indexer_kl_bwd_kernel", "bound": "alu",
@@ -640,6 +647,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the indexer training step (prefill_L16k)")
+    ap.add_argument("--train-only", action="store_true",
+                    help="profiling only: time just the indexer training step")
+    ap.add_argument("--train-len", type=int, default=16384,
+                    help="profiling only: sequence length of the training step")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--prefill-only", type=int, default=0, choices=[0, 1, 4, 5],
@@ -670,6 +681,15 @@ def main():
             torch.cuda.set_device(dev)
             line = run_prefill(args, dsa, dev, torch.cuda.current_stream(), read_peaks(), rank,
                                world)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            return
+        if args.train_only:
+            import sparse_attention_long_04_b200 as dsa
+            dev = torch.device("cuda", local_rank)
+            torch.cuda.set_device(dev)
+            line = run_indexer_train(args, dsa, dev, torch.cuda.current_stream(), read_peaks(),
+                                     rank, world, None, cpu_leg=rank == 0 and not args.no_cpu)
             if rank == 0:
                 print(json.dumps(line), flush=True)
             return
