@@ -13,14 +13,17 @@
 //   dk[s_e,:] += g_e sum_j w[t,j] [D[j,e] > 0] q[t,j,:]   (summed over rows with atomic adds)
 // The derivative of max(x, 0) at 0 is taken as 0.
 //
-// Design (first version, CUDA cores, fp32).  One CTA of 256 threads per query row.  The row's
+// Design (CUDA cores, fp32).  One CTA of 256 threads per query row, two CTAs per SM.  The row's
 // real-valued queries stay in shared memory (row stride D_I + 1 floats, so that lanes reading
-// one dim of consecutive heads hit distinct banks); keys come 32 at a time, decoded from e4m3 and
-// scaled into shared memory.  Pass 1 computes every S_e: warp w takes keys 4w..4w+3 of the
-// chunk, lane l heads l and l + 32, and the head sum is a butterfly over the lanes.  Block
-// reductions then give max S, the softmax normaliser, sum p, the loss and g.  Pass 2 recomputes
-// D chunk by chunk (the same instructions, so the same values and ReLU decisions as pass 1) and
-// forms coef[e][j] = g_e w_j [D > 0] in shared memory; dw accumulates in registers, dk (lanes over
+// one dim of consecutive heads hit distinct banks); keys come 64 at a time, decoded from e4m3 and
+// scaled into shared memory.  The loops are register-tiled so that shared-memory loads, not
+// FMAs, stop being the bound: each 4-dim step of the dot products loads 8 keys (broadcast) and
+// 2 heads' queries for 64 FMAs, dk loads the coefficients of 8 keys 4 heads at a time, dq those
+// of 8 heads per key.  Pass 1 computes every S_e: warp w takes keys 8w..8w+7 of the chunk, lane
+// l heads l and l + 32, and the head sum is a butterfly over the lanes.  Block reductions then
+// give max S, the softmax normaliser, sum p, the loss and g.  Pass 2 recomputes D chunk by chunk
+// (the same instructions, so the same values and ReLU decisions as pass 1) and forms
+// coef[e][j] = g_e w_j [D > 0] in shared memory; dw accumulates in registers, dk (lanes over
 // dims, per key) goes out with coalesced atomic adds, and dq (warp = 8 heads, lane = dims
 // l + 32 c) accumulates in registers over all chunks.  Chunks without a valid key are skipped.
 #pragma once
@@ -60,7 +63,7 @@ struct IdxBwdParams {
 template <int H_I, int D_I>
 struct IdxBwdCfg {
   static constexpr int THREADS = 256;
-  static constexpr int CH = 32;                       // keys per chunk
+  static constexpr int CH = 64;                       // keys per chunk
   static constexpr int KPW = CH / 8;                  // keys per warp
   static constexpr int HPL = (H_I + 31) / 32;         // heads per lane (D, coef)
   static constexpr int HPW = (H_I + 7) / 8;           // heads per warp (dq)
@@ -69,8 +72,8 @@ struct IdxBwdCfg {
   static constexpr int MAX_K = 2048;
   static constexpr int MAX_CH = MAX_K / CH;
   // floats: queries, key chunk, coef (the dw partials reuse it at the end), S / g, w; then
-  // ints: physical rows, chunk flags; then 32 floats of reduction scratch.  73 KB at
-  // (64, 128): three CTAs per SM.
+  // ints: physical rows, chunk flags; then 32 floats of reduction scratch.  97 KB at
+  // (64, 128): two CTAs per SM.
   static constexpr int SMEM_BYTES =
       4 * (H_I * QS + CH * D_I + CH * H_I + MAX_K + H_I) + 4 * (MAX_K + MAX_CH) + 4 * 32 + 16;
   static_assert(D_I % 32 == 0 && H_I <= 64 && H_I % 4 == 0, "shape");
@@ -78,20 +81,14 @@ struct IdxBwdCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// 16 e4m3 codes -> 16 floats times `scale`
-__device__ __forceinline__ void decode16_e4m3(const uint4 raw, float scale, float (&out)[16]) {
-  const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const __nv_fp8x2_storage_t two = static_cast<__nv_fp8x2_storage_t>(wds[q] >> (16 * h));
-      const __half2 hv = __half2(__nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3));
-      const float2 f = __half22float2(hv);
-      out[4 * q + 2 * h] = f.x * scale;
-      out[4 * q + 2 * h + 1] = f.y * scale;
-    }
-  }
+// 4 e4m3 codes (one 32-bit word, first code in the low byte) -> 4 floats times `scale`
+__device__ __forceinline__ float4 decode4_e4m3(uint32_t raw, float scale) {
+  const __half2 lo = __half2(__nv_cvt_fp8x2_to_halfraw2(
+      static_cast<__nv_fp8x2_storage_t>(raw & 0xFFFFu), __NV_E4M3));
+  const __half2 hi = __half2(__nv_cvt_fp8x2_to_halfraw2(
+      static_cast<__nv_fp8x2_storage_t>(raw >> 16), __NV_E4M3));
+  const float2 a = __half22float2(lo), b = __half22float2(hi);
+  return make_float4(a.x * scale, a.y * scale, b.x * scale, b.y * scale);
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -120,7 +117,7 @@ __device__ __forceinline__ float block_reduce(float x, float* scratch) {
 }
 
 template <int H_I, int D_I>
-__global__ void __launch_bounds__(256) dsa_indexer_kl_bwd_kernel(const IdxBwdParams p) {
+__global__ void __launch_bounds__(256, 2) dsa_indexer_kl_bwd_kernel(const IdxBwdParams p) {
   using C = IdxBwdCfg<H_I, D_I>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* sQ = reinterpret_cast<float*>(smem_raw);     // [H_I][QS]
@@ -160,13 +157,15 @@ __global__ void __launch_bounds__(256) dsa_indexer_kl_bwd_kernel(const IdxBwdPar
   // ---- queries (real-valued) and weights into shared memory
   {
     const uint8_t* qrow = p.q_idx + static_cast<int64_t>(row) * H_I * D_I;
-    for (int u = tid; u < H_I * D_I / 16; u += C::THREADS) {
-      const int j = (u * 16) / D_I, i0 = (u * 16) % D_I;
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow) + u);
-      float f[16];
-      decode16_e4m3(raw, __ldg(p.q_scale + static_cast<int64_t>(row) * H_I + j), f);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) sQ[j * C::QS + i0 + c] = f[c];
+    for (int u = tid; u < H_I * D_I / 4; u += C::THREADS) {
+      const int j = (u * 4) / D_I, i0 = (u * 4) % D_I;
+      const float4 f = decode4_e4m3(__ldg(reinterpret_cast<const uint32_t*>(qrow) + u),
+                                    __ldg(p.q_scale + static_cast<int64_t>(row) * H_I + j));
+      float* dst = sQ + j * C::QS + i0;
+      dst[0] = f.x;
+      dst[1] = f.y;
+      dst[2] = f.z;
+      dst[3] = f.w;
     }
     if (tid < H_I) sW[tid] = __ldg(p.w + static_cast<int64_t>(row) * H_I + tid);
   }
@@ -195,28 +194,24 @@ __global__ void __launch_bounds__(256) dsa_indexer_kl_bwd_kernel(const IdxBwdPar
   }
   __syncthreads();
   for (int c = warp; c < n_chunks; c += 8) {
-    const unsigned any = __ballot_sync(0xffffffffu, sPhys[c * C::CH + lane] >= 0);
+    const bool v = sPhys[c * C::CH + lane] >= 0 || sPhys[c * C::CH + 32 + lane] >= 0;
+    const unsigned any = __ballot_sync(0xffffffffu, v);
     if (lane == 0) sChunk[c] = any != 0u;
   }
   __syncthreads();
 
-  // one chunk of keys, decoded and scaled, into sK (unused keys: zeros)
+  // one chunk of keys, decoded and scaled, into sK (unused keys: zeros); consecutive lanes
+  // take consecutive 4-code words, so the float4 stores are conflict-free
   auto load_chunk = [&](int c) {
-    for (int u = tid; u < C::CH * D_I / 16; u += C::THREADS) {
-      const int e = (u * 16) / D_I, i0 = (u * 16) % D_I;
+    for (int u = tid; u < C::CH * D_I / 4; u += C::THREADS) {
+      const int e = (u * 4) / D_I, i0 = (u * 4) % D_I;
       const int32_t ph = sPhys[c * C::CH + e];
-      float f[16];
-      if (ph >= 0) {
-        const uint4 raw =
-            __ldg(reinterpret_cast<const uint4*>(p.k_idx + static_cast<int64_t>(ph) * D_I + i0));
-        decode16_e4m3(raw, __ldg(p.k_scale + ph), f);
-      } else {
-#pragma unroll
-        for (int x = 0; x < 16; ++x) f[x] = 0.f;
-      }
-      float4* dst = reinterpret_cast<float4*>(sK + e * D_I + i0);
-#pragma unroll
-      for (int x = 0; x < 4; ++x) dst[x] = make_float4(f[4 * x], f[4 * x + 1], f[4 * x + 2], f[4 * x + 3]);
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ph >= 0)
+        f = decode4_e4m3(__ldg(reinterpret_cast<const uint32_t*>(
+                             p.k_idx + static_cast<int64_t>(ph) * D_I + i0)),
+                         __ldg(p.k_scale + ph));
+      *reinterpret_cast<float4*>(sK + e * D_I + i0) = f;
     }
   };
   // D[j][e] for this warp's 4 keys and this lane's heads
@@ -342,7 +337,7 @@ __global__ void __launch_bounds__(256) dsa_indexer_kl_bwd_kernel(const IdxBwdPar
       }
     }
     __syncwarp();
-    // dk of this warp's keys: lanes over dims
+    // dk of this warp's keys: lanes over dims; coefficients 4 heads at a time
     {
       float kacc[C::KPW][C::DPL];
 #pragma unroll
@@ -350,16 +345,23 @@ __global__ void __launch_bounds__(256) dsa_indexer_kl_bwd_kernel(const IdxBwdPar
 #pragma unroll
         for (int dd = 0; dd < C::DPL; ++dd) kacc[kk][dd] = 0.f;
       const float* cw = sCoef + warp * C::KPW * H_I;
-#pragma unroll 4
-      for (int j = 0; j < H_I; ++j) {
-        float qv[C::DPL];
+#pragma unroll 1
+      for (int j0 = 0; j0 < H_I; j0 += 4) {
+        float4 cf[C::KPW];
 #pragma unroll
-        for (int dd = 0; dd < C::DPL; ++dd) qv[dd] = sQ[j * C::QS + lane + 32 * dd];
+        for (int kk = 0; kk < C::KPW; ++kk)
+          cf[kk] = *reinterpret_cast<const float4*>(cw + kk * H_I + j0);
 #pragma unroll
-        for (int kk = 0; kk < C::KPW; ++kk) {
-          const float cf = cw[kk * H_I + j];
+        for (int h = 0; h < 4; ++h) {
+          float qv[C::DPL];
 #pragma unroll
-          for (int dd = 0; dd < C::DPL; ++dd) kacc[kk][dd] = fmaf(cf, qv[dd], kacc[kk][dd]);
+          for (int dd = 0; dd < C::DPL; ++dd) qv[dd] = sQ[(j0 + h) * C::QS + lane + 32 * dd];
+#pragma unroll
+          for (int kk = 0; kk < C::KPW; ++kk) {
+            const float c = h == 0 ? cf[kk].x : h == 1 ? cf[kk].y : h == 2 ? cf[kk].z : cf[kk].w;
+#pragma unroll
+            for (int dd = 0; dd < C::DPL; ++dd) kacc[kk][dd] = fmaf(c, qv[dd], kacc[kk][dd]);
+          }
         }
       }
 #pragma unroll
@@ -378,13 +380,28 @@ __global__ void __launch_bounds__(256) dsa_indexer_kl_bwd_kernel(const IdxBwdPar
       float kv[C::DPL];
 #pragma unroll
       for (int dd = 0; dd < C::DPL; ++dd) kv[dd] = sK[e * D_I + lane + 32 * dd];
+      float cf[C::HPW];
+      if constexpr (C::HPW % 4 == 0) {   // this warp's heads are whole float4s of the row
 #pragma unroll
-      for (int h8 = 0; h8 < C::HPW; ++h8) {
-        const int j = warp * C::HPW + h8;
-        const float cf = j < H_I ? sCoef[e * H_I + j] : 0.f;
+        for (int q4 = 0; q4 < C::HPW / 4; ++q4) {
+          const float4 t =
+              *reinterpret_cast<const float4*>(sCoef + e * H_I + warp * C::HPW + 4 * q4);
+          cf[4 * q4] = t.x;
+          cf[4 * q4 + 1] = t.y;
+          cf[4 * q4 + 2] = t.z;
+          cf[4 * q4 + 3] = t.w;
+        }
+      } else {
 #pragma unroll
-        for (int dd = 0; dd < C::DPL; ++dd) dqacc[h8][dd] = fmaf(cf, kv[dd], dqacc[h8][dd]);
+        for (int h8 = 0; h8 < C::HPW; ++h8) {
+          const int j = warp * C::HPW + h8;
+          cf[h8] = j < H_I ? sCoef[e * H_I + j] : 0.f;
+        }
       }
+#pragma unroll
+      for (int h8 = 0; h8 < C::HPW; ++h8)
+#pragma unroll
+        for (int dd = 0; dd < C::DPL; ++dd) dqacc[h8][dd] = fmaf(cf[h8], kv[dd], dqacc[h8][dd]);
     }
     __syncthreads();   // sK and sCoef are rewritten by the next chunk
   }
