@@ -467,7 +467,12 @@ def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, clk, cpu_leg):
                         "achieved": round(b_tf, 2), "peak": round(fp32_peak, 1),
                         "unit": "TFLOP/s", "frac": round(b_tf / fp32_peak, 4),
                         "flops": f_b,
-                        "peak_note": f"fp32 FMA: {sms} SMs x 128 lanes x 2 FLOP x {mhz:.0f} MHz"},
+                        "peak_note": f"fp32 FMA: {sms} SMs x 128 lanes x 2 FLOP x {mhz:.0f} MHz",
+                        "vs_tensor": {"peak": round(peaks["bf16_sustained"] / 2, 1),
+                                      "frac": round(b_tf / (peaks["bf16_sustained"] / 2), 4),
+                                      "note": "tf32 tensor peak (half the measured bf16, the "
+                                              "nominal ratio): the bound once the three "
+                                              "contractions run on tensor cores"}},
            "target_roofline": {"kernel": "dsa_sparse_mla_kernel (target mode)",
                                "bound": "tensor", "achieved": round(t_tf, 1),
                                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
