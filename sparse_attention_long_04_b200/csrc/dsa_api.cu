@@ -12,6 +12,7 @@
 #include "cache_append.cuh"
 #include "indexer.cuh"
 #include "indexer_bwd.cuh"
+#include "indexer_bwd_tc.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
@@ -543,12 +544,19 @@ dsa_status_t target_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_
   return launch_status();
 }
 
-template <int H_I, int D_I>
-dsa_status_t kl_backward_impl(const IdxBwdParams& prm, cudaStream_t st) {
-  using C = IdxBwdCfg<H_I, D_I>;
-  auto k = dsa_indexer_kl_bwd_kernel<H_I, D_I>;
-  if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
-  k<<<prm.row_count, C::THREADS, C::SMEM_BYTES, st>>>(prm);
+// (64, 128): the tensor-core kernel; the small indexer shape (4 heads: too narrow an MMA N)
+// runs on the CUDA cores.
+dsa_status_t kl_backward_launch(bool full, const IdxBwdParams& prm, cudaStream_t st) {
+  if (full) {
+    auto k = dsa_indexer_kl_bwd_tc_kernel;
+    if (prepare_kernel(k, KlTcCfg::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
+    k<<<prm.row_count, KlTcCfg::THREADS, KlTcCfg::SMEM_BYTES, st>>>(prm);
+  } else {
+    using C = IdxBwdCfg<4, 32>;
+    auto k = dsa_indexer_kl_bwd_kernel<4, 32>;
+    if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
+    k<<<prm.row_count, C::THREADS, C::SMEM_BYTES, st>>>(prm);
+  }
   return launch_status();
 }
 
@@ -845,7 +853,7 @@ dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* s
   prm.num_kv_rows = s.num_kv_rows;
   prm.status = dev_status;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return full ? kl_backward_impl<64, 128>(prm, st) : kl_backward_impl<4, 32>(prm, st);
+  return kl_backward_launch(full, prm, st);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream) {

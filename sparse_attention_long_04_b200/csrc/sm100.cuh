@@ -334,6 +334,37 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------- warp sums
+
+// One step of a sum of 64 values per lane across the 32 lanes of a warp (a butterfly that
+// halves the values each step): each lane holds 2 LEN partial sums; it keeps LEN of them (the
+// upper half if lane bit LEN/2 is set), adds the partner lane's copy of the same entries and
+// hands its other half to the partner.  After the steps 32, 16, 8, 4, 2 lane l holds the warp
+// sums of entries e0 and e0 + 1, e0 = 32 b4 + 16 b3 + 8 b2 + 4 b1 + 2 b0 (b = the bits of l).
+template <int LEN>
+__device__ __forceinline__ void head_sum_step(float (&v)[64], int lane) {
+  const bool up = (lane & (LEN / 2)) != 0;
+#pragma unroll
+  for (int j = 0; j < LEN; ++j) {
+    const float send = up ? v[j] : v[j + LEN];
+    const float keep = up ? v[j + LEN] : v[j];
+    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, LEN / 2);
+  }
+}
+
+__device__ __forceinline__ void warp_sum64(float (&v)[64], int lane) {
+  head_sum_step<32>(v, lane);
+  head_sum_step<16>(v, lane);
+  head_sum_step<8>(v, lane);
+  head_sum_step<4>(v, lane);
+  head_sum_step<2>(v, lane);
+}
+
+__device__ __forceinline__ int warp_sum64_first(int lane) {
+  return ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
+         ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte-swizzled tile.
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);

@@ -111,20 +111,6 @@ struct MlaCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// One step of the head sum across a warp: each lane holds 2 LEN values (its partial sums of
-// 2 LEN keys); it keeps LEN of them (the upper half if lane bit LEN/2 is set), adds the partner
-// lane's copy of the same keys, and hands its other half to the partner.
-template <int LEN>
-__device__ __forceinline__ void head_sum_step(float (&v)[64], int lane) {
-  const bool up = (lane & (LEN / 2)) != 0;
-#pragma unroll
-  for (int j = 0; j < LEN; ++j) {
-    const float send = up ? v[j] : v[j + LEN];
-    const float keep = up ? v[j + LEN] : v[j];
-    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, LEN / 2);
-  }
-}
-
 template <int D_QK, int D_V, bool kTarget = false>
 __global__ void __launch_bounds__(512, 1)
     dsa_sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) {
@@ -464,8 +450,7 @@ __global__ void __launch_bounds__(512, 1)
         hrow < p.h ? p.lse_in[static_cast<int64_t>(row) * p.h + hrow] * 1.4426950408889634f
                    : INFINITY;
     // after the butterfly this lane holds the head sums of keys key0 and key0 + 1
-    const int key0 = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
-                     ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+    const int key0 = warp_sum64_first(lane);
     const float inv_h = 1.f / static_cast<float>(p.h);
     const float sc = p.scale_log2;
     bool ok = !abort_s;
@@ -491,11 +476,7 @@ __global__ void __launch_bounds__(512, 1)
           v[32 * hh + j] = ((vb >> j) & 1u) ? pr : 0.f;
         }
       }
-      head_sum_step<32>(v, lane);
-      head_sum_step<16>(v, lane);
-      head_sum_step<8>(v, lane);
-      head_sum_step<4>(v, lane);
-      head_sum_step<2>(v, lane);
+      warp_sum64(v, lane);
       // the 4 warps' sums meet in shared memory (double-buffered by tile parity)
       const int buf = i & 1;
       float* red = sRed + buf * 4 * C::BN;
