@@ -84,3 +84,16 @@ def test_two_ranks_gloo(tmp_path):
         assert np.array_equal(np.load(tmp_path / f"idx{rank}.npy"), idx[rows])
         assert np.array_equal(np.load(tmp_path / f"lse{rank}.npy"), lse[rows])
         assert np.array_equal(np.load(tmp_path / f"o{rank}.npy"), o[rows])
+
+
+def test_bench_work_models():
+    """The bench's FLOP counts and the KL backward roofline, on hand-countable cases."""
+    import bench
+    d = dict(h_idx=2, d_idx=4, topk=3, h=5, d_qk=6, d_v=4)
+    # one sequence of 5 rows, k = 3: selected (row, key) pairs = 1 + 2 + 3 + 3 + 3 = 12
+    f_t, f_b = bench.train_flops([5], d)
+    assert f_t == 2 * 5 * 6 * 12 and f_b == 3 * 2 * 2 * 4 * 12
+    roof = bench.kl_backward_roofline(3e12, 2.0, 1000.0)
+    # 1e12 e4m3 FLOP at 2000 TF/s + 2e12 bf16 FLOP at 1000 TF/s = 0.5 ms + 2 ms
+    assert roof["ideal_ms"] == pytest.approx(2.5) and roof["frac"] == pytest.approx(1.25)
+    assert roof["achieved"] == pytest.approx(1500.0) and roof["bound"] == "tensor"
