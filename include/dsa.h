@@ -27,6 +27,11 @@
  *                       rows) and decode (one new token per sequence, paged or contiguous
  *                       caches)
  *
+ * and, around the path: dsa_cache_append (the decode step that writes the new token's e4m3
+ * indexer key and latent row into the caches), and dsa_indexer_kl_target with
+ * dsa_indexer_kl_backward (the indexer's training step in the sparse stage), each documented
+ * where it is declared below.
+ *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and contiguous.
  *     The library allocates nothing and keeps no state apart from a per-device attribute

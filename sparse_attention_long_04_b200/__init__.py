@@ -3,7 +3,9 @@
 The library (``include/dsa.h``) runs the three DSA stages in hand-written CUDA kernels:
 the FP8 lightning indexer, the exact top-k selector and sparse MLA attention in MQA mode
 ("FP8 index -> top-k selection -> sparse core attention", "DeepSeek V3.2-Exp Cuts
-Long-Context Costs with DeepSeek Sparse Attention (DSA)", pipeline summary).
+Long-Context Costs with DeepSeek Sparse Attention (DSA)", pipeline summary), plus the decode
+cache append and the indexer's training step (KL target and backward, same page, "Training
+signal").
 
 This module only marshals arguments: the functions named like the C entry points take torch
 tensors (device memory owned by the caller), pass their pointers and the current CUDA stream,

@@ -13,6 +13,10 @@
 //   dk[s_e,:] += g_e sum_j w[t,j] [D[j,e] > 0] q[t,j,:]   (summed over rows with atomic adds)
 // The derivative of max(x, 0) at 0 is taken as 0.
 //
+// This CUDA-core kernel serves the small indexer shape (4 heads: too narrow an N for an MMA);
+// the 64 x 128 shape runs on the tensor cores (indexer_bwd_tc.cuh), which reuses the parameter
+// block and the e4m3 decoding below.
+//
 // Design (CUDA cores, fp32).  One CTA of 256 threads per query row, two CTAs per SM.  The row's
 // real-valued queries stay in shared memory (row stride D_I + 1 floats, so that lanes reading
 // one dim of consecutive heads hit distinct banks); keys come 64 at a time, decoded from e4m3 and
