@@ -1,8 +1,9 @@
 """NumPy twin of the C oracle, for tiny inputs -- TEST INFRASTRUCTURE ONLY.
 
-Vectorised fp64 restatements of the same three definitions (indexer, top-k, MQA-mode sparse
-attention; "DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention (DSA)",
-pipeline summary and "Instantiation").  Written independently of ``dsa_oracle.c`` so that the
+Vectorised fp64 restatements of the same definitions (indexer, top-k, MQA-mode sparse
+attention, and the indexer's training target and KL gradients; "DeepSeek V3.2-Exp Cuts
+Long-Context Costs with DeepSeek Sparse Attention (DSA)", pipeline summary, "Instantiation" and
+"Training signal").  Written independently of ``dsa_oracle.c`` so that the
 two cross-check each other; neither is the CUDA path.
 """
 from __future__ import annotations
@@ -59,3 +60,43 @@ def sparse_attention(q_bits, kv_bits, sel_rows, scale: float, d_v: int):
     p = np.exp(logits - m)
     den = p.sum(axis=1, keepdims=True)
     return (p @ kv[:, :d_v]) / den, (m + np.log(den))[:, 0]
+
+
+def kl_target(q_bits, kv_bits, sel_rows, scale: float) -> np.ndarray:
+    """The indexer's training target on one row's selection: the mean over heads of each
+    head's softmax over the selected latent rows ("Training signal").  q_bits [H, D_qk],
+    kv_bits [R, D_qk] bf16 codes; sel_rows physical rows (-1: unused, target 0)."""
+    sel_rows = np.asarray(sel_rows, dtype=np.int64)
+    out = np.zeros(len(sel_rows))
+    used = sel_rows >= 0
+    if not used.any():
+        return out
+    q = bf16_to_f64(q_bits)
+    kv = bf16_to_f64(kv_bits[sel_rows[used]])
+    logits = scale * (q @ kv.T)                      # [H, n]
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    out[used] = p.mean(axis=0)
+    return out
+
+
+def indexer_kl(q, w, keys, valid, target):
+    """KL(target || softmax of the indexer scores) on one row's selection and its gradients,
+    written with whole-array operations: q [H_I, D_I], w [H_I], keys [k, D_I] real-valued,
+    valid [k] bool, target [k].  Returns (loss, dw [H_I], dq [H_I, D_I], dk [k, D_I])."""
+    q, w, keys = (np.asarray(a, np.float64) for a in (q, w, keys))
+    valid = np.asarray(valid, bool)
+    p = np.where(valid, np.asarray(target, np.float64), 0.0)
+    dots = q @ keys.T                                # [H_I, k]
+    relu = np.maximum(dots, 0.0)
+    s = np.where(valid, w @ relu, -np.inf)
+    log_pi = s - (s.max() + np.log(np.exp(s - s.max()).sum())) if valid.any() else s
+    pi = np.where(valid, np.exp(log_pi), 0.0)
+    pos = p > 0
+    loss = float((p[pos] * (np.log(p[pos]) - log_pi[pos])).sum())
+    g = np.where(valid, pi * p.sum() - p, 0.0)
+    gate = (dots > 0).astype(np.float64)             # d ReLU / d x, 0 at x = 0
+    dw = relu @ g
+    dq = (w[:, None] * (gate * g[None, :])) @ keys
+    dk = (g[:, None] * (gate.T * w[None, :])) @ q
+    return loss, dw, dq, dk

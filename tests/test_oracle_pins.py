@@ -549,3 +549,24 @@ def test_indexer_kl_key_gradient_sums_over_rows():
     assert sorted(acc) == both["dk_rows"].tolist()
     for p, g in zip(both["dk_rows"], both["dk"]):
         np.testing.assert_allclose(g, acc[int(p)], rtol=1e-12, atol=1e-15)
+
+
+def test_training_oracle_matches_numpy_twin():
+    """The C oracle's target and KL gradients equal the independent NumPy twin's."""
+    wl = _tiny_attn_workload()
+    rows = [30, 39]
+    idx = np.array([[3, 11, 0, -1, 25, 7, 30, -1], [39, 38, 37, 4, -1, -1, -1, -1]], np.int32)
+    t = oracle.kl_target_rows(wl, rows, idx)
+    qb = wl.q.view(torch.int16).numpy().view(np.uint16)
+    kvb = wl.kv.view(torch.int16).numpy().view(np.uint16)
+    for i, r in enumerate(rows):   # a single prefill sequence: logical key s is physical row s
+        np.testing.assert_allclose(t[i], reference_np.kl_target(qb[r], kvb, idx[i], 0.3),
+                                   rtol=1e-12, atol=1e-15)
+    q, w, keys, valid, target = _random_real_case(13, n=3, h=4, d=6, k=9)
+    res = oracle.indexer_kl_real(q, w, keys, valid, target)
+    for i in range(3):
+        loss, dw, dq, dk = reference_np.indexer_kl(q[i], w[i], keys[i], valid[i] > 0, target[i])
+        assert res["loss"][i] == pytest.approx(loss, rel=1e-12, abs=1e-15)
+        np.testing.assert_allclose(res["dw"][i], dw, rtol=1e-11, atol=1e-14)
+        np.testing.assert_allclose(res["dq"][i], dq, rtol=1e-11, atol=1e-14)
+        np.testing.assert_allclose(res["dk"][i], dk, rtol=1e-11, atol=1e-14)
