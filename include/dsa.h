@@ -193,6 +193,11 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const ds
  * idx_out is NULL, split-KV partials).  Larger workspaces allow larger prefill chunks. */
 DSA_API size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs);
 
+/* The same size for a device with `sm_count` SMs, without touching any device (host-only; for
+ * sizing buffers before a device is chosen).  0 on invalid arguments or sm_count <= 0. */
+DSA_API size_t dsa_forward_workspace_size_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                              int32_t sm_count);
+
 /* The whole path for all seqs->total_rows query rows.  Inputs as for the three stages.
  *   idx_out  optional int32 [total_rows, topk]: the selected indices (NULL = not kept).
  *            When NULL, rows with at most topk prior keys (the first topk rows of each prefill

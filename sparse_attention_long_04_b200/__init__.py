@@ -40,7 +40,7 @@ EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_fwd", "dsa_forward_workspace_size", "dsa_forward",
             "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
             "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
-            "dsa_indexer_kl_target", "dsa_indexer_kl_backward")
+            "dsa_indexer_kl_target", "dsa_indexer_kl_backward", "dsa_forward_workspace_size_for")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -79,6 +79,7 @@ def _load():
         "dsa_sparse_mla_workspace_size": (SZ, [DP, SP, I32]),
         "dsa_sparse_mla_fwd": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, SZ, P, P]),
         "dsa_forward_workspace_size": (SZ, [DP, SP]),
+        "dsa_forward_workspace_size_for": (SZ, [DP, SP, I32]),
         "dsa_forward": (I32, [DP, SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_selftest_wait_timeout": (I32, [P, P]),
@@ -225,6 +226,11 @@ def dsa_sparse_mla_fwd_noalloc(pb: Problem, q, kv, idx, row_begin: int, row_coun
 
 def dsa_forward_workspace_size(pb: Problem) -> int:
     return int(lib.dsa_forward_workspace_size(ctypes.byref(pb.dims), ctypes.byref(pb.seqs)))
+
+
+def dsa_forward_workspace_size_for(pb: Problem, sm_count: int) -> int:
+    return int(lib.dsa_forward_workspace_size_for(ctypes.byref(pb.dims), ctypes.byref(pb.seqs),
+                                                  sm_count))
 
 
 def dsa_forward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, q, kv, idx_out, out, lse,

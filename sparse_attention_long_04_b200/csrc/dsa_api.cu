@@ -664,6 +664,12 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                       workspace_bytes, dev_status, reinterpret_cast<cudaStream_t>(stream), splits);
 }
 
+size_t dsa_forward_workspace_size_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                      int32_t sm_count) {
+  if (check_common(dims, seqs) != DSA_OK || sm_count <= 0) return 0;
+  return plan_forward(*dims, *seqs, sm_count).total;
+}
+
 size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs) {
   if (check_common(dims, seqs) != DSA_OK) return 0;
   DeviceInfo info;

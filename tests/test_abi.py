@@ -188,3 +188,35 @@ def test_indexer_training_argument_errors(dsa):
     assert backward(pb, [FAKE + 4] + ok[1:]) == dsa.DSA_ERR_MISALIGNED
     assert backward(pb, ok, rb=1) == dsa.DSA_ERR_INVALID_ARG
     assert backward(_pb(dsa, h_idx=32), ok) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_forward_workspace_plan_on_the_host(dsa):
+    """Workspace sizes of `dsa_forward` for a given SM count, with no device involved.  A decode
+    batch needs a score slab of every sequence's padded row and its indices; a prefill sequence
+    is cut into chunks of at most 256 MiB of fp32 scores, and a sequence that needs several
+    chunks gets a multiple of sm_count / 2 rows per chunk (whole waves of two-CTA rows)."""
+    full = dict(h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512, topk=2048, softmax_scale=0.04)
+    size = dsa.dsa_forward_workspace_size_for
+    # decode_B64_N128k shapes, contiguous caches: 128 attention CTAs fill one wave of 148 SMs,
+    # so no split-KV partials
+    dec = dsa.make_problem(mode="decode", num_kv_rows=64 * 131072, seqlens=[131072] * 64,
+                           seq_lens=FAKE, max_seqlen=131072, **full)
+    assert size(dec, 148) == 64 * 131072 * 4 + 64 * 2048 * 4
+    # a few long decode rows on many SMs are split, and the partials add to the workspace
+    few = dsa.make_problem(mode="decode", num_kv_rows=2 * 131072, seqlens=[131072] * 2,
+                           seq_lens=FAKE, max_seqlen=131072, **full)
+    assert size(few, 148) > 2 * 131072 * 4 + 2 * 2048 * 4
+    # prefill: 131072 rows need 512 rows of scores per 256 MiB; 148 SMs -> 444 (6 x 74) rows
+    pre = dsa.make_problem(mode="prefill", num_kv_rows=131072, seqlens=[131072],
+                           cu_seqlens=FAKE, **full)
+    assert size(pre, 148) == 444 * 131072 * 4 + 444 * 2048 * 4
+    assert size(pre, 132) == 462 * 131072 * 4 + 462 * 2048 * 4       # 7 x 66 rows
+    # a short sequence runs in one chunk; varlen sizes the slab for the largest chunk's scores
+    # and the indices for the chunk with the most rows (here the short sequence's 1000)
+    short = dsa.make_problem(mode="prefill", num_kv_rows=1000, seqlens=[1000], cu_seqlens=FAKE,
+                             **full)
+    assert size(short, 148) == 1000 * 1000 * 4 + 1000 * 2048 * 4
+    mix = dsa.make_problem(mode="prefill", num_kv_rows=132072, seqlens=[1000, 131072],
+                           cu_seqlens=FAKE, **full)
+    assert size(mix, 148) == 444 * 131072 * 4 + 1000 * 2048 * 4
+    assert size(pre, 0) == 0 and size(_pb(dsa, topk=100), 148) == 0
