@@ -269,8 +269,9 @@ DSA_API dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seq
  *   loss     fp32 [row_count];  dw fp32 [row_count, h_idx];  dq fp32 [row_count, h_idx, d_idx]
  *   dk       fp32 [num_kv_rows, d_idx]: ADDED to (zero it first); the order of the atomic
  *            additions is not fixed, so its last bits may vary from run to run
- * Indexer shapes (h_idx, d_idx) = (64, 128) or (4, 32), both modes.  All pointers 16-byte
- * aligned.  Out-of-range indices are skipped and set DSA_DEVICE_BAD_INDEX. */
+ * Indexer shapes (h_idx, d_idx) = (64, 128) with topk a multiple of 128, or (4, 32); both
+ * modes.  All pointers 16-byte aligned.  Out-of-range indices are skipped and set
+ * DSA_DEVICE_BAD_INDEX. */
 DSA_API dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                              const uint8_t* q_idx, const float* q_scale,
                                              const float* w, const uint8_t* k_idx,

@@ -823,6 +823,7 @@ dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* s
   const bool full = d.h_idx == 64 && d.d_idx == 128;
   const bool tiny = d.h_idx == 4 && d.d_idx == 32;
   if (!full && !tiny) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (full && d.topk % KlTcCfg::BK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;   // whole key tiles
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
   if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !idx || !target || !loss || !dw || !dq ||
       !dk)

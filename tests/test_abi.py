@@ -188,6 +188,8 @@ def test_indexer_training_argument_errors(dsa):
     assert backward(pb, [FAKE + 4] + ok[1:]) == dsa.DSA_ERR_MISALIGNED
     assert backward(pb, ok, rb=1) == dsa.DSA_ERR_INVALID_ARG
     assert backward(_pb(dsa, h_idx=32), ok) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    # the tensor-core kernel of the 64 x 128 indexer takes the selection in 128-key tiles
+    assert backward(_pb(dsa, topk=192), ok) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
 
 
 def test_forward_workspace_plan_on_the_host(dsa):
