@@ -263,7 +263,9 @@ DSA_API dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seq
  *   dk[row,:] += g_e sum_j w[t,j] [D[j,e] > 0] q[t,j,:]   for the physical row of idx[t,e]
  * (d/dx max(x, 0) = 0 at x = 0; the gradients are those of the real values, so a caller that
  * quantised q and k passes them straight through the rounding).
- *   q_idx, q_scale, w, k_idx, k_scale   as for dsa_indexer_scores (k_scale must not be NULL)
+ *   q_idx, q_scale, w, k_idx, k_scale   as for dsa_indexer_scores (k_scale must not be NULL;
+ *            the scales must be positive, as the e4m3 quantiser makes them: the ReLU masks
+ *            are taken from the e4m3 products)
  *   idx      int32 [row_count, topk], relative to row_begin, -1 = unused (required)
  *   target   fp32 [row_count, topk]
  *   loss     fp32 [row_count];  dw fp32 [row_count, h_idx];  dq fp32 [row_count, h_idx, d_idx]
