@@ -1,6 +1,7 @@
 // C ABI of the DSA hot path (see include/dsa.h): argument checks, planning and launches.
 // Nothing here allocates device memory; the only state is a per-device attribute cache.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -97,6 +98,15 @@ dsa_status_t prepare_kernel(Kernel k, int smem_bytes) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range around an entry point (host side: argument checks, planning and the launches it
+// enqueues); a no-op unless a profiler is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -608,6 +618,7 @@ dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                 const uint8_t* k_idx, const float* k_scale, int32_t row_begin,
                                 int32_t row_count, float* scores, int64_t ld_scores,
                                 int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_indexer_scores");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if (!indexer_shape_ok(*dims, seqs->mode)) return DSA_ERR_UNSUPPORTED_SHAPE;
@@ -625,6 +636,7 @@ dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
 dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
                       int64_t ld_scores, int32_t row_begin, int32_t row_count, int32_t* idx,
                       int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_topk");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
@@ -648,6 +660,7 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                 int32_t row_begin, int32_t row_count, uint16_t* out, float* lse,
                                 void* workspace, size_t workspace_bytes, int32_t* dev_status,
                                 dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_sparse_mla_fwd");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
@@ -682,6 +695,7 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
                          const float* k_scale, const uint16_t* q, const uint16_t* kv,
                          int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
                          size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_forward");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   const dsa_dims_t& d = *dims;
@@ -751,6 +765,7 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
 dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* k_new,
                               const uint16_t* kv_new, uint8_t* k_cache, float* k_scale_cache,
                               uint16_t* kv_cache, int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_cache_append");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   const dsa_dims_t& d = *dims;
@@ -791,6 +806,7 @@ dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seqs_t* seq
                                    const uint16_t* q, const uint16_t* kv, const int32_t* idx,
                                    const float* lse, int32_t row_begin, int32_t row_count,
                                    float* target, int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_indexer_kl_target");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
@@ -816,6 +832,7 @@ dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* s
                                      const int32_t* idx, const float* target, int32_t row_begin,
                                      int32_t row_count, float* loss, float* dw, float* dq,
                                      float* dk, int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_indexer_kl_backward");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   const dsa_dims_t& d = *dims;
@@ -913,6 +930,7 @@ dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const dsa_seqs_t
                                         const uint16_t* q, const uint16_t* kv, const int32_t* idx,
                                         int32_t row_begin, int32_t row_count, uint16_t* out,
                                         float* lse, int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_sparse_mla_fwd_noalloc");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
