@@ -183,6 +183,110 @@ def kl_backward_roofline(flops_3, ms, bf16_tflops):
 
 # ------------------------------------------------------------------------------ our arm
 
+class DecodeStep:
+    """The staged decode step on one workload: the indexer counting each row's first radix digit
+    as it writes the scores, the top-k starting from those counts, the sparse MLA forward (the
+    same kernels dsa_forward runs), with optional CUDA events between the calls."""
+
+    def __init__(self, dsa, wl, stream):
+        d = wl.dims
+        dev = wl.kv.device
+        self.dsa, self.wl, self.stream = dsa, wl, stream
+        self.pb = dsa.problem_of(wl)
+        B = wl.batch
+        self.ld = (wl.max_seqlen + 3) // 4 * 4
+        self.scores = torch.empty(B, self.ld, dtype=torch.float32, device=dev)
+        self.hist = torch.zeros(B, dsa.TOPK_HIST_BINS, dtype=torch.int32, device=dev)
+        self.idx = torch.empty(B, d["topk"], dtype=torch.int32, device=dev)
+        self.out = torch.empty(B, d["h"], d["d_v"], dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, d["h"], dtype=torch.float32, device=dev)
+        self.mla_ws_bytes = dsa.dsa_sparse_mla_workspace_size(self.pb, B)
+        self.mla_ws = torch.empty(max(self.mla_ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.launches = 3 + (1 if self.mla_ws_bytes > 0 else 0)
+
+    def __call__(self, ev=None):
+        dsa, wl, st, B = self.dsa, self.wl, self.stream, self.wl.batch
+        if ev is not None:
+            ev[0].record(st)
+        dsa.check(dsa.dsa_indexer_scores(self.pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx,
+                                         wl.k_scale, 0, B, self.scores, self.ld, self.status, st,
+                                         hist=self.hist), "indexer")
+        if ev is not None:
+            ev[1].record(st)
+        dsa.check(dsa.dsa_topk(self.pb, self.scores, self.ld, 0, B, self.idx, self.status, st,
+                               hist=self.hist), "topk")
+        if ev is not None:
+            ev[2].record(st)
+        dsa.check(dsa.dsa_sparse_mla_fwd(self.pb, wl.q, wl.kv, self.idx, 0, B, self.out,
+                                         self.lse, self.mla_ws, self.mla_ws_bytes, self.status,
+                                         st), "sparse_mla")
+        if ev is not None:
+            ev[3].record(st)
+
+
+class CudaTimer:
+    """CUDA events on the launching stream and device synchronisation (the bench's clock)."""
+
+    @staticmethod
+    def event():
+        return torch.cuda.Event(enable_timing=True)
+
+    @staticmethod
+    def sync():
+        torch.cuda.synchronize()
+
+
+def time_decode(args, dsa, step, world, dev, clocks=None, timer=CudaTimer):
+    """W warm-up steps, then K timed steps with events between the stages, bracketed by a
+    barrier and a device synchronisation on both sides.  Returns (ms per step (max over ranks),
+    mean ms per stage [indexer, top-k, sparse MLA], clocks)."""
+    stream = step.stream
+    for _ in range(args.warmup):
+        step()
+    timer.sync()
+    st, raw = step.dsa.dsa_read_device_status(step.status, stream)
+    step.dsa.check(st, "device status after warm-up")
+    evs = [[timer.event() for _ in range(4)] for _ in range(args.steps)]
+    start, end = timer.event(), timer.event()
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.25)
+    if world > 1:
+        torch.distributed.barrier()
+    timer.sync()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    timer.sync()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop() if clocks is not None else None
+    ms = start.elapsed_time(end)
+    k_ms = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+            for e in evs]
+    per_kernel = [sum(x[j] for x in k_ms) / len(k_ms) for j in range(3)]
+    st, raw = step.dsa.dsa_read_device_status(step.status, stream)
+    step.dsa.check(st, "device status after timing")
+    return max_over_ranks(ms, world, dev) / args.steps, per_kernel, clk
+
+
+def decode_rooflines(wl, ms_step, per_kernel, peaks, traffic=None):
+    work = decode_algorithmic_bytes(wl)
+    idx_gbs = work["indexer"] / (per_kernel[0] / 1e3) / 1e9
+    step_gbs = work["total"] / (ms_step / 1e3) / 1e9
+    roof = {"kernel": "dsa_indexer_kernel (decode)", "bound": "hbm",
+            "achieved": round(idx_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": round(idx_gbs / peaks["hbm"], 4), "traffic": traffic,
+            "peak_source": peaks["source"],
+            "algorithmic_bytes_per_launch": work["indexer"]}
+    step_roof = {"bound": "hbm", "achieved": round(step_gbs, 1), "unit": "GB/s",
+                 "frac": round(step_gbs / peaks["hbm"], 4),
+                 "algorithmic_bytes_per_step": work["total"]}
+    return roof, step_roof
+
+
 def run_ours(args, rank, world, local_rank):
     import sparse_attention_long_04_b200 as dsa
     from dsa_workloads import make_config, CONFIGS
@@ -202,61 +306,12 @@ def run_ours(args, rank, world, local_rank):
     else:
         wl = make_config(DECODE_CFG, device=dev, seed=rank_seed(DECODE_CFG, rank))
     d = wl.dims
-    pb = dsa.problem_of(wl)
     B = wl.batch
-    ld = (wl.max_seqlen + 3) // 4 * 4
-    scores = torch.empty(B, ld, dtype=torch.float32, device=dev)
-    idx = torch.empty(B, d["topk"], dtype=torch.int32, device=dev)
-    out = torch.empty(B, d["h"], d["d_v"], dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(B, d["h"], dtype=torch.float32, device=dev)
-    mla_ws_bytes = dsa.dsa_sparse_mla_workspace_size(pb, B)
-    mla_ws = torch.empty(max(mla_ws_bytes, 16), dtype=torch.uint8, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    launches_per_step = 3 + (1 if mla_ws_bytes > 0 else 0)
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        dsa.check(dsa.dsa_indexer_scores(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx, wl.k_scale,
-                                         0, B, scores, ld, status, stream), "indexer")
-        if ev is not None:
-            ev[1].record(stream)
-        dsa.check(dsa.dsa_topk(pb, scores, ld, 0, B, idx, status, stream), "topk")
-        if ev is not None:
-            ev[2].record(stream)
-        dsa.check(dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, idx, 0, B, out, lse, mla_ws,
-                                         mla_ws_bytes, status, stream), "sparse_mla")
-        if ev is not None:
-            ev[3].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    st, raw = dsa.dsa_read_device_status(status, stream)
-    dsa.check(st, "device status after warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    time.sleep(0.25)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop()
-    ms = start.elapsed_time(end)
-    k_ms = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
-            for e in evs]
-    per_kernel = [sum(x[j] for x in k_ms) / len(k_ms) for j in range(3)]
-    ms_step = max_over_ranks(ms, world, dev) / args.steps
+    step = DecodeStep(dsa, wl, stream)
+    ms_step, per_kernel, clk = time_decode(args, dsa, step, world, dev,
+                                           clocks=ClockSampler(local_rank))
     value = weak_value(world, B, ms_step)
+    out, lse = step.out, step.lse
 
     # ---- end to end through the public call, host buffers, copies inside the timed region.
     # Two buffer sets and three streams, as a serving loop runs it: step i+1's inputs go up
@@ -317,14 +372,10 @@ def run_ours(args, rank, world, local_rank):
     for st_b in sets:
         st_e, _ = dsa.dsa_read_device_status(st_b["fwd"].status, stream)
         dsa.check(st_e, "e2e device status")
-    fwd = sets[0]["fwd"]
-    st, raw = dsa.dsa_read_device_status(status, stream)
-    dsa.check(st, "device status after timing")
+    del sets
 
-    work = decode_algorithmic_bytes(wl)
-    idx_gbs = work["indexer"] / (per_kernel[0] / 1e3) / 1e9
-    step_gbs = work["total"] / (ms_step / 1e3) / 1e9
-    traffic = load_traffic("indexer_decode")
+    roof, step_roof = decode_rooflines(wl, ms_step, per_kernel, peaks,
+                                       traffic=load_traffic("indexer_decode"))
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -344,14 +395,8 @@ def run_ours(args, rank, world, local_rank):
                    "latent": d["d_qk"], "d_v": d["d_v"],
                    "l2": "inputs larger than L2 (11 GB of caches per step)",
                    "parallelism": f"replicas{world}"},
-        "roofline": {"kernel": "dsa_indexer_kernel (decode)", "bound": "hbm",
-                     "achieved": round(idx_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": round(idx_gbs / peaks["hbm"], 4),
-                     "traffic": traffic, "peak_source": peaks["source"],
-                     "algorithmic_bytes_per_launch": work["indexer"]},
-        "step_roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "unit": "GB/s",
-                          "frac": round(step_gbs / peaks["hbm"], 4),
-                          "algorithmic_bytes_per_step": work["total"]},
+        "roofline": roof,
+        "step_roofline": step_roof,
         "kernel_ms": {"indexer": round(per_kernel[0], 4), "topk": round(per_kernel[1], 4),
                       "sparse_mla": round(per_kernel[2], 4)},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -360,26 +405,177 @@ def run_ours(args, rank, world, local_rank):
                         "from pinned host memory, dsa_forward, out + lse copied back; the "
                         "paged caches stay resident; two buffer sets on three streams overlap "
                         "step i+1's upload and step i-1's download with step i"},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": step.launches * args.steps,
         "clocks": clk,
     }
-    del fwd
     line["cache_append"] = time_cache_append(args, dsa, wl, stream, peaks,
                                              cpu_leg=rank == 0 and not args.no_cpu)
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    del step, out, lse, wl
+    torch.cuda.empty_cache()
+    if not args.no_extra:
+        line["decode_B32_N32k"] = run_decode_extra(args, dsa, dev, stream, peaks, rank, world)
     if not args.no_prefill:
-        del scores, idx, out, lse
-        line["prefill"] = run_prefill(args, dsa, dev, stream, peaks, rank, world)
+        line["prefill"] = run_prefill(args, dsa, dev, stream, peaks, rank, world, PREFILL_CFG)
+        if not args.no_extra:
+            line["prefill_L16k"] = run_prefill(args, dsa, dev, stream, peaks, rank, world, 4)
     if not args.no_train:
         line["indexer_train"] = run_indexer_train(args, dsa, dev, stream, peaks, rank, world,
                                                   cpu_leg=rank == 0 and not args.no_cpu)
-    if rank == 0 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     return line
 
 
-def run_prefill(args, dsa, dev, stream, peaks, rank, world):
+def run_decode_extra(args, dsa, dev, stream, peaks, rank, world, cfg=2):
+    """decode_B32_N32k: the same staged step on the 32-sequence, 32k-context workload
+    (contiguous caches), with its rooflines and the oracle on a sample of its rows."""
     from dsa_workloads import make_config, CONFIGS
-    wl = make_config(PREFILL_CFG, device=dev, seed=rank_seed(PREFILL_CFG, rank))
+    import oracle
+    wl = make_config(cfg, device=dev, seed=rank_seed(cfg, rank))
+    step = DecodeStep(dsa, wl, stream)
+    ms_step, per_kernel, _ = time_decode(args, dsa, step, world, dev)
+    roof, step_roof = decode_rooflines(wl, ms_step, per_kernel, peaks)
+    res = {"workload": CONFIGS[cfg]["name"], "value": round(weak_value(world, wl.batch, ms_step), 1),
+           "unit": "tokens/s", "ms_per_step": round(ms_step, 4), "steps": args.steps,
+           "kernel_ms": {"indexer": round(per_kernel[0], 4), "topk": round(per_kernel[1], 4),
+                         "sparse_mla": round(per_kernel[2], 4)},
+           "roofline": roof, "step_roofline": step_roof,
+           "l2": "inputs larger than L2 (2.4 GB of latent rows, 138 MB of indexer keys)",
+           "gpu_launches_per_step": step.launches}
+    if rank == 0 and not args.no_cpu:
+        n = min(wl.batch, oracle.num_threads())
+        t0 = time.perf_counter()
+        oracle.forward_rows(wl, list(range(n)))
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": round(n / dt, 3), "unit": "tokens/s",
+                               "cores": oracle.num_threads(), "kind": "oracle",
+                               "sample": f"{n} of {wl.batch} decode rows (full 32768-key "
+                                         f"indexer, top-k, fp64 attention per row), {dt:.1f} s"}
+    del step, wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def prefill_stage_split(dsa, wl, stream, sm_count):
+    """One pass over the same row chunks dsa_forward runs (its own chunk plan), through the stage
+    calls with CUDA events around each launch: the dense attention of the first topk rows of
+    every sequence, then per chunk the indexer (counting the first digit), the top-k (from the
+    counts) and the sparse MLA forward.  Returns the summed ms per stage."""
+    pb = dsa.problem_of(wl)
+    d = wl.dims
+    K = d["topk"]
+    dev = wl.kv.device
+    plan, off = [], 0
+    for b, L in enumerate(wl.seqlens):
+        rows = dsa.dsa_forward_chunk_rows_for(pb, b, sm_count)
+        plan.append((off, L, rows))
+        off += L
+    ld_max = max((L + 3) // 4 * 4 * rows for _, L, rows in plan if L > K)
+    rows_max = max(rows for _, L, rows in plan)
+    slab = torch.empty(ld_max, dtype=torch.float32, device=dev)
+    hist = torch.zeros(rows_max, dsa.TOPK_HIST_BINS, dtype=torch.int32, device=dev)
+    idx = torch.empty(rows_max, K, dtype=torch.int32, device=dev)
+    out = torch.empty(wl.total_rows, d["h"], d["d_v"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wl.total_rows, d["h"], dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    marks = []   # (stage, start event, end event)
+
+    def timed(stage, fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dsa.check(fn(), stage)
+        b.record(stream)
+        marks.append((stage, a, b))
+
+    for c0, L, rows in plan:
+        nd = min(L, K)
+        timed("sparse_mla_dense", lambda: dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, None, c0, nd,
+                                                                 out, lse, None, 0, status,
+                                                                 stream))
+        ld = (L + 3) // 4 * 4
+        for r0 in range(nd, L, rows):
+            rb, n = c0 + r0, min(rows, L - r0)
+            timed("indexer", lambda: dsa.dsa_indexer_scores(pb, wl.q_idx, wl.q_scale, wl.w,
+                                                            wl.k_idx, wl.k_scale, rb, n, slab,
+                                                            ld, status, stream, hist=hist))
+            timed("topk", lambda: dsa.dsa_topk(pb, slab, ld, rb, n, idx, status, stream,
+                                               hist=hist))
+            timed("sparse_mla", lambda: dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, idx, rb, n, out,
+                                                               lse, None, 0, status, stream))
+    torch.cuda.synchronize()
+    st, _ = dsa.dsa_read_device_status(status, stream)
+    dsa.check(st, "staged prefill status")
+    split = {}
+    for stage, a, b in marks:
+        split[stage] = split.get(stage, 0.0) + a.elapsed_time(b)
+    return split, len(marks)
+
+
+def run_prefill_sharded(args, dsa, dev, stream, peaks, rank, world, cfg):
+    """N > 1: one prefill problem split over the ranks (strong scaling).  Each rank holds its
+    range of query rows and the key-side rows of that range; a step is the all-gather of the
+    key-side rows (NCCL) and dsa_forward_rows on the rank's rows.  Time: max over ranks."""
+    from dsa_workloads import make_config, CONFIGS
+    from sparse_attention_long_04_b200 import shard
+    wl = make_config(cfg, device=dev, seed=rank_seed(cfg, 0))      # the same problem everywhere
+    pb = dsa.problem_of(wl)
+    ranges = shard.split_rows(wl.seqlens, wl.dims, world)
+    rb, n = ranges[rank]
+    sl = slice(rb, rb + n)
+    local_keys = (wl.k_idx[sl].clone(), wl.k_scale[sl].clone(), wl.kv[sl].clone())
+    part = shard.ShardForward(dsa, pb, rb, n, wl.q_idx[sl], wl.q_scale[sl], wl.w[sl], wl.q[sl])
+    del wl
+    torch.cuda.empty_cache()
+
+    def step():
+        with torch.cuda.stream(stream):
+            keys = shard.gather_keys(*local_keys, ranges)
+        dsa.check(part(*keys, stream=stream), "sharded prefill")
+        return keys
+
+    steps = max(1, min(args.steps, args.prefill_steps))
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    torch.cuda.synchronize()
+    torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    torch.distributed.barrier()
+    ms_step = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    st, _ = dsa.dsa_read_device_status(part.status, stream)
+    dsa.check(st, "sharded prefill status")
+    seqlens = make_config_seqlens(cfg)
+    T = sum(seqlens)
+    from dsa_workloads import FULL
+    f8, f16 = prefill_flops(seqlens, FULL)
+    p8 = 2.0 * peaks["bf16_sustained"]
+    ideal_ms = (f8 / (p8 * 1e12) + f16 / (peaks["bf16_sustained"] * 1e12)) * 1e3 / world
+    res = {"workload": CONFIGS[cfg]["name"], "value": round(T / (ms_step / 1e3), 1),
+           "unit": "tokens/s", "ms_per_step": round(ms_step, 3), "steps": steps,
+           "scaling": "strong", "ranges": ranges,
+           "roofline": {"bound": "tensor", "frac": round(ideal_ms / ms_step, 4),
+                        "ideal_ms_per_gpu": round(ideal_ms, 3)},
+           "note": "one problem split over the ranks by query rows; each step all-gathers the "
+                   "key-side rows (NCCL) and runs dsa_forward_rows on the rank's rows"}
+    del part, local_keys
+    torch.cuda.empty_cache()
+    return res
+
+
+def make_config_seqlens(cfg):
+    from dsa_workloads import CONFIGS
+    return list(CONFIGS[cfg]["seqlens"])
+
+
+def run_prefill(args, dsa, dev, stream, peaks, rank, world, cfg):
+    if world > 1:
+        return run_prefill_sharded(args, dsa, dev, stream, peaks, rank, world, cfg)
+    from dsa_workloads import make_config, CONFIGS, sample_rows
+    wl = make_config(cfg, device=dev, seed=rank_seed(cfg, rank))
     fwd = dsa.Forward(wl, keep_idx=False)
     steps = max(1, min(args.steps, args.prefill_steps))
     for _ in range(max(1, min(args.warmup, 3))):
@@ -396,18 +592,38 @@ def run_prefill(args, dsa, dev, stream, peaks, rank, world):
     ms_step = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
     st, raw = dsa.dsa_read_device_status(fwd.status, stream)
     dsa.check(st, "prefill device status")
+    del fwd
+    sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    split, n_launch = prefill_stage_split(dsa, wl, stream, sm)
     f8, f16 = prefill_flops(wl.seqlens, wl.dims)
     p8 = 2.0 * peaks["bf16_sustained"]
     ideal_ms = (f8 / (p8 * 1e12) + f16 / (peaks["bf16_sustained"] * 1e12)) * 1e3
     T = wl.total_rows
-    res = {"workload": CONFIGS[PREFILL_CFG]["name"], "value": round(weak_value(world, T, ms_step), 1),
+    stage_sum = sum(split.values())
+    res = {"workload": CONFIGS[cfg]["name"], "value": round(weak_value(world, T, ms_step), 1),
            "unit": "tokens/s", "ms_per_step": round(ms_step, 3), "steps": steps,
            "roofline": {"bound": "tensor", "frac": round(ideal_ms / ms_step, 4),
                         "ideal_ms": round(ideal_ms, 3), "flops_fp8": f8, "flops_bf16": f16,
                         "peak_bf16_tflops": peaks["bf16_sustained"],
                         "peak_fp8_tflops": p8,
-                        "peak_note": "bf16 sustained measured; fp8 = 2x bf16 (nominal ratio)"}}
-    del fwd, wl
+                        "peak_note": "bf16 sustained measured; fp8 = 2x bf16 (nominal ratio)"},
+           "kernel_ms": {k: round(v, 3) for k, v in sorted(split.items())},
+           "kernel_share": {k: round(v / stage_sum, 4) for k, v in sorted(split.items())},
+           "kernel_ms_note": "one pass of the same chunks through the stage calls, CUDA events "
+                             "around every launch; summed per stage (the forward runs them "
+                             "back to back, so the sum is a little above ms_per_step)",
+           "gpu_launches_per_step": n_launch}
+    if rank == 0 and not args.no_cpu:
+        import oracle
+        rows = sample_rows(wl, 2)
+        t0 = time.perf_counter()
+        oracle.forward_rows(wl, rows)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": round(len(rows) / dt, 3), "unit": "tokens/s",
+                               "cores": oracle.num_threads(), "kind": "oracle",
+                               "sample": f"{len(rows)} sampled rows (2 per sequence; indexer over "
+                                         f"every prior key, top-k, fp64 attention), {dt:.1f} s"}
+    del wl
     torch.cuda.empty_cache()
     return res
 
@@ -646,6 +862,23 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(n: int) -> int:
+    """`--gpus N` without a launcher: start N ranks of this script on this node (one per GPU)
+    through torch.distributed.run, with the same arguments; rank 0 prints the line.  Never
+    reports a one-GPU number for N > 1."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -654,6 +887,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the secondary full-shape workloads (decode_B32_N32k, prefill_L16k)")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the indexer training step (prefill_L16k)")
     ap.add_argument("--train-only", action="store_true",
@@ -669,9 +904,13 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: one rank per GPU")
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
@@ -689,7 +928,7 @@ def main():
             dev = torch.device("cuda", local_rank)
             torch.cuda.set_device(dev)
             line = run_prefill(args, dsa, dev, torch.cuda.current_stream(), read_peaks(), rank,
-                               world)
+                               world, PREFILL_CFG)
             if rank == 0:
                 print(json.dumps(line), flush=True)
             return

@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 1
+#define DSA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define DSA_API __attribute__((visibility("default")))
@@ -128,25 +128,68 @@ typedef struct {
  *   k_idx   e4m3 [num_kv_rows, d_idx]            k_scale     fp32 [num_kv_rows]
  *   scores  fp32 [row_count, ld_scores]: scores[(t - row_begin) * ld + s] for s <= pos(t);
  *           entries past pos(t) are left untouched.  ld_scores >= max pos(t) + 1 over
- *           the rows and a multiple of 4. */
+ *           the rows and a multiple of 4.
+ *   hist    optional uint32 [row_count, DSA_TOPK_HIST_BINS], zero on entry: the indexer ADDS
+ *           to row t - row_begin the count of each written score in the bin of its first
+ *           radix digit (the top 11 bits of the order-preserving key the selection sorts on),
+ *           so that dsa_topk can start from exact per-row counts (the fused indexer + top-k).
+ *           (64, 128) indexer only: with (4, 32) a non-NULL hist is DSA_ERR_UNSUPPORTED_SHAPE.
+ *           NULL: no counting. */
+#define DSA_TOPK_HIST_BINS 2048
 DSA_API dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                 const uint8_t* q_idx, const float* q_scale, const float* w,
                                 const uint8_t* k_idx, const float* k_scale, int32_t row_begin,
                                 int32_t row_count, float* scores, int64_t ld_scores,
-                                int32_t* dev_status, dsa_stream_t stream);
+                                uint32_t* hist, int32_t* dev_status, dsa_stream_t stream);
 
 /* Stage 2.  Exact top-k of each row of `scores` (layout as written by dsa_indexer_scores)
  * over keys 0..pos(t).  idx int32 [row_count, topk]: the selected LOGICAL key indices in
  * increasing order, then -1 padding when pos(t) + 1 < topk.  The set is unique: larger
- * score first, equal scores broken by the smaller index (-0 and +0 compare equal). */
+ * score first, equal scores broken by the smaller index (-0 and +0 compare equal).
+ *   hist  optional: the histograms dsa_indexer_scores counted while writing these same rows
+ *         of `scores` (exact counts of each row's keys 0..pos(t); anything else gives a wrong
+ *         selection).  The selection then starts from them and reads each score once; on
+ *         return they are zero again, ready for the next dsa_indexer_scores.  NULL: the
+ *         selection counts the first digit itself (one more read of the scores). */
 DSA_API dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
-                      int64_t ld_scores, int32_t row_begin, int32_t row_count, int32_t* idx,
-                      int32_t* dev_status, dsa_stream_t stream);
+                      int64_t ld_scores, uint32_t* hist, int32_t row_begin, int32_t row_count,
+                      int32_t* idx, int32_t* dev_status, dsa_stream_t stream);
+
+/* Stages 1 and 2 fused: the indexer scores of rows [row_begin, row_begin + row_count) and their
+ * top-k, without the scores leaving the call.  The pages' selector keeps k tokens per query
+ * straight from the indexer's scores ("FP8 index -> top-k selection -> sparse core attention",
+ * "DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek Sparse Attention (DSA)", pipeline
+ * summary; "the Top-k selector keeps only k key-value pairs per query", maplevalley page,
+ * section 1).  As it writes each score into a slab in `workspace`, the indexer counts it in
+ * its row's histogram of the first radix digit (the top 11 bits of the order-preserving key);
+ * the selection then starts from those counts and reads the slab once.  Inputs as for
+ * dsa_indexer_scores; idx as written by dsa_topk (the same set, increasing order, -1 padding).
+ * workspace: at least dsa_indexer_topk_workspace_size(dims, seqs, row_count) bytes, 16-byte
+ * aligned, caller-owned, contents on entry irrelevant (too small: DSA_ERR_WORKSPACE_TOO_SMALL).
+ * With the (4, 32) indexer shape the selection builds its histograms itself. */
+DSA_API size_t dsa_indexer_topk_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                               int32_t row_count);
+DSA_API dsa_status_t dsa_indexer_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                      const uint8_t* q_idx, const float* q_scale, const float* w,
+                                      const uint8_t* k_idx, const float* k_scale,
+                                      int32_t row_begin, int32_t row_count, int32_t* idx,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, dsa_stream_t stream);
 
 /* Bytes of workspace dsa_sparse_mla_fwd needs for `row_count` rows (split-KV partials when
  * few rows leave SMs idle).  0 is a valid answer. */
 DSA_API size_t dsa_sparse_mla_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                      int32_t row_count);
+
+/* The same size for a device with `sm_count` SMs, without touching any device (host-only), when
+ * the partials may take at most `max_bytes` (SIZE_MAX: no limit, the answer
+ * dsa_sparse_mla_workspace_size gives on such a device).  The split count only changes speed:
+ * under a cap the fastest split count that fits is chosen, and one split needs no partials, so
+ * the answer never exceeds max_bytes.  dsa_sparse_mla_fwd_noalloc sizes its partials this way
+ * with max_bytes = DSA_NOALLOC_SCRATCH_BYTES.  0 on invalid arguments or sm_count <= 0. */
+DSA_API size_t dsa_sparse_mla_workspace_size_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                                 int32_t row_count, int32_t sm_count,
+                                                 size_t max_bytes);
 
 /* Stage 3.  Sparse MLA-MQA forward for rows [row_begin, row_begin + row_count).
  *   q    bf16 [total_rows, h, d_qk]   (indexed by absolute row)
@@ -177,8 +220,11 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t
  *   - The first call on a device looks up that device's copy of the array
  *     (cudaGetSymbolAddress, with that device current).  Make that first call before any stream
  *     capture.
- *   - A call whose split-KV partials would not fit the array returns
- *     DSA_ERR_WORKSPACE_TOO_SMALL before launching (on a 148-SM B200 every row count fits).
+ *   - The split-KV slicing is chosen so that the partials fit the array: the fastest split
+ *     count with splits * row_count * h * (d_v + 1) * 4 bytes (+256) within
+ *     DSA_NOALLOC_SCRATCH_BYTES (at full shapes, splits * row_count <= 79), else one split,
+ *     which needs no scratch at all.  Every row count therefore runs; large batches run
+ *     unsplit, exactly as dsa_sparse_mla_fwd runs them.
  *   - Every call shares the one array and each call overwrites the parts it uses, so nothing has
  *     to start at zero; two calls that overlap on the GPU (different streams, no ordering) race
  *     on it and give undefined results.  Calls on one stream are safe. */
@@ -198,6 +244,14 @@ DSA_API size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs
 DSA_API size_t dsa_forward_workspace_size_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                               int32_t sm_count);
 
+/* How dsa_forward cuts a prefill into row chunks, for a device with `sm_count` SMs (host-only):
+ * the rows per chunk of sequence `seq` (the last chunk of a sequence may be shorter; with
+ * idx_out NULL the first min(L, topk) rows run dense attention before the chunks start).  Each
+ * chunk is one indexer, one top-k and one attention launch over its rows.  DECODE: the batch
+ * (one chunk).  0 on invalid arguments. */
+DSA_API int32_t dsa_forward_chunk_rows_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                           int32_t seq, int32_t sm_count);
+
 /* The whole path for all seqs->total_rows query rows.  Inputs as for the three stages.
  *   idx_out  optional int32 [total_rows, topk]: the selected indices (NULL = not kept).
  *            When NULL, rows with at most topk prior keys (the first topk rows of each prefill
@@ -209,6 +263,26 @@ DSA_API dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                          const float* k_scale, const uint16_t* q, const uint16_t* kv,
                          int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
                          size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream);
+
+/* dsa_forward for query rows [row_begin, row_begin + row_count) only, with the query-side
+ * arrays holding just those rows: the building block of a prefill split across GPUs (each GPU
+ * takes a range of query rows; the keys are gathered first, since every row attends to the
+ * prior keys of its whole sequence).  The rows, chunks, selection and results are exactly those
+ * dsa_forward computes for the same rows.
+ *   q_idx [row_count, h_idx, d_idx], q_scale / w [row_count, h_idx], q [row_count, h, d_qk],
+ *   out [row_count, h, d_v], lse [row_count, h], idx_out (optional) [row_count, topk]: row i of
+ *   these is query row row_begin + i.
+ *   k_idx, k_scale, kv: the full key-side arrays (num_kv_rows physical rows), as for dsa_forward.
+ *   workspace: dsa_forward_workspace_size(dims, seqs) bytes suffice for every row range.
+ * DECODE: rows are sequences (a range of the batch). */
+DSA_API dsa_status_t dsa_forward_rows(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                      int32_t row_begin, int32_t row_count,
+                                      const uint8_t* q_idx, const float* q_scale, const float* w,
+                                      const uint8_t* k_idx, const float* k_scale,
+                                      const uint16_t* q, const uint16_t* kv, int32_t* idx_out,
+                                      uint16_t* out, float* lse, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status,
+                                      dsa_stream_t stream);
 
 /* Decode cache append, the step that fills the caches the path reads ("FP8 index -> top-k
  * selection -> sparse core attention", "DeepSeek V3.2-Exp Cuts Long-Context Costs with DeepSeek

@@ -33,6 +33,7 @@ DSA_ERR_TIMEOUT = 6
 DSA_ERR_CUDA = 7
 DSA_DEVICE_TIMEOUT = 1
 DSA_DEVICE_BAD_INDEX = 2
+TOPK_HIST_BINS = 2048
 DSA_PREFILL = 0
 DSA_DECODE = 1
 
@@ -40,7 +41,10 @@ EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_fwd", "dsa_forward_workspace_size", "dsa_forward",
             "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
             "dsa_sparse_mla_fwd_noalloc", "dsa_cache_append", "dsa_selftest_wait_timeout",
-            "dsa_indexer_kl_target", "dsa_indexer_kl_backward", "dsa_forward_workspace_size_for")
+            "dsa_indexer_kl_target", "dsa_indexer_kl_backward", "dsa_forward_workspace_size_for",
+            "dsa_sparse_mla_workspace_size_for", "dsa_indexer_topk",
+            "dsa_indexer_topk_workspace_size", "dsa_forward_chunk_rows_for",
+            "dsa_forward_rows")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -74,13 +78,18 @@ def _load():
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     DP, SP = ctypes.POINTER(dsa_dims_t), ctypes.POINTER(dsa_seqs_t)
     sig = {
-        "dsa_indexer_scores": (I32, [DP, SP, P, P, P, P, P, I32, I32, P, I64, P, P]),
-        "dsa_topk": (I32, [DP, SP, P, I64, I32, I32, P, P, P]),
+        "dsa_indexer_scores": (I32, [DP, SP, P, P, P, P, P, I32, I32, P, I64, P, P, P]),
+        "dsa_topk": (I32, [DP, SP, P, I64, P, I32, I32, P, P, P]),
+        "dsa_indexer_topk_workspace_size": (SZ, [DP, SP, I32]),
+        "dsa_indexer_topk": (I32, [DP, SP, P, P, P, P, P, I32, I32, P, P, SZ, P, P]),
         "dsa_sparse_mla_workspace_size": (SZ, [DP, SP, I32]),
         "dsa_sparse_mla_fwd": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, SZ, P, P]),
         "dsa_forward_workspace_size": (SZ, [DP, SP]),
         "dsa_forward_workspace_size_for": (SZ, [DP, SP, I32]),
+        "dsa_forward_chunk_rows_for": (I32, [DP, SP, I32, I32]),
+        "dsa_sparse_mla_workspace_size_for": (SZ, [DP, SP, I32, I32, SZ]),
         "dsa_forward": (I32, [DP, SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+        "dsa_forward_rows": (I32, [DP, SP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_selftest_wait_timeout": (I32, [P, P]),
         "dsa_indexer_kl_target": (I32, [DP, SP, P, P, P, P, I32, I32, P, P, P]),
@@ -187,23 +196,46 @@ def problem_of(wl) -> Problem:
 
 def dsa_indexer_scores(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, row_begin: int,
                        row_count: int, scores, ld_scores: int, dev_status=None,
-                       stream=None) -> int:
+                       stream=None, hist=None) -> int:
     return int(lib.dsa_indexer_scores(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
-        _ptr(k_idx), _ptr(k_scale), row_begin, row_count, _ptr(scores), ld_scores,
+        _ptr(k_idx), _ptr(k_scale), row_begin, row_count, _ptr(scores), ld_scores, _ptr(hist),
         _ptr(dev_status), _stream(stream)))
 
 
 def dsa_topk(pb: Problem, scores, ld_scores: int, row_begin: int, row_count: int, idx,
-             dev_status=None, stream=None) -> int:
+             dev_status=None, stream=None, hist=None) -> int:
     return int(lib.dsa_topk(ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(scores),
-                            ld_scores, row_begin, row_count, _ptr(idx), _ptr(dev_status),
-                            _stream(stream)))
+                            ld_scores, _ptr(hist), row_begin, row_count, _ptr(idx),
+                            _ptr(dev_status), _stream(stream)))
+
+
+def dsa_indexer_topk_workspace_size(pb: Problem, row_count: int) -> int:
+    return int(lib.dsa_indexer_topk_workspace_size(ctypes.byref(pb.dims), ctypes.byref(pb.seqs),
+                                                   row_count))
+
+
+def dsa_indexer_topk(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, row_begin: int,
+                     row_count: int, idx, workspace, workspace_bytes: int, dev_status=None,
+                     stream=None) -> int:
+    return int(lib.dsa_indexer_topk(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
+        _ptr(k_idx), _ptr(k_scale), row_begin, row_count, _ptr(idx), _ptr(workspace),
+        workspace_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def dsa_sparse_mla_workspace_size(pb: Problem, row_count: int) -> int:
     return int(lib.dsa_sparse_mla_workspace_size(ctypes.byref(pb.dims), ctypes.byref(pb.seqs),
                                                  row_count))
+
+
+def dsa_sparse_mla_workspace_size_for(pb: Problem, row_count: int, sm_count: int,
+                                      max_bytes: Optional[int] = None) -> int:
+    """Host-only sizing (no device needed); max_bytes None = no cap."""
+    cap = ctypes.c_size_t(-1).value if max_bytes is None else int(max_bytes)
+    return int(lib.dsa_sparse_mla_workspace_size_for(ctypes.byref(pb.dims),
+                                                     ctypes.byref(pb.seqs), row_count,
+                                                     sm_count, cap))
 
 
 def dsa_sparse_mla_fwd(pb: Problem, q, kv, idx, row_begin: int, row_count: int, out, lse,
@@ -233,12 +265,27 @@ def dsa_forward_workspace_size_for(pb: Problem, sm_count: int) -> int:
                                                   sm_count))
 
 
+def dsa_forward_chunk_rows_for(pb: Problem, seq: int, sm_count: int) -> int:
+    return int(lib.dsa_forward_chunk_rows_for(ctypes.byref(pb.dims), ctypes.byref(pb.seqs), seq,
+                                              sm_count))
+
+
 def dsa_forward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, q, kv, idx_out, out, lse,
                 workspace, workspace_bytes: int, dev_status=None, stream=None) -> int:
     return int(lib.dsa_forward(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
         _ptr(k_idx), _ptr(k_scale), _ptr(q), _ptr(kv), _ptr(idx_out), _ptr(out), _ptr(lse),
         _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def dsa_forward_rows(pb: Problem, row_begin: int, row_count: int, q_idx, q_scale, w, k_idx,
+                     k_scale, q, kv, idx_out, out, lse, workspace, workspace_bytes: int,
+                     dev_status=None, stream=None) -> int:
+    return int(lib.dsa_forward_rows(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), row_begin, row_count, _ptr(q_idx),
+        _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q), _ptr(kv), _ptr(idx_out),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes, _ptr(dev_status),
+        _stream(stream)))
 
 
 def dsa_cache_append(pb: Problem, k_new, kv_new, k_cache, k_scale_cache, kv_cache,

@@ -6,6 +6,8 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstdint>
+#include <climits>
 #include <cstring>
 #include <mutex>
 
@@ -66,34 +68,35 @@ dsa_status_t encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
   return DSA_OK;
 }
 
-// Per (kernel, device): the kernel's dynamic shared-memory limit has been raised.
+// Per (kernel, device): the dynamic shared-memory limit the kernel has been raised to.
 struct SmemRaised {
   const void* fn;
-  uint64_t devices;
+  int bytes[kMaxDevices];
 };
 SmemRaised g_raised[32];
 int g_n_raised = 0;
 
+// Raises the kernel's dynamic shared-memory limit to at least smem_bytes on the current device
+// (once per size increase).
 template <typename Kernel>
 dsa_status_t prepare_kernel(Kernel k, int smem_bytes) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
-  const uint64_t bit = uint64_t(1) << dev;
   const void* fn = reinterpret_cast<const void*>(k);
   std::lock_guard<std::mutex> lk(g_mu);
   int slot = -1;
   for (int i = 0; i < g_n_raised; ++i)
     if (g_raised[i].fn == fn) slot = i;
-  if (slot >= 0 && (g_raised[slot].devices & bit)) return DSA_OK;
+  if (slot >= 0 && g_raised[slot].bytes[dev] >= smem_bytes) return DSA_OK;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (slot < 0) {
     if (g_n_raised == 32) return DSA_OK;   // not cached: raised again next time
     slot = g_n_raised++;
-    g_raised[slot] = SmemRaised{fn, 0};
+    g_raised[slot] = SmemRaised{fn, {}};
   }
-  g_raised[slot].devices |= bit;
+  g_raised[slot].bytes[dev] = smem_bytes;
   return DSA_OK;
 }
 
@@ -253,11 +256,33 @@ dsa_status_t run_indexer_kernel(const CUtensorMap& kmap, const CUtensorMap& qmap
   return launch_status();
 }
 
+// Key tiles per CTA of the decode indexer.  The launch is HBM-bound and every CTA streams
+// tps tiles, so its time is about waves x (tps + c0): waves = ceil(rows x splits / slots) for
+// `slots` resident CTAs, c0 ~ 2 tiles of per-CTA set-up (barriers, TMEM, the query group).
+// Pick the split count with the smallest such makespan, so that the last wave is not a thin
+// tail of a few CTAs.
+int64_t decode_tiles_per_split(int64_t rows, int64_t tiles, int64_t slots) {
+  int64_t best_tps = tiles;
+  double best = 1e300;
+  for (int64_t sp = 1; sp <= tiles; ++sp) {
+    const int64_t tps = ceil_div(tiles, sp);
+    if (sp > 1 && tps == ceil_div(tiles, sp - 1)) continue;   // same split as sp - 1
+    const double waves = double(ceil_div(rows * ceil_div(tiles, tps), std::max<int64_t>(1, slots)));
+    const double t = waves * (double(tps) + 2.0);
+    if (t < best - 1e-9) {
+      best = t;
+      best_tps = tps;
+    }
+  }
+  return best_tps;
+}
+
 template <int H_I, int D_I, int QPG>
 dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
                           const float* q_scale, const float* w, const uint8_t* k_idx,
                           const float* k_scale, int32_t row_begin, int32_t row_count,
-                          float* scores, int64_t ld, int32_t* status, cudaStream_t st) {
+                          float* scores, int64_t ld, int32_t* status, cudaStream_t st,
+                          uint32_t* hist) {
   using C = IndexerCfg<H_I, D_I, QPG>;
   DeviceInfo info;
   if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
@@ -287,13 +312,13 @@ dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_
   prm.kv_stride = s.max_seqlen;
   prm.max_seqlen = s.max_seqlen;
   prm.num_kv_rows = s.num_kv_rows;
+  prm.hist = C::HIST ? hist : nullptr;
   const int ctas_per_sm = C::TMEM_COLS == 512 ? 1 : 2;
   const int64_t target = int64_t(info.sm_count) * ctas_per_sm * 4;
   if (s.mode == DSA_DECODE) {
     const int64_t tiles = ceil_div(s.max_seqlen, 128);
-    int64_t splits = std::min<int64_t>(tiles, std::max<int64_t>(1, ceil_div(target, row_count)));
-    const int64_t tps = ceil_div(tiles, splits);
-    splits = ceil_div(tiles, tps);
+    const int64_t tps = decode_tiles_per_split(row_count, tiles, int64_t(info.sm_count) * ctas_per_sm);
+    const int64_t splits = ceil_div(tiles, tps);
     prm.decode = 1;
     prm.row0 = row_begin;
     prm.nrows = row_count;
@@ -326,28 +351,72 @@ dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_
   return DSA_OK;
 }
 
+dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* scores, int64_t ld,
+                         int32_t row_begin, int32_t row_count, int32_t* idx, int32_t* status,
+                         cudaStream_t st, uint32_t* hist = nullptr);
+
+// Whether the indexer of these dims counts the first-digit histograms (the full 64 x 128 shape;
+// the 4 x 32 shape's 64-row query groups have no room for them).
+bool indexer_counts_hist(const dsa_dims_t& d) { return d.h_idx == 64 && d.d_idx == 128; }
+
 dsa_status_t indexer_dispatch(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
                               const float* q_scale, const float* w, const uint8_t* k_idx,
                               const float* k_scale, int32_t row_begin, int32_t row_count,
-                              float* scores, int64_t ld, int32_t* status, cudaStream_t st) {
+                              float* scores, int64_t ld, int32_t* status, cudaStream_t st,
+                              uint32_t* hist = nullptr) {
   if (row_count == 0) return DSA_OK;
   if (d.h_idx == 64 && d.d_idx == 128) {
     if (s.mode == DSA_DECODE)
       return indexer_impl<64, 128, 1>(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin,
-                                      row_count, scores, ld, status, st);
+                                      row_count, scores, ld, status, st, hist);
     return indexer_impl<64, 128, 4>(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin,
-                                    row_count, scores, ld, status, st);
+                                    row_count, scores, ld, status, st, hist);
   }
   return indexer_impl<4, 32, 64>(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
-                                 scores, ld, status, st);
+                                 scores, ld, status, st, nullptr);
+}
+
+// Indexer and top-k of rows [row_begin, row_begin + row_count) through a score slab, the
+// indexer counting each row's first digit as it writes the scores (`hist`: row_count rows of
+// kTopkBins words, zero on entry and zero again on return) when its shape allows.
+dsa_status_t indexer_topk(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
+                          const float* q_scale, const float* w, const uint8_t* k_idx,
+                          const float* k_scale, int32_t row_begin, int32_t row_count,
+                          float* slab, int64_t ld, uint32_t* hist, int32_t* idx,
+                          int32_t* status, cudaStream_t st) {
+  uint32_t* h = indexer_counts_hist(d) ? hist : nullptr;
+  dsa_status_t e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin,
+                                    row_count, slab, ld, status, st, h);
+  if (e != DSA_OK) return e;
+  return topk_launch(d, s, slab, ld, row_begin, row_count, idx, status, st, h);
 }
 
 // ------------------------------------------------------------------------ stage 2
 
+// Cluster size and slice of the top-k launch for rows of up to `longest` keys: slices of at
+// most 32768 keys (8 KB of bitmaps), then more CTAs per row while the rows alone leave SMs idle
+// and slices stay at least 4096 keys long.  Longer rows than 8 slices of 32768 take longer
+// slices (larger bitmaps), as far as shared memory allows.
+struct TopkShape {
+  int csize;
+  int slice;
+};
+TopkShape topk_shape(int64_t longest, int32_t row_count, int sm_count) {
+  int c = 1;
+  while (c < 8 && int64_t(c) * 32768 < longest) c *= 2;
+  while (c < 8 && int64_t(row_count) * c < sm_count && int64_t(c) * 4096 < longest) c *= 2;
+  const int64_t per = (ceil_div(std::max<int64_t>(1, longest), c) + 127) / 128 * 128;
+  return TopkShape{c, static_cast<int>(std::min<int64_t>(per, INT32_MAX / 2))};
+}
+
+// `hist`: per-row first-digit histograms written with the scores (the fused indexer), or null
+// (the top-k builds them itself).
 dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* scores, int64_t ld,
                          int32_t row_begin, int32_t row_count, int32_t* idx, int32_t* status,
-                         cudaStream_t st) {
+                         cudaStream_t st, uint32_t* hist) {
   if (row_count == 0) return DSA_OK;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
   TopkParams prm{};
   prm.scores = scores;
   prm.ld = ld;
@@ -360,20 +429,22 @@ dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* 
   prm.seq_lens = s.seq_lens;
   prm.max_seqlen = s.max_seqlen;
   prm.status = status;
-  // CTAs per row: enough that a row's slices fit shared memory (up to 8, the portable limit)
+  prm.hist = hist;
   const int64_t longest = std::min<int64_t>(max_keys(&s, row_begin, row_count), ld);
-  int csize = 1;
-  while (csize < 8 && int64_t(csize) * kTopkSlice < longest) csize *= 2;
-  prm.csize = csize;
-  if (prepare_kernel(dsa_topk_kernel, kTopkSmem) != DSA_OK) return DSA_ERR_CUDA;
+  const TopkShape shape = topk_shape(longest, row_count, info.sm_count);
+  prm.csize = shape.csize;
+  prm.slice = shape.slice;
+  const int64_t smem = topk_smem_bytes(shape.slice);
+  if (smem + 1024 > info.max_smem) return DSA_ERR_UNSUPPORTED_SHAPE;   // (+ static shared)
+  if (prepare_kernel(dsa_topk_kernel, static_cast<int>(smem)) != DSA_OK) return DSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(int64_t(row_count) * csize));
+  cfg.gridDim = dim3(static_cast<unsigned>(int64_t(row_count) * shape.csize));
   cfg.blockDim = dim3(kTopkThreads);
-  cfg.dynamicSmemBytes = kTopkSmem;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.x = shape.csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -384,7 +455,15 @@ dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* 
 
 // ------------------------------------------------------------------------ stage 3
 
-int mla_splits(const dsa_dims_t& d, const dsa_seqs_t& s, int32_t row_count, int sm_count) {
+size_t mla_ws_bytes(const dsa_dims_t& d, int splits, int32_t row_count) {
+  if (splits <= 1) return 0;
+  return size_t(splits) * row_count * d.h * (d.d_v + 1) * sizeof(float) + 256;
+}
+
+// Split-KV slices per decode row.  Only speed depends on the choice: one split needs no
+// partials, so a cap on the partials' bytes (max_ws) always leaves a valid answer.
+int mla_splits(const dsa_dims_t& d, const dsa_seqs_t& s, int32_t row_count, int sm_count,
+               size_t max_ws = SIZE_MAX) {
   if (s.mode != DSA_DECODE || row_count <= 0) return 1;
   // Two CTAs (one per value half) per row and split; one CTA per SM.  Pick the split count
   // with the smallest estimated makespan: waves x (prologue + tiles per split), in tile units
@@ -394,6 +473,7 @@ int mla_splits(const dsa_dims_t& d, const dsa_seqs_t& s, int32_t row_count, int 
   int best = 1;
   double best_t = 1e30;
   for (int sp = 1; sp <= std::min(16, std::max(1, tiles / 4)); ++sp) {
+    if (mla_ws_bytes(d, sp, row_count) > max_ws) continue;
     const double waves = std::ceil(2.0 * row_count * sp / sms);
     const double t = waves * (3.0 + std::ceil(double(tiles) / sp)) + (sp > 1 ? 2.0 : 0.0);
     if (t < best_t - 1e-9) {
@@ -402,11 +482,6 @@ int mla_splits(const dsa_dims_t& d, const dsa_seqs_t& s, int32_t row_count, int 
     }
   }
   return best;
-}
-
-size_t mla_ws_bytes(const dsa_dims_t& d, int splits, int32_t row_count) {
-  if (splits <= 1) return 0;
-  return size_t(splits) * row_count * d.h * (d.d_v + 1) * sizeof(float) + 256;
 }
 
 // The inputs and row geometry shared by the attention forward and the target pass.
@@ -486,6 +561,7 @@ struct ForwardPlan {
   int64_t idx_ints = 0;      // chunk indices when idx_out is null
   int mla_splits = 1;
   size_t mla_bytes = 0;
+  int64_t hist_rows = 0;     // first-digit histograms of one chunk's rows (fused indexer)
   size_t total = 0;
 };
 
@@ -509,6 +585,7 @@ ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count)
     p.idx_ints = int64_t(s.batch) * d.topk;
     p.mla_splits = mla_splits(d, s, s.batch, sm_count);
     p.mla_bytes = mla_ws_bytes(d, p.mla_splits, s.batch);
+    p.hist_rows = s.batch;
   } else {
     const int32_t* cu = s.cu_seqlens_host;
     int64_t max_rows = 0;
@@ -520,9 +597,12 @@ ForwardPlan plan_forward(const dsa_dims_t& d, const dsa_seqs_t& s, int sm_count)
       max_rows = std::max(max_rows, rows);
     }
     p.idx_ints = max_rows * d.topk;
+    p.hist_rows = max_rows;
   }
+  if (!indexer_counts_hist(d)) p.hist_rows = 0;
   auto align = [](size_t x) { return (x + 255) / 256 * 256; };
-  p.total = align(p.slab_floats * 4) + align(p.idx_ints * 4) + align(p.mla_bytes);
+  p.total = align(p.slab_floats * 4) + align(p.idx_ints * 4) + align(p.mla_bytes) +
+            size_t(p.hist_rows) * kTopkBins * 4;
   return p;
 }
 
@@ -568,6 +648,97 @@ dsa_status_t kl_backward_launch(bool full, const IdxBwdParams& prm, cudaStream_t
     k<<<prm.row_count, C::THREADS, C::SMEM_BYTES, st>>>(prm);
   }
   return launch_status();
+}
+
+// ------------------------------------------------------------------------ dsa_forward body
+
+// The whole path for query rows [w0, w1): the query-side pointers (q_idx, q_scale, w, q, out,
+// lse, idx_out) are indexed by absolute row, the key-side ones (k_idx, k_scale, kv) by physical
+// row.  Prefill: per sequence, the window's rows with at most topk prior keys run dense attention
+// (when no indices are kept), the rest in chunks of indexer + top-k (fused first digit) +
+// sparse attention.  Decode: the window's sequences in one chunk.
+dsa_status_t forward_window(const dsa_dims_t& d, const dsa_seqs_t& s, int64_t w0, int64_t w1,
+                            const uint8_t* q_idx, const float* q_scale, const float* w,
+                            const uint8_t* k_idx, const float* k_scale, const uint16_t* q,
+                            const uint16_t* kv, int32_t* idx_out, uint16_t* out, float* lse,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            cudaStream_t st) {
+  dsa_status_t e;
+  if (!indexer_shape_ok(d, s.mode) || !mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!q_idx || !q_scale || !w || !k_idx || !q || !kv || !out || !lse)
+    return DSA_ERR_INVALID_ARG;
+  if (k_scale == nullptr && !interleaved_ok(s)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(q) ||
+      !aligned16(kv) || !aligned16(out) || !aligned16(lse) || !aligned16(idx_out) ||
+      !aligned16(workspace) || !aligned16(q_scale) || !aligned16(w))
+    return DSA_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  const ForwardPlan plan = plan_forward(d, s, info.sm_count);
+  if (workspace == nullptr || workspace_bytes < plan.total) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (w1 <= w0) return DSA_OK;
+  auto align = [](size_t x) { return (x + 255) / 256 * 256; };
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  float* slab = reinterpret_cast<float*>(wsb);
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(wsb + align(plan.slab_floats * 4));
+  void* mla_ws = wsb + align(plan.slab_floats * 4) + align(plan.idx_ints * 4);
+  uint32_t* hist = plan.hist_rows > 0
+                       ? reinterpret_cast<uint32_t*>(wsb + align(plan.slab_floats * 4) +
+                                                     align(plan.idx_ints * 4) +
+                                                     align(plan.mla_bytes))
+                       : nullptr;
+  // the histograms start at zero; each top-k launch leaves its rows zeroed for the next chunk
+  if (hist != nullptr &&
+      cudaMemsetAsync(hist, 0, size_t(plan.hist_rows) * kTopkBins * 4, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+
+  if (s.mode == DSA_DECODE) {
+    const int32_t rb = static_cast<int32_t>(w0), rc = static_cast<int32_t>(w1 - w0);
+    // a window of fewer sequences may split more: as far as the planned partials allow
+    const int splits = rc == s.batch ? plan.mla_splits
+                                     : mla_splits(d, s, rc, info.sm_count, plan.mla_bytes);
+    const size_t mla_bytes = mla_ws_bytes(d, splits, rc);
+    if (idx_out == nullptr && s.max_seqlen <= d.topk)   // every context key is kept: dense
+      return mla_dispatch(d, s, q, kv, nullptr, rb, rc, out, lse, mla_ws, mla_bytes, dev_status,
+                          st, splits);
+    const int64_t ld = round4(s.max_seqlen);
+    int32_t* idx = idx_out ? idx_out + int64_t(rb) * d.topk : idx_ws;
+    if ((e = indexer_topk(d, s, q_idx, q_scale, w, k_idx, k_scale, rb, rc, slab, ld, hist, idx,
+                          dev_status, st)) != DSA_OK)
+      return e;
+    return mla_dispatch(d, s, q, kv, idx, rb, rc, out, lse, mla_ws, mla_bytes, dev_status, st,
+                        splits);
+  }
+  const int32_t* cu = s.cu_seqlens_host;
+  for (int b = 0; b < s.batch; ++b) {
+    const int64_t L = cu[b + 1] - cu[b];
+    // the window's rows of this sequence, as positions [p0, p1)
+    const int64_t p0 = std::max<int64_t>(w0, cu[b]) - cu[b];
+    const int64_t p1 = std::min<int64_t>(w1, cu[b + 1]) - cu[b];
+    if (L <= 0 || p1 <= p0) continue;
+    const int64_t ld = round4(p1);
+    const int64_t rows = chunk_rows_for(L, info.sm_count);
+    // rows with at most topk prior keys keep all of them: dense attention, no indexer or top-k
+    // (unless the caller wants the indices)
+    const int64_t dense_end = idx_out == nullptr ? std::min<int64_t>(p1, d.topk) : p0;
+    if (dense_end > p0 &&
+        (e = mla_dispatch(d, s, q, kv, nullptr, static_cast<int32_t>(cu[b] + p0),
+                          static_cast<int32_t>(dense_end - p0), out, lse, nullptr, 0, dev_status,
+                          st, 1)) != DSA_OK)
+      return e;
+    for (int64_t r0 = std::max(p0, dense_end); r0 < p1; r0 += rows) {
+      const int32_t row_begin = static_cast<int32_t>(cu[b] + r0);
+      const int32_t row_count = static_cast<int32_t>(std::min(rows, p1 - r0));
+      int32_t* idx = idx_out ? idx_out + int64_t(row_begin) * d.topk : idx_ws;
+      if ((e = indexer_topk(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
+                            slab, ld, hist, idx, dev_status, st)) != DSA_OK)
+        return e;
+      if ((e = mla_dispatch(d, s, q, kv, idx, row_begin, row_count, out, lse, nullptr, 0,
+                            dev_status, st, 1)) != DSA_OK)
+        return e;
+    }
+  }
+  return DSA_OK;
 }
 
 // ---------------------------------------------------------------- bounded-wait self-test
@@ -617,34 +788,75 @@ dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                 const uint8_t* q_idx, const float* q_scale, const float* w,
                                 const uint8_t* k_idx, const float* k_scale, int32_t row_begin,
                                 int32_t row_count, float* scores, int64_t ld_scores,
-                                int32_t* dev_status, dsa_stream_t stream) {
+                                uint32_t* hist, int32_t* dev_status, dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_indexer_scores");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if (!indexer_shape_ok(*dims, seqs->mode)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (hist != nullptr && !indexer_counts_hist(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
   if (!q_idx || !q_scale || !w || !k_idx || !scores) return DSA_ERR_INVALID_ARG;
   if (k_scale == nullptr && !interleaved_ok(*seqs)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(scores) ||
-      ld_scores % 4 != 0)
+      !aligned16(hist) || ld_scores % 4 != 0)
     return DSA_ERR_MISALIGNED;
   if (ld_scores < max_keys(seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
   return indexer_dispatch(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
-                          scores, ld_scores, dev_status, reinterpret_cast<cudaStream_t>(stream));
+                          scores, ld_scores, dev_status, reinterpret_cast<cudaStream_t>(stream),
+                          hist);
 }
 
 dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
-                      int64_t ld_scores, int32_t row_begin, int32_t row_count, int32_t* idx,
-                      int32_t* dev_status, dsa_stream_t stream) {
+                      int64_t ld_scores, uint32_t* hist, int32_t row_begin, int32_t row_count,
+                      int32_t* idx, int32_t* dev_status, dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_topk");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
   if (!scores || !idx) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(scores) || !aligned16(idx) || ld_scores % 4 != 0) return DSA_ERR_MISALIGNED;
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(hist) || ld_scores % 4 != 0)
+    return DSA_ERR_MISALIGNED;
   if (ld_scores < max_keys(seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
   return topk_launch(*dims, *seqs, scores, ld_scores, row_begin, row_count, idx, dev_status,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<cudaStream_t>(stream), hist);
+}
+
+size_t dsa_indexer_topk_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                       int32_t row_count) {
+  if (check_common(dims, seqs) != DSA_OK || row_count < 0) return 0;
+  const size_t slab = size_t(row_count) * size_t(round4(seqs->max_seqlen)) * 4;
+  return (slab + 255) / 256 * 256 + size_t(row_count) * kTopkBins * 4;
+}
+
+dsa_status_t dsa_indexer_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
+                              const float* q_scale, const float* w, const uint8_t* k_idx,
+                              const float* k_scale, int32_t row_begin, int32_t row_count,
+                              int32_t* idx, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_indexer_topk");
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (!indexer_shape_ok(*dims, seqs->mode)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q_idx || !q_scale || !w || !k_idx || !idx) return DSA_ERR_INVALID_ARG;
+  if (k_scale == nullptr && !interleaved_ok(*seqs)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(idx) ||
+      !aligned16(workspace))
+    return DSA_ERR_MISALIGNED;
+  if (row_count == 0) return DSA_OK;
+  const size_t need = dsa_indexer_topk_workspace_size(dims, seqs, row_count);
+  if (workspace == nullptr || workspace_bytes < need) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  const int64_t ld = round4(max_keys(seqs, row_begin, row_count));
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  float* slab = reinterpret_cast<float*>(wsb);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(
+      wsb + (size_t(row_count) * size_t(round4(seqs->max_seqlen)) * 4 + 255) / 256 * 256);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (indexer_counts_hist(*dims) &&
+      cudaMemsetAsync(hist, 0, size_t(row_count) * kTopkBins * 4, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return indexer_topk(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count, slab,
+                      ld, hist, idx, dev_status, st);
 }
 
 size_t dsa_sparse_mla_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
@@ -677,10 +889,25 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                       workspace_bytes, dev_status, reinterpret_cast<cudaStream_t>(stream), splits);
 }
 
+size_t dsa_sparse_mla_workspace_size_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                         int32_t row_count, int32_t sm_count, size_t max_bytes) {
+  if (check_common(dims, seqs) != DSA_OK || sm_count <= 0 || row_count < 0) return 0;
+  return mla_ws_bytes(*dims, mla_splits(*dims, *seqs, row_count, sm_count, max_bytes), row_count);
+}
+
 size_t dsa_forward_workspace_size_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                       int32_t sm_count) {
   if (check_common(dims, seqs) != DSA_OK || sm_count <= 0) return 0;
   return plan_forward(*dims, *seqs, sm_count).total;
+}
+
+int32_t dsa_forward_chunk_rows_for(const dsa_dims_t* dims, const dsa_seqs_t* seqs, int32_t seq,
+                                   int32_t sm_count) {
+  if (check_common(dims, seqs) != DSA_OK || sm_count <= 0) return 0;
+  if (seqs->mode != DSA_PREFILL) return seqs->batch;
+  if (seq < 0 || seq >= seqs->batch) return 0;
+  const int64_t L = seqs->cu_seqlens_host[seq + 1] - seqs->cu_seqlens_host[seq];
+  return L <= 0 ? 0 : static_cast<int32_t>(chunk_rows_for(L, sm_count));
 }
 
 size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs) {
@@ -698,68 +925,45 @@ dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const u
   NvtxRange nvtx_range("dsa_forward");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
-  const dsa_dims_t& d = *dims;
-  const dsa_seqs_t& s = *seqs;
-  if (!indexer_shape_ok(d, s.mode) || !mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (!q_idx || !q_scale || !w || !k_idx || !q || !kv || !out || !lse)
-    return DSA_ERR_INVALID_ARG;
-  if (k_scale == nullptr && !interleaved_ok(s)) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(q) ||
-      !aligned16(kv) ||
-      !aligned16(out) || !aligned16(lse) || !aligned16(idx_out) || !aligned16(workspace))
-    return DSA_ERR_MISALIGNED;
-  DeviceInfo info;
-  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
-  const ForwardPlan plan = plan_forward(d, s, info.sm_count);
-  if (workspace == nullptr || workspace_bytes < plan.total) return DSA_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  auto align = [](size_t x) { return (x + 255) / 256 * 256; };
-  uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  float* slab = reinterpret_cast<float*>(wsb);
-  int32_t* idx_ws = reinterpret_cast<int32_t*>(wsb + align(plan.slab_floats * 4));
-  void* mla_ws = wsb + align(plan.slab_floats * 4) + align(plan.idx_ints * 4);
+  return forward_window(*dims, *seqs, 0, seqs->total_rows, q_idx, q_scale, w, k_idx, k_scale, q,
+                        kv, idx_out, out, lse, workspace, workspace_bytes, dev_status,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
 
-  if (s.mode == DSA_DECODE) {
-    if (idx_out == nullptr && s.max_seqlen <= d.topk)   // every context key is kept: dense
-      return mla_dispatch(d, s, q, kv, nullptr, 0, s.batch, out, lse, mla_ws, plan.mla_bytes,
-                          dev_status, st, plan.mla_splits);
-    const int64_t ld = round4(s.max_seqlen);
-    int32_t* idx = idx_out ? idx_out : idx_ws;
-    if ((e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, 0, s.batch, slab, ld,
-                              dev_status, st)) != DSA_OK)
-      return e;
-    if ((e = topk_launch(d, s, slab, ld, 0, s.batch, idx, dev_status, st)) != DSA_OK) return e;
-    return mla_dispatch(d, s, q, kv, idx, 0, s.batch, out, lse, mla_ws, plan.mla_bytes,
-                        dev_status, st, plan.mla_splits);
-  }
-  const int32_t* cu = s.cu_seqlens_host;
-  for (int b = 0; b < s.batch; ++b) {
-    const int64_t L = cu[b + 1] - cu[b];
-    if (L <= 0) continue;
-    const int64_t ld = round4(L);
-    const int64_t rows = chunk_rows_for(L, info.sm_count);
-    // rows with at most topk prior keys keep all of them: dense attention, no indexer or top-k
-    // (unless the caller wants the indices)
-    const int64_t n_dense = idx_out == nullptr ? std::min<int64_t>(L, d.topk) : 0;
-    if (n_dense > 0 &&
-        (e = mla_dispatch(d, s, q, kv, nullptr, cu[b], static_cast<int32_t>(n_dense), out, lse,
-                          nullptr, 0, dev_status, st, 1)) != DSA_OK)
-      return e;
-    for (int64_t r0 = n_dense; r0 < L; r0 += rows) {
-      const int32_t row_begin = static_cast<int32_t>(cu[b] + r0);
-      const int32_t row_count = static_cast<int32_t>(std::min(rows, L - r0));
-      int32_t* idx = idx_out ? idx_out + int64_t(row_begin) * d.topk : idx_ws;
-      if ((e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
-                                slab, ld, dev_status, st)) != DSA_OK)
-        return e;
-      if ((e = topk_launch(d, s, slab, ld, row_begin, row_count, idx, dev_status, st)) != DSA_OK)
-        return e;
-      if ((e = mla_dispatch(d, s, q, kv, idx, row_begin, row_count, out, lse, nullptr, 0,
-                            dev_status, st, 1)) != DSA_OK)
-        return e;
-    }
-  }
-  return DSA_OK;
+dsa_status_t dsa_forward_rows(const dsa_dims_t* dims, const dsa_seqs_t* seqs, int32_t row_begin,
+                              int32_t row_count, const uint8_t* q_idx, const float* q_scale,
+                              const float* w, const uint8_t* k_idx, const float* k_scale,
+                              const uint16_t* q, const uint16_t* kv, int32_t* idx_out,
+                              uint16_t* out, float* lse, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_forward_rows");
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
+  if (!q_idx || !q_scale || !w || !q || !out || !lse) return DSA_ERR_INVALID_ARG;
+  const dsa_dims_t& d = *dims;
+  // the query-side arrays hold rows [row_begin, row_begin + row_count); the kernels index them
+  // by absolute row, so they get bases moved back by row_begin rows (computed as integers; only
+  // the caller's rows are ever addressed from them)
+  auto back = [&](const void* p, size_t row_bytes) -> uintptr_t {
+    return reinterpret_cast<uintptr_t>(p) - uintptr_t(row_begin) * row_bytes;
+  };
+  const size_t hi = size_t(d.h_idx);
+  const uintptr_t q_idx_a = back(q_idx, hi * d.d_idx);
+  const uintptr_t q_scale_a = back(q_scale, hi * 4);
+  const uintptr_t w_a = back(w, hi * 4);
+  const uintptr_t q_a = back(q, size_t(d.h) * d.d_qk * 2);
+  const uintptr_t out_a = back(out, size_t(d.h) * d.d_v * 2);
+  const uintptr_t lse_a = back(lse, size_t(d.h) * 4);
+  const uintptr_t idx_a = idx_out ? back(idx_out, size_t(d.topk) * 4) : 0;
+  return forward_window(d, *seqs, row_begin, row_begin + row_count,
+                        reinterpret_cast<const uint8_t*>(q_idx_a),
+                        reinterpret_cast<const float*>(q_scale_a),
+                        reinterpret_cast<const float*>(w_a), k_idx, k_scale,
+                        reinterpret_cast<const uint16_t*>(q_a), kv,
+                        reinterpret_cast<int32_t*>(idx_a), reinterpret_cast<uint16_t*>(out_a),
+                        reinterpret_cast<float*>(lse_a), workspace, workspace_bytes, dev_status,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_cache_append(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* k_new,
@@ -941,9 +1145,11 @@ dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_dims_t* dims, const dsa_seqs_t
     return DSA_ERR_MISALIGNED;
   DeviceInfo info;
   if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
-  const int splits = mla_splits(*dims, *seqs, row_count, info.sm_count);
+  // the fastest split count whose partials fit the built-in array (one split needs none)
+  const int splits =
+      mla_splits(*dims, *seqs, row_count, info.sm_count, DSA_NOALLOC_SCRATCH_BYTES);
   const size_t need = mla_ws_bytes(*dims, splits, row_count);
-  if (need > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (need > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE_TOO_SMALL;   // unreachable
   void* scratch = nullptr;
   if (need > 0 && (e = noalloc_scratch(&scratch)) != DSA_OK) return e;
   return mla_dispatch(*dims, *seqs, q, kv, idx, row_begin, row_count, out, lse, scratch,

@@ -19,6 +19,12 @@
 // accumulators are a ring of ACC buffers in TMEM so the epilogue of tile i overlaps the MMA of
 // later tiles.  Decode (one query row, N = 64) runs two epilogue warpgroups on alternate tiles;
 // prefill (N = 256) splits each tile's columns over four warpgroups, one query row each.
+//
+// Fused first digit of the top-k (when `hist` is given): as it writes a score, each epilogue
+// thread also counts it in its query row's histogram of the top 11 bits of the order-preserving
+// key (the first radix digit the top-k selects on), kept in shared memory; at the end the CTA
+// adds the non-zero bins into the row's global histogram.  The top-k then starts from exact
+// per-row counts and classifies the slab in a single pass.
 #pragma once
 #include "sm100.cuh"
 
@@ -46,12 +52,22 @@ struct IndexerParams {
   int32_t max_seqlen;     // decode: a seq_lens entry above this is clamped and reported
   int64_t num_kv_rows;
   int32_t tiles_per_split;
+  uint32_t* hist;         // optional: [slab rows][kIdxHistBins] first-digit counts (added to)
 };
+
+constexpr int kIdxHistBins = 2048;   // top 11 bits of the order-preserving score key
+
+// Order-preserving 32-bit key of a score (unsigned order = float order, -0 folded onto +0).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0) u = 0;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 template <int H_I, int D_I, int QPG>
 struct IndexerCfg {
   static constexpr int N = H_I * QPG;                 // MMA N: (row, head) columns
-  static constexpr int STAGES = QPG == 1 ? 6 : 8;
+  static constexpr int STAGES = QPG == 1 ? 5 : 8;
   static constexpr int ACC = QPG == 1 ? 4 : 2;        // TMEM accumulator ring
   static constexpr int EPI_WARPS = QPG == 1 ? 8 : 16;    // prefill: one query row per warpgroup
   static constexpr bool TILE_SPLIT = QPG == 1;        // warpgroups take alternate tiles
@@ -64,9 +80,13 @@ struct IndexerCfg {
   static constexpr uint32_t SBO = 8 * D_I;            // next 8-row group
   static constexpr int TMEM_COLS = ACC * N;
   static constexpr int SCALE_FLOATS = 2 * 80;         // per stage: 2 boxes x (64 + slack)
+  // per query row of the group, the first-digit histogram (full shapes; the 64-row groups of
+  // the small shape have no room for it and run the top-k's own histogram instead)
+  static constexpr bool HIST = QPG <= 4;
+  static constexpr int HIST_BYTES = HIST ? QPG * kIdxHistBins * 4 : 0;
   static constexpr int SMEM_BYTES =
       1024 + Q_BYTES + STAGES * TILE_BYTES + STAGES * SCALE_FLOATS * 4 + STAGES * 2 * 16 +
-      N * 4 + 512;
+      N * 4 + 512 + HIST_BYTES;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   static_assert(Q_BYTES % 1024 == 0 && TILE_BYTES % 1024 == 0, "1024-byte aligned tiles");
@@ -98,6 +118,8 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
   uint64_t* tempty = tfull + C::ACC;          // [ACC] accumulator drained by the epilogue
   uint64_t* qbar = tempty + C::ACC;           // Q group landed
   uint64_t* done = qbar + 1;                  // every MMA of this CTA completed
+  uint32_t* sHist = reinterpret_cast<uint32_t*>(done + 1);   // [QPG][kIdxHistBins]
+  const bool hist_on = C::HIST && p.hist != nullptr;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
@@ -145,6 +167,8 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
     abort_s = 0;
     fence_mbar_init();
   }
+  if (hist_on)
+    for (int i = threadIdx.x; i < C::HIST_BYTES / 4; i += C::THREADS) sHist[i] = 0;
   if (warp == 2) tmem_alloc(smem_u32(&tmem_base_s), C::TMEM_COLS);
   if (warp == 3) {
     for (int i = lane; i < N; i += 32) {
@@ -364,9 +388,11 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
             }
           }
           const int rr = (part * COLS) / H_I + q;
-          if (rr < rows_in_group && key <= pos_first + rr)
-            p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] =
-                ks * ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
+          if (rr < rows_in_group && key <= pos_first + rr) {
+            const float sc = ks * ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
+            p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] = sc;
+            if (hist_on) atomicAdd(&sHist[rr * kIdxHistBins + (order_key(sc) >> 21)], 1u);
+          }
         }
         continue;
       }
@@ -389,9 +415,11 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
           }
           if ((col + 32) % H_I == 0) {       // a query row's heads are complete
             const int rr = col / H_I;
-            if (rr < rows_in_group && key <= pos_first + rr)
-              p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] =
-                  ks * acc;
+            if (rr < rows_in_group && key <= pos_first + rr) {
+              const float sc = ks * acc;
+              p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] = sc;
+              if (hist_on) atomicAdd(&sHist[rr * kIdxHistBins + (order_key(sc) >> 21)], 1u);
+            }
             acc = 0.f;
           }
         } else {
@@ -418,6 +446,18 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (hist_on) {
+    // this CTA's counts into the rows' global histograms (only the bins it saw)
+    for (int i = threadIdx.x; i < rows_in_group * kIdxHistBins; i += C::THREADS) {
+      const uint32_t v = sHist[i];
+      if (v != 0) {
+        const int rr = i / kIdxHistBins;
+        atomicAdd(p.hist + static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * kIdxHistBins +
+                      (i % kIdxHistBins),
+                  v);
+      }
+    }
   }
 }
 

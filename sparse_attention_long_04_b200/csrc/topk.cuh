@@ -5,18 +5,28 @@
 // page, section 1.)
 //
 // Radix select, no sort.  Each score maps to a 32-bit key whose unsigned order is the float
-// order (-0 folded onto +0).  A row is split over a cluster of C CTAs (C = 1..8); CTA c reads
-// its slice of the row from global memory once and keeps the keys in shared memory, building
-// the histogram of the first digit (the top 11 bits) while it loads.  The C histograms are
-// summed through distributed shared memory (each CTA adds its non-zero bins into every CTA)
-// and every CTA picks the bin holding the k-th largest key.  The keys of that bin are few:
-// every CTA appends its own into CTA 0's candidate buffer, CTA 0 resolves the remaining 21
-// bits (digits of 11 and 10 bits) locally and broadcasts the exact k-th key tau and the count
-// of keys == tau still needed.  (If the bin is too crowded for the buffer, e.g. mass ties, the
-// CTAs resolve the remaining digits together with filtered scans and cluster-summed
-// histograms instead.)  The output pass takes every key > tau and the first `need` keys == tau in index
-// order (the smallest indices): per-warp counts give each warp's output offset (an exclusive
-// scan over the cluster in index order), and the indices come out in increasing order.
+// order (-0 folded onto +0).  A row is split over a cluster of C CTAs (C = 1..8), CTA c owning
+// the slice [c per, (c+1) per) of the row.
+//   1. First digit (the top 11 bits of the key).  Its per-row histogram either comes with the
+//      scores (the indexer counts each score as it writes it) or is built here with one pass
+//      over the slice and summed over the cluster through distributed shared memory.  Every CTA
+//      finds the bin b holding the k-th largest key and the count above it.
+//   2. One classifying pass over the slice: keys of a bin above b are taken (a bit in the
+//      slice's "taken" bitmap); keys of bin b are candidates, kept in shared memory with their
+//      positions.  When bin b holds exactly the keys still needed, all of it is taken instead.
+//      Bitmap layout: a block of 128 keys is 4 words; key 4 l + e of the block is bit l of word
+//      e, so that lane l of a warp reading the block as float4 contributes bit l of each word.
+//   3. The candidates of the cluster are few (1-6k): their keys go to CTA 0, which resolves the
+//      remaining 21 bits (digits of 11 and 10 bits) and broadcasts the exact k-th key tau and the
+//      number of keys equal to tau still needed.  Each CTA marks its candidates above tau as
+//      taken and those equal to tau as ties (a second bitmap).  A bin too crowded for the
+//      buffers (mass ties) is resolved instead with filtered passes over the slice and
+//      cluster-summed histograms, followed by a marking pass.
+//   4. Output from the bitmaps alone: every taken key, and the first `need` ties in index order
+//      (the smaller indices), at positions given by exclusive scans of the per-word counts over
+//      the CTA and the cluster, so the indices come out in increasing order.
+// The scores are read from global memory once (twice without a given histogram, three times in
+// the crowded case), never held in shared memory.
 #pragma once
 #include "sm100.cuh"
 
@@ -35,15 +45,24 @@ struct TopkParams {
   int32_t max_seqlen;
   int32_t* status;
   int32_t csize;           // CTAs per row (the cluster size)
+  int32_t slice;           // keys per CTA slice (a multiple of 128), sizes the bitmaps
+  uint32_t* hist;          // optional [row_count][kTopkBins] first-digit counts of each row's
+                           // scores; read, then zeroed for the next use
 };
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkSlice = 16384;          // keys a CTA keeps in shared memory
 constexpr int kTopkBins = 2048;
-constexpr int kTopkCand = 8192;           // candidate keys CTA 0 gathers after the first digit
-// 112.5 KiB: two CTAs still fit on one SM
-constexpr int kTopkSmem = kTopkSlice * 4 + kTopkCand * 4 + 2 * kTopkBins * 4 + 512;
+constexpr int kTopkLocal = 4096;     // candidates (key, position) a CTA keeps
+constexpr int kTopkGather = 12288;   // candidate keys CTA 0 gathers from the cluster
+constexpr int kTopkFixedSmem =
+    2 * kTopkBins * 4 + 2 * kTopkLocal * 4 + kTopkGather * 4 + 512;
+
+// Dynamic shared memory of a launch whose slices hold `slice` keys: the fixed part plus the two
+// bitmaps of the slice.
+__host__ __device__ constexpr int topk_smem_bytes(int slice) {
+  return kTopkFixedSmem + 2 * ((slice + 31) / 32) * 4;
+}
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -51,14 +70,10 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
+// Bitmap position of key i of a slice (see the layout above).
+__device__ __forceinline__ int bm_word(int i) { return (i >> 7) * 4 + (i & 3); }
+__device__ __forceinline__ uint32_t bm_bit(int i) { return 1u << ((i >> 2) & 31); }
+
 __device__ __forceinline__ void st_cluster_u4(uint32_t addr, uint4 v) {
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w)
@@ -66,6 +81,9 @@ __device__ __forceinline__ void st_cluster_u4(uint32_t addr, uint4 v) {
 }
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // Exclusive scan over the CTA's threads (one value each); *total receives the sum.
@@ -97,10 +115,6 @@ __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t* tmp, uin
   return res;
 }
 
-__device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
-  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 // Sums the cluster's histograms (nb bins) into every CTA's hsum, which the caller zeroed before
 // the histogram was built: every CTA adds its non-zero bins into every CTA's hsum.
 __device__ __forceinline__ void cluster_hist_sum(uint32_t* hist, uint32_t* hsum, uint32_t nb,
@@ -120,24 +134,22 @@ __device__ __forceinline__ void cluster_hist_sum(uint32_t* hist, uint32_t* hsum,
   }
 }
 
-__device__ __forceinline__ uint32_t atom_cluster_add(uint32_t addr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v)
-               : "memory");
-  return old;
-}
-
 // Bin holding the need-th largest key of hsum (nb bins, descending cumulative counts); all
-// threads of the CTA call it and all get the same (bin, count above the bin).
+// threads of the CTA call it and all get the same (bin, count above the bin).  A histogram
+// holding fewer than `need` keys (inconsistent input) gives bin 0.
 __device__ __forceinline__ void find_bin(const uint32_t* hsum, uint32_t nb, uint32_t need,
                                          uint32_t* tmp, uint32_t* s_bin, uint32_t* s_above,
                                          uint32_t* bin, uint32_t* above) {
   const int tid = threadIdx.x;
   const uint32_t bpt = nb / kTopkThreads;         // 4 or 2 bins per thread
+  if (tid == 0) {
+    *s_bin = 0;
+    *s_above = 0;
+  }
   uint32_t mine = 0;
   for (uint32_t j = 0; j < bpt; ++j) mine += hsum[nb - 1 - (tid * bpt + j)];
   uint32_t tot;
-  const uint32_t before = cta_excl_scan(mine, tmp, &tot);
+  const uint32_t before = cta_excl_scan(mine, tmp, &tot);   // (syncs: s_bin init visible)
   if (before < need && before + mine >= need) {
     uint32_t c = before;
     for (uint32_t j = 0; j < bpt; ++j) {
@@ -156,18 +168,24 @@ __device__ __forceinline__ void find_bin(const uint32_t* hsum, uint32_t nb, uint
   __syncthreads();
 }
 
+__device__ __forceinline__ void cta_or_cluster_sync(int C) {
+  if (C > 1) cluster_sync(); else __syncthreads();
+}
+
 __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(topk_smem);           // [kTopkSlice]
-  uint32_t* cand = keys + kTopkSlice;                                // [kTopkCand] (CTA 0)
-  uint32_t* hist = cand + kTopkCand;                                 // [kTopkBins] this CTA
-  uint32_t* hsum = hist + kTopkBins;                                 // [kTopkBins] cluster sum
-  uint32_t* tmp = hsum + kTopkBins;                                  // [40] scan scratch
-  uint32_t* wgt = tmp + 40;                                          // [16] per-warp > tau
-  uint32_t* weq = wgt + 16;                                          // [16] per-warp == tau
-  uint32_t* cnt = weq + 16;                                          // [16] per-CTA (gt, eq)
-  uint32_t* bc = cnt + 16;                                           // [4] broadcast result
-  __shared__ uint32_t s_bin, s_above, s_ncand, s_base;
+  uint32_t* hsum = reinterpret_cast<uint32_t*>(topk_smem);          // [kTopkBins] row / digit
+  uint32_t* hloc = hsum + kTopkBins;                                 // [kTopkBins] this slice
+  uint32_t* ckey = hloc + kTopkBins;                                 // [kTopkLocal] candidates
+  int32_t* cpos = reinterpret_cast<int32_t*>(ckey + kTopkLocal);     // [kTopkLocal] positions
+  uint32_t* gath = reinterpret_cast<uint32_t*>(cpos + kTopkLocal);   // [kTopkGather] (CTA 0)
+  uint32_t* tmp = gath + kTopkGather;                                // [40] scan scratch
+  uint32_t* cnt = tmp + 40;                                          // [4][8] per-CTA counts
+  uint32_t* bc = cnt + 32;                                           // [4] broadcast result
+  uint32_t* bm_take = reinterpret_cast<uint32_t*>(topk_smem + kTopkFixedSmem);  // [words]
+  const int words = (p.slice + 31) / 32;
+  uint32_t* bm_tie = bm_take + words;                                // [words]
+  __shared__ uint32_t s_bin, s_above, s_nloc, s_over;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = p.csize;
@@ -191,147 +209,151 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   }
   const float* srow = p.scores + static_cast<int64_t>(r) * p.ld;
   int32_t* out = p.idx + static_cast<int64_t>(r) * p.topk;
+  uint32_t* grow_hist = p.hist ? p.hist + static_cast<int64_t>(r) * kTopkBins : nullptr;
   const int K = p.topk;
   if (n <= K) {                                    // uniform over the cluster: no barrier used
     for (int j = crank * kTopkThreads + tid; j < K; j += C * kTopkThreads)
       out[j] = j < n ? j : -1;
+    if (grow_hist != nullptr && crank == 0)        // leave the histogram zeroed for reuse
+      for (int i = tid; i < kTopkBins; i += kTopkThreads) grow_hist[i] = 0;
     return;
   }
-  // this CTA's slice [s0, s1); a multiple of 4 long so every slice starts 16-byte aligned
-  const int per = ((n + C - 1) / C + 3) / 4 * 4;
+  // this CTA's slice [s0, s0 + m); per is a multiple of 128 (no larger than p.slice)
+  const int per = ((n + C - 1) / C + 127) / 128 * 128;
   const int s0 = min(n, crank * per);
-  const int s1 = min(n, s0 + per);
-  const int m = s1 - s0;
-  const bool cached = m <= kTopkSlice;
-  auto key_at = [&](int i) -> uint32_t {
-    return cached ? keys[i] : score_key(srow[s0 + i]);
-  };
-  auto key4_at = [&](int i) -> uint4 {            // i multiple of 4, i < m
-    if (cached) return *reinterpret_cast<const uint4*>(keys + i);
-    if (i + 3 < m) {                              // a streamed slice: one 16-byte load
-      const float4 v = *reinterpret_cast<const float4*>(srow + s0 + i);
-      return make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
-    }
-    uint4 k = make_uint4(0, 0, 0, 0);
-    if (i + 0 < m) k.x = score_key(srow[s0 + i + 0]);
-    if (i + 1 < m) k.y = score_key(srow[s0 + i + 1]);
-    if (i + 2 < m) k.z = score_key(srow[s0 + i + 2]);
-    if (i + 3 < m) k.w = score_key(srow[s0 + i + 3]);
-    return k;
-  };
+  const int m = min(n, s0 + per) - s0;
+  const int nrounds = (m + 127) / 128;           // 128-key blocks: lane l reads keys 4l..4l+3
 
-  // ---- digit 1 (top 11 bits): load + histogram in one pass
-  for (int i = tid; i < kTopkBins; i += kTopkThreads) {
-    hist[i] = 0;
-    hsum[i] = 0;
+  for (int i = tid; i < words; i += kTopkThreads) {
+    bm_take[i] = 0;
+    bm_tie[i] = 0;
   }
-  if (tid == 0) s_ncand = 0;
-  __syncthreads();
-  if (cached) {
-    constexpr int kVec = kTopkSlice / 4 / kTopkThreads;   // float4 per thread (8)
-    float4 v[kVec];
-#pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-      const int i4 = (u * kTopkThreads + tid) * 4;
-      v[u] = i4 < m ? *reinterpret_cast<const float4*>(srow + s0 + i4)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-      const int i4 = (u * kTopkThreads + tid) * 4;
-      if (i4 < m) {
-        const uint4 k = make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z),
-                                   score_key(v[u].w));
-        *reinterpret_cast<uint4*>(keys + i4) = k;
-        atomicAdd(&hist[k.x >> 21], 1u);
-        if (i4 + 1 < m) atomicAdd(&hist[k.y >> 21], 1u);
-        if (i4 + 2 < m) atomicAdd(&hist[k.z >> 21], 1u);
-        if (i4 + 3 < m) atomicAdd(&hist[k.w >> 21], 1u);
-      }
-    }
+  if (tid == 0) {
+    s_nloc = 0;
+    s_over = 0;
+  }
+
+  // ---- 1. first digit
+  if (grow_hist != nullptr) {
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) hsum[i] = __ldcg(grow_hist + i);
+    __syncthreads();
   } else {
-    // a slice longer than shared memory holds: streamed with 16-byte loads, 4 in flight
-    for (int base = tid * 4; base < m; base += kTopkThreads * 16) {
-      uint4 k[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i4 = base + u * kTopkThreads * 4;
-        k[u] = i4 < m ? key4_at(i4) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i4 = base + u * kTopkThreads * 4;
-        if (i4 < m) atomicAdd(&hist[k[u].x >> 21], 1u);
-        if (i4 + 1 < m) atomicAdd(&hist[k[u].y >> 21], 1u);
-        if (i4 + 2 < m) atomicAdd(&hist[k[u].z >> 21], 1u);
-        if (i4 + 3 < m) atomicAdd(&hist[k[u].w >> 21], 1u);
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) {
+      hloc[i] = 0;
+      hsum[i] = 0;
+    }
+    __syncthreads();
+    for (int rd = warp; rd < nrounds; rd += kTopkWarps) {
+      const int i4 = rd * 128 + 4 * lane;
+      if (i4 < m) {
+        const float4 v = *reinterpret_cast<const float4*>(srow + s0 + i4);
+        atomicAdd(&hloc[score_key(v.x) >> 21], 1u);
+        if (i4 + 1 < m) atomicAdd(&hloc[score_key(v.y) >> 21], 1u);
+        if (i4 + 2 < m) atomicAdd(&hloc[score_key(v.z) >> 21], 1u);
+        if (i4 + 3 < m) atomicAdd(&hloc[score_key(v.w) >> 21], 1u);
       }
     }
+    cluster_hist_sum(hloc, hsum, kTopkBins, C);
   }
-  cluster_hist_sum(hist, hsum, kTopkBins, C);
   uint32_t bin, above;
   find_bin(hsum, kTopkBins, K, tmp, &s_bin, &s_above, &bin, &above);
   uint32_t need = K - above;
+  const bool whole_bin = hsum[bin] == need;      // every key of the bin is taken
   uint32_t prefix = bin << 21, mask = 0xFFE00000u;
-  const uint32_t in_bin_total = hsum[bin];
-  const uint32_t in_bin_local = hist[bin];
+
+  // ---- 2. classify the slice: above the bin -> taken; in the bin -> candidate
+  constexpr int U = 4;                             // blocks in flight per warp
+  for (int rd0 = warp; rd0 < nrounds; rd0 += U * kTopkWarps) {
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i4 = (rd0 + u * kTopkWarps) * 128 + 4 * lane;
+      v[u] = i4 < m ? __ldcs(reinterpret_cast<const float4*>(srow + s0 + i4))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int rd = rd0 + u * kTopkWarps;
+      if (rd >= nrounds) break;
+      const float ve[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rd * 128 + 4 * lane + e;
+        const uint32_t k = score_key(ve[e]);
+        const uint32_t b = k >> 21;
+        const bool in = i < m;
+        const bool take = in && (b > bin || (whole_bin && b == bin));
+        const bool cand = in && !whole_bin && b == bin;
+        const uint32_t tw = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) bm_take[rd * 4 + e] = tw;
+        const uint32_t cw = __ballot_sync(0xffffffffu, cand);
+        if (cw != 0) {
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(&s_nloc, static_cast<uint32_t>(__popc(cw)));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (cand) {
+            const uint32_t slot = base + __popc(cw & ((1u << lane) - 1u));
+            if (slot < static_cast<uint32_t>(kTopkLocal)) {
+              ckey[slot] = k;
+              cpos[slot] = i;
+            } else {
+              s_over = 1;
+            }
+          }
+        }
+      }
+    }
+  }
   __syncthreads();
 
-  if (in_bin_total != need) {                     // else: every key of the bin is taken
-    if (in_bin_total + 3u * C <= static_cast<uint32_t>(kTopkCand)) {
-      // ---- gather the bin's keys into CTA 0 and resolve the last 21 bits there.  Each CTA
-      // reserves a multiple of 4 slots, compacts its keys locally (CTA 0: in place), pads with
-      // a key outside the bin and copies 16 bytes at a time into CTA 0's buffer.
-      const uint32_t n4 = (in_bin_local + 3u) & ~3u;
-      const uint32_t pad_key = bin == 0 ? 0xFFFFFFFFu : 0u;   // never matches the bin
-      if (tid == 0)
-        s_base = n4 ? (C > 1 ? atom_cluster_add(map_to_rank(smem_u32(&s_ncand), 0), n4)
-                             : atomicAdd(&s_ncand, n4))
-                    : 0u;
-      if (C > 1) cluster_sync(); else __syncthreads();   // reservations done (CTA 0's count)
-      uint32_t mine = 0;                           // this thread's matches, in its 4-key groups
-      const int nrounds = (m + kTopkThreads * 4 - 1) / (kTopkThreads * 4);
-      for (int u = 0; u < nrounds; ++u) {
-        const int i4 = (u * kTopkThreads + tid) * 4;
-        if (i4 < m) {
-          const uint4 k = key4_at(i4);
-          mine += (k.x & mask) == prefix;
-          mine += i4 + 1 < m && (k.y & mask) == prefix;
-          mine += i4 + 2 < m && (k.z & mask) == prefix;
-          mine += i4 + 3 < m && (k.w & mask) == prefix;
+  // ---- 3. resolve tau within the bin
+  if (!whole_bin) {
+    const uint32_t nloc = min(s_nloc, static_cast<uint32_t>(kTopkLocal));
+    const uint32_t n4 = (nloc + 3u) & ~3u;
+    // every CTA learns every CTA's candidate count and overflow flag
+    if (tid == 0) {
+      for (int c = 0; c < C; ++c) {
+        const uint32_t a = C > 1 ? map_to_rank(smem_u32(cnt), c) : smem_u32(cnt);
+        if (C > 1) {
+          st_cluster_u32(a + 4 * crank, n4);
+          st_cluster_u32(a + 4 * (8 + crank), s_over);
+        } else {
+          cnt[0] = n4;
+          cnt[8] = s_over;
         }
       }
-      uint32_t tot;
-      const uint32_t lbase = crank == 0 ? s_base : 0u;   // where this CTA compacts locally
-      uint32_t slot = lbase + cta_excl_scan(mine, tmp, &tot);
-      for (int u = 0; u < nrounds && mine; ++u) {
-        const int i4 = (u * kTopkThreads + tid) * 4;
-        if (i4 < m) {
-          const uint4 k = key4_at(i4);
-          const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (i4 + e < m && (kk[e] & mask) == prefix) cand[slot++] = kk[e];
-        }
-      }
-      if (tid < static_cast<int>(n4 - in_bin_local)) cand[lbase + in_bin_local + tid] = pad_key;
+    }
+    cta_or_cluster_sync(C);
+    uint32_t total = 0, off = 0, over = 0;
+    for (int c = 0; c < C; ++c) {
+      if (c < crank) off += cnt[c];
+      total += cnt[c];
+      over |= cnt[8 + c];
+    }
+    const bool crowded = over != 0 || total > static_cast<uint32_t>(kTopkGather);
+    if (!crowded) {
+      // candidates' keys into CTA 0 (padded to 4 with a key outside the bin), 16 B at a time
+      const uint32_t pad_key = bin == 0 ? 0xFFFFFFFFu : 0u;
+      for (uint32_t j = nloc + tid; j < n4; j += kTopkThreads) ckey[j] = pad_key;
       __syncthreads();
-      if (C > 1 && crank != 0) {
-        const uint32_t dst0 = map_to_rank(smem_u32(cand), 0) + s_base * 4;
-        const uint4* src4 = reinterpret_cast<const uint4*>(cand);
+      const uint4* src4 = reinterpret_cast<const uint4*>(ckey);
+      if (C > 1) {
+        const uint32_t dst0 = map_to_rank(smem_u32(gath), 0) + off * 4;
         for (uint32_t j = tid; j < n4 / 4; j += kTopkThreads) st_cluster_u4(dst0 + j * 16, src4[j]);
+      } else {
+        for (uint32_t j = tid; j < n4 / 4; j += kTopkThreads)
+          reinterpret_cast<uint4*>(gath)[j] = src4[j];
       }
-      if (C > 1) cluster_sync(); else __syncthreads();   // CTA 0 holds every candidate
+      cta_or_cluster_sync(C);                      // CTA 0 holds every candidate
       if (crank == 0) {
-        // digits 2 and 3 over the candidates, locally
         constexpr int kShift[2] = {10, 0};
         constexpr int kBits[2] = {11, 10};
         for (int pass = 0; pass < 2; ++pass) {
           const uint32_t nb = 1u << kBits[pass];
           for (uint32_t i = tid; i < nb; i += kTopkThreads) hsum[i] = 0;
           __syncthreads();
-          for (uint32_t i = tid; i < s_ncand; i += kTopkThreads) {
-            const uint32_t k = cand[i];
+          for (uint32_t i = tid; i < total; i += kTopkThreads) {
+            const uint32_t k = gath[i];
             if ((k & mask) == prefix) atomicAdd(&hsum[(k >> kShift[pass]) & (nb - 1)], 1u);
           }
           __syncthreads();
@@ -346,11 +368,11 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
         }
         if (tid == 0)
           for (int c = 0; c < C; ++c) {
-            const uint32_t base = C > 1 ? map_to_rank(smem_u32(bc), c) : smem_u32(bc);
             if (C > 1) {
-              st_cluster_u32(base + 0, prefix);
-              st_cluster_u32(base + 4, mask);
-              st_cluster_u32(base + 8, need);
+              const uint32_t a = map_to_rank(smem_u32(bc), c);
+              st_cluster_u32(a + 0, prefix);
+              st_cluster_u32(a + 4, mask);
+              st_cluster_u32(a + 8, need);
             } else {
               bc[0] = prefix;
               bc[1] = mask;
@@ -358,26 +380,34 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
             }
           }
       }
-      if (C > 1) cluster_sync(); else __syncthreads();   // the broadcast has landed
+      cta_or_cluster_sync(C);                      // the broadcast has landed
       prefix = bc[0];
       mask = bc[1];
       need = bc[2];
+      // mark the candidates: above tau -> taken, equal -> tie
+      for (uint32_t j = tid; j < nloc; j += kTopkThreads) {
+        const uint32_t km = ckey[j] & mask;
+        const int i = cpos[j];
+        if (km > prefix) atomicOr(&bm_take[bm_word(i)], bm_bit(i));
+        else if (km == prefix) atomicOr(&bm_tie[bm_word(i)], bm_bit(i));
+      }
     } else {
-      // ---- crowded bin: the remaining digits with filtered scans and cluster sums
+      // crowded bin: the remaining digits with filtered passes and cluster sums, then a pass
+      // that marks the bin's keys
       constexpr int kShift[2] = {10, 0};
       constexpr int kBits[2] = {11, 10};
       for (int pass = 0; pass < 2; ++pass) {
         const uint32_t nb = 1u << kBits[pass];
         for (uint32_t i = tid; i < nb; i += kTopkThreads) {
-          hist[i] = 0;
+          hloc[i] = 0;
           hsum[i] = 0;
         }
         __syncthreads();
         for (int i = tid; i < m; i += kTopkThreads) {
-          const uint32_t k = key_at(i);
-          if ((k & mask) == prefix) atomicAdd(&hist[(k >> kShift[pass]) & (nb - 1)], 1u);
+          const uint32_t k = score_key(srow[s0 + i]);
+          if ((k & mask) == prefix) atomicAdd(&hloc[(k >> kShift[pass]) & (nb - 1)], 1u);
         }
-        cluster_hist_sum(hist, hsum, nb, C);
+        cluster_hist_sum(hloc, hsum, nb, C);
         uint32_t b2, ab2;
         find_bin(hsum, nb, need, tmp, &s_bin, &s_above, &b2, &ab2);
         need -= ab2;
@@ -387,122 +417,76 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
         __syncthreads();
         if (exact) break;
       }
-    }
-  }
-
-  // ---- output: keys > tau, then the first `need` keys == tau in index order
-  const int wn = ((m + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;   // per warp, x128
-  const int w0 = min(m, warp * wn), w1 = min(m, w0 + wn);
-  uint32_t gt = 0, eq = 0;
-  for (int i4 = w0 + lane * 4; i4 < w1; i4 += 128) {
-    const uint4 k = key4_at(i4);
-    const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (i4 + e < w1) {
-        const uint32_t km = kk[e] & mask;
-        gt += km > prefix;
-        eq += km == prefix;
+      for (int i = tid; i < m; i += kTopkThreads) {
+        const uint32_t k = score_key(srow[s0 + i]);
+        if ((k >> 21) != bin) continue;            // the bin's keys only (above: taken already)
+        const uint32_t km = k & mask;
+        if (km > prefix) atomicOr(&bm_take[bm_word(i)], bm_bit(i));
+        else if (km == prefix) atomicOr(&bm_tie[bm_word(i)], bm_bit(i));
       }
     }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    gt += __shfl_xor_sync(0xffffffffu, gt, o);
-    eq += __shfl_xor_sync(0xffffffffu, eq, o);
-  }
-  if (lane == 0) {
-    wgt[warp] = gt;
-    weq[warp] = eq;
   }
   __syncthreads();
+
+  // ---- 4. output: taken keys and the first `need` ties, in index order
+  // thread t owns the 128-key blocks [t bpt, (t+1) bpt) of the slice
+  const int nblk = words / 4;
+  const int bpt = (nblk + kTopkThreads - 1) / kTopkThreads;
+  const int b0 = min(nblk, tid * bpt), b1 = min(nblk, b0 + bpt);
+  uint32_t tk = 0, te = 0;
+  for (int w = 4 * b0; w < 4 * b1; ++w) {
+    tk += __popc(bm_take[w]);
+    te += __popc(bm_tie[w]);
+  }
+  uint32_t tk_tot, te_tot;
+  uint32_t tk_before = cta_excl_scan(tk, tmp, &tk_tot);
+  uint32_t te_before = cta_excl_scan(te, tmp, &te_tot);
   if (tid == 0) {
-    uint32_t g = 0, e = 0;
-    for (int w = 0; w < kTopkWarps; ++w) {
-      g += wgt[w];
-      e += weq[w];
-    }
-    if (C > 1) {
-      for (int c = 0; c < C; ++c) {
-        st_cluster_u32(map_to_rank(smem_u32(cnt + crank), c), g);
-        st_cluster_u32(map_to_rank(smem_u32(cnt + 8 + crank), c), e);
+    for (int c = 0; c < C; ++c) {
+      if (C > 1) {
+        const uint32_t a = map_to_rank(smem_u32(cnt), c);
+        st_cluster_u32(a + 4 * (16 + crank), tk_tot);
+        st_cluster_u32(a + 4 * (24 + crank), te_tot);
+      } else {
+        cnt[16] = tk_tot;
+        cnt[24] = te_tot;
       }
-    } else {
-      cnt[0] = g;
-      cnt[8] = e;
     }
   }
-  if (C > 1) cluster_sync(); else __syncthreads();
-  // every key == tau is taken when the cluster holds exactly `need` of them (the usual case)
-  uint32_t eq_all = 0;
-  for (int c = 0; c < C; ++c) eq_all += cnt[8 + c];
-  const bool all_eq = eq_all == need;
-  // offsets: keys taken by the CTAs, then the warps, before this one (index order)
-  uint32_t w_out = 0, w_eq = 0;
+  cta_or_cluster_sync(C);
   for (int c = 0; c < crank; ++c) {
-    w_out += cnt[c] + (need > w_eq ? min(need - w_eq, cnt[8 + c]) : 0u);
-    w_eq += cnt[8 + c];
+    tk_before += cnt[16 + c];
+    te_before += cnt[24 + c];
   }
-  for (int w = 0; w < warp; ++w) {
-    w_out += wgt[w] + (need > w_eq ? min(need - w_eq, weq[w]) : 0u);
-    w_eq += weq[w];
-  }
-  // 128 keys per round: lane j holds keys 4j..4j+3 of the round (index order = lane order).
-  // Few keys are taken (topk of the row): a warp with none skips the loop, a round with none
-  // skips the scans.
-  const bool warp_has = wgt[warp] + weq[warp] != 0;
-  for (int b0 = w0; warp_has && b0 < w1; b0 += 128) {
-    const int i4 = b0 + lane * 4;
-    const uint4 k = i4 < w1 ? key4_at(i4) : make_uint4(0, 0, 0, 0);
-    const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
-    uint32_t gtm = 0, eqm = 0;
+  if (grow_hist != nullptr && crank == 0)         // every CTA has read it: zero for reuse
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) grow_hist[i] = 0;
+  for (int blk = b0; blk < b1; ++blk) {
+    uint32_t t[4], e[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (i4 + e < w1) {
-        const uint32_t km = kk[e] & mask;
-        gtm |= (km > prefix ? 1u : 0u) << e;
-        eqm |= (km == prefix ? 1u : 0u) << e;
-      }
+    for (int q = 0; q < 4; ++q) {
+      t[q] = bm_take[4 * blk + q];
+      e[q] = bm_tie[4 * blk + q];
     }
-    if (!__any_sync(0xffffffffu, (gtm | eqm) != 0)) continue;   // nothing here: offsets unchanged
-    // counts over the lanes before this one (index order) from one ballot per key slot
-    const uint32_t lt = (1u << lane) - 1u;
-    uint32_t take = gtm | eqm;
-    uint32_t round_eq = 0;
-    if (!all_eq) {
-      uint32_t eq_before = 0;
+    uint32_t any = (t[0] | e[0]) | (t[1] | e[1]) | (t[2] | e[2]) | (t[3] | e[3]);
+    while (any) {                                  // key 4 l + q of the block, l ascending
+      const int l = __ffs(any) - 1;
+      any &= any - 1;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t be = __ballot_sync(0xffffffffu, (eqm >> e) & 1u);
-        eq_before += __popc(be & lt);
-        round_eq += __popc(be);
-      }
-      uint32_t eq_rank = w_eq + eq_before;      // rank of this lane's first key == tau
-      take = gtm;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((eqm >> e) & 1u) {
-          if (eq_rank < need) take |= 1u << e;
-          ++eq_rank;
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pos = 0xFFFFFFFFu;
+        if ((t[q] >> l) & 1u) {
+          pos = tk_before + min(te_before, need);
+          ++tk_before;
+        } else if ((e[q] >> l) & 1u) {
+          if (te_before < need) pos = tk_before + te_before;
+          ++te_before;
         }
-    }
-    uint32_t before = 0, round_take = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t bt = __ballot_sync(0xffffffffu, (take >> e) & 1u);
-      before += __popc(bt & lt);
-      round_take += __popc(bt);
-    }
-    uint32_t pos = w_out + before;
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if ((take >> e) & 1u) {
-        if (pos < static_cast<uint32_t>(K)) out[pos] = s0 + i4 + e;
-        ++pos;
+        if (pos < static_cast<uint32_t>(K)) out[pos] = s0 + blk * 128 + 4 * l + q;
       }
-    w_out += round_take;
-    if (!all_eq) w_eq += round_eq;
+    }
   }
+  // no CTA may leave while a peer can still write into its shared memory: the last remote
+  // writes were the counts above, ordered before the barrier that every CTA has passed
 }
 
 }  // namespace dsa

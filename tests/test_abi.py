@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(dsa):
     for n in declared_symbols():
         assert hasattr(lib, n), n
     assert set(dsa.EXPORTED) >= set(declared_symbols())
-    assert dsa.abi_version() == 1
+    assert dsa.abi_version() == 2
     assert dsa.status_string(0) == "ok"
     assert "workspace" in dsa.status_string(3)
 
@@ -201,24 +201,96 @@ def test_forward_workspace_plan_on_the_host(dsa):
     size = dsa.dsa_forward_workspace_size_for
     # decode_B64_N128k shapes, contiguous caches: 128 attention CTAs fill one wave of 148 SMs,
     # so no split-KV partials
+    # (+ the fused indexer's first-digit histograms: 2048 words per row of a chunk)
+    H = 2048 * 4
     dec = dsa.make_problem(mode="decode", num_kv_rows=64 * 131072, seqlens=[131072] * 64,
                            seq_lens=FAKE, max_seqlen=131072, **full)
-    assert size(dec, 148) == 64 * 131072 * 4 + 64 * 2048 * 4
+    assert size(dec, 148) == 64 * 131072 * 4 + 64 * 2048 * 4 + 64 * H
     # a few long decode rows on many SMs are split, and the partials add to the workspace
     few = dsa.make_problem(mode="decode", num_kv_rows=2 * 131072, seqlens=[131072] * 2,
                            seq_lens=FAKE, max_seqlen=131072, **full)
-    assert size(few, 148) > 2 * 131072 * 4 + 2 * 2048 * 4
+    assert size(few, 148) > 2 * 131072 * 4 + 2 * 2048 * 4 + 2 * H
     # prefill: 131072 rows need 512 rows of scores per 256 MiB; 148 SMs -> 444 (6 x 74) rows
     pre = dsa.make_problem(mode="prefill", num_kv_rows=131072, seqlens=[131072],
                            cu_seqlens=FAKE, **full)
-    assert size(pre, 148) == 444 * 131072 * 4 + 444 * 2048 * 4
-    assert size(pre, 132) == 462 * 131072 * 4 + 462 * 2048 * 4       # 7 x 66 rows
+    assert size(pre, 148) == 444 * 131072 * 4 + 444 * 2048 * 4 + 444 * H
+    assert size(pre, 132) == 462 * 131072 * 4 + 462 * 2048 * 4 + 462 * H   # 7 x 66 rows
     # a short sequence runs in one chunk; varlen sizes the slab for the largest chunk's scores
     # and the indices for the chunk with the most rows (here the short sequence's 1000)
     short = dsa.make_problem(mode="prefill", num_kv_rows=1000, seqlens=[1000], cu_seqlens=FAKE,
                              **full)
-    assert size(short, 148) == 1000 * 1000 * 4 + 1000 * 2048 * 4
+    assert size(short, 148) == 1000 * 1000 * 4 + 1000 * 2048 * 4 + 1000 * H
     mix = dsa.make_problem(mode="prefill", num_kv_rows=132072, seqlens=[1000, 131072],
                            cu_seqlens=FAKE, **full)
-    assert size(mix, 148) == 444 * 131072 * 4 + 1000 * 2048 * 4
+    assert size(mix, 148) == 444 * 131072 * 4 + 1000 * 2048 * 4 + 1000 * H
+    # the small indexer shape builds its histograms in the top-k: none in the workspace
+    tiny = dsa.make_problem(mode="prefill", num_kv_rows=1024, seqlens=[1024], cu_seqlens=FAKE,
+                            h_idx=4, d_idx=32, h=16, d_qk=160, d_v=128, topk=64,
+                            softmax_scale=0.08)
+    assert size(tiny, 148) == 1024 * 1024 * 4 + 1024 * 64 * 4
     assert size(pre, 0) == 0 and size(_pb(dsa, topk=100), 148) == 0
+    # the chunk plan itself: rows per chunk of each sequence
+    rows = dsa.dsa_forward_chunk_rows_for
+    assert rows(pre, 0, 148) == 444 and rows(pre, 0, 132) == 462
+    assert rows(mix, 0, 148) == 1000 and rows(mix, 1, 148) == 444
+    assert rows(mix, 2, 148) == 0 and rows(dec, 0, 148) == 64
+
+
+def test_noalloc_partials_fit_the_builtin_array_for_every_batch(dsa):
+    """The allocation-free attention entry point sizes its split-KV partials to its built-in
+    array: for every decode batch of 1..4096 rows at full shapes, on 148 and 132 SMs, the capped
+    choice fits DSA_NOALLOC_SCRATCH_BYTES, equals the uncapped choice whenever that one fits,
+    and falls back to no partials at all otherwise."""
+    full = dict(h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512, topk=2048, softmax_scale=0.04)
+    cap = dsa.NOALLOC_SCRATCH_BYTES
+    per_split_row = 128 * 513 * 4
+    for sms in (148, 132):
+        for rows in range(1, 4097):
+            pb = dsa.make_problem(mode="decode", num_kv_rows=rows * 8192, seqlens=[8192] * rows,
+                                  seq_lens=FAKE, max_seqlen=8192, **full)
+            free = dsa.dsa_sparse_mla_workspace_size_for(pb, rows, sms)
+            capped = dsa.dsa_sparse_mla_workspace_size_for(pb, rows, sms, cap)
+            assert capped <= cap, (sms, rows, capped)
+            if free <= cap:
+                assert capped == free, (sms, rows)
+            assert capped == 0 or (capped - 256) % (rows * per_split_row) == 0
+    # the bound at full shapes: splits * rows * 128 * 513 * 4 + 256 <= 20 MiB -> <= 79 row-splits
+    assert (cap - 256) // per_split_row == 79
+
+
+def test_fused_indexer_topk_arguments(dsa):
+    """dsa_indexer_topk: workspace sizing on the host (slab of the rows at max_seqlen keys plus
+    2048 histogram words per row) and argument errors before any launch."""
+    pb = _pb(dsa)
+    need = dsa.dsa_indexer_topk_workspace_size(pb, 2)
+    assert need == 2 * 4096 * 4 + 2 * 2048 * 4
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE]        # q_idx, q_scale, w, k_idx, k_scale
+
+    def call(p, a, rb=0, n=2, idx=FAKE, ws=FAKE, wsb=None):
+        return dsa.dsa_indexer_topk(p, *a, rb, n, idx, ws, need if wsb is None else wsb, None, 0)
+
+    assert call(pb, args, idx=None) == dsa.DSA_ERR_INVALID_ARG
+    assert call(pb, [None] + args[1:]) == dsa.DSA_ERR_INVALID_ARG
+    assert call(pb, args, wsb=need - 1) == dsa.DSA_ERR_WORKSPACE_TOO_SMALL
+    assert call(pb, args, ws=None) == dsa.DSA_ERR_WORKSPACE_TOO_SMALL
+    assert call(pb, args, ws=FAKE + 8) == dsa.DSA_ERR_MISALIGNED
+    assert call(pb, args, rb=1) == dsa.DSA_ERR_INVALID_ARG
+    assert call(_pb(dsa, h_idx=32), args) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+    assert call(pb, args, n=0) == dsa.DSA_OK        # nothing to do, nothing launched
+
+
+def test_stage_histogram_arguments(dsa):
+    """The optional first-digit histograms of dsa_indexer_scores / dsa_topk: 16-byte alignment,
+    and only the 64 x 128 indexer counts them."""
+    pb = _pb(dsa)
+    st = dsa.dsa_indexer_scores(pb, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE, 4096, None, 0,
+                                hist=FAKE + 4)
+    assert st == dsa.DSA_ERR_MISALIGNED
+    st = dsa.dsa_topk(pb, FAKE, 4096, 0, 2, FAKE, None, 0, hist=FAKE + 4)
+    assert st == dsa.DSA_ERR_MISALIGNED
+    tiny = dsa.make_problem(mode="prefill", num_kv_rows=1024, seqlens=[1024], cu_seqlens=FAKE,
+                            h_idx=4, d_idx=32, h=16, d_qk=160, d_v=128, topk=64,
+                            softmax_scale=0.08)
+    st = dsa.dsa_indexer_scores(tiny, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE, 1024, None, 0,
+                                hist=FAKE)
+    assert st == dsa.DSA_ERR_UNSUPPORTED_SHAPE

@@ -351,7 +351,7 @@ def _check_forward(wl, f, rows, overlap_min=0.999):
 def test_forward_tiny_prefill_all_rows(dsa):
     wl = make_config(1, device="cuda")
     f = _forward(dsa, wl)
-    _check_forward(wl, f, list(range(0, 1024, 3)) + [1023])
+    _check_forward(wl, f, list(range(wl.total_rows)))
 
 
 def test_forward_small_decode_full_dims(dsa):
@@ -366,6 +366,38 @@ def test_forward_small_prefill_full_dims(dsa):
     f = _forward(dsa, wl)
     rows = [0, 1, 63, 2046, 2047, 2048, 2100, 2499, 2500, 2799]
     _check_forward(wl, f, rows)
+
+
+# ------------------------------------------------------ per-head query scales of the indexer
+
+def per_head_q_scale(wl, seed):
+    """The workload with a different fp32 scale for every (query row, indexer head): the
+    generator draws one scale per token (copied over the heads); here each head's scale is
+    multiplied by its own seeded power-of-two-spread factor in [1/8, 8).  Both sides read the
+    same modified array."""
+    g = torch.Generator(device=wl.q_scale.device).manual_seed(seed)
+    f = torch.exp2(torch.rand(wl.q_scale.shape, generator=g, device=wl.q_scale.device) * 6 - 3)
+    wl.q_scale = (wl.q_scale * f).contiguous()
+    assert (wl.q_scale[:, 0] != wl.q_scale[:, 1]).any()
+    return wl
+
+
+def test_indexer_per_head_q_scale(dsa):
+    _indexer_case(dsa, per_head_q_scale(make_config(1, device="cuda"), 5), list(range(1024)))
+    wl = make_prefill(11, [130, 7, 600, 1, 515], FULL, needles=8, device="cuda")
+    _indexer_case(dsa, per_head_q_scale(wl, 6), list(range(wl.total_rows)))
+    for lay in ("separate", "interleaved"):
+        wl = make_decode(17, 5, [3000, 64, 1, 200, 131], FULL, boost=0.01, paged=True,
+                         device="cuda", scale_layout=lay)
+        _indexer_case(dsa, per_head_q_scale(wl, 7), list(range(5)))
+
+
+def test_forward_per_head_q_scale(dsa):
+    wl = per_head_q_scale(make_decode(21, 5, [7000, 2048, 2049, 100, 1], FULL, boost=0.01,
+                                      paged=True, device="cuda"), 8)
+    _check_forward(wl, _forward(dsa, wl), [0, 1, 2, 3, 4])
+    wl = per_head_q_scale(make_prefill(22, [2500, 300], FULL, needles=8, device="cuda"), 9)
+    _check_forward(wl, _forward(dsa, wl), [0, 1, 63, 2046, 2047, 2048, 2100, 2499, 2500, 2799])
 
 
 # --------------------------------------------------------------- dense (short-row) attention

@@ -3,10 +3,12 @@
 dsa_sparse_mla_fwd_noalloc exists for callers that may not allocate device memory at all (work
 recorded into a CUDA graph, runtimes that own every byte through a fixed pool, plugins whose host
 forbids allocator calls on the hot path).  It keeps its split-KV partials in a scratch array built
-into the library instead of a caller workspace.  This test runs it on a few decode rows (few rows,
-so the partials path and therefore the built-in scratch is used), twice in a row with different
-selections, and compares each result with dsa_sparse_mla_fwd given a normal workspace, within the
-attention tolerance of the parity tests.  The file is named so that pytest collects it last.
+into the library instead of a caller workspace, choosing a split count whose partials fit it.  This
+test runs it on decode batches of 3 rows (split, the partials in the built-in scratch), 37 rows
+(the largest split batch that still fits), 40 rows (whose unconstrained split would not fit, so it
+runs with fewer splits) and 64 rows (unsplit), twice in a row with different selections, and
+compares each result with dsa_sparse_mla_fwd given a normal workspace, within the attention
+tolerance of the parity tests.  The file is named so that pytest collects it last.
 """
 import pytest
 import torch
@@ -27,21 +29,27 @@ def _selection(lens, k, seed):
     return idx.cuda()
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+def _lens(rows):
+    base = [6000, 2048, 300]
+    return base if rows == 3 else [base[i % 3] + 37 * i for i in range(rows)]
+
+
+@pytest.mark.parametrize("rows", [3, 37, 40, 64])
+def test_noalloc_matches_workspace_entry_point_on_two_calls(rows):
     import sparse_attention_long_04_b200 as dsa
-    lens = [6000, 2048, 300]
+    lens = _lens(rows)
     wl = make_decode(41, len(lens), lens, FULL, boost=0.0, paged=True, device="cuda")
     pb = dsa.problem_of(wl)
-    rows = len(lens)
     ws_bytes = dsa.dsa_sparse_mla_workspace_size(pb, rows)
-    assert 0 < ws_bytes <= dsa.NOALLOC_SCRATCH_BYTES      # the path that needs scratch
+    if rows == 3:
+        assert 0 < ws_bytes <= dsa.NOALLOC_SCRATCH_BYTES      # the path that needs scratch
     d = wl.dims
     for call, seed in enumerate((1, 2)):
         idx = _selection(lens, d["topk"], seed)
         ref_out = torch.full((rows, d["h"], d["d_v"]), float("nan"), dtype=torch.bfloat16,
                              device="cuda")
         ref_lse = torch.full((rows, d["h"]), float("nan"), device="cuda")
-        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
         assert dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, idx, 0, rows, ref_out, ref_lse, ws,
                                       ws_bytes) == dsa.DSA_OK
         out = torch.full_like(ref_out, float("nan"))
