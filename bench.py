@@ -410,6 +410,7 @@ def run_ours(args, rank, world, local_rank):
     }
     line["cache_append"] = time_cache_append(args, dsa, wl, stream, peaks,
                                              cpu_leg=rank == 0 and not args.no_cpu)
+    line["probes"] = {"dsmem": probe_dsmem(dsa, dev, stream)}
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     del step, out, lse, wl
@@ -771,6 +772,24 @@ def time_cache_append(args, dsa, wl, stream, peaks, cpu_leg):
         res["cpu_baseline"] = {"us_per_call": round((time.perf_counter() - t0) / reps * 1e6, 1),
                                "kind": "oracle", "cores": 1,
                                "sample": f"the same {B} tokens, host caches"}
+    return res
+
+
+def probe_dsmem(dsa, dev, stream, nbytes=32 * 1024, reps=256):
+    """Distributed-shared-memory exchange rate between the two CTAs (two SMs) of a cluster, both
+    directions at once: one cluster alone and one per SM pair; per SM = bytes it sends / time."""
+    sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    res = {"bytes_per_round": nbytes, "rounds": reps}
+    for name, clusters in (("one_pair", 1), ("all_pairs", sm // 2)):
+        ns = torch.zeros(clusters, dtype=torch.int64, device=dev)
+        bad = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(2):   # the first launch warms up
+            dsa.check(dsa.dsa_probe_dsmem(clusters, nbytes, reps, ns, bad, stream), "dsmem probe")
+        torch.cuda.synchronize()
+        dsa.check(0 if int(bad.item()) == 0 else dsa.DSA_ERR_CUDA, "dsmem probe words")
+        t = ns.double().mean().item()
+        res[name] = {"clusters": clusters, "gbs_per_sm": round(nbytes * reps / t, 2),
+                     "gbs_total": round(2 * clusters * nbytes * reps / t, 1)}
     return res
 
 

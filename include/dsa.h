@@ -196,9 +196,9 @@ DSA_API size_t dsa_sparse_mla_workspace_size_for(const dsa_dims_t* dims, const d
  *   kv   bf16 [num_kv_rows, d_qk]
  *   idx  int32 [row_count, topk] logical key indices (-1 = unused), relative to row_begin,
  *        or NULL: every prior key of each row (dense causal attention), which is exactly the
- *        top-k's selection when no row has more than topk prior keys; with NULL a row range
- *        holding a row with more than topk prior keys (decode: max_seqlen > topk) returns
- *        DSA_ERR_INVALID_ARG
+ *        top-k's selection when no row has more than topk prior keys, and the dense model's
+ *        attention (the training's warm-up stage) when rows are longer.  PREFILL rows of any
+ *        length; DECODE with NULL needs max_seqlen <= topk (else DSA_ERR_INVALID_ARG)
  *   out  bf16 [total_rows, h, d_v] and lse fp32 [total_rows, h] (absolute rows); a row
  *        with no valid index gets out = 0 and lse = -inf. */
 DSA_API dsa_status_t dsa_sparse_mla_fwd(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
@@ -357,6 +357,37 @@ DSA_API dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_s
                                              float* dq, float* dk, int32_t* dev_status,
                                              dsa_stream_t stream);
 
+/* The dense warm-up stage of the indexer's training ("DeepSeek V3.2-Exp Cuts Long-Context Costs
+ * with DeepSeek Sparse Attention (DSA)", "Training signal": before the sparse stage the indexer
+ * learns to imitate the dense attention, over every prior key).  PREFILL only.  The entries of
+ * query row t are its keys 0..pos(t), in position order; target rows have one entry per key.
+ *
+ * Target: target[t - row_begin, s] = (1/h) sum_h exp(sigma q[t,h,:] . kv[s,:] - lse[t,h]) for
+ * s <= pos(t), with lse from dsa_sparse_mla_fwd with idx = NULL (the dense attention of the
+ * same rows).  target fp32 [row_count, ld_target], ld_target a multiple of 64 (else
+ * DSA_ERR_MISALIGNED), at least topk and the longest row's key count rounded up to 64 (else
+ * DSA_ERR_INVALID_ARG); entries past pos(t) are 0 or left untouched. */
+DSA_API dsa_status_t dsa_indexer_kl_target_dense(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                                 const uint16_t* q, const uint16_t* kv,
+                                                 const float* lse, int32_t row_begin,
+                                                 int32_t row_count, float* target,
+                                                 int64_t ld_target, int32_t* dev_status,
+                                                 dsa_stream_t stream);
+
+/* Loss and gradients of the same KL as dsa_indexer_kl_backward, over every prior key of each row
+ * (entry s = key s, target [row_count, ld_target] as written by dsa_indexer_kl_target_dense,
+ * ld_target a multiple of 4 and at least the longest row's key count).  Outputs as for
+ * dsa_indexer_kl_backward.  The (64, 128) indexer takes rows of any length; the (4, 32) shape
+ * rows of at most 2048 keys (else DSA_ERR_UNSUPPORTED_SHAPE). */
+DSA_API dsa_status_t dsa_indexer_kl_backward_dense(const dsa_dims_t* dims,
+                                                   const dsa_seqs_t* seqs, const uint8_t* q_idx,
+                                                   const float* q_scale, const float* w,
+                                                   const uint8_t* k_idx, const float* k_scale,
+                                                   const float* target, int64_t ld_target,
+                                                   int32_t row_begin, int32_t row_count,
+                                                   float* loss, float* dw, float* dq, float* dk,
+                                                   int32_t* dev_status, dsa_stream_t stream);
+
 /* Synchronises `stream`, reads the device status word and maps it: 0 -> DSA_OK,
  * DSA_DEVICE_TIMEOUT -> DSA_ERR_TIMEOUT, DSA_DEVICE_BAD_INDEX -> DSA_ERR_BAD_INDEX.
  * *raw (optional, host) receives the word. */
@@ -370,6 +401,17 @@ DSA_API dsa_status_t dsa_read_device_status(const int32_t* dev_status, dsa_strea
  * context usable.  Asynchronous on `stream`, which stays busy for about 2 s; read the word with
  * dsa_read_device_status, which then returns DSA_ERR_TIMEOUT. */
 DSA_API dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream);
+
+/* Diagnostics: the rate of distributed-shared-memory traffic between the two CTAs of a cluster,
+ * the figure that decides whether the two CTAs of an attention row can exchange partial logits
+ * instead of each computing all of them.  Launches `clusters` clusters of two 512-thread CTAs
+ * (one CTA per SM); the two CTAs of each cluster store `bytes` (a multiple of 16, at most the
+ * device's shared memory per CTA) of 16-byte words into each other's shared memory `reps` times,
+ * both at once.  ns (device, uint64 [clusters]) receives each cluster's exchange time in
+ * nanoseconds; bad (device int32, zero it first) receives the count of words that did not land
+ * as written (0 expected).  Asynchronous on `stream`. */
+DSA_API dsa_status_t dsa_probe_dsmem(int32_t clusters, int32_t bytes, int32_t reps, uint64_t* ns,
+                                     int32_t* bad, dsa_stream_t stream);
 
 DSA_API const char* dsa_status_string(dsa_status_t status);
 DSA_API int32_t dsa_abi_version(void);

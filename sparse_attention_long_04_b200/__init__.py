@@ -44,7 +44,8 @@ EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_indexer_kl_target", "dsa_indexer_kl_backward", "dsa_forward_workspace_size_for",
             "dsa_sparse_mla_workspace_size_for", "dsa_indexer_topk",
             "dsa_indexer_topk_workspace_size", "dsa_forward_chunk_rows_for",
-            "dsa_forward_rows")
+            "dsa_forward_rows", "dsa_indexer_kl_target_dense", "dsa_indexer_kl_backward_dense",
+            "dsa_probe_dsmem")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -92,7 +93,11 @@ def _load():
         "dsa_forward_rows": (I32, [DP, SP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_selftest_wait_timeout": (I32, [P, P]),
+        "dsa_probe_dsmem": (I32, [I32, I32, I32, P, P, P]),
         "dsa_indexer_kl_target": (I32, [DP, SP, P, P, P, P, I32, I32, P, P, P]),
+        "dsa_indexer_kl_target_dense": (I32, [DP, SP, P, P, P, I32, I32, P, I64, P, P]),
+        "dsa_indexer_kl_backward_dense": (I32, [DP, SP, P, P, P, P, P, P, I64, I32, I32, P, P, P,
+                                                P, P, P]),
         "dsa_indexer_kl_backward": (I32, [DP, SP, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P,
                                           P]),
         "dsa_status_string": (ctypes.c_char_p, [I32]),
@@ -311,8 +316,28 @@ def dsa_indexer_kl_backward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, idx,
         _ptr(dw), _ptr(dq), _ptr(dk), _ptr(dev_status), _stream(stream)))
 
 
+def dsa_indexer_kl_target_dense(pb: Problem, q, kv, lse, row_begin: int, row_count: int, target,
+                                ld_target: int, dev_status=None, stream=None) -> int:
+    return int(lib.dsa_indexer_kl_target_dense(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q), _ptr(kv), _ptr(lse), row_begin,
+        row_count, _ptr(target), ld_target, _ptr(dev_status), _stream(stream)))
+
+
+def dsa_indexer_kl_backward_dense(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, target,
+                                  ld_target: int, row_begin: int, row_count: int, loss, dw, dq,
+                                  dk, dev_status=None, stream=None) -> int:
+    return int(lib.dsa_indexer_kl_backward_dense(
+        ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
+        _ptr(k_idx), _ptr(k_scale), _ptr(target), ld_target, row_begin, row_count, _ptr(loss),
+        _ptr(dw), _ptr(dq), _ptr(dk), _ptr(dev_status), _stream(stream)))
+
+
 def dsa_selftest_wait_timeout(dev_status, stream=None) -> int:
     return int(lib.dsa_selftest_wait_timeout(_ptr(dev_status), _stream(stream)))
+
+
+def dsa_probe_dsmem(clusters: int, bytes_: int, reps: int, ns, bad, stream=None) -> int:
+    return int(lib.dsa_probe_dsmem(clusters, bytes_, reps, _ptr(ns), _ptr(bad), _stream(stream)))
 
 
 def dsa_read_device_status(dev_status, stream=None):

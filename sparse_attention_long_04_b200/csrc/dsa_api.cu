@@ -177,9 +177,17 @@ int64_t max_keys(const dsa_seqs_t* s, int32_t row_begin, int32_t row_count) {
   return m;
 }
 
-// Without an index array sparse attention runs dense: every prior key of each row, which is only
-// the top-k's selection when no row has more than topk prior keys.
+// Without an index array attention runs dense: every prior key of each row (the top-k's
+// selection when no row has more than topk prior keys; dense causal attention in general).
+// Decode rows take at most topk keys that way (resolved through the block table up front);
+// prefill rows of any length (their keys are consecutive packed rows, streamed past topk).
 bool dense_ok(const dsa_dims_t& d, const dsa_seqs_t* s, int32_t row_begin, int32_t row_count) {
+  return s->mode == DSA_PREFILL || max_keys(s, row_begin, row_count) <= d.topk;
+}
+
+// The training target without indices writes topk entries per row: rows of at most topk keys.
+bool dense_target_ok(const dsa_dims_t& d, const dsa_seqs_t* s, int32_t row_begin,
+                     int32_t row_count) {
   return max_keys(s, row_begin, row_count) <= d.topk;
 }
 
@@ -509,6 +517,7 @@ MlaParams mla_params(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q
   prm.block_size = d.block_size > 0 ? d.block_size : 64;
   prm.num_kv_rows = s.num_kv_rows;
   prm.status = status;
+  prm.ld_target = d.topk;
   return prm;
 }
 
@@ -618,13 +627,14 @@ int target_splits(const dsa_dims_t& d, int32_t row_count, int sm_count) {
 template <int D_QK, int D_V>
 dsa_status_t target_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
                          const uint16_t* kv, const int32_t* idx, const float* lse,
-                         int32_t row_begin, int32_t row_count, float* target, int32_t* status,
-                         cudaStream_t st, int sm_count) {
+                         int32_t row_begin, int32_t row_count, float* target, int64_t ld_target,
+                         int32_t* status, cudaStream_t st, int sm_count) {
   using C = MlaCfg<D_QK, D_V>;
   const int splits = target_splits(d, row_count, sm_count);
   MlaParams prm = mla_params(d, s, q, kv, idx, row_begin, row_count, splits, status);
   prm.lse_in = lse;
   prm.target = target;
+  prm.ld_target = ld_target;
   CUtensorMap q_map;
   if (make_row_map(&q_map, q, uint64_t(s.total_rows) * d.h, D_QK * 2, 128, 128) != DSA_OK)
     return DSA_ERR_CUDA;
@@ -741,6 +751,79 @@ dsa_status_t forward_window(const dsa_dims_t& d, const dsa_seqs_t& s, int64_t w0
   return DSA_OK;
 }
 
+// ------------------------------------------------------------------- training entry bodies
+
+dsa_status_t kl_target_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* q,
+                            const uint16_t* kv, const int32_t* idx, const float* lse,
+                            int32_t row_begin, int32_t row_count, float* target,
+                            int64_t ld_target, int32_t* status, cudaStream_t st) {
+  if (!mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  dsa_status_t e;
+  if ((e = check_rows(&s, row_begin, row_count)) != DSA_OK) return e;
+  if (!q || !kv || !lse || !target) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(lse) || !aligned16(target))
+    return DSA_ERR_MISALIGNED;
+  if (row_count == 0) return DSA_OK;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  if (d.d_qk == 576)
+    return target_impl<576, 512>(d, s, q, kv, idx, lse, row_begin, row_count, target, ld_target,
+                                 status, st, info.sm_count);
+  return target_impl<160, 128>(d, s, q, kv, idx, lse, row_begin, row_count, target, ld_target,
+                               status, st, info.sm_count);
+}
+
+// idx NULL: dense mode (every prior key of each row, the caller checked the geometry)
+dsa_status_t kl_backward_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
+                              const float* q_scale, const float* w, const uint8_t* k_idx,
+                              const float* k_scale, const int32_t* idx, const float* target,
+                              int64_t ld_target, int32_t row_begin, int32_t row_count,
+                              float* loss, float* dw, float* dq, float* dk, int32_t* status,
+                              cudaStream_t st) {
+  const bool full = d.h_idx == 64 && d.d_idx == 128;
+  const bool tiny = d.h_idx == 4 && d.d_idx == 32;
+  if (!full && !tiny) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (full && d.topk % KlTcCfg::BK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;   // whole key tiles
+  dsa_status_t e;
+  if ((e = check_rows(&s, row_begin, row_count)) != DSA_OK) return e;
+  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !target || !loss || !dw || !dq || !dk)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx) || !aligned16(target) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(q_scale) || !aligned16(w) ||
+      !aligned16(k_scale) || !aligned16(loss) || !aligned16(dw))
+    return DSA_ERR_MISALIGNED;
+  if (row_count == 0) return DSA_OK;
+  IdxBwdParams prm{};
+  prm.q_idx = q_idx;
+  prm.q_scale = q_scale;
+  prm.w = w;
+  prm.k_idx = k_idx;
+  prm.k_scale = k_scale;
+  prm.idx = idx;
+  prm.target = target;
+  prm.ld_target = ld_target;
+  prm.dense = idx == nullptr;
+  prm.loss = loss;
+  prm.dw = dw;
+  prm.dq = dq;
+  prm.dk = dk;
+  prm.row_begin = row_begin;
+  prm.row_count = row_count;
+  prm.topk = d.topk;
+  prm.decode = s.mode == DSA_DECODE;
+  prm.batch = s.batch;
+  prm.cu_seqlens = s.cu_seqlens;
+  prm.seq_lens = s.seq_lens;
+  prm.block_table = s.block_table;
+  prm.max_blocks = s.max_blocks;
+  prm.kv_stride = s.max_seqlen;
+  prm.max_seqlen = s.max_seqlen;
+  prm.block_size = d.block_size > 0 ? d.block_size : 64;
+  prm.num_kv_rows = s.num_kv_rows;
+  prm.status = status;
+  return kl_backward_launch(full, prm, st);
+}
+
 // ---------------------------------------------------------------- bounded-wait self-test
 
 // One CTA waits on an mbarrier that nothing arrives at, with the wait every kernel here uses
@@ -760,6 +843,48 @@ __global__ void __launch_bounds__(64) dsa_selftest_wait_kernel(int32_t* status) 
     abort_flag = 1;
     atomicOr(status, kStatusTimeout);
   }
+}
+
+// ------------------------------------------------------- distributed shared memory probe
+
+// Each cluster of two CTAs (one per SM) exchanges `bytes` of its shared memory with its partner
+// `reps` times over distributed shared memory: every thread stores 16-byte words into the
+// partner's buffer (st.shared::cluster.v4), both CTAs at once, the traffic pattern of a logit
+// exchange between the two CTAs of an attention row.  ns[cluster] = the exchange time of the
+// cluster (%globaltimer between two cluster barriers, CTA 0); after the last round every CTA
+// checks that its buffer holds its partner's last pattern and adds the mismatching words to *bad.
+constexpr int kProbeThreads = 512;
+__global__ void __launch_bounds__(kProbeThreads) dsa_probe_dsmem_kernel(int32_t bytes,
+                                                                       int32_t reps,
+                                                                       uint64_t* ns,
+                                                                       int32_t* bad) {
+  extern __shared__ __align__(16) uint8_t probe_smem[];
+  uint4* buf = reinterpret_cast<uint4*>(probe_smem);
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int words = bytes / 16;
+  const uint32_t dst = map_to_rank(smem_u32(buf), peer);
+  cluster_sync();
+  const uint64_t t0 = global_timer_ns();
+  for (int r = 0; r < reps; ++r) {
+    for (int j = threadIdx.x; j < words; j += kProbeThreads) {
+      const uint32_t v = (uint32_t(r) << 20) ^ (uint32_t(j) << 1) ^ rank;
+      asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + j * 16),
+                   "r"(v), "r"(v + 1u), "r"(v + 2u), "r"(v + 3u)
+                   : "memory");
+    }
+  }
+  cluster_sync();
+  const uint64_t t1 = global_timer_ns();
+  if (rank == 0 && threadIdx.x == 0) ns[blockIdx.x / 2] = t1 - t0;
+  int miss = 0;
+  for (int j = threadIdx.x; j < words; j += kProbeThreads) {
+    const uint32_t v = (uint32_t(reps - 1) << 20) ^ (uint32_t(j) << 1) ^ peer;
+    const uint4 w = buf[j];
+    miss += (w.x != v) + (w.y != v + 1u) + (w.z != v + 2u) + (w.w != v + 3u);
+  }
+  if (miss) atomicAdd(bad, miss);
+  cluster_sync();   // no CTA leaves while its partner may still read nothing of it (symmetry)
 }
 
 }  // namespace
@@ -1013,21 +1138,27 @@ dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seqs_t* seq
   NvtxRange nvtx_range("dsa_indexer_kl_target");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
-  if (!mla_shape_ok(*dims)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (idx == nullptr && !dense_target_ok(*dims, seqs, row_begin, row_count))
+    return DSA_ERR_INVALID_ARG;
+  return kl_target_impl(*dims, *seqs, q, kv, idx, lse, row_begin, row_count, target, dims->topk,
+                        dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_indexer_kl_target_dense(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                         const uint16_t* q, const uint16_t* kv, const float* lse,
+                                         int32_t row_begin, int32_t row_count, float* target,
+                                         int64_t ld_target, int32_t* dev_status,
+                                         dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_indexer_kl_target_dense");
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (seqs->mode != DSA_PREFILL) return DSA_ERR_INVALID_ARG;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
-  if (!q || !kv || !lse || !target) return DSA_ERR_INVALID_ARG;
-  if (idx == nullptr && !dense_ok(*dims, seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(lse) || !aligned16(target))
-    return DSA_ERR_MISALIGNED;
-  if (row_count == 0) return DSA_OK;
-  DeviceInfo info;
-  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dims->d_qk == 576)
-    return target_impl<576, 512>(*dims, *seqs, q, kv, idx, lse, row_begin, row_count, target,
-                                 dev_status, st, info.sm_count);
-  return target_impl<160, 128>(*dims, *seqs, q, kv, idx, lse, row_begin, row_count, target,
-                               dev_status, st, info.sm_count);
+  if (ld_target % 64 != 0) return DSA_ERR_MISALIGNED;
+  if (ld_target < (max_keys(seqs, row_begin, row_count) + 63) / 64 * 64 || ld_target < dims->topk)
+    return DSA_ERR_INVALID_ARG;
+  return kl_target_impl(*dims, *seqs, q, kv, nullptr, lse, row_begin, row_count, target,
+                        ld_target, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
@@ -1039,49 +1170,32 @@ dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* s
   NvtxRange nvtx_range("dsa_indexer_kl_backward");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
-  const dsa_dims_t& d = *dims;
-  const dsa_seqs_t& s = *seqs;
-  const bool full = d.h_idx == 64 && d.d_idx == 128;
-  const bool tiny = d.h_idx == 4 && d.d_idx == 32;
-  if (!full && !tiny) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (full && d.topk % KlTcCfg::BK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;   // whole key tiles
+  if (idx == nullptr) return DSA_ERR_INVALID_ARG;
+  return kl_backward_impl(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, idx, target,
+                          dims->topk, row_begin, row_count, loss, dw, dq, dk, dev_status,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_indexer_kl_backward_dense(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
+                                           const uint8_t* q_idx, const float* q_scale,
+                                           const float* w, const uint8_t* k_idx,
+                                           const float* k_scale, const float* target,
+                                           int64_t ld_target, int32_t row_begin,
+                                           int32_t row_count, float* loss, float* dw, float* dq,
+                                           float* dk, int32_t* dev_status, dsa_stream_t stream) {
+  NvtxRange nvtx_range("dsa_indexer_kl_backward_dense");
+  dsa_status_t e = check_common(dims, seqs);
+  if (e != DSA_OK) return e;
+  if (seqs->mode != DSA_PREFILL) return DSA_ERR_INVALID_ARG;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
-  if (!q_idx || !q_scale || !w || !k_idx || !k_scale || !idx || !target || !loss || !dw || !dq ||
-      !dk)
-    return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx) || !aligned16(target) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(q_scale) || !aligned16(w) ||
-      !aligned16(k_scale) || !aligned16(loss) || !aligned16(dw))
-    return DSA_ERR_MISALIGNED;
-  if (row_count == 0) return DSA_OK;
-  IdxBwdParams prm{};
-  prm.q_idx = q_idx;
-  prm.q_scale = q_scale;
-  prm.w = w;
-  prm.k_idx = k_idx;
-  prm.k_scale = k_scale;
-  prm.idx = idx;
-  prm.target = target;
-  prm.loss = loss;
-  prm.dw = dw;
-  prm.dq = dq;
-  prm.dk = dk;
-  prm.row_begin = row_begin;
-  prm.row_count = row_count;
-  prm.topk = d.topk;
-  prm.decode = s.mode == DSA_DECODE;
-  prm.batch = s.batch;
-  prm.cu_seqlens = s.cu_seqlens;
-  prm.seq_lens = s.seq_lens;
-  prm.block_table = s.block_table;
-  prm.max_blocks = s.max_blocks;
-  prm.kv_stride = s.max_seqlen;
-  prm.max_seqlen = s.max_seqlen;
-  prm.block_size = d.block_size > 0 ? d.block_size : 64;
-  prm.num_kv_rows = s.num_kv_rows;
-  prm.status = dev_status;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return kl_backward_launch(full, prm, st);
+  if (ld_target % 4 != 0) return DSA_ERR_MISALIGNED;
+  const int64_t longest = max_keys(seqs, row_begin, row_count);
+  if (ld_target < longest) return DSA_ERR_INVALID_ARG;
+  // the CUDA-core kernel of the small shape keeps every entry in shared memory
+  if (dims->h_idx == 4 && longest > IdxBwdCfg<4, 32>::MAX_K) return DSA_ERR_UNSUPPORTED_SHAPE;
+  return kl_backward_impl(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, nullptr, target,
+                          ld_target, row_begin, row_count, loss, dw, dq, dk, dev_status,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream) {
@@ -1089,6 +1203,35 @@ dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t stream)
   if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
     return DSA_ERR_MISALIGNED;
   dsa_selftest_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(dev_status);
+  return launch_status();
+}
+
+dsa_status_t dsa_probe_dsmem(int32_t clusters, int32_t bytes, int32_t reps, uint64_t* ns,
+                             int32_t* bad, dsa_stream_t stream) {
+  if (clusters <= 0 || reps <= 0 || bytes <= 0 || bytes % 16 != 0 || !ns || !bad)
+    return DSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ns) & 7u) != 0 || (reinterpret_cast<uintptr_t>(bad) & 3u) != 0)
+    return DSA_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  // at least 116 KB each, so that one CTA runs per SM: the two CTAs of a pair sit on two SMs
+  const int smem = std::max(bytes, 116 * 1024);
+  if (smem > info.max_smem - 1024) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (prepare_kernel(dsa_probe_dsmem_kernel, smem) != DSA_OK) return DSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+  cfg.blockDim = dim3(kProbeThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dsa_probe_dsmem_kernel, bytes, reps, ns, bad) != cudaSuccess)
+    return DSA_ERR_CUDA;
   return launch_status();
 }
 

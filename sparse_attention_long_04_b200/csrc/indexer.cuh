@@ -11,7 +11,8 @@
 //   D[key, (row, head)] = K_tile[128 x D_I] * Q_group[N x D_I]^T,   N = QPG * H_I
 // with e4m3 operands in 128-byte (or 32-byte for D_I = 32) swizzled shared memory and an fp32
 // accumulator in Tensor Memory (TMEM lane = key).  Each epilogue thread then owns one key and
-// reduces its row's heads with no cross-thread traffic: 2 ALU ops (max, fma) per head.
+// reduces its row's heads with no cross-thread traffic: per head a max (the ReLU) and half of a
+// packed fp32x2 FMA (two heads per instruction).
 //
 // Roles: warp 0 issues TMA (Q once, then per tile two 64-row key boxes plus a bulk copy of each
 // box's k_scale), warp 1 issues the tcgen05.mma, warp 2 owns the TMEM allocation, warp 3
@@ -189,6 +190,9 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // decode streams the key cache once: evict-first, so that the score slab the top-k reads
+      // next stays in L2
+      const uint64_t pol = l2_evict_first();
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&qmap);
       mbar_arrive_expect_tx(smem_u32(qbar), C::Q_BYTES);
@@ -254,10 +258,11 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
             for (int hlf = 0; hlf < 2; ++hlf) {
               if (!ok[hlf]) continue;
               const int64_t blk = y[hlf] / 64;
-              tma_load_3d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
-                          smem_u32(&full[s]), 0, 0, static_cast<int32_t>(blk));
-              bulk_load_g2s(smem_u32(sbuf + hlf * 80),
-                            p.k_blocks + blk * kBlockBytes + 64 * D_I, 256, smem_u32(&full[s]));
+              tma_load_3d_hint(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
+                               smem_u32(&full[s]), 0, 0, static_cast<int32_t>(blk), pol);
+              bulk_load_g2s_hint(smem_u32(sbuf + hlf * 80),
+                                 p.k_blocks + blk * kBlockBytes + 64 * D_I, 256,
+                                 smem_u32(&full[s]), pol);
             }
           } else {
           // each box's 64 scales: a 16-byte-aligned superset of the rows, inside the cache
@@ -276,11 +281,11 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
           mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
           for (int hlf = 0; hlf < 2; ++hlf) {
             if (ok[hlf])
-              tma_load_2d(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
-                          smem_u32(&full[s]), 0, static_cast<int32_t>(y[hlf]));
+              tma_load_2d_hint(smem_u32(sK + s * C::TILE_BYTES + hlf * 64 * D_I), &kmap,
+                               smem_u32(&full[s]), 0, static_cast<int32_t>(y[hlf]), pol);
             if (sb[hlf] > 0)
-              bulk_load_g2s(smem_u32(sbuf + hlf * 80), p.k_scale + a0[hlf], sb[hlf],
-                            smem_u32(&full[s]));
+              bulk_load_g2s_hint(smem_u32(sbuf + hlf * 80), p.k_scale + a0[hlf], sb[hlf],
+                                 smem_u32(&full[s]), pol);
           }
           }
         }
@@ -328,6 +333,7 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
     const int grp = (warp - 4) / 4;          // warpgroup
     const int part = C::TILE_SPLIT ? 0 : grp;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint64_t slab_pol = l2_evict_last();   // the decode slab stays in L2 for the top-k
     for (int it = C::TILE_SPLIT ? grp : 0; it < n_tiles; it += C::TILE_SPLIT ? 2 : 1) {
       const int a = it % C::ACC;
       const int s = it % C::STAGES;
@@ -374,29 +380,34 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
         constexpr int CPR = H_I / 32;          // chunks per query row
 #pragma unroll
         for (int q = 0; q < NCH / CPR; ++q) {
-          float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+          // heads in pairs: one packed fp32x2 FMA per two heads (ReLU stays scalar)
+          float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int c = q * CPR; c < (q + 1) * CPR; ++c) {
             const float4* cc = reinterpret_cast<const float4*>(sC + part * COLS + c * 32);
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               const float4 c4 = cc[j / 4];
-              acc4[0] = fmaf(c4.x, fmaxf(__uint_as_float(r[c][j + 0]), 0.f), acc4[0]);
-              acc4[1] = fmaf(c4.y, fmaxf(__uint_as_float(r[c][j + 1]), 0.f), acc4[1]);
-              acc4[2] = fmaf(c4.z, fmaxf(__uint_as_float(r[c][j + 2]), 0.f), acc4[2]);
-              acc4[3] = fmaf(c4.w, fmaxf(__uint_as_float(r[c][j + 3]), 0.f), acc4[3]);
+              a01 = __ffma2_rn(make_float2(c4.x, c4.y),
+                               make_float2(fmaxf(__uint_as_float(r[c][j + 0]), 0.f),
+                                           fmaxf(__uint_as_float(r[c][j + 1]), 0.f)),
+                               a01);
+              a23 = __ffma2_rn(make_float2(c4.z, c4.w),
+                               make_float2(fmaxf(__uint_as_float(r[c][j + 2]), 0.f),
+                                           fmaxf(__uint_as_float(r[c][j + 3]), 0.f)),
+                               a23);
             }
           }
           const int rr = (part * COLS) / H_I + q;
           if (rr < rows_in_group && key <= pos_first + rr) {
-            const float sc = ks * ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]));
+            const float sc = ks * ((a01.x + a01.y) + (a23.x + a23.y));
             p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] = sc;
             if (hist_on) atomicAdd(&sHist[rr * kIdxHistBins + (order_key(sc) >> 21)], 1u);
           }
         }
         continue;
       }
-      float acc = 0.f;
+      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);   // heads in pairs
 #pragma unroll 1
       for (int c0 = 0; c0 < COLS; c0 += 32) {
         const int col = part * COLS + c0;
@@ -408,19 +419,27 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
             const float4 c4 = cc[j / 4];
-            acc = fmaf(c4.x, fmaxf(__uint_as_float(r[j + 0]), 0.f), acc);
-            acc = fmaf(c4.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), acc);
-            acc = fmaf(c4.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), acc);
-            acc = fmaf(c4.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), acc);
+            a01 = __ffma2_rn(make_float2(c4.x, c4.y),
+                             make_float2(fmaxf(__uint_as_float(r[j + 0]), 0.f),
+                                         fmaxf(__uint_as_float(r[j + 1]), 0.f)),
+                             a01);
+            a23 = __ffma2_rn(make_float2(c4.z, c4.w),
+                             make_float2(fmaxf(__uint_as_float(r[j + 2]), 0.f),
+                                         fmaxf(__uint_as_float(r[j + 3]), 0.f)),
+                             a23);
           }
           if ((col + 32) % H_I == 0) {       // a query row's heads are complete
             const int rr = col / H_I;
+            const float acc = (a01.x + a01.y) + (a23.x + a23.y);
+            a01 = make_float2(0.f, 0.f);
+            a23 = make_float2(0.f, 0.f);
             if (rr < rows_in_group && key <= pos_first + rr) {
               const float sc = ks * acc;
-              p.scores[static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key] = sc;
+              float* dst = p.scores + static_cast<int64_t>(p.out_row0 + (grow0 - p.row0) + rr) * p.ld + key;
+              if (C::TILE_SPLIT) st_global_hint(dst, sc, slab_pol);   // decode: read next
+              else *dst = sc;
               if (hist_on) atomicAdd(&sHist[rr * kIdxHistBins + (order_key(sc) >> 21)], 1u);
             }
-            acc = 0.f;
           }
         } else {
 #pragma unroll

@@ -30,6 +30,7 @@
 // coef[e][j] = g_e w_j [D > 0] in shared memory; dw accumulates in registers, dk (lanes over
 // dims, per key) goes out with coalesced atomic adds, and dq (warp = 8 heads, lane = dims
 // l + 32 c) accumulates in registers over all chunks.  Chunks without a valid key are skipped.
+// Dense mode (no index array): the entries are the row's keys 0..pos(t), at most MAX_K.
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -62,6 +63,8 @@ struct IdxBwdParams {
   int32_t block_size;
   int64_t num_kv_rows;
   int32_t* status;
+  int64_t ld_target;           // target row stride (topk; dense: >= every row's key count)
+  int32_t dense;               // 1: every prior key of each row (prefill), no idx
 };
 
 template <int H_I, int D_I>
@@ -137,9 +140,6 @@ __global__ void __launch_bounds__(256, 2) dsa_indexer_kl_bwd_kernel(const IdxBwd
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int r = blockIdx.x;
   const int row = p.row_begin + r;
-  const int K = p.topk;
-  const int n_chunks = K / C::CH;
-
   // ---- row geometry
   int b, n_keys;
   int64_t key_base = 0;
@@ -157,6 +157,10 @@ __global__ void __launch_bounds__(256, 2) dsa_indexer_kl_bwd_kernel(const IdxBwd
     n_keys = row - p.cu_seqlens[lo] + 1;
     key_base = p.cu_seqlens[lo];
   }
+  // entries of the row: the selection (topk slots), or in dense mode its keys 0..pos (at most
+  // MAX_K, checked by the caller), padded to whole chunks
+  const int K = p.dense ? (min(n_keys, C::MAX_K) + C::CH - 1) / C::CH * C::CH : p.topk;
+  const int n_chunks = K / C::CH;
 
   // ---- queries (real-valued) and weights into shared memory
   {
@@ -176,9 +180,9 @@ __global__ void __launch_bounds__(256, 2) dsa_indexer_kl_bwd_kernel(const IdxBwd
   // ---- selected keys -> physical rows (-1: unused or out of range)
   {
     bool bad = false;
-    const int32_t* irow = p.idx + static_cast<int64_t>(r) * K;
+    const int32_t* irow = p.dense ? nullptr : p.idx + static_cast<int64_t>(r) * K;
     for (int e = tid; e < K; e += C::THREADS) {
-      const int v = __ldg(irow + e);
+      const int v = p.dense ? (e < n_keys ? e : -1) : __ldg(irow + e);
       int64_t ph = -1;
       if (v >= n_keys) bad = true;
       if (v >= 0 && v < n_keys) {
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(256, 2) dsa_indexer_kl_bwd_kernel(const IdxBwd
   __syncthreads();
 
   // ---- softmax, loss and g = dloss/dS
-  const float* trow = p.target + static_cast<int64_t>(r) * K;
+  const float* trow = p.target + static_cast<int64_t>(r) * p.ld_target;
   float m = -INFINITY;
   for (int e = tid; e < K; e += C::THREADS) m = fmaxf(m, sG[e]);
   m = block_reduce<true>(m, sScr);

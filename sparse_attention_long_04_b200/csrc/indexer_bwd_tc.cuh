@@ -16,12 +16,20 @@
 // warp 1 owns TMEM, warps 2-3 gather the selected key rows (16-byte cp.async into 128-byte-
 // swizzled tiles, two stages; unused keys are zero-filled), warps 4-7 are the epilogue with
 // thread = TMEM lane.  Pass 1 runs D^T for every tile and the epilogue forms the scores S
-// (thread = key); the 128 epilogue threads then take the softmax, the loss and g.  Pass 2 runs
-// D^T again per tile; the epilogue writes A1 (TMEM, thread = key), B2 (shared memory, row =
-// key) and Kh^T (TMEM, thread = dim, read column-wise out of the key tile), sums dw over the
-// tile's keys with a butterfly across lanes, and after the dk/dq MMAs adds its key's dk row to
-// global memory with 16-byte atomic adds.  At the end thread = dim writes dq.  Every wait is
-// bounded.
+// (thread = key), keeping per thread the running softmax statistics of its keys (max, the sum
+// of exp(S - max), and the target's sum, sum p S and sum p ln p); the 128 epilogue threads then
+// combine them into the normaliser and the loss.  No per-key value is stored, so a row may have
+// any number of entries.  Pass 2 runs D^T again per tile, recomputes S with the same
+// instructions (so the same value and ReLU decisions), forms g; the epilogue writes A1 (TMEM,
+// thread = key), B2 (shared memory, row = key) and Kh^T (TMEM, thread = dim, read column-wise
+// out of the key tile), sums dw over the tile's keys with a butterfly across lanes, and after
+// the dk/dq MMAs adds its key's dk row to global memory with 16-byte atomic adds.  At the end
+// thread = dim writes dq.  Every wait is bounded.
+//
+// Dense mode (the warm-up stage of the training, "Training signal": the indexer imitates the
+// dense attention over every prior key): no index array; the entries of row t are its keys
+// 0..pos(t) (prefill: consecutive packed rows), in 128-key tiles computed on the fly, and the
+// target row has one entry per key.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -50,8 +58,7 @@ struct KlTcCfg {
   static constexpr int OFF_QB = OFF_Q8 + H * D;                // [2 dim blocks][64 heads][128 B]
   static constexpr int OFF_KT = OFF_QB + 2 * H * 128;          // [STAGES][128 keys][128 B] e4m3
   static constexpr int OFF_B2 = OFF_KT + STAGES * TILE_BYTES;  // [hi, lo][128 keys][128 B] bf16
-  static constexpr int OFF_S = OFF_B2 + 2 * BK * 128;          // [MAX_K] f32: S, then g
-  static constexpr int OFF_PHYS = OFF_S + 4 * MAX_K;           // [MAX_K] i32
+  static constexpr int OFF_PHYS = OFF_B2 + 2 * BK * 128;       // [MAX_K] i32 (selected keys)
   static constexpr int OFF_TILES = OFF_PHYS + 4 * MAX_K;       // [MAX_TILES] i32
   static constexpr int OFF_W = OFF_TILES + 4 * MAX_TILES;      // [64] w
   static constexpr int OFF_SQ = OFF_W + 4 * H;                 // [64] s_q
@@ -90,7 +97,6 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
   uint8_t* sQb = smem + C::OFF_QB;
   uint8_t* sKt = smem + C::OFF_KT;
   uint8_t* sB2 = smem + C::OFF_B2;
-  float* sS = reinterpret_cast<float*>(smem + C::OFF_S);
   int32_t* sPhys = reinterpret_cast<int32_t*>(smem + C::OFF_PHYS);
   int32_t* sTiles = reinterpret_cast<int32_t*>(smem + C::OFF_TILES);
   float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
@@ -114,7 +120,7 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int r = blockIdx.x;
   const int row = p.row_begin + r;
-  const int K = p.topk;
+  const bool dense = p.dense != 0;
 
   // ---- row geometry
   int b, n_keys;
@@ -153,7 +159,8 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     sW[tid] = __ldg(p.w + static_cast<int64_t>(row) * C::H + tid);
     sSq[tid] = __ldg(p.q_scale + static_cast<int64_t>(row) * C::H + tid);
   }
-  {
+  const int K = dense ? n_keys : p.topk;   // entries of the row
+  if (!dense) {
     bool bad = false;
     const int32_t* irow = p.idx + static_cast<int64_t>(r) * K;
     for (int e = tid; e < K; e += C::THREADS) {
@@ -172,7 +179,6 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
         if (ph < 0) bad = true;
       }
       sPhys[e] = static_cast<int32_t>(ph);
-      sS[e] = -INFINITY;
     }
     if (bad && p.status) atomicOr(p.status, kStatusBadIndex);
   }
@@ -196,13 +202,23 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
   __syncthreads();
   if (tid == 0) {
     int n = 0;
-    for (int t = 0; t < K / C::BK; ++t) {
-      bool any = false;
-      for (int e = 0; e < C::BK && !any; ++e) any = sPhys[t * C::BK + e] >= 0;
-      if (any) sTiles[n++] = t;
+    if (dense) {
+      n = (n_keys + C::BK - 1) / C::BK;
+    } else {
+      for (int t = 0; t < K / C::BK; ++t) {
+        bool any = false;
+        for (int e = 0; e < C::BK && !any; ++e) any = sPhys[t * C::BK + e] >= 0;
+        if (any) sTiles[n++] = t;
+      }
     }
     n_act_s = n;
   }
+  // tile of step i and physical row of entry e (-1: unused entry)
+  auto tile_at = [&](int i) -> int { return dense ? i : sTiles[i]; };
+  auto phys_at = [&](int e) -> int64_t {
+    if (!dense) return sPhys[e];
+    return e < n_keys ? key_base + e : -1;
+  };
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -274,12 +290,12 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
         ok = false;
         break;
       }
-      const int tile = sTiles[it % n];
+      const int tile = tile_at(it % n);
       const uint32_t dst = smem_u32(sKt + s * C::TILE_BYTES);
 #pragma unroll 4
       for (int q = 0; q < C::BK / 8; ++q) {
         const int rr = r0 + 8 * q;
-        const int32_t ph = sPhys[tile * C::BK + rr];
+        const int64_t ph = phys_at(tile * C::BK + rr);
         const void* src = ph >= 0 ? static_cast<const void*>(p.k_idx + static_cast<int64_t>(ph) *
                                                                          C::D + c * 16)
                                   : static_cast<const void*>(p.k_idx);
@@ -304,7 +320,19 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       return r2;
     };
     bool ok = true;
-    // ---- pass 1: S_e = s_k sum_j w_j s_q,j max(D_je, 0), thread = key
+    // ---- pass 1: S_e = s_k sum_j w_j s_q,j max(D_je, 0), thread = key; running statistics
+    const float* trow = p.target + static_cast<int64_t>(r) * p.ld_target;
+    // (explicitly rounded products: pass 2 must get the bits of pass 1, so the compiler may not
+    // fuse them into the arithmetic that follows either call)
+    auto score = [&](const uint32_t (&du)[2][32], int64_t ph) -> float {
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < C::H; ++j)
+        acc = fmaf(__fmul_rn(sW[j], sSq[j]), fmaxf(__uint_as_float(du[j >> 5][j & 31]), 0.f),
+                   acc);
+      return __fmul_rn(__ldg(p.k_scale + ph), acc);
+    };
+    float m = -INFINITY, z = 0.f, psum = 0.f, sps = 0.f, splp = 0.f;
     for (int it = 0; it < n && ok; ++it) {
       const int s = it % C::STAGES;
       ok = warp_mbar_wait(smem_u32(d_full), it & 1, &abort_s);
@@ -317,54 +345,48 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       tc_fence_before();
       mbar_arrive(smem_u32(d_empty));
       mbar_arrive(smem_u32(&kempty[s]));
-      const int e = sTiles[it] * C::BK + et;
-      const int32_t ph = sPhys[e];
-      float acc = 0.f;
-#pragma unroll
-      for (int j = 0; j < C::H; ++j)
-        acc = fmaf(sW[j] * sSq[j], fmaxf(__uint_as_float(du[j >> 5][j & 31]), 0.f), acc);
-      sS[e] = ph >= 0 ? __ldg(p.k_scale + ph) * acc : -INFINITY;
+      const int e = tile_at(it) * C::BK + et;
+      const int64_t ph = phys_at(e);
+      if (ph >= 0) {
+        const float S = score(du, ph);
+        if (S > m) {
+          z = z * expf(m - S) + 1.f;
+          m = S;
+        } else {
+          z += expf(S - m);
+        }
+        const float pe = __ldg(trow + e);
+        psum += pe;
+        sps += pe * S;
+        if (pe > 0.f) splp += pe * logf(pe);
+      }
     }
-    // ---- softmax over the selection, loss, g (each thread owns entries et + 128 q)
-    const float* trow = p.target + static_cast<int64_t>(r) * K;
-    float m = -INFINITY;
-    for (int e = et; e < K; e += C::BK) m = fmaxf(m, sS[e]);
-    m = warp_max(m);
-    if (lane == 0) sScr[ew] = m;
+    // ---- the row's normaliser and loss from the 128 threads' statistics
+    const float wm = warp_max(m);
+    float zz = m == -INFINITY ? 0.f : z * expf(m - wm);
+    zz = warp_sum(zz);
+    psum = warp_sum(psum);
+    sps = warp_sum(sps);
+    splp = warp_sum(splp);
+    if (lane == 0) {
+      sScr[ew] = wm;
+      sScr[4 + ew] = zz;
+      sScr[8 + ew] = psum;
+      sScr[12 + ew] = sps;
+      sScr[16 + ew] = splp;
+    }
     ok = ok && epi_sync();
     m = fmaxf(fmaxf(sScr[0], sScr[1]), fmaxf(sScr[2], sScr[3]));
-    float z = 0.f, psum = 0.f;
-    if (m != -INFINITY)
-      for (int e = et; e < K; e += C::BK)
-        if (sPhys[e] >= 0) {
-          z += expf(sS[e] - m);
-          psum += __ldg(trow + e);
-        }
-    z = warp_sum(z);
-    psum = warp_sum(psum);
-    if (lane == 0) {
-      sScr[4 + ew] = z;
-      sScr[8 + ew] = psum;
-    }
-    ok = ok && epi_sync();
-    z = (sScr[4] + sScr[5]) + (sScr[6] + sScr[7]);
+    z = 0.f;
+#pragma unroll
+    for (int w4 = 0; w4 < 4; ++w4)
+      if (sScr[w4] != -INFINITY) z += sScr[4 + w4] * expf(sScr[w4] - m);
     psum = (sScr[8] + sScr[9]) + (sScr[10] + sScr[11]);
+    sps = (sScr[12] + sScr[13]) + (sScr[14] + sScr[15]);
+    splp = (sScr[16] + sScr[17]) + (sScr[18] + sScr[19]);
     const float log_z = m == -INFINITY ? 0.f : m + logf(z);
-    float l = 0.f;
-    for (int e = et; e < K; e += C::BK) {
-      float g = 0.f;
-      if (sPhys[e] >= 0) {
-        const float pe = __ldg(trow + e);
-        const float log_pi = sS[e] - log_z;
-        if (pe > 0.f) l += pe * (logf(pe) - log_pi);
-        g = expf(log_pi) * psum - pe;
-      }
-      sS[e] = g;
-    }
-    l = warp_sum(l);
-    if (lane == 0) sScr[12 + ew] = l;
-    ok = ok && epi_sync();
-    if (et == 0) p.loss[r] = (sScr[12] + sScr[13]) + (sScr[14] + sScr[15]);
+    // loss = sum p (ln p - ln pi), ln pi = S - log_z
+    if (et == 0) p.loss[r] = (m == -INFINITY || !ok) ? 0.f : splp - sps + psum * log_z;
 
     // ---- pass 2: coefficients, dw, dk; dq accumulates in TMEM
     const int h0 = warp_sum64_first(lane);   // this lane's two heads of the warp's dw sums
@@ -380,9 +402,10 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(d_empty));
-      const int e = sTiles[i2] * C::BK + et;
-      const int32_t ph = sPhys[e];
-      const float g = sS[e];                                   // 0 for unused keys
+      const int e = tile_at(i2) * C::BK + et;
+      const int64_t ph = phys_at(e);
+      // g = pi psum - p, from the same score as in pass 1 (0 for unused entries)
+      const float g = ph >= 0 ? expf(score(du, ph) - log_z) * psum - __ldg(trow + e) : 0.f;
       const float gsk = ph >= 0 ? g * __ldg(p.k_scale + ph) : 0.f;
       // dw: g s_k max(D, 0) summed over the tile's keys (s_q applied at the end)
       {

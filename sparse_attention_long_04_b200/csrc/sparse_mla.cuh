@@ -32,7 +32,9 @@
 // the keys, then gather rows [16w, 16w + 16) of every tile: warps 8-11 the QK-only dims,
 // warps 12-15 the value dims.  Grid: x = 2 * row + v, y = split-KV slice.
 // Without an index array the selection is every prior key (dense causal attention), which is
-// what the top-k keeps whenever a row has at most topk prior keys.
+// what the top-k keeps whenever a row has at most topk prior keys.  A dense row with more keys
+// than topk (prefill only: its keys are consecutive packed rows) is streamed: its tiles, their
+// valid-key masks and physical rows are computed on the fly instead of resolved up front.
 //
 // Target mode (kTarget): the indexer's training target on the same selection, the main
 // attention's distribution summed over heads and normalised ("DeepSeek V3.2-Exp Cuts
@@ -74,7 +76,8 @@ struct MlaParams {
   int64_t num_kv_rows;
   int32_t* status;
   const float* lse_in;         // target mode: the forward's LSE [T, H]
-  float* target;               // target mode: [row_count, topk], relative to row_begin
+  float* target;               // target mode: [row_count, ld_target], relative to row_begin
+  int64_t ld_target;           // target mode: row stride (topk; dense: >= the longest row)
 };
 
 template <int D_QK, int D_V>
@@ -85,6 +88,7 @@ struct MlaCfg {
   static constexpr int KK = KB_ALL - VKB;             // QK-only k-blocks
   static constexpr int BN = 64;                       // keys per tile
   static constexpr int STAGES = 2;
+  static constexpr int PREFETCH = 3;                  // tiles ahead whose rows go to L2
   static constexpr int MAX_TILES = 32;                // topk <= 2048
   static constexpr int THREADS = 512;
   static constexpr int S_COL = V_HALF;
@@ -171,6 +175,18 @@ __global__ void __launch_bounds__(512, 1)
     key_base = p.cu_seqlens[lo];
   }
 
+  // a dense prefill row longer than the resolved-key arrays: tiles computed on the fly
+  const bool stream_dense = dense && !p.decode && n_keys > p.topk;
+  __shared__ int t0_s;
+  auto tile_at = [&](int i) -> int {
+    return stream_dense ? t0_s + (kTarget ? 2 * i + vh : i) : sTiles[i];
+  };
+  auto mask_of = [&](int t) -> uint64_t {
+    if (!stream_dense) return sMask[t];
+    const int rem = n_keys - t * C::BN;
+    return rem >= C::BN ? ~0ull : ((1ull << rem) - 1ull);
+  };
+
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(smem_u32(&k_full[i]), 128);
@@ -203,7 +219,7 @@ __global__ void __launch_bounds__(512, 1)
       tma_load_2d(smem_u32(dst), &q_map, smem_u32(q_bar), kb * 128, row * p.h);
     }
   }
-  if (warp >= 8) {
+  if (warp >= 8 && !stream_dense) {
     // ---- every selected key -> physical row (or -1): 8 keys per thread, all index loads in
     // flight together, then all block-table loads
     const int t = threadIdx.x - 256;
@@ -243,7 +259,7 @@ __global__ void __launch_bounds__(512, 1)
     if (bad_idx && p.status) atomicOr(p.status, kStatusBadIndex);
   }
   __syncthreads();
-  if (warp >= 8) {
+  if (warp >= 8 && !stream_dense) {
     // ---- per tile: the valid-key mask; invalid keys borrow the tile's first valid row
     for (int tt = warp - 8; tt < n_tiles_all; tt += 8) {
       int32_t* ph = sPhys + tt * C::BN;
@@ -259,8 +275,9 @@ __global__ void __launch_bounds__(512, 1)
         if (a1 < 0) ph[32 + lane] = fb;
       }
       if (lane == 0) sMask[tt] = m;
-      if (kTarget && m == 0 && vh == 0 && split == 0) {   // no valid key: targets are 0
-        float* tg = p.target + static_cast<int64_t>(r) * p.topk + tt * C::BN;
+      if (kTarget && m == 0 && vh == 0 && split == 0 &&   // no valid key: targets are 0
+          static_cast<int64_t>(tt + 1) * C::BN <= p.ld_target) {
+        float* tg = p.target + static_cast<int64_t>(r) * p.ld_target + tt * C::BN;
         tg[lane] = 0.f;
         tg[32 + lane] = 0.f;
       }
@@ -270,17 +287,27 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 0 && lane == 0) {
     // ---- the active tiles of this split, identical in both CTAs of the row
     int cnt = 0;
-    for (int t = 0; t < n_tiles_all; ++t)
-      if (sMask[t] != 0) {
-        sTiles[cnt] = t;
-        ++cnt;
-      }
+    if (stream_dense) {
+      cnt = (n_keys + C::BN - 1) / C::BN;
+    } else {
+      for (int t = 0; t < n_tiles_all; ++t)
+        if (sMask[t] != 0) {
+          sTiles[cnt] = t;
+          ++cnt;
+        }
+    }
     const int per = (cnt + p.splits - 1) / p.splits;
     const int t0 = min(cnt, split * per);
     const int t1 = min(cnt, t0 + per);
     int m = 0;   // target mode: the two CTAs of a row take alternate tiles
-    for (int i = t0; i < t1; ++i)
-      if (!kTarget || ((i - t0) & 1) == vh) sTiles[m++] = sTiles[i];
+    if (stream_dense) {
+      t0_s = t0;
+      m = kTarget ? (t1 - t0 - vh + 1) / 2 : t1 - t0;
+      if (m < 0) m = 0;
+    } else {
+      for (int i = t0; i < t1; ++i)
+        if (!kTarget || ((i - t0) & 1) == vh) sTiles[m++] = sTiles[i];
+    }
     n_act_s = m;
   }
   if (warp >= 4 && warp < 8) {
@@ -400,12 +427,12 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* full = part == 0 ? k_full : v_full;
     uint64_t* empty = part == 0 ? k_empty : v_empty;
     // one tile's part: rows [16 pw, 16 pw + 16), NKB k-blocks (latent-row block kb_of(ks))
-    auto copy_part = [&](auto nkb_c, uint8_t* dst, const int32_t* ph, auto kb_of) {
+    auto copy_part = [&](auto nkb_c, uint8_t* dst, auto phys_of, auto kb_of) {
       constexpr int NKB = decltype(nkb_c)::value;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int rr = rsub + 4 * j;
-        const __nv_bfloat16* src = p.kv + static_cast<int64_t>(ph[rr]) * D_QK + ch * 8;
+        const __nv_bfloat16* src = p.kv + phys_of(rr) * D_QK + ch * 8;
         const uint32_t drow = smem_u32(dst) + sw128_offset(pw * 16 + rr, ch);
 #pragma unroll
         for (int ks = 0; ks < NKB; ++ks) {
@@ -426,14 +453,43 @@ __global__ void __launch_bounds__(512, 1)
         ok = false;
         break;
       }
-      const int32_t* ph = sPhys + sTiles[i] * C::BN + pw * 16;
+      const int tile = tile_at(i);
+      const int32_t* ph = sPhys + tile * C::BN + pw * 16;
+      // physical row of row rr of this warp's 16: resolved up front, or (streamed dense rows)
+      // consecutive packed rows, keys past the row borrowing the tile's first key
+      auto phys_of = [&](int rr) -> int64_t {
+        if (!stream_dense) return ph[rr];
+        const int key = tile * C::BN + pw * 16 + rr;
+        return key_base + (key < n_keys ? key : tile * C::BN);
+      };
       if (part == 0)   // the QK-only k-blocks: all but this CTA's value blocks
-        copy_part(std::integral_constant<int, C::KK>{}, sK + s * C::K_SLOT_BYTES, ph,
+        copy_part(std::integral_constant<int, C::KK>{}, sK + s * C::K_SLOT_BYTES, phys_of,
                   [&](int ks) { return ks < vh * C::VKB ? ks : ks + C::VKB; });
       else             // this CTA's value k-blocks
-        copy_part(std::integral_constant<int, C::VKB>{}, sV + s * C::V_SLOT_BYTES, ph,
+        copy_part(std::integral_constant<int, C::VKB>{}, sV + s * C::V_SLOT_BYTES, phys_of,
                   [&](int ks) { return vh * C::VKB + ks; });
       cp_async_arrive_noinc(smem_u32(&full[s]));
+      // the rows of the tile PREFETCH steps ahead into L2 (its slot is not free yet): one
+      // thread per row of the K-part warps, each CTA of the pair half of the row, so that the
+      // gather of that tile reads L2 instead of HBM
+      if (part == 0 && i + C::PREFETCH < n) {
+        const int t2 = tile_at(i + C::PREFETCH);
+        const int rr = (warp - 8) * 32 + lane;      // 0..127: rows 0..63 only
+        if (rr < C::BN) {
+          int64_t row2;
+          if (!stream_dense) {
+            row2 = sPhys[t2 * C::BN + rr];
+          } else {
+            const int key = t2 * C::BN + rr;
+            row2 = key_base + (key < n_keys ? key : t2 * C::BN);
+          }
+          constexpr uint32_t kHalf = (D_QK * 2 / 2 + 15) / 16 * 16;
+          const uint32_t off = vh * kHalf;
+          const uint32_t bytes = vh == 0 ? kHalf : D_QK * 2 - kHalf;
+          if (bytes > 0)
+            prefetch_l2(reinterpret_cast<const uint8_t*>(p.kv + row2 * D_QK) + off, bytes);
+        }
+      }
     }
     if (!ok) {
       abort_s = 1;
@@ -465,7 +521,7 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_empty));
-      const uint64_t vmask = sMask[sTiles[i]];
+      const uint64_t vmask = mask_of(tile_at(i));
       float v[64];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -490,7 +546,7 @@ __global__ void __launch_bounds__(512, 1)
       if (w4 == 0) {
         ok = (warp_mbar_wait(smem_u32(&red_full[buf]), (i >> 1) & 1, &abort_s));
         if (!ok) break;
-        float* tg = p.target + static_cast<int64_t>(r) * p.topk + sTiles[i] * C::BN;
+        float* tg = p.target + static_cast<int64_t>(r) * p.ld_target + tile_at(i) * C::BN;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int e = lane + 32 * c;
@@ -521,7 +577,7 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_empty));
-      const uint64_t vmask = sMask[sTiles[i]];
+      const uint64_t vmask = mask_of(tile_at(i));
       // the tile max of the unscaled logits (sigma log2 e > 0), as 8 independent partial maxima
       float mm[8];
 #pragma unroll

@@ -13,7 +13,8 @@
 //      finds the bin b holding the k-th largest key and the count above it.
 //   2. One classifying pass over the slice: keys of a bin above b are taken (a bit in the
 //      slice's "taken" bitmap); keys of bin b are candidates, kept in shared memory with their
-//      positions.  When bin b holds exactly the keys still needed, all of it is taken instead.
+//      positions, each warp in its own region (no shared counter).  When bin b holds exactly
+//      the keys still needed, all of it is taken instead.
 //      Bitmap layout: a block of 128 keys is 4 words; key 4 l + e of the block is bit l of word
 //      e, so that lane l of a warp reading the block as float4 contributes bit l of each word.
 //   3. The candidates of the cluster are few (1-6k): their keys go to CTA 0, which resolves the
@@ -54,6 +55,7 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 2048;
 constexpr int kTopkLocal = 4096;     // candidates (key, position) a CTA keeps
+constexpr int kTopkPerWarp = kTopkLocal / kTopkWarps;   // each warp's own candidate region
 constexpr int kTopkGather = 12288;   // candidate keys CTA 0 gathers from the cluster
 constexpr int kTopkFixedSmem =
     2 * kTopkBins * 4 + 2 * kTopkLocal * 4 + kTopkGather * 4 + 512;
@@ -68,6 +70,17 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
   if ((u << 1) == 0) u = 0;                       // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The smallest float whose order key is >= t (t <= 2^32): scores compare against it as floats
+// exactly as their keys compare against t.  NaN (no float reaches it) for t = 2^32 or inside the
+// NaN range of positive keys; -inf when only NaN patterns lie below t (negative keys).
+__device__ __forceinline__ float key_floor_float(uint64_t t) {
+  if (t >= (uint64_t(1) << 32)) return __int_as_float(0x7fffffff);
+  const uint32_t k = static_cast<uint32_t>(t);
+  if (k & 0x80000000u) return __uint_as_float(k & 0x7fffffffu);
+  const float f = __uint_as_float(~k);
+  return f != f ? -INFINITY : f;
 }
 
 // Bitmap position of key i of a slice (see the layout above).
@@ -172,7 +185,8 @@ __device__ __forceinline__ void cta_or_cluster_sync(int C) {
   if (C > 1) cluster_sync(); else __syncthreads();
 }
 
-__global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams p) {
+// two CTAs per SM (64 registers a thread): a row's slices fill one wave in decode
+__global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
   uint32_t* hsum = reinterpret_cast<uint32_t*>(topk_smem);          // [kTopkBins] row / digit
   uint32_t* hloc = hsum + kTopkBins;                                 // [kTopkBins] this slice
@@ -185,13 +199,22 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   uint32_t* bm_take = reinterpret_cast<uint32_t*>(topk_smem + kTopkFixedSmem);  // [words]
   const int words = (p.slice + 31) / 32;
   uint32_t* bm_tie = bm_take + words;                                // [words]
-  __shared__ uint32_t s_bin, s_above, s_nloc, s_over;
+  __shared__ uint32_t s_bin, s_above, s_over;
+  __shared__ uint32_t s_wcnt[kTopkWarps];          // candidates of each warp (its region)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = p.csize;
   const int crank = static_cast<int>(blockIdx.x) % C;
   const int r = blockIdx.x / C;
   const int row = p.row_begin + r;
+  uint32_t* grow_hist = p.hist ? p.hist + static_cast<int64_t>(r) * kTopkBins : nullptr;
+  // the row's first-digit counts are loaded before anything else (their latency then overlaps
+  // the row geometry's)
+  constexpr int kHpt = kTopkBins / kTopkThreads;
+  uint32_t hreg[kHpt];
+  if (grow_hist != nullptr)
+#pragma unroll
+    for (int j = 0; j < kHpt; ++j) hreg[j] = __ldcg(grow_hist + j * kTopkThreads + tid);
   int n;
   if (p.decode) {
     n = p.seq_lens[row];
@@ -209,7 +232,6 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   }
   const float* srow = p.scores + static_cast<int64_t>(r) * p.ld;
   int32_t* out = p.idx + static_cast<int64_t>(r) * p.topk;
-  uint32_t* grow_hist = p.hist ? p.hist + static_cast<int64_t>(r) * kTopkBins : nullptr;
   const int K = p.topk;
   if (n <= K) {                                    // uniform over the cluster: no barrier used
     for (int j = crank * kTopkThreads + tid; j < K; j += C * kTopkThreads)
@@ -228,14 +250,12 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
     bm_take[i] = 0;
     bm_tie[i] = 0;
   }
-  if (tid == 0) {
-    s_nloc = 0;
-    s_over = 0;
-  }
+  if (tid == 0) s_over = 0;
 
   // ---- 1. first digit
   if (grow_hist != nullptr) {
-    for (int i = tid; i < kTopkBins; i += kTopkThreads) hsum[i] = __ldcg(grow_hist + i);
+#pragma unroll
+    for (int j = 0; j < kHpt; ++j) hsum[j * kTopkThreads + tid] = hreg[j];
     __syncthreads();
   } else {
     for (int i = tid; i < kTopkBins; i += kTopkThreads) {
@@ -262,6 +282,14 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
   uint32_t prefix = bin << 21, mask = 0xFFE00000u;
 
   // ---- 2. classify the slice: above the bin -> taken; in the bin -> candidate
+  // (take: key >= t_hi, candidate: t_lo <= key < t_hi; compared as floats, the keys' order,
+  // through the smallest float of each threshold's bin)
+  const uint32_t t_lo = bin << 21;
+  const uint64_t t_hi = whole_bin ? uint64_t(bin) << 21 : (uint64_t(bin) + 1) << 21;
+  const float f_lo = key_floor_float(t_lo), f_hi = key_floor_float(t_hi);
+  uint32_t* wkey = ckey + warp * kTopkPerWarp;
+  int32_t* wpos = cpos + warp * kTopkPerWarp;
+  uint32_t wn = 0;                                 // this warp's candidates so far
   constexpr int U = 4;                             // blocks in flight per warp
   for (int rd0 = warp; rd0 < nrounds; rd0 += U * kTopkWarps) {
     float4 v[U];
@@ -276,40 +304,47 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
       const int rd = rd0 + u * kTopkWarps;
       if (rd >= nrounds) break;
       const float ve[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t cw[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = rd * 128 + 4 * lane + e;
-        const uint32_t k = score_key(ve[e]);
-        const uint32_t b = k >> 21;
         const bool in = i < m;
-        const bool take = in && (b > bin || (whole_bin && b == bin));
-        const bool cand = in && !whole_bin && b == bin;
-        const uint32_t tw = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) bm_take[rd * 4 + e] = tw;
-        const uint32_t cw = __ballot_sync(0xffffffffu, cand);
-        if (cw != 0) {
-          uint32_t base = 0;
-          if (lane == 0) base = atomicAdd(&s_nloc, static_cast<uint32_t>(__popc(cw)));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (cand) {
-            const uint32_t slot = base + __popc(cw & ((1u << lane) - 1u));
-            if (slot < static_cast<uint32_t>(kTopkLocal)) {
-              ckey[slot] = k;
-              cpos[slot] = i;
-            } else {
-              s_over = 1;
+        const bool above = ve[e] >= f_hi;
+        const uint32_t tw = __ballot_sync(0xffffffffu, in && above);
+        if (lane == e) bm_take[rd * 4 + e] = tw;
+        cw[e] = __ballot_sync(0xffffffffu, in && !above && ve[e] >= f_lo);
+      }
+      if ((cw[0] | cw[1] | cw[2] | cw[3]) != 0) {
+        // this lane's candidates, in key order (lane-major, then e), into the warp's region
+        uint32_t before = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) before += __popc(cw[e] & ((1u << lane) - 1u));
+        uint32_t slot = wn + before;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if ((cw[e] >> lane) & 1u) {
+            if (slot < static_cast<uint32_t>(kTopkPerWarp)) {
+              wkey[slot] = score_key(ve[e]);
+              wpos[slot] = rd * 128 + 4 * lane + e;
             }
+            ++slot;
           }
-        }
+        wn += __popc(cw[0]) + __popc(cw[1]) + __popc(cw[2]) + __popc(cw[3]);
       }
     }
+  }
+  if (lane == 0) {
+    s_wcnt[warp] = min(wn, static_cast<uint32_t>(kTopkPerWarp));
+    if (wn > static_cast<uint32_t>(kTopkPerWarp)) s_over = 1;
   }
   __syncthreads();
 
   // ---- 3. resolve tau within the bin
   if (!whole_bin) {
-    const uint32_t nloc = min(s_nloc, static_cast<uint32_t>(kTopkLocal));
-    const uint32_t n4 = (nloc + 3u) & ~3u;
+    // each warp's segment padded to a multiple of 4 with a key outside the bin
+    const uint32_t pad_key = bin == 0 ? 0xFFFFFFFFu : 0u;
+    uint32_t n4 = 0;
+    for (int w = 0; w < kTopkWarps; ++w) n4 += (s_wcnt[w] + 3u) & ~3u;
     // every CTA learns every CTA's candidate count and overflow flag
     if (tid == 0) {
       for (int c = 0; c < C; ++c) {
@@ -332,17 +367,21 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
     }
     const bool crowded = over != 0 || total > static_cast<uint32_t>(kTopkGather);
     if (!crowded) {
-      // candidates' keys into CTA 0 (padded to 4 with a key outside the bin), 16 B at a time
-      const uint32_t pad_key = bin == 0 ? 0xFFFFFFFFu : 0u;
-      for (uint32_t j = nloc + tid; j < n4; j += kTopkThreads) ckey[j] = pad_key;
-      __syncthreads();
-      const uint4* src4 = reinterpret_cast<const uint4*>(ckey);
-      if (C > 1) {
-        const uint32_t dst0 = map_to_rank(smem_u32(gath), 0) + off * 4;
-        for (uint32_t j = tid; j < n4 / 4; j += kTopkThreads) st_cluster_u4(dst0 + j * 16, src4[j]);
-      } else {
-        for (uint32_t j = tid; j < n4 / 4; j += kTopkThreads)
-          reinterpret_cast<uint4*>(gath)[j] = src4[j];
+      // candidates' keys into CTA 0, each warp its own padded segment, 16 B at a time
+      {
+        uint32_t woff = off;                       // this warp's segment in CTA 0's buffer
+        for (int w = 0; w < warp; ++w) woff += (s_wcnt[w] + 3u) & ~3u;
+        const uint32_t wc = s_wcnt[warp], w4 = (wc + 3u) & ~3u;
+        if (lane < static_cast<int>(w4 - wc)) wkey[wc + lane] = pad_key;
+        __syncwarp();
+        const uint4* src4 = reinterpret_cast<const uint4*>(wkey);
+        if (C > 1) {
+          const uint32_t dst0 = map_to_rank(smem_u32(gath), 0) + woff * 4;
+          for (uint32_t j = lane; j < w4 / 4; j += 32) st_cluster_u4(dst0 + j * 16, src4[j]);
+        } else {
+          for (uint32_t j = lane; j < w4 / 4; j += 32)
+            reinterpret_cast<uint4*>(gath + woff)[j] = src4[j];
+        }
       }
       cta_or_cluster_sync(C);                      // CTA 0 holds every candidate
       if (crank == 0) {
@@ -385,9 +424,9 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const TopkParams
       mask = bc[1];
       need = bc[2];
       // mark the candidates: above tau -> taken, equal -> tie
-      for (uint32_t j = tid; j < nloc; j += kTopkThreads) {
-        const uint32_t km = ckey[j] & mask;
-        const int i = cpos[j];
+      for (uint32_t j = lane; j < s_wcnt[warp]; j += 32) {
+        const uint32_t km = wkey[j] & mask;
+        const int i = wpos[j];
         if (km > prefix) atomicOr(&bm_take[bm_word(i)], bm_bit(i));
         else if (km == prefix) atomicOr(&bm_tie[bm_word(i)], bm_bit(i));
       }

@@ -131,19 +131,32 @@ def test_cache_append_argument_errors(dsa):
     assert call(odd, ok) == dsa.DSA_ERR_UNSUPPORTED_SHAPE
 
 
-def test_dense_attention_needs_short_rows(dsa):
-    """Sparse attention without an index array means every prior key; a row range with a row
-    of more than topk prior keys is refused before any launch."""
+def test_dense_attention_row_rules(dsa):
+    """Attention without an index array means every prior key.  Prefill rows may be of any
+    length (dense causal attention); a decode batch whose contexts exceed topk, and the training
+    target without indices over a row of more than topk keys (it writes topk entries per row),
+    are refused before any launch; the dense warm-up calls check their row strides."""
     pre = dsa.make_problem(mode="prefill", h_idx=64, d_idx=128, h=128, d_qk=576, d_v=512,
                            topk=2048, softmax_scale=0.04, num_kv_rows=1 << 20,
                            seqlens=[5000], cu_seqlens=FAKE)
-    ws = [FAKE, FAKE]
-    # rows 0..2047 have at most 2048 prior keys; row 2048 has 2049
-    args = lambda rb, rc: (pre, FAKE, FAKE, None, rb, rc, FAKE, FAKE, None, 0, None, 0)
-    assert dsa.dsa_sparse_mla_fwd(*args(2000, 100)) == dsa.DSA_ERR_INVALID_ARG
     dec = _pb(dsa, max_seqlen=4096)
     assert dsa.dsa_sparse_mla_fwd(dec, FAKE, FAKE, None, 0, 2, FAKE, FAKE, None, 0, None,
                                   0) == dsa.DSA_ERR_INVALID_ARG
+    # rows 0..2047 have at most 2048 prior keys; row 2048 has 2049
+    assert dsa.dsa_indexer_kl_target(pre, FAKE, FAKE, None, FAKE, 2000, 100, FAKE, None,
+                                     0) == dsa.DSA_ERR_INVALID_ARG
+    tgt = dsa.dsa_indexer_kl_target_dense
+    assert tgt(pre, FAKE, FAKE, FAKE, 2000, 100, FAKE, 2048, None, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert tgt(pre, FAKE, FAKE, FAKE, 2000, 100, FAKE, 2110, None, 0) == dsa.DSA_ERR_MISALIGNED
+    assert tgt(dec, FAKE, FAKE, FAKE, 0, 2, FAKE, 4096, None, 0) == dsa.DSA_ERR_INVALID_ARG
+    bwd = dsa.dsa_indexer_kl_backward_dense
+    f = [FAKE] * 5
+    out = [FAKE] * 4
+    assert bwd(pre, *f, FAKE, 2048, 2000, 100, *out, None, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert bwd(pre, *f, FAKE, 2102, 2000, 100, *out, None, 0) == dsa.DSA_ERR_MISALIGNED
+    assert bwd(dec, *f, FAKE, 4096, 0, 2, *out, None, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert dsa.dsa_indexer_kl_backward(pre, *f, None, FAKE, 0, 2, *out, None,
+                                       0) == dsa.DSA_ERR_INVALID_ARG
 
 
 def test_scales_inside_key_blocks_only_for_paged_decode(dsa):

@@ -11,13 +11,15 @@ Tolerances (derived from the arithmetic):
   loss     |L_gpu - L_ref| <= 1e-3 |L_ref| + 1e-5: the fp32 indexer scores carry the indexer's
            1e-3 relative tolerance into the softmax
   grads    element by element, |g_gpu - g_ref| <= 2e-3 |g_ref| + 1e-4 M, with M = max|g_ref|
-           over the element's query row for dw and dq, and over every touched key for dk; and
-           per row rel-L2 <= 2e-3.  The coefficient g_e = pi_e sum p - p_e of a key cancels to ~0
-           where the indexer already matches the target, so an element's own size is no scale
-           for its error: an absolute score error eta moves g_e by up to 2 eta pi_e, a shift set
-           by the row's probabilities, not by g_e.  A dk row gathers such terms from every query
-           row that selected the key, so its floor is the tensor's scale, not the row's own
-           (which can cancel to ~0 as a whole); dw and dq rows sum over 2048 keys of one row.
+           over the whole gradient tensor (dw, dq, or every touched key of dk); and per row
+           rel-L2 <= 2e-3 in the sparse stage.  The coefficient g_e = pi_e sum p - p_e of a key
+           cancels to ~0 where the indexer already matches the target, so an element's own size
+           is no scale for its error: an absolute score error eta moves g_e by up to 2 eta pi_e,
+           a shift set by the row's probabilities, not by g_e.  A gradient row sums such terms
+           over up to 2048 selected keys (the dense warm-up: every prior key) and can cancel as a
+           whole (g sums to 0 over a row whose target sums to 1), so the floor is the tensor's
+           scale, not the row's own.  The dense warm-up's rows sum every prior key: there the
+           floor is 1e-3 of the tensor's scale, with the per-row rel-L2 bound beside it.
 """
 import numpy as np
 import pytest
@@ -34,6 +36,7 @@ T_REL, T_ABS = 1e-4, 1e-7
 L_REL, L_ABS = 1e-3, 1e-5
 G_REL_L2 = 2e-3
 G_REL, G_FLOOR = 2e-3, 1e-4
+DENSE_FLOOR = 1e-3
 
 
 @pytest.fixture(scope="module")
@@ -135,14 +138,14 @@ def _rel_l2(a, b):
     return np.linalg.norm(a - b) / nb if nb > 0 else np.linalg.norm(a)
 
 
-def _check_elementwise(got, ref, what, per_row=True):
-    """|got - ref| <= G_REL |ref| + G_FLOOR M, element by element; M = max|ref| of the element's
+def _check_elementwise(got, ref, what, per_row=False, floor=G_FLOOR):
+    """|got - ref| <= G_REL |ref| + floor M, element by element; M = max|ref| of the element's
     row (first axis) or, with per_row False, of the whole tensor."""
     got = np.asarray(got, np.float64).reshape(len(ref), -1)
     ref = np.asarray(ref, np.float64).reshape(len(ref), -1)
     scale = (np.abs(ref).max(axis=1, keepdims=True) if per_row
              else np.abs(ref).max(initial=0.0))
-    tol = G_REL * np.abs(ref) + G_FLOOR * scale
+    tol = G_REL * np.abs(ref) + floor * scale
     err = np.abs(got - ref)
     bad = np.argwhere(err > tol)
     assert len(bad) == 0, (what, len(bad), bad[:3].tolist(),
@@ -161,7 +164,7 @@ def _check_backward(dsa, wl, rb, n):
         assert _rel_l2(dq[i], ref["dq"][i]) <= G_REL_L2, ("dq", rows[i])
     _check_elementwise(dw, ref["dw"], "dw")
     _check_elementwise(dq, ref["dq"], "dq")
-    _check_elementwise(dk[ref["dk_rows"]], ref["dk"], "dk", per_row=False)
+    _check_elementwise(dk[ref["dk_rows"]], ref["dk"], "dk")
     assert _rel_l2(dk[ref["dk_rows"]], ref["dk"]) <= G_REL_L2
     untouched = np.setdiff1d(np.arange(dk.shape[0]), ref["dk_rows"])
     assert not dk[untouched].any()
@@ -219,3 +222,96 @@ def test_kl_backward_bad_index_reported(dsa):
     torch.cuda.synchronize()
     assert int(status.item()) & dsa.DSA_DEVICE_BAD_INDEX
     np.testing.assert_allclose(to_np(loss), ref["loss"], rtol=L_REL, atol=L_ABS)
+
+
+# ------------------------------------------------------------------ dense warm-up stage
+
+def _dense_idx(wl, rows):
+    """Every prior key of each row, in position order, padded with -1 to the longest row."""
+    from tests.parity import n_valid_of
+    n = [n_valid_of(wl, r) for r in rows]
+    idx = np.full((len(rows), max(n)), -1, np.int32)
+    for i, m in enumerate(n):
+        idx[i, :m] = np.arange(m)
+    return idx
+
+
+def _dense_case(dsa, wl, rb, n):
+    """Dense attention (the LSE the warm-up target needs), the dense target and the dense KL
+    backward of rows [rb, rb + n) against the oracle over every prior key."""
+    from tests.parity import check_attention
+    rows = list(range(rb, rb + n))
+    idx = _dense_idx(wl, rows)
+    ld = (idx.shape[1] + 63) // 64 * 64
+    ld = max(ld, wl.dims["topk"])
+    pb = dsa.problem_of(wl)
+    d = wl.dims
+    # 1. dense attention: out and LSE over every prior key
+    o_ref, l_ref = oracle.sparse_mla_rows(wl, rows, idx)
+    out = torch.full((wl.total_rows, d["h"], d["d_v"]), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    lse = torch.full((wl.total_rows, d["h"]), float("nan"), device="cuda")
+    assert dsa.dsa_sparse_mla_fwd(pb, wl.q, wl.kv, None, rb, n, out, lse) == dsa.DSA_OK
+    torch.cuda.synchronize()
+    o, l = to_np(out), to_np(lse)
+    for i, r in enumerate(rows):
+        check_attention(o[r], l[r], o_ref[i], l_ref[i], d["h"], f"dense row {r}")
+    # 2. the dense target from the oracle's LSE
+    lse_d = torch.zeros(wl.total_rows, d["h"], device="cuda")
+    lse_d[rb:rb + n] = torch.tensor(l_ref, dtype=torch.float32, device="cuda")
+    tgt = torch.full((n, ld), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = dsa.dsa_indexer_kl_target_dense(pb, wl.q, wl.kv, lse_d, rb, n, tgt, ld, status)
+    assert st == dsa.DSA_OK, dsa.status_string(st)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_t = oracle.kl_target_rows(wl, rows, idx)
+    got_t = to_np(tgt)
+    for i in range(n):
+        m = int((idx[i] >= 0).sum())
+        _check_target(got_t[i:i + 1, :m], ref_t[i:i + 1, :m], idx[i:i + 1, :m])
+        assert np.allclose(ref_t[i, :m].sum(), 1.0)
+    # 3. the dense KL backward on the oracle's target
+    target = ref_t.astype(np.float32)
+    ref = oracle.indexer_kl_rows(wl, rows, idx, target.astype(np.float64))
+    t_pad = np.zeros((n, ld), np.float32)
+    t_pad[:, :target.shape[1]] = target
+    loss = torch.full((n,), float("nan"), device="cuda")
+    dw = torch.full((n, d["h_idx"]), float("nan"), device="cuda")
+    dq = torch.full((n, d["h_idx"], d["d_idx"]), float("nan"), device="cuda")
+    dk = torch.zeros(wl.kv.shape[0], d["d_idx"], device="cuda")
+    st = dsa.dsa_indexer_kl_backward_dense(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx, wl.k_scale,
+                                           torch.tensor(t_pad, device="cuda"), ld, rb, n, loss,
+                                           dw, dq, dk, status)
+    assert st == dsa.DSA_OK, dsa.status_string(st)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    loss, dw, dq, dk = to_np(loss), to_np(dw), to_np(dq), to_np(dk)
+    np.testing.assert_allclose(loss, ref["loss"], rtol=L_REL, atol=L_ABS)
+    # a dense row sums every prior key (up to 4096 here, where the sparse stage sums at most
+    # 2048): per row rel-L2 <= 2e-3 and, element by element, a floor of 1e-3 of the tensor's
+    # largest element (the sums cancel further over more keys)
+    for i in range(n):
+        assert _rel_l2(dw[i], ref["dw"][i]) <= G_REL_L2, ("dw", rows[i])
+        assert _rel_l2(dq[i], ref["dq"][i]) <= G_REL_L2, ("dq", rows[i])
+    assert _rel_l2(dk[ref["dk_rows"]], ref["dk"]) <= G_REL_L2
+    _check_elementwise(dw, ref["dw"], "dw", floor=DENSE_FLOOR)
+    _check_elementwise(dq, ref["dq"], "dq", floor=DENSE_FLOOR)
+    _check_elementwise(dk[ref["dk_rows"]], ref["dk"], "dk", floor=DENSE_FLOOR)
+    untouched = np.setdiff1d(np.arange(dk.shape[0]), ref["dk_rows"])
+    assert not dk[untouched].any()
+
+
+def test_dense_warmup_full_dims_4096_rows(dsa):
+    """The warm-up stage on a 4096-row sequence at full shapes: rows around pos + 1 = topk and
+    at the end of the sequence, where every row has more than topk prior keys."""
+    wl = make_prefill(23, [4096], FULL, needles=8, device="cuda")
+    _dense_case(dsa, wl, 2040, 16)
+    _dense_case(dsa, wl, 4088, 8)
+
+
+def test_dense_warmup_small_shape(dsa):
+    """The same at the small shapes (topk 64, rows of up to 1024 keys: the CUDA-core backward)."""
+    wl = make_config(1, device="cuda")
+    _dense_case(dsa, wl, 980, 44)
+    _dense_case(dsa, wl, 30, 40)
