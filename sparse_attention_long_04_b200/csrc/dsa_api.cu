@@ -113,6 +113,25 @@ struct NvtxRange {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Launch with programmatic stream serialization: the kernel may start while the previous kernel
+// of the stream is finishing; it waits for it (griddepcontrol.wait) before reading anything.
+template <typename Kernel, typename... Args>
+dsa_status_t launch_pdl(Kernel k, dim3 grid, int threads, int smem, cudaStream_t st,
+                        Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k, args...) != cudaSuccess) return DSA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 dsa_status_t launch_status() {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -450,13 +469,16 @@ dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* 
   cfg.blockDim = dim3(kTopkThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = shape.csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // may launch while the previous kernel finishes (the kernel waits for it before any read)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, dsa_topk_kernel, prm) != cudaSuccess) return DSA_ERR_CUDA;
   return launch_status();
 }
@@ -542,8 +564,9 @@ dsa_status_t mla_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint16_t* 
     return DSA_ERR_CUDA;
   auto k = dsa_sparse_mla_kernel<D_QK, D_V>;
   if (prepare_kernel(k, C::SMEM_BYTES) != DSA_OK) return DSA_ERR_CUDA;
-  k<<<dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st>>>(q_map, prm);
-  if (launch_status() != DSA_OK) return DSA_ERR_CUDA;
+  if (launch_pdl(k, dim3(2 * row_count, splits), C::THREADS, C::SMEM_BYTES, st, q_map, prm) !=
+      DSA_OK)
+    return DSA_ERR_CUDA;
   if (splits > 1) {
     dsa_mla_combine_kernel<D_V><<<dim3(row_count, d.h), 128, 0, st>>>(prm);
     return launch_status();

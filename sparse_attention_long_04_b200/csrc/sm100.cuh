@@ -114,6 +114,13 @@ __device__ __forceinline__ bool warp_mbar_wait(uint32_t bar, uint32_t parity,
   return ok != 0;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the previous kernel of the stream is still running; it waits here, before reading
+// anything, until that kernel has completed and its writes are visible (a no-op otherwise).
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------- proxies, cluster
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

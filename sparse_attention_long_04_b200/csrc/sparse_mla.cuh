@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(512, 1)
   __shared__ int abort_s;
   __shared__ int n_act_s;
 
+  wait_prior_grid();   // (launched early: the indices come from the previous kernel)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int vh = static_cast<int>(blockIdx.x & 1u);   // value half
   const int split = blockIdx.y;

@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
   __shared__ uint32_t s_bin, s_above, s_over;
   __shared__ uint32_t s_wcnt[kTopkWarps];          // candidates of each warp (its region)
 
+  wait_prior_grid();   // (launched early: the scores come from the previous kernel)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = p.csize;
   const int crank = static_cast<int>(blockIdx.x) % C;
@@ -477,9 +478,20 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
     tk += __popc(bm_take[w]);
     te += __popc(bm_tie[w]);
   }
-  uint32_t tk_tot, te_tot;
-  uint32_t tk_before = cta_excl_scan(tk, tmp, &tk_tot);
-  uint32_t te_before = cta_excl_scan(te, tmp, &te_tot);
+  // one scan of both counts packed in 16-bit halves when a slice cannot hold 65536 keys of a
+  // kind (taken keys are at most topk), else two scans
+  uint32_t tk_before, te_before, tk_tot, te_tot;
+  if (m < 65536) {
+    uint32_t both_tot;
+    const uint32_t both_before = cta_excl_scan(tk | (te << 16), tmp, &both_tot);
+    tk_before = both_before & 0xffffu;
+    te_before = both_before >> 16;
+    tk_tot = both_tot & 0xffffu;
+    te_tot = both_tot >> 16;
+  } else {
+    tk_before = cta_excl_scan(tk, tmp, &tk_tot);
+    te_before = cta_excl_scan(te, tmp, &te_tot);
+  }
   if (tid == 0) {
     for (int c = 0; c < C; ++c) {
       if (C > 1) {
