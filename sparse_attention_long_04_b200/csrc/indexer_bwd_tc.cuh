@@ -16,20 +16,21 @@
 //
 // One CTA per query row (1 per SM: it allocates all 512 TMEM columns).  Warp 0 issues the MMAs,
 // warp 1 owns TMEM, warps 2-3 gather each tile (16-byte cp.async of the selected key rows into
-// a 128-byte-swizzled tile, 4-byte copies of their scales and of the tile's targets; two
-// stages; unused entries are zero-filled), warps 4-7 are the epilogue with thread = TMEM lane.
-// Pass 1 runs D^T for every tile and the epilogue forms the scores S (thread = key), keeping per
-// thread the running softmax statistics of its keys (max, the sum of exp(S - max), and the
-// target's sum, sum p S and sum p ln p); the 128 epilogue threads then combine them into the
-// normaliser and the loss.  No per-key value is stored, so a row may have any number of
-// entries.  Pass 2 runs D^T again per tile, recomputes S with the same instructions (so the
-// same value and ReLU decisions) and forms g; the epilogue sums dw over the tile's keys with a
-// butterfly across lanes and writes M1 (TMEM, thread = key), B2 and the key tile in bf16
-// (shared memory, row = key).  The dk accumulator is double-buffered: while the tensor cores
-// run tile i's dk and dq, the epilogue drains tile i-1's dk rows (times g) through shared
-// memory into global memory with bulk reductions (one 512-byte cp.reduce.async.bulk per key),
-// then forms tile i+1's operands.  At the end the epilogue writes dq (hi + lo, times w) and dw.
-// Every wait is bounded.
+// a 128-byte-swizzled tile and of the tile's targets, 4-byte copies of the keys' scales; 8
+// stages in pass 1, 2 in pass 2; unused entries read as zeros), warps 4-7 are the epilogue with
+// thread = TMEM lane.
+// Pass 1 runs D^T for every tile (4 accumulators in rotation, so the MMAs run ahead of the
+// epilogue) and the epilogue forms the scores S (thread = key), keeping per thread the running
+// softmax statistics of its keys (max, the sum of exp(S - max), and the target's sum, sum p S
+// and sum p ln p); the 128 epilogue threads then combine them into the normaliser and the loss.
+// No per-key value is stored, so a row may have any number of entries.  Pass 2 runs D^T again
+// per tile, recomputes S with the same instructions (so the same value and ReLU decisions) and
+// forms g; the epilogue sums dw over the tile's keys with a butterfly across lanes and writes
+// M1 (TMEM, thread = key), B2 and the key tile in bf16 (shared memory, row = key).  The dk
+// accumulator is double-buffered: while the tensor cores run tile i's dk and dq, the epilogue
+// drains tile i-1's dk rows (times g) through shared memory into global memory with bulk
+// reductions (one 512-byte cp.reduce.async.bulk per key), then forms tile i+1's operands.  At
+// the end the epilogue writes dq (hi + lo, times w) and dw.  Every wait is bounded.
 //
 // Dense mode (the warm-up stage of the training, "Training signal": the indexer imitates the
 // dense attention over every prior key): no index array; the entries of row t are its keys
@@ -48,7 +49,10 @@ struct KlTcCfg {
   static constexpr int BK = 128;                   // keys per tile (MMA M of D^T and dk)
   static constexpr int MAX_K = 2048;
   static constexpr int MAX_TILES = MAX_K / BK;
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = 2;                 // key stages of pass 2
+  static constexpr int STAGES1 = 8;                // key stages of pass 1: the 2 above and 6
+                                                   // over the pass-2 buffers B2 and staging
+  static constexpr int ND1 = 4;                    // D^T buffers of pass 1 (over dk, dq)
   static constexpr int THREADS = 256;
   static constexpr int TILE_BYTES = BK * D;        // e4m3 key rows, 16 KB
   static constexpr int BF_TILE = 2 * BK * 128;     // bf16 [2 blocks of 64][128 rows][128 B]
@@ -66,22 +70,43 @@ struct KlTcCfg {
   static constexpr int OFF_KH = OFF_KT + STAGES * TILE_BYTES;  // key tile in bf16, MN-major
   static constexpr int OFF_B2 = OFF_KH + BF_TILE;              // B2 hi/lo, MN-major bf16
   static constexpr int OFF_STG = OFF_B2 + BF_TILE;             // [128 keys][STAGE_ROW] dk rows
-  static constexpr int OFF_KS = OFF_STG + BK * STAGE_ROW;      // [STAGES][128] k_scale
-  static constexpr int OFF_TG = OFF_KS + STAGES * BK * 4;      // [STAGES][128] target
-  static constexpr int OFF_PHYS = OFF_TG + STAGES * BK * 4;    // [MAX_K] i32 (selected keys)
+  static constexpr int OFF_KS = OFF_STG + BK * STAGE_ROW;      // [STAGES1][128] k_scale
+  static constexpr int OFF_TG = OFF_KS + STAGES1 * BK * 4;     // [STAGES1][128] target
+  static constexpr int OFF_PHYS = OFF_TG + STAGES1 * BK * 4;   // [MAX_K] i32 (selected keys)
   static constexpr int OFF_TILES = OFF_PHYS + 4 * MAX_K;       // [MAX_TILES] i32
   static constexpr int OFF_W = OFF_TILES + 4 * MAX_TILES;      // [64] w
   static constexpr int OFF_SQ = OFF_W + 4 * H;                 // [64] s_q
   static constexpr int OFF_DWP = OFF_SQ + 4 * H;               // [4 warps][64] dw partials
   static constexpr int OFF_SCR = OFF_DWP + 4 * 4 * H;          // [32] reduction scratch
   static constexpr int OFF_BAR = OFF_SCR + 4 * 32;             // barriers
-  static constexpr int N_BAR = 16;
+  static constexpr int N_BAR = 2 * STAGES1 + 2 * ND1 + 8;
   static constexpr int USED = OFF_BAR + 8 * N_BAR;
   static constexpr int SMEM_BYTES = 1024 + USED;
   static_assert(OFF_QW % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_KH % 1024 == 0 &&
                 OFF_B2 % 1024 == 0, "tiles");
   static_assert(OFF_STG % 16 == 0 && STAGE_ROW % 16 == 0, "bulk sources");
   static_assert(OFF_BAR % 8 == 0, "barriers");
+  static_assert((STAGES1 - STAGES) * TILE_BYTES <= BF_TILE + BK * STAGE_ROW &&
+                    OFF_STG == OFF_B2 + BF_TILE,
+                "pass-1 stages over B2 and the staging rows");
+  static_assert(D_COL == 0 && (ND1 - 1) * 64 <= DQ_COL - DK_COL + 64, "pass-1 D^T buffers");
+  // key stage of step `it` (pass 1: it < n; pass 2: it = n + i) and how often that stage was
+  // used before it (the parity of its barriers)
+  __device__ static int stage_of(int it, int n) {
+    return it < n ? it % STAGES1 : (it - n) % STAGES;
+  }
+  __device__ static int use_of(int it, int n) {
+    if (it < n) return it / STAGES1;
+    const int s = (it - n) % STAGES;
+    const int used1 = n > s ? (n - 1 - s) / STAGES1 + 1 : 0;
+    return used1 + (it - n) / STAGES;
+  }
+  // D^T buffer of step `it` (pass 1 rotates over ND1 buffers at columns 64 b; pass 2 uses
+  // buffer 0) and how often that buffer was used before it
+  __device__ static int dbuf_of(int it, int n) { return it < n ? it % ND1 : 0; }
+  __device__ static int duse_of(int it, int n) {
+    return it < n ? it / ND1 : (n + ND1 - 1) / ND1 + (it - n);
+  }
   static_assert(SMEM_BYTES > 116 * 1024, "one CTA per SM (its TMEM allocation never waits)");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
@@ -128,15 +153,15 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
   float* sDwp = reinterpret_cast<float*>(smem + C::OFF_DWP);
   float* sScr = reinterpret_cast<float*>(smem + C::OFF_SCR);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;            // [2] 64 gathering threads (each when its copies land)
-  uint64_t* kempty = bars + 2;      // [2] 128 epilogue threads: the stage is no longer read
-  uint64_t* d_full = bars + 4;      // D^T MMA commit
-  uint64_t* d_empty = bars + 5;     // 128 epilogue threads: D^T read
-  uint64_t* coef_full = bars + 6;   // 128 epilogue threads: M1, B2, Kh written (and the dk
-                                    // buffer of two tiles back drained)
-  uint64_t* mma_done = bars + 7;    // dk / dq MMA commit
-  uint64_t* ep_bar = bars + 8;      // 128 epilogue threads meet
-  uint64_t* fin = bars + 9;         // the MMA issuer's last commit
+  uint64_t* full = bars;            // [STAGES1] 64 gathering threads (each when its copies land)
+  uint64_t* kempty = full + C::STAGES1;   // [STAGES1] 128 epilogue threads: stage no longer read
+  uint64_t* d_full = kempty + C::STAGES1;   // [ND1] D^T MMA commit
+  uint64_t* d_empty = d_full + C::ND1;      // [ND1] 128 epilogue threads: D^T read
+  uint64_t* coef_full = d_empty + C::ND1;   // 128 epilogue threads: M1, B2, Kh written (and
+                                            // the dk buffer of two tiles back drained)
+  uint64_t* mma_done = coef_full + 1;  // dk / dq MMA commit
+  uint64_t* ep_bar = coef_full + 2;    // 128 epilogue threads meet
+  uint64_t* fin = coef_full + 3;       // the MMA issuer's last commit
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int n_act_s;
@@ -216,12 +241,14 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     if (bad && p.status) atomicOr(p.status, kStatusBadIndex);
   }
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::STAGES1; ++i) {
       mbar_init(smem_u32(&full[i]), 64);
       mbar_init(smem_u32(&kempty[i]), 128);
     }
-    mbar_init(smem_u32(d_full), 1);
-    mbar_init(smem_u32(d_empty), 128);
+    for (int i = 0; i < C::ND1; ++i) {
+      mbar_init(smem_u32(&d_full[i]), 1);
+      mbar_init(smem_u32(&d_empty[i]), 128);
+    }
     mbar_init(smem_u32(coef_full), 128);
     mbar_init(smem_u32(mma_done), 1);
     mbar_init(smem_u32(ep_bar), 128);
@@ -257,6 +284,11 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
   const uint32_t tmem = tmem_base_s;
   const int n = n_act_s;
   const int steps = 2 * n;   // pass 1 then pass 2 over the same tiles
+  // e4m3 key tile of stage s (stages 2.. lie over B2 and the staging rows, which only the
+  // epilogue writes, in pass 2, after every pass-1 MMA has completed)
+  auto key_tile = [&](int s) -> uint8_t* {
+    return s < C::STAGES ? sKt + s * C::TILE_BYTES : sB2 + (s - C::STAGES) * C::TILE_BYTES;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -271,18 +303,19 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       bool ok = true;
       for (int it = 0; it <= steps && ok; ++it) {
         if (it < steps) {
-          const int s = it % C::STAGES;
-          ok = mbar_wait(smem_u32(&full[s]), (it / C::STAGES) & 1, &abort_s);
-          if (ok && it >= 1) ok = mbar_wait(smem_u32(d_empty), (it - 1) & 1, &abort_s);
+          const int s = C::stage_of(it, n);
+          const int db = C::dbuf_of(it, n), du = C::duse_of(it, n);
+          ok = mbar_wait(smem_u32(&full[s]), C::use_of(it, n) & 1, &abort_s);
+          if (ok && du >= 1) ok = mbar_wait(smem_u32(&d_empty[db]), (du - 1) & 1, &abort_s);
           if (!ok) break;
           tc_fence_after();
           fence_proxy_async_smem();   // the key tile was written by cp.async
-          const uint32_t kt = smem_u32(sKt + s * C::TILE_BYTES);
+          const uint32_t kt = smem_u32(key_tile(s));
 #pragma unroll
           for (int k = 0; k < C::D / 32; ++k)
-            umma_e4m3(tmem + C::D_COL, sdesc_sw128(kt + k * 32, 16, 1024),
+            umma_e4m3(tmem + C::D_COL + 64 * db, sdesc_sw128(kt + k * 32, 16, 1024),
                       sdesc_sw128(q8 + k * 32, 16, 1024), id_d, k > 0);
-          umma_commit(smem_u32(d_full));
+          umma_commit(smem_u32(&d_full[db]));
         }
         const int i2 = it - 1 - n;   // pass-2 tile whose dk and dq run now
         if (i2 < 0) continue;
@@ -310,21 +343,20 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ gather
-    // thread pt copies 16-byte chunk (pt & 7) of rows (pt >> 3) + 8 q of every tile, and the
-    // scales and targets of entries pt and pt + 64
+    // thread pt copies 16-byte chunk (pt & 7) of rows (pt >> 3) + 8 q of every tile, the scales
+    // of entries pt and pt + 64 (4 bytes each) and, pt < 32, 16-byte chunk pt of the targets
     const int pt = tid - 64;
     const int c = pt & 7, r0 = pt >> 3;
     const float* trow = p.target + static_cast<int64_t>(r) * p.ld_target;
     bool ok = true;
     for (int it = 0; it < steps && ok; ++it) {
-      const int s = it % C::STAGES;
-      if (it >= C::STAGES &&
-          !warp_mbar_wait(smem_u32(&kempty[s]), ((it / C::STAGES) - 1) & 1, &abort_s)) {
+      const int s = C::stage_of(it, n), u = C::use_of(it, n);
+      if (u >= 1 && !warp_mbar_wait(smem_u32(&kempty[s]), (u - 1) & 1, &abort_s)) {
         ok = false;
         break;
       }
       const int tile = tile_at(it % n);
-      const uint32_t dst = smem_u32(sKt + s * C::TILE_BYTES);
+      const uint32_t dst = smem_u32(key_tile(s));
 #pragma unroll 4
       for (int q = 0; q < C::BK / 8; ++q) {
         const int rr = r0 + 8 * q;
@@ -336,11 +368,16 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       }
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        const int ee = pt + 64 * q, e = tile * C::BK + ee;
-        const int64_t ph = phys_at(e);
+        const int ee = pt + 64 * q;
+        const int64_t ph = phys_at(tile * C::BK + ee);
         cp_async_4(smem_u32(sKs + s * C::BK + ee), ph >= 0 ? p.k_scale + ph : p.k_scale,
                    ph >= 0 ? 4u : 0u);
-        cp_async_4(smem_u32(sTg + s * C::BK + ee), e < K ? trow + e : trow, e < K ? 4u : 0u);
+      }
+      if (pt < C::BK / 4) {
+        // targets [tile 128 + 4 pt, +4): within the row's stride (a multiple of 4), else zeros
+        const int64_t e4 = static_cast<int64_t>(tile) * C::BK + 4 * pt;
+        const bool in = e4 < p.ld_target;
+        cp_async_16(smem_u32(sTg + s * C::BK + 4 * pt), in ? trow + e4 : trow, in ? 16u : 0u);
       }
       cp_async_arrive_noinc(smem_u32(&full[s]));
     }
@@ -375,15 +412,16 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     // this step's D^T, its scale and target (the stage's barrier, already complete, orders the
     // cp.async data before the shared-memory reads)
     auto read_step = [&](int it, uint32_t (&du)[2][32], float& ks, float& tg) -> bool {
-      const int s = it % C::STAGES;
-      if (!warp_mbar_wait(smem_u32(d_full), it & 1, &abort_s)) return false;
+      const int s = C::stage_of(it, n);
+      const int db = C::dbuf_of(it, n);
+      if (!warp_mbar_wait(smem_u32(&d_full[db]), C::duse_of(it, n) & 1, &abort_s)) return false;
       tc_fence_after();
-      tmem_ld32(la + C::D_COL, du[0]);
-      tmem_ld32(la + C::D_COL + 32, du[1]);
+      tmem_ld32(la + C::D_COL + 64 * db, du[0]);
+      tmem_ld32(la + C::D_COL + 64 * db + 32, du[1]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(d_empty));
-      if (!warp_mbar_wait(smem_u32(&full[s]), (it / C::STAGES) & 1, &abort_s)) return false;
+      mbar_arrive(smem_u32(&d_empty[db]));
+      if (!warp_mbar_wait(smem_u32(&full[s]), C::use_of(it, n) & 1, &abort_s)) return false;
       ks = sKs[s * C::BK + et];
       tg = sTg[s * C::BK + et];
       return true;
@@ -394,7 +432,7 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       float ks, pe;
       ok = read_step(it, du, ks, pe);
       if (!ok) break;
-      mbar_arrive(smem_u32(&kempty[it % C::STAGES]));
+      mbar_arrive(smem_u32(&kempty[C::stage_of(it, n)]));
       if (phys_at(tile_at(it) * C::BK + et) >= 0) {
         const float S = score(du, ks);
         if (S > m) {
@@ -442,15 +480,19 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     auto drain = [&](int buf, float g, int64_t ph) {
       bulk_wait_read_all();   // the previous reduction has read this staging row
 #pragma unroll
-      for (int q = 0; q < C::D / 32; ++q) {
-        uint32_t u[32];
-        tmem_ld32(la + C::DK_COL + 128 * buf + 32 * q, u);
+      for (int hh = 0; hh < 2; ++hh) {   // 64 columns per wait
+        uint32_t u[2][32];
+        tmem_ld32(la + C::DK_COL + 128 * buf + 64 * hh, u[0]);
+        tmem_ld32(la + C::DK_COL + 128 * buf + 64 * hh + 32, u[1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4)
-          *reinterpret_cast<float4*>(my_stage + 128 * q + 16 * c4) =
-              make_float4(g * __uint_as_float(u[4 * c4]), g * __uint_as_float(u[4 * c4 + 1]),
-                          g * __uint_as_float(u[4 * c4 + 2]), g * __uint_as_float(u[4 * c4 + 3]));
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            *reinterpret_cast<float4*>(my_stage + 256 * hh + 128 * q + 16 * c4) =
+                make_float4(g * __uint_as_float(u[q][4 * c4]), g * __uint_as_float(u[q][4 * c4 + 1]),
+                            g * __uint_as_float(u[q][4 * c4 + 2]),
+                            g * __uint_as_float(u[q][4 * c4 + 3]));
       }
       fence_proxy_async_smem();   // the staging row is read by the bulk engine
       if (ph >= 0 && g != 0.f) {
@@ -463,7 +505,7 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     float g_prev = 0.f;
     int64_t ph_prev = -1;
     for (int i2 = 0; i2 < n && ok; ++i2) {
-      const int it = n + i2, s = it % C::STAGES;
+      const int it = n + i2, s = C::stage_of(it, n);
       uint32_t du[2][32];
       float ks, tg;
       ok = read_step(it, du, ks, tg);
@@ -523,7 +565,7 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       }
       // Kh: this thread's key row of the tile in bf16 (exact), row et of the two dim blocks
       {
-        const uint8_t* tb = sKt + s * C::TILE_BYTES;
+        const uint8_t* tb = key_tile(s);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 v = *reinterpret_cast<const uint4*>(tb + sw128_offset(et, c));
