@@ -632,7 +632,7 @@ def run_prefill(args, dsa, dev, stream, peaks, rank, world, cfg):
 def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, cpu_leg):
     """One training step of the indexer (sparse stage) on prefill_L16k: the KL target from the
     main attention and the KL loss with its gradients (both on the tensor cores),
-    after one forward pass that keeps the selection and the LSE.  dk is zeroed inside the
+    after one forward pass that keeps the selection, the selected keys' scores and the LSE.  dk is zeroed inside the
     step (the backward adds into it)."""
     from dsa_workloads import make_config, make_prefill, CONFIGS, FULL
     if args.train_len == CONFIGS[TRAIN_CFG]["seqlens"][0]:
@@ -645,7 +645,7 @@ def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, cpu_leg):
                           seed=rank_seed(TRAIN_CFG, rank), name=name)
     d = wl.dims
     T, K = wl.total_rows, d["topk"]
-    fwd = dsa.Forward(wl, keep_idx=True)
+    fwd = dsa.Forward(wl, keep_idx=True, keep_sel=True)
     dsa.check(fwd(stream), "forward for the training step")
     pb = fwd.pb
     target = torch.empty(T, K, dtype=torch.float32, device=dev)
@@ -666,7 +666,7 @@ def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, cpu_leg):
             dk.zero_()
         dsa.check(dsa.dsa_indexer_kl_backward(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx,
                                               wl.k_scale, fwd.idx, target, 0, T, loss, dw, dq,
-                                              dk, status, stream), "kl backward")
+                                              dk, status, stream, sel=fwd.sel), "kl backward")
         if ev is not None:
             ev[2].record(stream)
 
@@ -699,8 +699,9 @@ def run_indexer_train(args, dsa, dev, stream, peaks, rank, world, cpu_leg):
                                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
                                "frac": round(t_tf / peaks["bf16_sustained"], 4), "flops": f_t},
            "gpu_launches_per_step": 2,
-           "note": "after one forward that keeps the selection and LSE; per step: target, "
-                   "dk zeroed (a torch memset), backward"}
+           "note": "after one forward that keeps the selection, its scores and the LSE; per "
+                   "step: target, dk zeroed (a torch memset), backward (softmax over the kept "
+                   "scores)"}
     if cpu_leg:
         import oracle
         rows = [int(x) for x in np.linspace(T // 2, T - 1, 16)]

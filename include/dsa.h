@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 2
+#define DSA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define DSA_API __attribute__((visibility("default")))
@@ -150,10 +150,13 @@ DSA_API dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t
  *         of `scores` (exact counts of each row's keys 0..pos(t); anything else gives a wrong
  *         selection).  The selection then starts from them and reads each score once; on
  *         return they are zero again, ready for the next dsa_indexer_scores.  NULL: the
- *         selection counts the first digit itself (one more read of the scores). */
+ *         selection counts the first digit itself (one more read of the scores).
+ *   sel_out  optional fp32 [row_count, topk]: the score of each selected key (sel_out[t][e] =
+ *         scores[t][idx[t][e]], the value the selection compared), 0 where idx is -1; the
+ *         indexer's training step takes them (dsa_indexer_kl_backward).  NULL: not written. */
 DSA_API dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
                       int64_t ld_scores, uint32_t* hist, int32_t row_begin, int32_t row_count,
-                      int32_t* idx, int32_t* dev_status, dsa_stream_t stream);
+                      int32_t* idx, float* sel_out, int32_t* dev_status, dsa_stream_t stream);
 
 /* Stages 1 and 2 fused: the indexer scores of rows [row_begin, row_begin + row_count) and their
  * top-k, without the scores leaving the call.  The pages' selector keeps k tokens per query
@@ -163,7 +166,8 @@ DSA_API dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, co
  * section 1).  As it writes each score into a slab in `workspace`, the indexer counts it in
  * its row's histogram of the first radix digit (the top 11 bits of the order-preserving key);
  * the selection then starts from those counts and reads the slab once.  Inputs as for
- * dsa_indexer_scores; idx as written by dsa_topk (the same set, increasing order, -1 padding).
+ * dsa_indexer_scores; idx and the optional sel_out as written by dsa_topk (the same set,
+ * increasing order, -1 padding).
  * workspace: at least dsa_indexer_topk_workspace_size(dims, seqs, row_count) bytes, 16-byte
  * aligned, caller-owned, contents on entry irrelevant (too small: DSA_ERR_WORKSPACE_TOO_SMALL).
  * With the (4, 32) indexer shape the selection builds its histograms itself. */
@@ -173,7 +177,7 @@ DSA_API dsa_status_t dsa_indexer_topk(const dsa_dims_t* dims, const dsa_seqs_t* 
                                       const uint8_t* q_idx, const float* q_scale, const float* w,
                                       const uint8_t* k_idx, const float* k_scale,
                                       int32_t row_begin, int32_t row_count, int32_t* idx,
-                                      void* workspace, size_t workspace_bytes,
+                                      float* sel_out, void* workspace, size_t workspace_bytes,
                                       int32_t* dev_status, dsa_stream_t stream);
 
 /* Bytes of workspace dsa_sparse_mla_fwd needs for `row_count` rows (split-KV partials when
@@ -257,12 +261,15 @@ DSA_API int32_t dsa_forward_chunk_rows_for(const dsa_dims_t* dims, const dsa_seq
  *            When NULL, rows with at most topk prior keys (the first topk rows of each prefill
  *            sequence; a decode batch whose max_seqlen <= topk) skip the indexer and the top-k,
  *            whose selection would be all of their keys, and run dense attention.
+ *   sel_out  optional fp32 [total_rows, topk]: the indexer score of each selected key, as
+ *            dsa_topk writes it (requires idx_out; else DSA_ERR_INVALID_ARG).
  *   out, lse as for dsa_sparse_mla_fwd. */
 DSA_API dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
                          const float* q_scale, const float* w, const uint8_t* k_idx,
                          const float* k_scale, const uint16_t* q, const uint16_t* kv,
-                         int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
-                         size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream);
+                         int32_t* idx_out, float* sel_out, uint16_t* out, float* lse,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         dsa_stream_t stream);
 
 /* dsa_forward for query rows [row_begin, row_begin + row_count) only, with the query-side
  * arrays holding just those rows: the building block of a prefill split across GPUs (each GPU
@@ -270,8 +277,8 @@ DSA_API dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
  * prior keys of its whole sequence).  The rows, chunks, selection and results are exactly those
  * dsa_forward computes for the same rows.
  *   q_idx [row_count, h_idx, d_idx], q_scale / w [row_count, h_idx], q [row_count, h, d_qk],
- *   out [row_count, h, d_v], lse [row_count, h], idx_out (optional) [row_count, topk]: row i of
- *   these is query row row_begin + i.
+ *   out [row_count, h, d_v], lse [row_count, h], idx_out and sel_out (optional) [row_count,
+ *   topk]: row i of these is query row row_begin + i.
  *   k_idx, k_scale, kv: the full key-side arrays (num_kv_rows physical rows), as for dsa_forward.
  *   workspace: dsa_forward_workspace_size(dims, seqs) bytes suffice for every row range.
  * DECODE: rows are sequences (a range of the batch). */
@@ -280,7 +287,7 @@ DSA_API dsa_status_t dsa_forward_rows(const dsa_dims_t* dims, const dsa_seqs_t* 
                                       const uint8_t* q_idx, const float* q_scale, const float* w,
                                       const uint8_t* k_idx, const float* k_scale,
                                       const uint16_t* q, const uint16_t* kv, int32_t* idx_out,
-                                      uint16_t* out, float* lse, void* workspace,
+                                      float* sel_out, uint16_t* out, float* lse, void* workspace,
                                       size_t workspace_bytes, int32_t* dev_status,
                                       dsa_stream_t stream);
 
@@ -341,6 +348,11 @@ DSA_API dsa_status_t dsa_indexer_kl_target(const dsa_dims_t* dims, const dsa_seq
  *            the scales must be positive, as the e4m3 quantiser makes them: the ReLU masks
  *            are taken from the e4m3 products)
  *   idx      int32 [row_count, topk], relative to row_begin, -1 = unused (required)
+ *   sel_scores  optional fp32 [row_count, topk]: the indexer scores S of the selected keys, as
+ *            the forward's selection wrote them (dsa_topk, dsa_indexer_topk, dsa_forward
+ *            sel_out).  Given, pi is the softmax of these values and the keys are read once
+ *            (the D products are still recomputed for the ReLU masks and the gradients); NULL:
+ *            S is recomputed from q and k (two reads of the keys).  Both agree up to rounding.
  *   target   fp32 [row_count, topk]
  *   loss     fp32 [row_count];  dw fp32 [row_count, h_idx];  dq fp32 [row_count, h_idx, d_idx]
  *   dk       fp32 [num_kv_rows, d_idx]: ADDED to (zero it first); the order of the atomic
@@ -352,10 +364,10 @@ DSA_API dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_s
                                              const uint8_t* q_idx, const float* q_scale,
                                              const float* w, const uint8_t* k_idx,
                                              const float* k_scale, const int32_t* idx,
-                                             const float* target, int32_t row_begin,
-                                             int32_t row_count, float* loss, float* dw,
-                                             float* dq, float* dk, int32_t* dev_status,
-                                             dsa_stream_t stream);
+                                             const float* sel_scores, const float* target,
+                                             int32_t row_begin, int32_t row_count, float* loss,
+                                             float* dw, float* dq, float* dk,
+                                             int32_t* dev_status, dsa_stream_t stream);
 
 /* The dense warm-up stage of the indexer's training ("DeepSeek V3.2-Exp Cuts Long-Context Costs
  * with DeepSeek Sparse Attention (DSA)", "Training signal": before the sparse stage the indexer

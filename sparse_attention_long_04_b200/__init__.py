@@ -80,17 +80,18 @@ def _load():
     DP, SP = ctypes.POINTER(dsa_dims_t), ctypes.POINTER(dsa_seqs_t)
     sig = {
         "dsa_indexer_scores": (I32, [DP, SP, P, P, P, P, P, I32, I32, P, I64, P, P, P]),
-        "dsa_topk": (I32, [DP, SP, P, I64, P, I32, I32, P, P, P]),
+        "dsa_topk": (I32, [DP, SP, P, I64, P, I32, I32, P, P, P, P]),
         "dsa_indexer_topk_workspace_size": (SZ, [DP, SP, I32]),
-        "dsa_indexer_topk": (I32, [DP, SP, P, P, P, P, P, I32, I32, P, P, SZ, P, P]),
+        "dsa_indexer_topk": (I32, [DP, SP, P, P, P, P, P, I32, I32, P, P, P, SZ, P, P]),
         "dsa_sparse_mla_workspace_size": (SZ, [DP, SP, I32]),
         "dsa_sparse_mla_fwd": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, SZ, P, P]),
         "dsa_forward_workspace_size": (SZ, [DP, SP]),
         "dsa_forward_workspace_size_for": (SZ, [DP, SP, I32]),
         "dsa_forward_chunk_rows_for": (I32, [DP, SP, I32, I32]),
         "dsa_sparse_mla_workspace_size_for": (SZ, [DP, SP, I32, I32, SZ]),
-        "dsa_forward": (I32, [DP, SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
-        "dsa_forward_rows": (I32, [DP, SP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+        "dsa_forward": (I32, [DP, SP, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+        "dsa_forward_rows": (I32, [DP, SP, I32, I32, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P,
+                                   P]),
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_selftest_wait_timeout": (I32, [P, P]),
         "dsa_probe_dsmem": (I32, [I32, I32, I32, P, P, P]),
@@ -98,8 +99,8 @@ def _load():
         "dsa_indexer_kl_target_dense": (I32, [DP, SP, P, P, P, I32, I32, P, I64, P, P]),
         "dsa_indexer_kl_backward_dense": (I32, [DP, SP, P, P, P, P, P, P, I64, I32, I32, P, P, P,
                                                 P, P, P]),
-        "dsa_indexer_kl_backward": (I32, [DP, SP, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P,
-                                          P]),
+        "dsa_indexer_kl_backward": (I32, [DP, SP, P, P, P, P, P, P, P, P, I32, I32, P, P, P, P,
+                                          P, P]),
         "dsa_status_string": (ctypes.c_char_p, [I32]),
         "dsa_abi_version": (I32, []),
         "dsa_sparse_mla_fwd_noalloc": (I32, [DP, SP, P, P, P, I32, I32, P, P, P, P]),
@@ -209,10 +210,10 @@ def dsa_indexer_scores(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, row_begin
 
 
 def dsa_topk(pb: Problem, scores, ld_scores: int, row_begin: int, row_count: int, idx,
-             dev_status=None, stream=None, hist=None) -> int:
+             dev_status=None, stream=None, hist=None, sel_out=None) -> int:
     return int(lib.dsa_topk(ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(scores),
                             ld_scores, _ptr(hist), row_begin, row_count, _ptr(idx),
-                            _ptr(dev_status), _stream(stream)))
+                            _ptr(sel_out), _ptr(dev_status), _stream(stream)))
 
 
 def dsa_indexer_topk_workspace_size(pb: Problem, row_count: int) -> int:
@@ -222,11 +223,11 @@ def dsa_indexer_topk_workspace_size(pb: Problem, row_count: int) -> int:
 
 def dsa_indexer_topk(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, row_begin: int,
                      row_count: int, idx, workspace, workspace_bytes: int, dev_status=None,
-                     stream=None) -> int:
+                     stream=None, sel_out=None) -> int:
     return int(lib.dsa_indexer_topk(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
-        _ptr(k_idx), _ptr(k_scale), row_begin, row_count, _ptr(idx), _ptr(workspace),
-        workspace_bytes, _ptr(dev_status), _stream(stream)))
+        _ptr(k_idx), _ptr(k_scale), row_begin, row_count, _ptr(idx), _ptr(sel_out),
+        _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def dsa_sparse_mla_workspace_size(pb: Problem, row_count: int) -> int:
@@ -276,20 +277,21 @@ def dsa_forward_chunk_rows_for(pb: Problem, seq: int, sm_count: int) -> int:
 
 
 def dsa_forward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, q, kv, idx_out, out, lse,
-                workspace, workspace_bytes: int, dev_status=None, stream=None) -> int:
+                workspace, workspace_bytes: int, dev_status=None, stream=None,
+                sel_out=None) -> int:
     return int(lib.dsa_forward(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
-        _ptr(k_idx), _ptr(k_scale), _ptr(q), _ptr(kv), _ptr(idx_out), _ptr(out), _ptr(lse),
-        _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream)))
+        _ptr(k_idx), _ptr(k_scale), _ptr(q), _ptr(kv), _ptr(idx_out), _ptr(sel_out), _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def dsa_forward_rows(pb: Problem, row_begin: int, row_count: int, q_idx, q_scale, w, k_idx,
                      k_scale, q, kv, idx_out, out, lse, workspace, workspace_bytes: int,
-                     dev_status=None, stream=None) -> int:
+                     dev_status=None, stream=None, sel_out=None) -> int:
     return int(lib.dsa_forward_rows(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), row_begin, row_count, _ptr(q_idx),
         _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q), _ptr(kv), _ptr(idx_out),
-        _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes, _ptr(dev_status),
+        _ptr(sel_out), _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes, _ptr(dev_status),
         _stream(stream)))
 
 
@@ -309,11 +311,12 @@ def dsa_indexer_kl_target(pb: Problem, q, kv, idx, lse, row_begin: int, row_coun
 
 def dsa_indexer_kl_backward(pb: Problem, q_idx, q_scale, w, k_idx, k_scale, idx, target,
                             row_begin: int, row_count: int, loss, dw, dq, dk, dev_status=None,
-                            stream=None) -> int:
+                            stream=None, sel=None) -> int:
+    """sel: optional [row_count, topk] scores of the selected keys (the forward's sel_out)."""
     return int(lib.dsa_indexer_kl_backward(
         ctypes.byref(pb.dims), ctypes.byref(pb.seqs), _ptr(q_idx), _ptr(q_scale), _ptr(w),
-        _ptr(k_idx), _ptr(k_scale), _ptr(idx), _ptr(target), row_begin, row_count, _ptr(loss),
-        _ptr(dw), _ptr(dq), _ptr(dk), _ptr(dev_status), _stream(stream)))
+        _ptr(k_idx), _ptr(k_scale), _ptr(idx), _ptr(sel), _ptr(target), row_begin, row_count,
+        _ptr(loss), _ptr(dw), _ptr(dq), _ptr(dk), _ptr(dev_status), _stream(stream)))
 
 
 def dsa_indexer_kl_target_dense(pb: Problem, q, kv, lse, row_begin: int, row_count: int, target,
@@ -357,7 +360,7 @@ class Forward:
     """Owns the outputs and workspace of ``dsa_forward`` for one workload shape (allocated with
     torch, once), so repeated calls allocate nothing."""
 
-    def __init__(self, wl, keep_idx: bool = True):
+    def __init__(self, wl, keep_idx: bool = True, keep_sel: bool = False):
         dev = wl.q.device
         d = wl.dims
         T = wl.total_rows
@@ -371,10 +374,13 @@ class Forward:
         self.lse = torch.empty(T, d["h"], dtype=torch.float32, device=dev)
         self.idx = (torch.empty(T, d["topk"], dtype=torch.int32, device=dev)
                     if keep_idx else None)
+        # the selected keys' scores (the indexer's training step takes them)
+        self.sel = (torch.empty(T, d["topk"], dtype=torch.float32, device=dev)
+                    if keep_idx and keep_sel else None)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def __call__(self, stream=None) -> int:
         wl = self.wl
         return dsa_forward(self.pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx, wl.k_scale, wl.q,
                            wl.kv, self.idx, self.out, self.lse, self.ws, self.ws_bytes,
-                           self.status, stream)
+                           self.status, stream, sel_out=self.sel)

@@ -380,7 +380,7 @@ dsa_status_t indexer_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_
 
 dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* scores, int64_t ld,
                          int32_t row_begin, int32_t row_count, int32_t* idx, int32_t* status,
-                         cudaStream_t st, uint32_t* hist = nullptr);
+                         cudaStream_t st, uint32_t* hist = nullptr, float* sel = nullptr);
 
 // Whether the indexer of these dims counts the first-digit histograms (the full 64 x 128 shape;
 // the 4 x 32 shape's 64-row query groups have no room for them).
@@ -409,13 +409,13 @@ dsa_status_t indexer_dispatch(const dsa_dims_t& d, const dsa_seqs_t& s, const ui
 dsa_status_t indexer_topk(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
                           const float* q_scale, const float* w, const uint8_t* k_idx,
                           const float* k_scale, int32_t row_begin, int32_t row_count,
-                          float* slab, int64_t ld, uint32_t* hist, int32_t* idx,
+                          float* slab, int64_t ld, uint32_t* hist, int32_t* idx, float* sel,
                           int32_t* status, cudaStream_t st) {
   uint32_t* h = indexer_counts_hist(d) ? hist : nullptr;
   dsa_status_t e = indexer_dispatch(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin,
                                     row_count, slab, ld, status, st, h);
   if (e != DSA_OK) return e;
-  return topk_launch(d, s, slab, ld, row_begin, row_count, idx, status, st, h);
+  return topk_launch(d, s, slab, ld, row_begin, row_count, idx, status, st, h, sel);
 }
 
 // ------------------------------------------------------------------------ stage 2
@@ -437,10 +437,10 @@ TopkShape topk_shape(int64_t longest, int32_t row_count, int sm_count) {
 }
 
 // `hist`: per-row first-digit histograms written with the scores (the fused indexer), or null
-// (the top-k builds them itself).
+// (the top-k builds them itself).  `sel`: optional scores of the selected keys.
 dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* scores, int64_t ld,
                          int32_t row_begin, int32_t row_count, int32_t* idx, int32_t* status,
-                         cudaStream_t st, uint32_t* hist) {
+                         cudaStream_t st, uint32_t* hist, float* sel) {
   if (row_count == 0) return DSA_OK;
   DeviceInfo info;
   if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
@@ -448,6 +448,7 @@ dsa_status_t topk_launch(const dsa_dims_t& d, const dsa_seqs_t& s, const float* 
   prm.scores = scores;
   prm.ld = ld;
   prm.idx = idx;
+  prm.sel = sel;
   prm.topk = d.topk;
   prm.decode = s.mode == DSA_DECODE;
   prm.row_begin = row_begin;
@@ -693,17 +694,18 @@ dsa_status_t kl_backward_launch(bool full, const IdxBwdParams& prm, cudaStream_t
 dsa_status_t forward_window(const dsa_dims_t& d, const dsa_seqs_t& s, int64_t w0, int64_t w1,
                             const uint8_t* q_idx, const float* q_scale, const float* w,
                             const uint8_t* k_idx, const float* k_scale, const uint16_t* q,
-                            const uint16_t* kv, int32_t* idx_out, uint16_t* out, float* lse,
-                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                            cudaStream_t st) {
+                            const uint16_t* kv, int32_t* idx_out, float* sel_out, uint16_t* out,
+                            float* lse, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, cudaStream_t st) {
   dsa_status_t e;
   if (!indexer_shape_ok(d, s.mode) || !mla_shape_ok(d)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (!q_idx || !q_scale || !w || !k_idx || !q || !kv || !out || !lse)
     return DSA_ERR_INVALID_ARG;
+  if (sel_out != nullptr && idx_out == nullptr) return DSA_ERR_INVALID_ARG;
   if (k_scale == nullptr && !interleaved_ok(s)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(q) ||
       !aligned16(kv) || !aligned16(out) || !aligned16(lse) || !aligned16(idx_out) ||
-      !aligned16(workspace) || !aligned16(q_scale) || !aligned16(w))
+      !aligned16(sel_out) || !aligned16(workspace) || !aligned16(q_scale) || !aligned16(w))
     return DSA_ERR_MISALIGNED;
   DeviceInfo info;
   if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
@@ -736,8 +738,9 @@ dsa_status_t forward_window(const dsa_dims_t& d, const dsa_seqs_t& s, int64_t w0
                           st, splits);
     const int64_t ld = round4(s.max_seqlen);
     int32_t* idx = idx_out ? idx_out + int64_t(rb) * d.topk : idx_ws;
+    float* sel = sel_out ? sel_out + int64_t(rb) * d.topk : nullptr;
     if ((e = indexer_topk(d, s, q_idx, q_scale, w, k_idx, k_scale, rb, rc, slab, ld, hist, idx,
-                          dev_status, st)) != DSA_OK)
+                          sel, dev_status, st)) != DSA_OK)
       return e;
     return mla_dispatch(d, s, q, kv, idx, rb, rc, out, lse, mla_ws, mla_bytes, dev_status, st,
                         splits);
@@ -763,8 +766,9 @@ dsa_status_t forward_window(const dsa_dims_t& d, const dsa_seqs_t& s, int64_t w0
       const int32_t row_begin = static_cast<int32_t>(cu[b] + r0);
       const int32_t row_count = static_cast<int32_t>(std::min(rows, p1 - r0));
       int32_t* idx = idx_out ? idx_out + int64_t(row_begin) * d.topk : idx_ws;
+      float* sel = sel_out ? sel_out + int64_t(row_begin) * d.topk : nullptr;
       if ((e = indexer_topk(d, s, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count,
-                            slab, ld, hist, idx, dev_status, st)) != DSA_OK)
+                            slab, ld, hist, idx, sel, dev_status, st)) != DSA_OK)
         return e;
       if ((e = mla_dispatch(d, s, q, kv, idx, row_begin, row_count, out, lse, nullptr, 0,
                             dev_status, st, 1)) != DSA_OK)
@@ -799,7 +803,8 @@ dsa_status_t kl_target_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint
 // idx NULL: dense mode (every prior key of each row, the caller checked the geometry)
 dsa_status_t kl_backward_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_t* q_idx,
                               const float* q_scale, const float* w, const uint8_t* k_idx,
-                              const float* k_scale, const int32_t* idx, const float* target,
+                              const float* k_scale, const int32_t* idx, const float* sel,
+                              const float* target,
                               int64_t ld_target, int32_t row_begin, int32_t row_count,
                               float* loss, float* dw, float* dq, float* dk, int32_t* status,
                               cudaStream_t st) {
@@ -824,6 +829,7 @@ dsa_status_t kl_backward_impl(const dsa_dims_t& d, const dsa_seqs_t& s, const ui
   prm.k_scale = k_scale;
   prm.idx = idx;
   prm.target = target;
+  prm.sel = idx != nullptr ? sel : nullptr;
   prm.ld_target = ld_target;
   prm.dense = idx == nullptr;
   prm.loss = loss;
@@ -956,17 +962,18 @@ dsa_status_t dsa_indexer_scores(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
 
 dsa_status_t dsa_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const float* scores,
                       int64_t ld_scores, uint32_t* hist, int32_t row_begin, int32_t row_count,
-                      int32_t* idx, int32_t* dev_status, dsa_stream_t stream) {
+                      int32_t* idx, float* sel_out, int32_t* dev_status, dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_topk");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if ((e = check_rows(seqs, row_begin, row_count)) != DSA_OK) return e;
   if (!scores || !idx) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(scores) || !aligned16(idx) || !aligned16(hist) || ld_scores % 4 != 0)
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(hist) || !aligned16(sel_out) ||
+      ld_scores % 4 != 0)
     return DSA_ERR_MISALIGNED;
   if (ld_scores < max_keys(seqs, row_begin, row_count)) return DSA_ERR_INVALID_ARG;
   return topk_launch(*dims, *seqs, scores, ld_scores, row_begin, row_count, idx, dev_status,
-                     reinterpret_cast<cudaStream_t>(stream), hist);
+                     reinterpret_cast<cudaStream_t>(stream), hist, sel_out);
 }
 
 size_t dsa_indexer_topk_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
@@ -979,8 +986,8 @@ size_t dsa_indexer_topk_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t*
 dsa_status_t dsa_indexer_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
                               const float* q_scale, const float* w, const uint8_t* k_idx,
                               const float* k_scale, int32_t row_begin, int32_t row_count,
-                              int32_t* idx, void* workspace, size_t workspace_bytes,
-                              int32_t* dev_status, dsa_stream_t stream) {
+                              int32_t* idx, float* sel_out, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_indexer_topk");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
@@ -989,7 +996,7 @@ dsa_status_t dsa_indexer_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, co
   if (!q_idx || !q_scale || !w || !k_idx || !idx) return DSA_ERR_INVALID_ARG;
   if (k_scale == nullptr && !interleaved_ok(*seqs)) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_scale) || !aligned16(idx) ||
-      !aligned16(workspace))
+      !aligned16(sel_out) || !aligned16(workspace))
     return DSA_ERR_MISALIGNED;
   if (row_count == 0) return DSA_OK;
   const size_t need = dsa_indexer_topk_workspace_size(dims, seqs, row_count);
@@ -1004,7 +1011,7 @@ dsa_status_t dsa_indexer_topk(const dsa_dims_t* dims, const dsa_seqs_t* seqs, co
       cudaMemsetAsync(hist, 0, size_t(row_count) * kTopkBins * 4, st) != cudaSuccess)
     return DSA_ERR_CUDA;
   return indexer_topk(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, row_begin, row_count, slab,
-                      ld, hist, idx, dev_status, st);
+                      ld, hist, idx, sel_out, dev_status, st);
 }
 
 size_t dsa_sparse_mla_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
@@ -1068,13 +1075,14 @@ size_t dsa_forward_workspace_size(const dsa_dims_t* dims, const dsa_seqs_t* seqs
 dsa_status_t dsa_forward(const dsa_dims_t* dims, const dsa_seqs_t* seqs, const uint8_t* q_idx,
                          const float* q_scale, const float* w, const uint8_t* k_idx,
                          const float* k_scale, const uint16_t* q, const uint16_t* kv,
-                         int32_t* idx_out, uint16_t* out, float* lse, void* workspace,
-                         size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream) {
+                         int32_t* idx_out, float* sel_out, uint16_t* out, float* lse,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_forward");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   return forward_window(*dims, *seqs, 0, seqs->total_rows, q_idx, q_scale, w, k_idx, k_scale, q,
-                        kv, idx_out, out, lse, workspace, workspace_bytes, dev_status,
+                        kv, idx_out, sel_out, out, lse, workspace, workspace_bytes, dev_status,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1082,8 +1090,8 @@ dsa_status_t dsa_forward_rows(const dsa_dims_t* dims, const dsa_seqs_t* seqs, in
                               int32_t row_count, const uint8_t* q_idx, const float* q_scale,
                               const float* w, const uint8_t* k_idx, const float* k_scale,
                               const uint16_t* q, const uint16_t* kv, int32_t* idx_out,
-                              uint16_t* out, float* lse, void* workspace, size_t workspace_bytes,
-                              int32_t* dev_status, dsa_stream_t stream) {
+                              float* sel_out, uint16_t* out, float* lse, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_status, dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_forward_rows");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
@@ -1104,13 +1112,15 @@ dsa_status_t dsa_forward_rows(const dsa_dims_t* dims, const dsa_seqs_t* seqs, in
   const uintptr_t out_a = back(out, size_t(d.h) * d.d_v * 2);
   const uintptr_t lse_a = back(lse, size_t(d.h) * 4);
   const uintptr_t idx_a = idx_out ? back(idx_out, size_t(d.topk) * 4) : 0;
+  const uintptr_t sel_a = sel_out ? back(sel_out, size_t(d.topk) * 4) : 0;
   return forward_window(d, *seqs, row_begin, row_begin + row_count,
                         reinterpret_cast<const uint8_t*>(q_idx_a),
                         reinterpret_cast<const float*>(q_scale_a),
                         reinterpret_cast<const float*>(w_a), k_idx, k_scale,
                         reinterpret_cast<const uint16_t*>(q_a), kv,
-                        reinterpret_cast<int32_t*>(idx_a), reinterpret_cast<uint16_t*>(out_a),
-                        reinterpret_cast<float*>(lse_a), workspace, workspace_bytes, dev_status,
+                        reinterpret_cast<int32_t*>(idx_a), reinterpret_cast<float*>(sel_a),
+                        reinterpret_cast<uint16_t*>(out_a), reinterpret_cast<float*>(lse_a),
+                        workspace, workspace_bytes, dev_status,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1187,15 +1197,17 @@ dsa_status_t dsa_indexer_kl_target_dense(const dsa_dims_t* dims, const dsa_seqs_
 dsa_status_t dsa_indexer_kl_backward(const dsa_dims_t* dims, const dsa_seqs_t* seqs,
                                      const uint8_t* q_idx, const float* q_scale, const float* w,
                                      const uint8_t* k_idx, const float* k_scale,
-                                     const int32_t* idx, const float* target, int32_t row_begin,
-                                     int32_t row_count, float* loss, float* dw, float* dq,
-                                     float* dk, int32_t* dev_status, dsa_stream_t stream) {
+                                     const int32_t* idx, const float* sel_scores,
+                                     const float* target, int32_t row_begin, int32_t row_count,
+                                     float* loss, float* dw, float* dq, float* dk,
+                                     int32_t* dev_status, dsa_stream_t stream) {
   NvtxRange nvtx_range("dsa_indexer_kl_backward");
   dsa_status_t e = check_common(dims, seqs);
   if (e != DSA_OK) return e;
   if (idx == nullptr) return DSA_ERR_INVALID_ARG;
-  return kl_backward_impl(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, idx, target,
-                          dims->topk, row_begin, row_count, loss, dw, dq, dk, dev_status,
+  if (!aligned16(sel_scores)) return DSA_ERR_MISALIGNED;
+  return kl_backward_impl(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, idx, sel_scores,
+                          target, dims->topk, row_begin, row_count, loss, dw, dq, dk, dev_status,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1216,8 +1228,8 @@ dsa_status_t dsa_indexer_kl_backward_dense(const dsa_dims_t* dims, const dsa_seq
   if (ld_target < longest) return DSA_ERR_INVALID_ARG;
   // the CUDA-core kernel of the small shape keeps every entry in shared memory
   if (dims->h_idx == 4 && longest > IdxBwdCfg<4, 32>::MAX_K) return DSA_ERR_UNSUPPORTED_SHAPE;
-  return kl_backward_impl(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, nullptr, target,
-                          ld_target, row_begin, row_count, loss, dw, dq, dk, dev_status,
+  return kl_backward_impl(*dims, *seqs, q_idx, q_scale, w, k_idx, k_scale, nullptr, nullptr,
+                          target, ld_target, row_begin, row_count, loss, dw, dq, dk, dev_status,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 

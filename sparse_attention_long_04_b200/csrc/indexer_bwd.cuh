@@ -47,6 +47,8 @@ struct IdxBwdParams {
   const float* k_scale;        // [R]
   const int32_t* idx;          // [row_count, topk] logical keys, -1 = unused
   const float* target;         // [row_count, topk]
+  const float* sel;            // optional [row_count, topk]: the indexer scores of the selected
+                               // keys (the forward's); the softmax is taken over them
   float* loss;                 // [row_count]
   float* dw;                   // [row_count, H_I]
   float* dq;                   // [row_count, H_I, D_I]
@@ -258,8 +260,12 @@ __global__ void __launch_bounds__(256, 2) dsa_indexer_kl_bwd_kernel(const IdxBwd
     }
   };
 
-  // ---- pass 1: the scores S_e
-  for (int c = 0; c < n_chunks; ++c) {
+  // ---- pass 1: the scores S_e (given: read them)
+  const bool have_sel = p.sel != nullptr && !p.dense;
+  if (have_sel)
+    for (int e = tid; e < K; e += C::THREADS)
+      sG[e] = sPhys[e] >= 0 ? __ldg(p.sel + static_cast<int64_t>(r) * K + e) : -INFINITY;
+  for (int c = 0; c < n_chunks && !have_sel; ++c) {
     if (!sChunk[c]) {
       if (tid < C::CH) sG[c * C::CH + tid] = -INFINITY;
       continue;

@@ -23,9 +23,10 @@
 // epilogue) and the epilogue forms the scores S (thread = key), keeping per thread the running
 // softmax statistics of its keys (max, the sum of exp(S - max), and the target's sum, sum p S
 // and sum p ln p); the 128 epilogue threads then combine them into the normaliser and the loss.
-// No per-key value is stored, so a row may have any number of entries.  Pass 2 runs D^T again
-// per tile, recomputes S with the same instructions (so the same value and ReLU decisions) and
-// forms g; the epilogue sums dw over the tile's keys with a butterfly across lanes and writes
+// No per-key value is stored, so a row may have any number of entries.  When the selected keys'
+// scores are given (the forward's top-k keeps them), pass 1 reads them instead, with no gather
+// and no MMA, and pass 2 takes S from them too.  Pass 2 runs D^T again per tile, recomputes S
+// with the same instructions (so the same value and ReLU decisions) and forms g; the epilogue sums dw over the tile's keys with a butterfly across lanes and writes
 // M1 (TMEM, thread = key), B2 and the key tile in bf16 (shared memory, row = key).  The dk
 // accumulator is double-buffered: while the tensor cores run tile i's dk and dq, the epilogue
 // drains tile i-1's dk rows (times g) through shared memory into global memory with bulk
@@ -91,21 +92,22 @@ struct KlTcCfg {
                 "pass-1 stages over B2 and the staging rows");
   static_assert(D_COL == 0 && (ND1 - 1) * 64 <= DQ_COL - DK_COL + 64, "pass-1 D^T buffers");
   // key stage of step `it` (pass 1: it < n; pass 2: it = n + i) and how often that stage was
-  // used before it (the parity of its barriers)
+  // used before it (the parity of its barriers); n1 = the pass-1 steps that ran on the keys
+  // (n, or 0 when the scores are given)
   __device__ static int stage_of(int it, int n) {
     return it < n ? it % STAGES1 : (it - n) % STAGES;
   }
-  __device__ static int use_of(int it, int n) {
+  __device__ static int use_of(int it, int n, int n1) {
     if (it < n) return it / STAGES1;
     const int s = (it - n) % STAGES;
-    const int used1 = n > s ? (n - 1 - s) / STAGES1 + 1 : 0;
+    const int used1 = n1 > s ? (n1 - 1 - s) / STAGES1 + 1 : 0;
     return used1 + (it - n) / STAGES;
   }
   // D^T buffer of step `it` (pass 1 rotates over ND1 buffers at columns 64 b; pass 2 uses
   // buffer 0) and how often that buffer was used before it
   __device__ static int dbuf_of(int it, int n) { return it < n ? it % ND1 : 0; }
-  __device__ static int duse_of(int it, int n) {
-    return it < n ? it / ND1 : (n + ND1 - 1) / ND1 + (it - n);
+  __device__ static int duse_of(int it, int n, int n1) {
+    return it < n ? it / ND1 : (n1 + ND1 - 1) / ND1 + (it - n);
   }
   static_assert(SMEM_BYTES > 116 * 1024, "one CTA per SM (its TMEM allocation never waits)");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -284,6 +286,12 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
   const uint32_t tmem = tmem_base_s;
   const int n = n_act_s;
   const int steps = 2 * n;   // pass 1 then pass 2 over the same tiles
+  // with the selected keys' scores given, pass 1 reads them instead of the keys: the gather and
+  // the MMAs start at pass 2
+  const bool have_sel = p.sel != nullptr && !dense;
+  const int n1 = have_sel ? 0 : n;
+  const int it0 = n - n1;
+  const float* selrow = have_sel ? p.sel + static_cast<int64_t>(r) * K : nullptr;
   // e4m3 key tile of stage s (stages 2.. lie over B2 and the staging rows, which only the
   // epilogue writes, in pass 2, after every pass-1 MMA has completed)
   auto key_tile = [&](int s) -> uint8_t* {
@@ -301,11 +309,11 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
       const uint32_t q8 = smem_u32(sQ8), qw = smem_u32(sQw), b2 = smem_u32(sB2),
                      kh = smem_u32(sKh);
       bool ok = true;
-      for (int it = 0; it <= steps && ok; ++it) {
+      for (int it = it0; it <= steps && ok; ++it) {
         if (it < steps) {
           const int s = C::stage_of(it, n);
-          const int db = C::dbuf_of(it, n), du = C::duse_of(it, n);
-          ok = mbar_wait(smem_u32(&full[s]), C::use_of(it, n) & 1, &abort_s);
+          const int db = C::dbuf_of(it, n), du = C::duse_of(it, n, n1);
+          ok = mbar_wait(smem_u32(&full[s]), C::use_of(it, n, n1) & 1, &abort_s);
           if (ok && du >= 1) ok = mbar_wait(smem_u32(&d_empty[db]), (du - 1) & 1, &abort_s);
           if (!ok) break;
           tc_fence_after();
@@ -349,8 +357,8 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     const int c = pt & 7, r0 = pt >> 3;
     const float* trow = p.target + static_cast<int64_t>(r) * p.ld_target;
     bool ok = true;
-    for (int it = 0; it < steps && ok; ++it) {
-      const int s = C::stage_of(it, n), u = C::use_of(it, n);
+    for (int it = it0; it < steps && ok; ++it) {
+      const int s = C::stage_of(it, n), u = C::use_of(it, n, n1);
       if (u >= 1 && !warp_mbar_wait(smem_u32(&kempty[s]), (u - 1) & 1, &abort_s)) {
         ok = false;
         break;
@@ -414,37 +422,54 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     auto read_step = [&](int it, uint32_t (&du)[2][32], float& ks, float& tg) -> bool {
       const int s = C::stage_of(it, n);
       const int db = C::dbuf_of(it, n);
-      if (!warp_mbar_wait(smem_u32(&d_full[db]), C::duse_of(it, n) & 1, &abort_s)) return false;
+      if (!warp_mbar_wait(smem_u32(&d_full[db]), C::duse_of(it, n, n1) & 1, &abort_s))
+        return false;
       tc_fence_after();
       tmem_ld32(la + C::D_COL + 64 * db, du[0]);
       tmem_ld32(la + C::D_COL + 64 * db + 32, du[1]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&d_empty[db]));
-      if (!warp_mbar_wait(smem_u32(&full[s]), C::use_of(it, n) & 1, &abort_s)) return false;
+      if (!warp_mbar_wait(smem_u32(&full[s]), C::use_of(it, n, n1) & 1, &abort_s)) return false;
       ks = sKs[s * C::BK + et];
       tg = sTg[s * C::BK + et];
       return true;
     };
     float m = -INFINITY, z = 0.f, psum = 0.f, sps = 0.f, splp = 0.f;
-    for (int it = 0; it < n && ok; ++it) {
+    auto stats = [&](float S, float pe) {
+      if (S > m) {
+        z = z * expf(m - S) + 1.f;
+        m = S;
+      } else {
+        z += expf(S - m);
+      }
+      psum += pe;
+      sps += pe * S;
+      if (pe > 0.f) splp += pe * logf(pe);
+    };
+    if (have_sel) {
+      // the scores and targets of this thread's entries, straight from global memory
+      const float* trow = p.target + static_cast<int64_t>(r) * p.ld_target;
+      for (int it = 0; it < n; it += 4) {
+        float sv[4], pv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = it + u < n ? tile_at(it + u) * C::BK + et : -1;
+          sv[u] = e >= 0 && phys_at(e) >= 0 ? __ldg(selrow + e) : 0.f;
+          pv[u] = e >= 0 && phys_at(e) >= 0 ? __ldg(trow + e) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (it + u < n && phys_at(tile_at(it + u) * C::BK + et) >= 0) stats(sv[u], pv[u]);
+      }
+    }
+    for (int it = 0; it < n1 && ok; ++it) {
       uint32_t du[2][32];
       float ks, pe;
       ok = read_step(it, du, ks, pe);
       if (!ok) break;
       mbar_arrive(smem_u32(&kempty[C::stage_of(it, n)]));
-      if (phys_at(tile_at(it) * C::BK + et) >= 0) {
-        const float S = score(du, ks);
-        if (S > m) {
-          z = z * expf(m - S) + 1.f;
-          m = S;
-        } else {
-          z += expf(S - m);
-        }
-        psum += pe;
-        sps += pe * S;
-        if (pe > 0.f) splp += pe * logf(pe);
-      }
+      if (phys_at(tile_at(it) * C::BK + et) >= 0) stats(score(du, ks), pe);
     }
     // ---- the row's normaliser and loss from the 128 threads' statistics
     const float wm = warp_max(m);
@@ -506,13 +531,16 @@ __global__ void __launch_bounds__(256, 1) dsa_indexer_kl_bwd_tc_kernel(const Idx
     int64_t ph_prev = -1;
     for (int i2 = 0; i2 < n && ok; ++i2) {
       const int it = n + i2, s = C::stage_of(it, n);
+      const int e2 = tile_at(i2) * C::BK + et;
+      const int64_t ph = phys_at(e2);
+      const float s_given = have_sel && ph >= 0 ? __ldg(selrow + e2) : 0.f;
       uint32_t du[2][32];
       float ks, tg;
       ok = read_step(it, du, ks, tg);
       if (!ok) break;
-      const int64_t ph = phys_at(tile_at(i2) * C::BK + et);
       // g = pi psum - p, from the same score as in pass 1 (0 for unused entries)
-      const float g = ph >= 0 ? expf(score(du, ks) - log_z) * psum - tg : 0.f;
+      const float g = ph >= 0 ? expf((have_sel ? s_given : score(du, ks)) - log_z) * psum - tg
+                              : 0.f;
       const float gsk = g * ks;
       // dw: g s_k max(D, 0) summed over the tile's keys (s_q applied at the end)
       {

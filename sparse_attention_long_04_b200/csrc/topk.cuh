@@ -37,6 +37,7 @@ struct TopkParams {
   const float* scores;     // slab row 0
   int64_t ld;
   int32_t* idx;            // [row_count, topk]
+  float* sel;              // optional [row_count, topk]: the score of each selected key
   int32_t topk;
   int32_t decode;
   int32_t row_begin;
@@ -233,10 +234,13 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
   }
   const float* srow = p.scores + static_cast<int64_t>(r) * p.ld;
   int32_t* out = p.idx + static_cast<int64_t>(r) * p.topk;
+  float* sel = p.sel != nullptr ? p.sel + static_cast<int64_t>(r) * p.topk : nullptr;
   const int K = p.topk;
   if (n <= K) {                                    // uniform over the cluster: no barrier used
-    for (int j = crank * kTopkThreads + tid; j < K; j += C * kTopkThreads)
+    for (int j = crank * kTopkThreads + tid; j < K; j += C * kTopkThreads) {
       out[j] = j < n ? j : -1;
+      if (sel != nullptr) sel[j] = j < n ? srow[j] : 0.f;
+    }
     if (grow_hist != nullptr && crank == 0)        // leave the histogram zeroed for reuse
       for (int i = tid; i < kTopkBins; i += kTopkThreads) grow_hist[i] = 0;
     return;
@@ -532,7 +536,11 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
           if (te_before < need) pos = tk_before + te_before;
           ++te_before;
         }
-        if (pos < static_cast<uint32_t>(K)) out[pos] = s0 + blk * 128 + 4 * l + q;
+        if (pos < static_cast<uint32_t>(K)) {
+          const int key = s0 + blk * 128 + 4 * l + q;
+          out[pos] = key;
+          if (sel != nullptr) sel[pos] = srow[key];
+        }
       }
     }
   }

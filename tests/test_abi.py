@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(dsa):
     for n in declared_symbols():
         assert hasattr(lib, n), n
     assert set(dsa.EXPORTED) >= set(declared_symbols())
-    assert dsa.abi_version() == 2
+    assert dsa.abi_version() == 3
     assert dsa.status_string(0) == "ok"
     assert "workspace" in dsa.status_string(3)
 
@@ -67,7 +67,7 @@ def test_null_pointers_rejected(dsa):
     st = dsa.dsa_sparse_mla_fwd(pb, FAKE, FAKE, FAKE, 0, 2, FAKE, None, None, 0, None, 0)
     assert st == dsa.DSA_ERR_INVALID_ARG
     lib = dsa.lib
-    assert lib.dsa_forward(None, None, *([None] * 11), 0, None, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_forward(None, None, *([None] * 12), 0, None, None) == dsa.DSA_ERR_INVALID_ARG
 
 
 def test_bad_shapes_rejected(dsa):
@@ -307,3 +307,26 @@ def test_stage_histogram_arguments(dsa):
     st = dsa.dsa_indexer_scores(tiny, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE, 1024, None, 0,
                                 hist=FAKE)
     assert st == dsa.DSA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_selected_scores_arguments(dsa):
+    """The optional scores of the selected keys (sel_out of the selection and the forward,
+    sel_scores of the KL backward): 16-byte alignment, and the forward keeps them only with the
+    indices."""
+    pb = _pb(dsa)
+    assert dsa.dsa_topk(pb, FAKE, 4096, 0, 2, FAKE, None, 0,
+                        sel_out=FAKE + 4) == dsa.DSA_ERR_MISALIGNED
+    need = dsa.dsa_indexer_topk_workspace_size(pb, 2)
+    assert dsa.dsa_indexer_topk(pb, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, FAKE, FAKE, need, None, 0,
+                                sel_out=FAKE + 8) == dsa.DSA_ERR_MISALIGNED
+    # q_idx, q_scale, w, k_idx, k_scale, q, kv, idx_out = None, out, lse, workspace, sel_out
+    st = dsa.dsa_forward(pb, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
+                         1 << 30, None, 0, sel_out=FAKE)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    st = dsa.dsa_forward_rows(pb, 0, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                              FAKE, FAKE, 1 << 30, None, 0, sel_out=FAKE)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    out = [FAKE] * 4                              # loss, dw, dq, dk
+    st = dsa.dsa_indexer_kl_backward(pb, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, *out,
+                                     None, 0, sel=FAKE + 4)
+    assert st == dsa.DSA_ERR_MISALIGNED

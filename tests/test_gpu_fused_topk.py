@@ -29,19 +29,29 @@ def dsa():
     return m
 
 
-def _fused(dsa, wl, rb, n):
+def _fused(dsa, wl, rb, n, with_sel=False):
     pb = dsa.problem_of(wl)
     ws_bytes = dsa.dsa_indexer_topk_workspace_size(pb, n)
     assert ws_bytes > 0
     ws = torch.full((ws_bytes,), 0xA5, dtype=torch.uint8, device="cuda")   # junk on entry
     idx = torch.full((n, wl.dims["topk"]), -7, dtype=torch.int32, device="cuda")
+    sel = (torch.full((n, wl.dims["topk"]), float("nan"), device="cuda") if with_sel
+           else None)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     st = dsa.dsa_indexer_topk(pb, wl.q_idx, wl.q_scale, wl.w, wl.k_idx, wl.k_scale, rb, n, idx,
-                              ws, ws_bytes, status)
+                              ws, ws_bytes, status, sel_out=sel)
     assert st == dsa.DSA_OK, dsa.status_string(st)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    return to_np(idx)
+    return (to_np(idx), to_np(sel)) if with_sel else to_np(idx)
+
+
+def _check_sel(idx, sel, sc):
+    """sel[t][e] = the slab's score of key idx[t][e], bit for bit; 0 where idx is -1."""
+    for i in range(idx.shape[0]):
+        ok = idx[i] >= 0
+        assert np.array_equal(sel[i, ok].view(np.uint32), sc[i, idx[i, ok]].view(np.uint32)), i
+        assert not sel[i, ~ok].any(), i
 
 
 def _unfused(dsa, wl, rb, n):
@@ -57,10 +67,11 @@ def _unfused(dsa, wl, rb, n):
 
 
 def _check(dsa, wl, rb, n, oracle_rows=None, overlap=True):
-    got = _fused(dsa, wl, rb, n)
+    got, sel = _fused(dsa, wl, rb, n, with_sel=True)
     sc, ref_idx = _unfused(dsa, wl, rb, n)
     k = wl.dims["topk"]
     assert np.array_equal(got, ref_idx)
+    _check_sel(got, sel, sc)
     for i in range(n):
         nv = n_valid_of(wl, rb + i)
         check_topk_exact(got[i], sc[i, :nv], k, f"row {rb + i}")
@@ -118,14 +129,15 @@ def test_forward_chunked_prefill_reuses_histograms(dsa):
     equals the fused call's on the same rows (the forward keeps its indices)."""
     wl = make_prefill(66, [70000], FULL, needles=8, device="cuda")
     pb = dsa.problem_of(wl)
-    f = dsa.Forward(wl)
+    f = dsa.Forward(wl, keep_sel=True)
     assert f() == dsa.DSA_OK
     torch.cuda.synchronize()
     assert int(f.status.item()) == 0
-    gidx = to_np(f.idx)
-    for rb, n in ((2048, 300), (40000, 200), (69800, 200)):
-        got = _fused(dsa, wl, rb, n)
+    gidx, gsel = to_np(f.idx), to_np(f.sel)
+    for rb, n in ((0, 100), (2048, 300), (40000, 200), (69800, 200)):
+        got, sel = _fused(dsa, wl, rb, n, with_sel=True)
         assert np.array_equal(gidx[rb:rb + n], got), rb
+        assert np.array_equal(gsel[rb:rb + n].view(np.uint32), sel.view(np.uint32)), rb
     rows = [2048, 30000, 69999]
     ref = oracle.indexer_rows(wl, rows)
     for r in rows:
@@ -156,9 +168,11 @@ def test_staged_calls_with_histograms(dsa):
         ref_h = np.bincount((key >> 21).astype(np.int64), minlength=2048)
         assert np.array_equal(h_np[i], ref_h), i
     idx = torch.empty(n, 2048, dtype=torch.int32, device="cuda")
-    assert dsa.dsa_topk(pb, sc, ld, 0, n, idx, hist=hist) == dsa.DSA_OK
+    sel = torch.full((n, 2048), float("nan"), device="cuda")
+    assert dsa.dsa_topk(pb, sc, ld, 0, n, idx, hist=hist, sel_out=sel) == dsa.DSA_OK
     torch.cuda.synchronize()
     assert not hist.any()
+    _check_sel(to_np(idx), to_np(sel), s_np)
     assert np.array_equal(to_np(idx), _fused(dsa, wl, 0, n))
     for i, L in enumerate(wl.seqlens):
         check_topk_exact(to_np(idx)[i], s_np[i, :L], 2048, f"row {i}")

@@ -114,11 +114,12 @@ def test_kl_target_dense_without_indices(dsa):
     _check_target(to_np(tgt), oracle.kl_target_rows(wl, rows, idx), idx)
 
 
-def _gpu_backward(dsa, wl, rb, idx, target):
+def _gpu_backward(dsa, wl, rb, idx, target, sel=None):
     n, k = idx.shape
     d = wl.dims
     dev = "cuda"
     idx_d = torch.tensor(idx, device=dev)
+    sel_d = None if sel is None else torch.tensor(sel, dtype=torch.float32, device=dev)
     tgt = torch.tensor(target, dtype=torch.float32, device=dev)
     loss = torch.full((n,), float("nan"), device=dev)
     dw = torch.full((n, d["h_idx"]), float("nan"), device=dev)
@@ -126,7 +127,8 @@ def _gpu_backward(dsa, wl, rb, idx, target):
     dk = torch.zeros(wl.kv.shape[0], d["d_idx"], device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     st = dsa.dsa_indexer_kl_backward(dsa.problem_of(wl), wl.q_idx, wl.q_scale, wl.w, wl.k_idx,
-                                     wl.k_scale, idx_d, tgt, rb, n, loss, dw, dq, dk, status, 0)
+                                     wl.k_scale, idx_d, tgt, rb, n, loss, dw, dq, dk, status, 0,
+                                     sel=sel_d)
     assert st == dsa.DSA_OK, dsa.status_string(st)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
@@ -152,12 +154,20 @@ def _check_elementwise(got, ref, what, per_row=False, floor=G_FLOOR):
                            float((err / np.maximum(tol, 1e-30)).max()))
 
 
-def _check_backward(dsa, wl, rb, n):
+def _check_backward(dsa, wl, rb, n, with_sel=False):
+    """with_sel: the selected keys' scores are passed in (the oracle's, in fp32), as the forward's
+    selection hands them over; the kernel then takes the softmax over them."""
     rows = list(range(rb, rb + n))
-    _, idx, _ = _oracle_selection(wl, rows)
+    sc, idx, _ = _oracle_selection(wl, rows)
     target = oracle.kl_target_rows(wl, rows, idx).astype(np.float32)
     ref = oracle.indexer_kl_rows(wl, rows, idx, target.astype(np.float64))
-    loss, dw, dq, dk = _gpu_backward(dsa, wl, rb, idx, target)
+    sel = None
+    if with_sel:
+        sel = np.zeros(idx.shape, np.float32)
+        for i, r in enumerate(rows):
+            ok = idx[i] >= 0
+            sel[i, ok] = sc[r][idx[i, ok]]
+    loss, dw, dq, dk = _gpu_backward(dsa, wl, rb, idx, target, sel)
     np.testing.assert_allclose(loss, ref["loss"], rtol=L_REL, atol=L_ABS)
     for i in range(n):
         assert _rel_l2(dw[i], ref["dw"][i]) <= G_REL_L2, ("dw", rows[i])
@@ -196,6 +206,19 @@ def test_kl_backward_full_dims_paged_decode(dsa):
     wl = make_decode(21, 5, [7000, 2048, 2049, 100, 1], FULL, boost=0.01, paged=True,
                      device="cuda")
     _check_backward(dsa, wl, 0, 5)
+
+
+def test_kl_backward_with_selected_scores(dsa):
+    """The scores of the selected keys given (the forward's sel_out): pass 1 reads them instead
+    of the keys; the same tolerances hold."""
+    wl = make_config(1, device="cuda")
+    _check_backward(dsa, wl, 980, 44, with_sel=True)
+    wl = make_prefill(22, [2500, 300], FULL, needles=8, device="cuda")
+    _check_backward(dsa, wl, 2040, 16, with_sel=True)
+    _check_backward(dsa, wl, 2490, 20, with_sel=True)
+    wl = make_decode(21, 5, [7000, 2048, 2049, 100, 1], FULL, boost=0.01, paged=True,
+                     device="cuda")
+    _check_backward(dsa, wl, 0, 5, with_sel=True)
 
 
 def test_kl_backward_bad_index_reported(dsa):
