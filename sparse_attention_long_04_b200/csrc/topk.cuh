@@ -509,10 +509,13 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
     }
   }
   cta_or_cluster_sync(C);
+  uint32_t tk0 = 0, te0 = 0;                       // the CTAs before this one
   for (int c = 0; c < crank; ++c) {
-    tk_before += cnt[16 + c];
-    te_before += cnt[24 + c];
+    tk0 += cnt[16 + c];
+    te0 += cnt[24 + c];
   }
+  tk_before += tk0;
+  te_before += te0;
   if (grow_hist != nullptr && crank == 0)         // every CTA has read it: zero for reuse
     for (int i = tid; i < kTopkBins; i += kTopkThreads) grow_hist[i] = 0;
   for (int blk = b0; blk < b1; ++blk) {
@@ -536,13 +539,19 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
           if (te_before < need) pos = tk_before + te_before;
           ++te_before;
         }
-        if (pos < static_cast<uint32_t>(K)) {
-          const int key = s0 + blk * 128 + 4 * l + q;
-          out[pos] = key;
-          if (sel != nullptr) sel[pos] = srow[key];
-        }
+        if (pos < static_cast<uint32_t>(K)) out[pos] = s0 + blk * 128 + 4 * l + q;
       }
     }
+  }
+  if (sel != nullptr) {
+    // the slice's outputs are one contiguous range of positions (keys in increasing order):
+    // every thread fetches scores of it, all loads in flight together
+    const uint32_t ties = need > te0 ? min(need - te0, te_tot) : 0u;
+    const uint32_t begin = tk0 + min(te0, need), count = tk_tot + ties;
+    __syncthreads();                               // this CTA's indices are written
+    for (uint32_t j = begin + tid; j < begin + count && j < static_cast<uint32_t>(K);
+         j += kTopkThreads)
+      sel[j] = srow[out[j]];
   }
   // no CTA may leave while a peer can still write into its shared memory: the last remote
   // writes were the counts above, ordered before the barrier that every CTA has passed
