@@ -238,9 +238,11 @@ class CudaTimer:
 
 
 def time_decode(args, dsa, step, world, dev, clocks=None, timer=CudaTimer):
-    """W warm-up steps, then K timed steps with events between the stages, bracketed by a
-    barrier and a device synchronisation on both sides.  Returns (ms per step (max over ranks),
-    mean ms per stage [indexer, top-k, sparse MLA], clocks)."""
+    """W warm-up steps, then K timed steps back to back (nothing between them but the launches,
+    so each kernel's dependent launch overlaps the previous one's tail), bracketed by a barrier
+    and a device synchronisation on both sides; then K more steps with events between the stages
+    for the per-kernel split.  Returns (ms per step (max over ranks), mean ms per stage
+    [indexer, top-k, sparse MLA], clocks)."""
     stream = step.stream
     for _ in range(args.warmup):
         step()
@@ -257,13 +259,16 @@ def time_decode(args, dsa, step, world, dev, clocks=None, timer=CudaTimer):
     timer.sync()
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step()
     end.record(stream)
     timer.sync()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop() if clocks is not None else None
     ms = start.elapsed_time(end)
+    for i in range(args.steps):           # the per-stage split, in a pass of its own
+        step(evs[i])
+    timer.sync()
     k_ms = [[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
             for e in evs]
     per_kernel = [sum(x[j] for x in k_ms) / len(k_ms) for j in range(3)]

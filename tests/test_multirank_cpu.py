@@ -258,13 +258,13 @@ def _bench_worker(rank, world, port, out_dir):
 def test_bench_timed_loop_two_ranks_gloo(tmp_path):
     """bench.time_decode on two gloo ranks with the kernels stubbed: W warm-up + K timed steps on
     every rank, barriers around the timed region, the job time is the slower rank's on both, and
-    the per-stage split comes from the events between the stages."""
+    the per-stage split comes from K more steps with events between the stages."""
     port = _free_port()
     mp.start_processes(_bench_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True,
                        start_method="spawn")
     import json
     r = [json.load(open(tmp_path / f"b{k}.json")) for k in (0, 1)]
-    assert r[0]["calls"] == r[1]["calls"] == 3 + 4
+    assert r[0]["calls"] == r[1]["calls"] == 3 + 4 + 4
     assert r[0]["ms"] == r[1]["ms"]                     # max over ranks, on both
     assert r[0]["ms"] >= 3 * 2.0 * 0.99                 # rank 1: three 2 ms stages per step
     assert all(x >= 1.9 for x in r[1]["per_kernel"]) and all(x >= 0.9 for x in r[0]["per_kernel"])
