@@ -279,8 +279,8 @@ dsa_status_t run_indexer_kernel(const CUtensorMap& kmap, const CUtensorMap& qmap
   if (C::TMEM_COLS == 512) smem = std::max(smem, 120 * 1024);   // one CTA per SM
   auto k = dsa_indexer_kernel<H_I, D_I, QPG>;
   if (prepare_kernel(k, smem) != DSA_OK) return DSA_ERR_CUDA;
-  k<<<grid, C::THREADS, smem, st>>>(kmap, qmap, prm);
-  return launch_status();
+  // may launch while the previous kernel finishes (the kernel waits for it before any read)
+  return launch_pdl(k, grid, C::THREADS, smem, st, kmap, qmap, prm);
 }
 
 // Key tiles per CTA of the decode indexer.  The launch is HBM-bound and every CTA streams

@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
                        const __grid_constant__ CUtensorMap qmap, const IndexerParams p) {
   using C = IndexerCfg<H_I, D_I, QPG>;
   constexpr int N = C::N;
+  wait_prior_grid();   // (launched early: anything before it in the stream is complete here)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
