@@ -188,6 +188,19 @@ __global__ void __launch_bounds__(512, 1)
     return rem >= C::BN ? ~0ull : ((1ull << rem) - 1ull);
   };
 
+  // the selected keys' indices (8 per thread of warps 8-15), loaded before the set-up and the Q
+  // load, so that their latency overlaps both
+  constexpr int KPT = C::MAX_TILES * C::BN / 256;
+  int v[KPT];
+  if (warp >= 8 && !stream_dense) {
+    const int t = threadIdx.x - 256;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int e = t + 256 * j;
+      v[j] = e >= p.topk ? -1 : dense ? (e < n_keys ? e : -1) : irow[e];
+    }
+  }
+
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(smem_u32(&k_full[i]), 128);
@@ -221,16 +234,9 @@ __global__ void __launch_bounds__(512, 1)
     }
   }
   if (warp >= 8 && !stream_dense) {
-    // ---- every selected key -> physical row (or -1): 8 keys per thread, all index loads in
-    // flight together, then all block-table loads
+    // ---- every selected key -> physical row (or -1): the indices loaded above, then all
+    // block-table loads in flight together
     const int t = threadIdx.x - 256;
-    constexpr int KPT = C::MAX_TILES * C::BN / 256;
-    int v[KPT];
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) {
-      const int e = t + 256 * j;
-      v[j] = e >= p.topk ? -1 : dense ? (e < n_keys ? e : -1) : irow[e];
-    }
     int64_t phys[KPT];
     bool bad_idx = false;
 #pragma unroll
