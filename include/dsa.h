@@ -426,6 +426,11 @@ DSA_API dsa_status_t dsa_probe_dsmem(int32_t clusters, int32_t bytes, int32_t re
                                      int32_t* bad, dsa_stream_t stream);
 
 DSA_API const char* dsa_status_string(dsa_status_t status);
+
+/* DSA_ABI_VERSION of the built library.  2: first-digit histograms (hist of dsa_indexer_scores
+ * and dsa_topk), dsa_indexer_topk, dsa_forward_rows, the dense warm-up entry points;
+ * 3: the scores of the selected keys (sel_out of dsa_topk, dsa_indexer_topk, dsa_forward and
+ * dsa_forward_rows; sel_scores of dsa_indexer_kl_backward). */
 DSA_API int32_t dsa_abi_version(void);
 
 #ifdef __cplusplus
