@@ -421,16 +421,18 @@ dsa_status_t indexer_topk(const dsa_dims_t& d, const dsa_seqs_t& s, const uint8_
 // ------------------------------------------------------------------------ stage 2
 
 // Cluster size and slice of the top-k launch for rows of up to `longest` keys: slices of at
-// most 32768 keys (8 KB of bitmaps), then more CTAs per row while the rows alone leave SMs idle
-// and slices stay at least 4096 keys long.  Longer rows than 8 slices of 32768 take longer
-// slices (larger bitmaps), as far as shared memory allows.
+// most 32768 keys (8 KB of bitmaps; 65536 when the launch has rows for two full waves, where
+// fewer CTAs per row pay the per-CTA phases fewer times), then more CTAs per row while the rows
+// alone leave SMs idle and slices stay at least 4096 keys long.  Longer rows than 8 slices take
+// longer slices (larger bitmaps), as far as shared memory allows.
 struct TopkShape {
   int csize;
   int slice;
 };
 TopkShape topk_shape(int64_t longest, int32_t row_count, int sm_count) {
+  const int64_t max_slice = int64_t(row_count) >= 2 * int64_t(sm_count) ? 65536 : 32768;
   int c = 1;
-  while (c < 8 && int64_t(c) * 32768 < longest) c *= 2;
+  while (c < 8 && int64_t(c) * max_slice < longest) c *= 2;
   while (c < 8 && int64_t(row_count) * c < sm_count && int64_t(c) * 4096 < longest) c *= 2;
   const int64_t per = (ceil_div(std::max<int64_t>(1, longest), c) + 127) / 128 * 128;
   return TopkShape{c, static_cast<int>(std::min<int64_t>(per, INT32_MAX / 2))};
