@@ -100,7 +100,10 @@ __device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
   asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// Exclusive scan over the CTA's threads (one value each); *total receives the sum.
+// Exclusive scan over the CTA's threads (one value each); *total receives the sum.  With
+// kReuse the scratch may be used again right after the call (a third barrier); without it the
+// caller passes another barrier before tmp is written again.
+template <bool kReuse = true>
 __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
@@ -125,7 +128,7 @@ __device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t* tmp, uin
   __syncthreads();
   const uint32_t res = tmp[warp] + x - v;
   *total = tmp[32];
-  __syncthreads();
+  if (kReuse) __syncthreads();
   return res;
 }
 
@@ -148,38 +151,65 @@ __device__ __forceinline__ void cluster_hist_sum(uint32_t* hist, uint32_t* hsum,
   }
 }
 
-// Bin holding the need-th largest key of hsum (nb bins, descending cumulative counts); all
-// threads of the CTA call it and all get the same (bin, count above the bin).  A histogram
-// holding fewer than `need` keys (inconsistent input) gives bin 0.
-__device__ __forceinline__ void find_bin(const uint32_t* hsum, uint32_t nb, uint32_t need,
-                                         uint32_t* tmp, uint32_t* s_bin, uint32_t* s_above,
-                                         uint32_t* bin, uint32_t* above) {
-  const int tid = threadIdx.x;
-  const uint32_t bpt = nb / kTopkThreads;         // 4 or 2 bins per thread
-  if (tid == 0) {
-    *s_bin = 0;
-    *s_above = 0;
-  }
+// Bin holding the need-th largest key of a histogram of BPT x kTopkThreads bins held in the
+// CTA's registers, thread t holding bins [BPT t, BPT t + BPT) in v; every thread gets the same
+// (bin, keys in the bins above it, keys in it).  need >= 1.  A histogram holding fewer than
+// `need` keys (inconsistent input) gives bin 0 with nothing above it.  Two barriers; the
+// scratch (wtot: kTopkWarps words, res: 3) may be written again by the next call at once: its
+// reads all precede the second barrier, and the next call writes res only after its first.
+template <int BPT>
+__device__ __forceinline__ void find_bin(const uint32_t (&v)[BPT], uint32_t need, uint32_t* wtot,
+                                         uint32_t* res, uint32_t* bin, uint32_t* above,
+                                         uint32_t* in_bin) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t mine = 0;
-  for (uint32_t j = 0; j < bpt; ++j) mine += hsum[nb - 1 - (tid * bpt + j)];
-  uint32_t tot;
-  const uint32_t before = cta_excl_scan(mine, tmp, &tot);   // (syncs: s_bin init visible)
-  if (before < need && before + mine >= need) {
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) mine += v[j];
+  uint32_t x = mine;                              // this lane's and the higher lanes' keys
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) wtot[warp] = x;
+  __syncthreads();
+  uint32_t before = x - mine;                     // keys in the bins above this thread's
+  for (int w = warp + 1; w < kTopkWarps; ++w) before += wtot[w];
+  if (before < need && before + mine >= need) {   // exactly one thread holds the crossing
     uint32_t c = before;
-    for (uint32_t j = 0; j < bpt; ++j) {
-      const uint32_t b = nb - 1 - (tid * bpt + j);
-      if (c + hsum[b] >= need) {
-        *s_bin = b;
-        *s_above = c;
-        break;
+    bool found = false;
+#pragma unroll
+    for (int j = BPT - 1; j >= 0; --j) {
+      if (!found && c + v[j] >= need) {
+        res[0] = static_cast<uint32_t>(BPT * tid + j);
+        res[1] = c;
+        res[2] = v[j];
+        found = true;
       }
-      c += hsum[b];
+      c += v[j];
     }
+  } else if (tid == 0 && before + mine < need) {  // fewer keys than needed in all
+    res[0] = 0;
+    res[1] = 0;
+    res[2] = v[0];
   }
   __syncthreads();
-  *bin = *s_bin;
-  *above = *s_above;
-  __syncthreads();
+  *bin = res[0];
+  *above = res[1];
+  *in_bin = res[2];
+}
+
+// A histogram in shared memory into the registers find_bin takes.
+template <int BPT>
+__device__ __forceinline__ void load_bins(const uint32_t* h, uint32_t (&v)[BPT]) {
+  static_assert(BPT == 2 || BPT == 4, "2 or 4 bins a thread");
+  if constexpr (BPT == 4) {
+    const uint4 x = reinterpret_cast<const uint4*>(h)[threadIdx.x];
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const uint2 x = reinterpret_cast<const uint2*>(h)[threadIdx.x];
+    v[0] = x.x; v[1] = x.y;
+  }
 }
 
 __device__ __forceinline__ void cta_or_cluster_sync(int C) {
@@ -200,7 +230,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
   uint32_t* bm_take = reinterpret_cast<uint32_t*>(topk_smem + kTopkFixedSmem);  // [words]
   const int words = (p.slice + 31) / 32;
   uint32_t* bm_tie = bm_take + words;                                // [words]
-  __shared__ uint32_t s_bin, s_above, s_over;
+  uint32_t* fres = tmp + 36;                                         // [3] find_bin's result
+  __shared__ uint32_t s_over;
   __shared__ uint32_t s_wcnt[kTopkWarps];          // candidates of each warp (its region)
 
   wait_prior_grid();   // (launched early: the scores come from the previous kernel)
@@ -211,12 +242,17 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
   const int row = p.row_begin + r;
   uint32_t* grow_hist = p.hist ? p.hist + static_cast<int64_t>(r) * kTopkBins : nullptr;
   // the row's first-digit counts are loaded before anything else (their latency then overlaps
-  // the row geometry's)
+  // the row geometry's); thread t holds bins 4t..4t+3
   constexpr int kHpt = kTopkBins / kTopkThreads;
+  static_assert(kHpt == 4, "four first-digit bins a thread");
   uint32_t hreg[kHpt];
-  if (grow_hist != nullptr)
-#pragma unroll
-    for (int j = 0; j < kHpt; ++j) hreg[j] = __ldcg(grow_hist + j * kTopkThreads + tid);
+  if (grow_hist != nullptr) {
+    const uint4 h4 = __ldcg(reinterpret_cast<const uint4*>(grow_hist) + tid);
+    hreg[0] = h4.x;
+    hreg[1] = h4.y;
+    hreg[2] = h4.z;
+    hreg[3] = h4.w;
+  }
   int n;
   if (p.decode) {
     n = p.seq_lens[row];
@@ -258,11 +294,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
   if (tid == 0) s_over = 0;
 
   // ---- 1. first digit
-  if (grow_hist != nullptr) {
-#pragma unroll
-    for (int j = 0; j < kHpt; ++j) hsum[j * kTopkThreads + tid] = hreg[j];
-    __syncthreads();
-  } else {
+  if (grow_hist == nullptr) {
     for (int i = tid; i < kTopkBins; i += kTopkThreads) {
       hloc[i] = 0;
       hsum[i] = 0;
@@ -279,11 +311,18 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
       }
     }
     cluster_hist_sum(hloc, hsum, kTopkBins, C);
+    load_bins(hsum, hreg);
   }
-  uint32_t bin, above;
-  find_bin(hsum, kTopkBins, K, tmp, &s_bin, &s_above, &bin, &above);
+  uint32_t bin, above, in_bin;
+  find_bin(hreg, K, tmp, fres, &bin, &above, &in_bin);
   uint32_t need = K - above;
-  const bool whole_bin = hsum[bin] == need;      // every key of the bin is taken
+  const bool whole_bin = in_bin == need;         // every key of the bin is taken
+  if (crank == 0 && !whole_bin) {
+    // CTA 0's histograms of the second (hloc, 2048 bins) and third (hsum, 1024 bins) digits,
+    // zeroed now: the barriers up to the resolution order these stores before its counts
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) hloc[i] = 0;
+    for (int i = tid; i < kTopkBins / 2; i += kTopkThreads) hsum[i] = 0;
+  }
   uint32_t prefix = bin << 21, mask = 0xFFE00000u;
 
   // ---- 2. classify the slice: above the bin -> taken; in the bin -> candidate
@@ -390,25 +429,31 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
       }
       cta_or_cluster_sync(C);                      // CTA 0 holds every candidate
       if (crank == 0) {
-        constexpr int kShift[2] = {10, 0};
-        constexpr int kBits[2] = {11, 10};
-        for (int pass = 0; pass < 2; ++pass) {
-          const uint32_t nb = 1u << kBits[pass];
-          for (uint32_t i = tid; i < nb; i += kTopkThreads) hsum[i] = 0;
-          __syncthreads();
+        // second digit (11 bits) into hloc, then, unless its bin is exact, the third (10 bits)
+        // into hsum; both were zeroed before the classifying pass
+        for (uint32_t i = tid; i < total; i += kTopkThreads) {
+          const uint32_t k = gath[i];
+          if ((k & mask) == prefix) atomicAdd(&hloc[(k >> 10) & 2047u], 1u);
+        }
+        __syncthreads();
+        uint32_t v2[4], b2, ab2, nb2;
+        load_bins(hloc, v2);
+        find_bin(v2, need, tmp, fres, &b2, &ab2, &nb2);
+        need -= ab2;
+        prefix |= b2 << 10;
+        mask |= 2047u << 10;
+        if (nb2 != need) {
           for (uint32_t i = tid; i < total; i += kTopkThreads) {
             const uint32_t k = gath[i];
-            if ((k & mask) == prefix) atomicAdd(&hsum[(k >> kShift[pass]) & (nb - 1)], 1u);
+            if ((k & mask) == prefix) atomicAdd(&hsum[k & 1023u], 1u);
           }
           __syncthreads();
-          uint32_t b2, ab2;
-          find_bin(hsum, nb, need, tmp, &s_bin, &s_above, &b2, &ab2);
-          need -= ab2;
-          prefix |= b2 << kShift[pass];
-          mask |= (nb - 1) << kShift[pass];
-          const bool exact = hsum[b2] == need;
-          __syncthreads();
-          if (exact) break;
+          uint32_t v3[2], b3, ab3, nb3;
+          load_bins(hsum, v3);
+          find_bin(v3, need, tmp, fres, &b3, &ab3, &nb3);
+          need -= ab3;
+          prefix |= b3;
+          mask |= 1023u;
         }
         if (tid == 0)
           for (int c = 0; c < C; ++c) {
@@ -452,14 +497,20 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
           if ((k & mask) == prefix) atomicAdd(&hloc[(k >> kShift[pass]) & (nb - 1)], 1u);
         }
         cluster_hist_sum(hloc, hsum, nb, C);
-        uint32_t b2, ab2;
-        find_bin(hsum, nb, need, tmp, &s_bin, &s_above, &b2, &ab2);
+        uint32_t b2, ab2, nb2;
+        if (pass == 0) {
+          uint32_t v2[4];
+          load_bins(hsum, v2);
+          find_bin(v2, need, tmp, fres, &b2, &ab2, &nb2);
+        } else {
+          uint32_t v3[2];
+          load_bins(hsum, v3);
+          find_bin(v3, need, tmp, fres, &b2, &ab2, &nb2);
+        }
         need -= ab2;
         prefix |= b2 << kShift[pass];
         mask |= (nb - 1) << kShift[pass];
-        const bool exact = hsum[b2] == need;
-        __syncthreads();
-        if (exact) break;
+        if (nb2 == need) break;
       }
       for (int i = tid; i < m; i += kTopkThreads) {
         const uint32_t k = score_key(srow[s0 + i]);
@@ -486,15 +537,15 @@ __global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const TopkPar
   // kind (taken keys are at most topk), else two scans
   uint32_t tk_before, te_before, tk_tot, te_tot;
   if (m < 65536) {
-    uint32_t both_tot;
-    const uint32_t both_before = cta_excl_scan(tk | (te << 16), tmp, &both_tot);
+    uint32_t both_tot;   // (tmp is not written again before the next barrier)
+    const uint32_t both_before = cta_excl_scan<false>(tk | (te << 16), tmp, &both_tot);
     tk_before = both_before & 0xffffu;
     te_before = both_before >> 16;
     tk_tot = both_tot & 0xffffu;
     te_tot = both_tot >> 16;
   } else {
     tk_before = cta_excl_scan(tk, tmp, &tk_tot);
-    te_before = cta_excl_scan(te, tmp, &te_tot);
+    te_before = cta_excl_scan<false>(te, tmp, &te_tot);
   }
   if (tid == 0) {
     for (int c = 0; c < C; ++c) {
