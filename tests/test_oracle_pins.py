@@ -245,6 +245,24 @@ def test_attention_k1_and_identical_rows_closed_forms():
     np.testing.assert_allclose(lse[0], math.log(5) + 0.3 * qd[30] @ kvd[9], rtol=1e-13)
 
 
+def test_attention_uniform_logit_shift():
+    """Adding the same amount to every logit of a row leaves O unchanged and moves LSE by that
+    amount: every key row gets 1 in a non-value dim, and the query's entry there goes from 0.5
+    to 2.5 (both exact in bf16), a shift of 0.3 * 2 = 0.6 of each scaled logit."""
+    wl = _tiny_attn_workload()
+    wl.kv[:, 23] = 1.0                                  # d_qk = 24, d_v = 16: not a value dim
+    wl.q[:, :, 23] = 0.5
+    rows = [5, 30, 39]
+    sel = np.array([[0, 1, 2, 3, 4, 5, -1, -1],
+                    [3, 11, 0, 25, 7, 30, 29, 2],
+                    [39, 38, 1, 12, -1, 20, 22, 9]], np.int32)
+    o1, l1 = oracle.sparse_mla_rows(wl, rows, sel)
+    wl.q[:, :, 23] = 2.5
+    o2, l2 = oracle.sparse_mla_rows(wl, rows, sel)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l2, l1 + 0.6, rtol=1e-12, atol=1e-12)
+
+
 def test_attention_order_and_padding_invariance_and_numpy_twin():
     wl = _tiny_attn_workload()
     sel = np.array([[3, 11, 0, 25, 7, 30, -1, -1]], np.int32)
