@@ -415,7 +415,8 @@ def run_ours(args, rank, world, local_rank):
     }
     line["cache_append"] = time_cache_append(args, dsa, wl, stream, peaks,
                                              cpu_leg=rank == 0 and not args.no_cpu)
-    line["probes"] = {"dsmem": probe_dsmem(dsa, dev, stream)}
+    line["probes"] = {"dsmem": probe_dsmem(dsa, dev, stream),
+                      "page_stream": probe_page_stream(dsa, wl, dev, stream, roof)}
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     del step, out, lse, wl
@@ -796,6 +797,45 @@ def probe_dsmem(dsa, dev, stream, nbytes=32 * 1024, reps=256):
         t = ns.double().mean().item()
         res[name] = {"clusters": clusters, "gbs_per_sm": round(nbytes * reps / t, 2),
                      "gbs_total": round(2 * clusters * nbytes * reps / t, 1)}
+    return res
+
+
+def probe_page_stream(dsa, wl, dev, stream, roof, reps=5):
+    """Read rate of the decode indexer's key pages (each 64-row page with its 64 scales, in
+    block-table order) with the indexer producer's copies and no arithmetic: the practical
+    ceiling of the indexer's stream on this access pattern, with 1 to 8 CTAs per SM (fewer
+    pages in flight per CTA as they grow); the indexer's own rate is reported as a fraction of
+    the best.  The 1.1 GB of pages exceed L2, so no flush is needed."""
+    if wl.block_table is None or wl.k_scale is not None:
+        return None
+    nb = [(L + 63) // 64 for L in wl.seqlens]
+    ids = torch.cat([wl.block_table[b, :n] for b, n in enumerate(nb)]).contiguous()
+    bb = int(wl.k_idx.shape[1])
+    nbytes = ids.numel() * bb
+    res = {"blocks": ids.numel(), "block_bytes": bb}
+    bad = torch.zeros(1, dtype=torch.int32, device=dev)
+    best = 0.0
+
+    def launch(cps):
+        dsa.check(dsa.dsa_probe_page_stream(wl.k_idx, ids, int(wl.k_idx.shape[0]),
+                                            wl.dims["d_idx"], cps, bad, stream),
+                  "page stream probe")
+
+    for cps in (1, 2, 3, 4, 6, 8):
+        for _ in range(2):                       # warm-up
+            launch(cps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            launch(cps)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        gbs = nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+        res[f"gbs_ctas_per_sm_{cps}"] = round(gbs, 1)
+        best = max(best, gbs)
+    dsa.check(0 if int(bad.item()) == 0 else dsa.DSA_ERR_CUDA, "page stream probe ids")
+    res["gbs"] = round(best, 1)
+    res["indexer_frac_of_stream"] = round(roof["achieved"] / best, 4)
     return res
 
 

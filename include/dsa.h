@@ -425,6 +425,23 @@ DSA_API dsa_status_t dsa_selftest_wait_timeout(int32_t* dev_status, dsa_stream_t
 DSA_API dsa_status_t dsa_probe_dsmem(int32_t clusters, int32_t bytes, int32_t reps, uint64_t* ns,
                                      int32_t* bad, dsa_stream_t stream);
 
+/* Diagnostics: the read rate of the decode indexer's key stream with no arithmetic, the
+ * practical ceiling of that access pattern.  Reads pages of an interleaved indexer key cache
+ * (k_blocks, device, 16-byte aligned, n_blocks pages of 64 key rows of d_idx bytes followed by
+ * their 64 fp32 scales; d_idx 32 or 128) in the order of block_ids (device int32 [n_ids]: page
+ * ids, e.g. the block-table rows of a decode batch) into shared memory with the indexer
+ * producer's copies (one TMA box for the rows, one bulk copy for the scales) and discards them.
+ * ctas_per_sm (1..8) CTAs per SM, each taking a contiguous range of block_ids and keeping as many
+ * pages in flight as fit its share of the SM's shared memory (at most 32;
+ * DSA_ERR_UNSUPPORTED_SHAPE when fewer than 2 fit).  An id outside [0, n_blocks) is skipped; bad
+ * (device int32, zero it first) receives the number of skipped ids plus one per CTA whose bounded
+ * wait ran out (0 expected).  Nothing is written but *bad.  Asynchronous on `stream`: time it
+ * with events on that stream. */
+DSA_API dsa_status_t dsa_probe_page_stream(const void* k_blocks, const int32_t* block_ids,
+                                           int64_t n_ids, int64_t n_blocks, int32_t d_idx,
+                                           int32_t ctas_per_sm, int32_t* bad,
+                                           dsa_stream_t stream);
+
 DSA_API const char* dsa_status_string(dsa_status_t status);
 
 /* DSA_ABI_VERSION of the built library.  2: first-digit histograms (hist of dsa_indexer_scores

@@ -45,7 +45,7 @@ EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_workspace_size",
             "dsa_sparse_mla_workspace_size_for", "dsa_indexer_topk",
             "dsa_indexer_topk_workspace_size", "dsa_forward_chunk_rows_for",
             "dsa_forward_rows", "dsa_indexer_kl_target_dense", "dsa_indexer_kl_backward_dense",
-            "dsa_probe_dsmem")
+            "dsa_probe_dsmem", "dsa_probe_page_stream")
 NOALLOC_SCRATCH_BYTES = 20 << 20
 
 
@@ -95,6 +95,7 @@ def _load():
         "dsa_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "dsa_selftest_wait_timeout": (I32, [P, P]),
         "dsa_probe_dsmem": (I32, [I32, I32, I32, P, P, P]),
+        "dsa_probe_page_stream": (I32, [P, P, I64, I64, I32, I32, P, P]),
         "dsa_indexer_kl_target": (I32, [DP, SP, P, P, P, P, I32, I32, P, P, P]),
         "dsa_indexer_kl_target_dense": (I32, [DP, SP, P, P, P, I32, I32, P, I64, P, P]),
         "dsa_indexer_kl_backward_dense": (I32, [DP, SP, P, P, P, P, P, P, I64, I32, I32, P, P, P,
@@ -341,6 +342,13 @@ def dsa_selftest_wait_timeout(dev_status, stream=None) -> int:
 
 def dsa_probe_dsmem(clusters: int, bytes_: int, reps: int, ns, bad, stream=None) -> int:
     return int(lib.dsa_probe_dsmem(clusters, bytes_, reps, _ptr(ns), _ptr(bad), _stream(stream)))
+
+
+def dsa_probe_page_stream(k_blocks, block_ids, n_blocks: int, d_idx: int, ctas_per_sm: int,
+                          bad, stream=None) -> int:
+    return int(lib.dsa_probe_page_stream(_ptr(k_blocks), _ptr(block_ids), block_ids.numel(),
+                                         n_blocks, d_idx, ctas_per_sm, _ptr(bad),
+                                         _stream(stream)))
 
 
 def dsa_read_device_status(dev_status, stream=None):

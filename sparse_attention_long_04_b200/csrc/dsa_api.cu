@@ -918,6 +918,74 @@ __global__ void __launch_bounds__(kProbeThreads) dsa_probe_dsmem_kernel(int32_t 
   cluster_sync();   // no CTA leaves while its partner may still read nothing of it (symmetry)
 }
 
+// ------------------------------------------------------- key-page stream probe
+
+// Reads the pages of an interleaved indexer key cache (each page 64 key rows of d_idx bytes,
+// then their 64 fp32 scales) into shared memory exactly as the decode indexer's producer does
+// (one 3-D TMA box for the rows and a 256-byte bulk copy for the scales, both evict-first) and
+// computes nothing: the read rate of the indexer's key stream with no arithmetic and no
+// consumer, the practical ceiling of that access pattern.  CTA c takes a contiguous range of
+// the page ids, as an indexer CTA takes a range of one row's pages; its warp loads 32 ids at a
+// time and lane 0 issues their copies into a ring of `slots` page buffers.  An id outside
+// [0, n_blocks) is skipped and counted in *bad, and so is a CTA whose bounded wait ran out (it
+// then stops issuing and waits, again bounded, for the copies in flight).
+constexpr int kStreamMaxSlots = 32;
+__global__ void __launch_bounds__(32) dsa_probe_stream_kernel(
+    const __grid_constant__ CUtensorMap kmap, const uint8_t* k_blocks, const int32_t* ids,
+    int64_t n_ids, int64_t n_blocks, int32_t d_idx, int32_t slots, int32_t* bad) {
+  extern __shared__ uint8_t stream_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(stream_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[kStreamMaxSlots];
+  const int lane = threadIdx.x;
+  const uint32_t key_bytes = 64u * static_cast<uint32_t>(d_idx);
+  const int64_t page_bytes = key_bytes + 256;
+  const uint32_t slot_bytes = (key_bytes + 256u + 1023u) & ~1023u;   // swizzle-atom aligned
+  const int64_t per = (n_ids + gridDim.x - 1) / gridDim.x;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t i1 = i0 + per < n_ids ? i0 + per : n_ids;
+  uint64_t pol = 0;
+  if (lane == 0) {
+    for (int s = 0; s < slots; ++s) mbar_init(smem_u32(&bars[s]), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&kmap);
+    pol = l2_evict_first();
+  }
+  __syncwarp();
+  int issued = 0, miss = 0, ok = 1;
+  for (int64_t c0 = i0; c0 < i1 && ok; c0 += 32) {
+    const int64_t mine = c0 + lane < i1 ? ids[c0 + lane] : 0;
+    const int cnt = i1 - c0 < 32 ? static_cast<int>(i1 - c0) : 32;
+    for (int j = 0; j < cnt; ++j) {
+      const int64_t id = __shfl_sync(0xffffffffu, mine, j);
+      if (lane != 0 || !ok) continue;
+      if (id < 0 || id >= n_blocks) {
+        ++miss;
+        continue;
+      }
+      const int s = issued % slots;
+      if (issued >= slots &&
+          !mbar_wait(smem_u32(&bars[s]), ((issued / slots) - 1) & 1, nullptr)) {
+        ok = 0;
+        continue;
+      }
+      const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * slot_bytes);
+      mbar_arrive_expect_tx(smem_u32(&bars[s]), key_bytes + 256u);
+      tma_load_3d_hint(dst, &kmap, smem_u32(&bars[s]), 0, 0, static_cast<int32_t>(id), pol);
+      bulk_load_g2s_hint(dst + key_bytes, k_blocks + id * page_bytes + key_bytes, 256u,
+                         smem_u32(&bars[s]), pol);
+      ++issued;
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+  }
+  if (lane != 0) return;
+  // never leave a copy in flight into the shared memory of an exiting CTA
+  for (int k = max(0, issued - slots); k < issued; ++k)
+    if (!mbar_wait(smem_u32(&bars[k % slots]), (k / slots) & 1, nullptr)) ok = 0;
+  if (!ok) ++miss;
+  if (miss) atomicAdd(bad, miss);
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -1269,6 +1337,37 @@ dsa_status_t dsa_probe_dsmem(int32_t clusters, int32_t bytes, int32_t reps, uint
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, dsa_probe_dsmem_kernel, bytes, reps, ns, bad) != cudaSuccess)
     return DSA_ERR_CUDA;
+  return launch_status();
+}
+
+dsa_status_t dsa_probe_page_stream(const void* k_blocks, const int32_t* block_ids,
+                                   int64_t n_ids, int64_t n_blocks, int32_t d_idx,
+                                   int32_t ctas_per_sm, int32_t* bad, dsa_stream_t stream) {
+  if (!k_blocks || !block_ids || !bad || n_ids <= 0 || n_blocks <= 0 ||
+      n_blocks > INT32_MAX || (d_idx != 32 && d_idx != 128) || ctas_per_sm < 1 ||
+      ctas_per_sm > 8)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_blocks) || (reinterpret_cast<uintptr_t>(block_ids) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(bad) & 3u) != 0)
+    return DSA_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (device_info(&info) != DSA_OK) return DSA_ERR_CUDA;
+  // the SM's shared memory split over its CTAs (1 KB of each reserved by the hardware, the
+  // barriers static, 1 KB of alignment slack)
+  const int64_t slot_bytes = (64 * d_idx + 256 + 1023) / 1024 * 1024;
+  const int64_t budget = (int64_t(info.max_smem) + 1024) / ctas_per_sm - 1024 - 512 - 1024;
+  const int64_t slots = std::min<int64_t>(kStreamMaxSlots, budget / slot_bytes);
+  if (slots < 2) return DSA_ERR_UNSUPPORTED_SHAPE;
+  const int smem = static_cast<int>(slots * slot_bytes + 1024);
+  CUtensorMap kmap;
+  if (make_block_map(&kmap, k_blocks, uint64_t(n_blocks), uint32_t(d_idx)) != DSA_OK)
+    return DSA_ERR_CUDA;
+  if (prepare_kernel(dsa_probe_stream_kernel, smem) != DSA_OK) return DSA_ERR_CUDA;
+  const int64_t grid = std::min<int64_t>(int64_t(info.sm_count) * ctas_per_sm, n_ids);
+  dsa_probe_stream_kernel<<<static_cast<unsigned>(grid), 32, smem,
+                            reinterpret_cast<cudaStream_t>(stream)>>>(
+      kmap, static_cast<const uint8_t*>(k_blocks), block_ids, n_ids, n_blocks, d_idx,
+      static_cast<int32_t>(slots), bad);
   return launch_status();
 }
 

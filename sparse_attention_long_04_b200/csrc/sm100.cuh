@@ -214,8 +214,8 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tiled load of the box at (x = inner element, y = row) into shared memory; completion is
-// counted in bytes on `bar`.  x * element size must be a multiple of 16 bytes.
+// 3-D tiled load of the box at (x = inner element, y = row, z = plane) into shared memory;
+// completion is counted in bytes on `bar`.  x * element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t x, int32_t y, int32_t z) {
   asm volatile(
@@ -225,6 +225,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 2-D tiled load of the box at (x = inner element, y = row); as tma_load_3d.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t x, int32_t y) {
   asm volatile(

@@ -176,6 +176,28 @@ def test_wait_selftest_argument_errors(dsa):
     assert dsa.dsa_selftest_wait_timeout(FAKE + 2, 0) == dsa.DSA_ERR_MISALIGNED
 
 
+def test_probe_argument_errors(dsa):
+    """The two diagnostics check counts, sizes and alignment before any launch."""
+    lib, INV, MIS = dsa.lib, dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_MISALIGNED
+    ok = dict(base=FAKE, ids=FAKE, n_ids=4, n_blocks=4, d_idx=128, cps=2, bad=FAKE)
+
+    def stream(**kw):
+        a = dict(ok, **kw)
+        return lib.dsa_probe_page_stream(a["base"], a["ids"], a["n_ids"], a["n_blocks"],
+                                         a["d_idx"], a["cps"], a["bad"], 0)
+
+    for kw in (dict(base=None), dict(ids=None), dict(bad=None), dict(n_ids=0),
+               dict(n_blocks=0), dict(n_blocks=1 << 31), dict(d_idx=0), dict(d_idx=64),
+               dict(cps=0), dict(cps=9)):
+        assert stream(**kw) == INV, kw
+    for kw in (dict(base=FAKE + 8), dict(ids=FAKE + 2), dict(bad=FAKE + 2)):
+        assert stream(**kw) == MIS, kw
+    assert lib.dsa_probe_dsmem(0, 32768, 4, FAKE, FAKE, 0) == INV
+    assert lib.dsa_probe_dsmem(1, 100, 4, FAKE, FAKE, 0) == INV
+    assert lib.dsa_probe_dsmem(1, 32768, 0, FAKE, FAKE, 0) == INV
+    assert lib.dsa_probe_dsmem(1, 32768, 4, FAKE + 4, FAKE, 0) == MIS
+
+
 def test_indexer_training_argument_errors(dsa):
     """The target and backward calls check their pointers, alignment, shapes and rows before
     any launch."""
