@@ -16,7 +16,9 @@
 //
 // Roles: warp 0 issues TMA (Q once, then per tile two 64-row key boxes plus a bulk copy of each
 // box's k_scale), warp 1 issues the tcgen05.mma, warp 2 owns the TMEM allocation, warp 3
-// computes c[t,j], warps 4.. run the epilogue.  Key stages are a ring of STAGES buffers; the
+// computes c[t,j] (and in decode then issues the tiles of odd index while warp 0 issues the
+// even ones: the key stream's rate grows with the threads that issue copies), warps 4.. run the
+// epilogue.  Key stages are a ring of STAGES buffers; the
 // accumulators are a ring of ACC buffers in TMEM so the epilogue of tile i overlaps the MMA of
 // later tiles.  Decode (one query row, N = 64) runs two epilogue warpgroups on alternate tiles;
 // prefill (N = 256) splits each tile's columns over four warpgroups, one query row each.
@@ -69,6 +71,9 @@ template <int H_I, int D_I, int QPG>
 struct IndexerCfg {
   static constexpr int N = H_I * QPG;                 // MMA N: (row, head) columns
   static constexpr int STAGES = QPG == 1 ? 5 : 8;
+  // decode streams its keys from two producer warps (tiles of even and odd index), which keeps
+  // more page copies moving than one issuing thread does
+  static constexpr int PRODUCERS = QPG == 1 ? 2 : 1;
   static constexpr int ACC = QPG == 1 ? 4 : 2;        // TMEM accumulator ring
   static constexpr int EPI_WARPS = QPG == 1 ? 8 : 16;    // prefill: one query row per warpgroup
   static constexpr bool TILE_SPLIT = QPG == 1;        // warpgroups take alternate tiles
@@ -124,6 +129,7 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
   const bool hist_on = C::HIST && p.hist != nullptr;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ int last_s[2];   // the last tile each producer issued (-1: none)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -188,19 +194,23 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 0 || (C::PRODUCERS > 1 && warp == 3)) {
+    // ------------------------------------------------------------------ TMA producers
+    // producer pr issues tiles pr, pr + PRODUCERS, ... (warp 3 has finished c[t,j] above)
+    const int pr = warp == 0 ? 0 : 1;
+    int last = -1;
     if (lane == 0) {
       // decode streams the key cache once: evict-first, so that the score slab the top-k reads
       // next stays in L2
       const uint64_t pol = l2_evict_first();
       tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&qmap);
-      mbar_arrive_expect_tx(smem_u32(qbar), C::Q_BYTES);
-      tma_load_2d(smem_u32(sQ), &qmap, smem_u32(qbar), 0, grow0 * H_I);
-      int issued = 0;
+      if (pr == 0) {
+        tma_prefetch_desc(&qmap);
+        mbar_arrive_expect_tx(smem_u32(qbar), C::Q_BYTES);
+        tma_load_2d(smem_u32(sQ), &qmap, smem_u32(qbar), 0, grow0 * H_I);
+      }
       const int n_blocks = (n_keys + 63) / 64;
-      for (int it = 0; it < n_tiles; ++it) {
+      for (int it = pr; it < n_tiles; it += C::PRODUCERS) {
         const int s = it % C::STAGES;
         if (it >= C::STAGES &&
             !mbar_wait(smem_u32(&empty[s]), ((it / C::STAGES) - 1) & 1, &abort_s)) {
@@ -290,13 +300,35 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, QPG>::THREADS, QPG == 1 ?
           }
           }
         }
-        ++issued;
+        last = it;
       }
-      // drain: never leave a copy in flight into shared memory of an exiting CTA
-      for (int it = max(0, issued - C::STAGES); it < issued; ++it)
-        mbar_wait(smem_u32(&full[it % C::STAGES]), (it / C::STAGES) & 1, nullptr);
-      mbar_wait(smem_u32(qbar), 0, nullptr);
     }
+    // drain: never leave a copy in flight into shared memory of an exiting CTA.  Each stage
+    // waits for the last tile issued into it (every earlier use was consumed before that tile
+    // could be issued, so only this phase can be outstanding).
+    if constexpr (C::PRODUCERS == 1) {
+      if (lane == 0)
+        for (int it = max(0, last + 1 - C::STAGES); it <= last; ++it)
+          mbar_wait(smem_u32(&full[it % C::STAGES]), (it / C::STAGES) & 1, nullptr);
+    } else {
+      if (lane == 0) last_s[pr] = last;
+      __syncwarp();
+      named_bar_sync(1, 64);                   // both producer warps are done issuing
+      if (pr == 0 && lane == 0)
+        for (int st = 0; st < C::STAGES; ++st) {
+          int t_last = -1;
+          for (int q = 0; q < C::PRODUCERS; ++q)
+            for (int t = last_s[q]; t >= 0 && t > last_s[q] - C::PRODUCERS * C::STAGES;
+                 t -= C::PRODUCERS)
+              if (t % C::STAGES == st) {
+                t_last = max(t_last, t);
+                break;
+              }
+          if (t_last >= 0)
+            mbar_wait(smem_u32(&full[st]), (t_last / C::STAGES) & 1, nullptr);
+        }
+    }
+    if (pr == 0 && lane == 0) mbar_wait(smem_u32(qbar), 0, nullptr);
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {

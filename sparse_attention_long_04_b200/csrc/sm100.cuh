@@ -114,6 +114,12 @@ __device__ __forceinline__ bool warp_mbar_wait(uint32_t bar, uint32_t parity,
   return ok != 0;
 }
 
+// Barrier `id` (1..15; 0 is __syncthreads) over `count` threads (a multiple of 32): the warps
+// of a subset of the CTA, each arriving whole.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Programmatic dependent launch: a kernel launched with programmatic stream serialization may
 // start while the previous kernel of the stream is still running; it waits here, before reading
 // anything, until that kernel has completed and its writes are visible (a no-op otherwise).
